@@ -1,0 +1,215 @@
+"""fp64 CPU oracle of the TurboQuant KV-vector hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import this package. It shares no code with the CUDA library: the arithmetic lives in
+``tq_oracle.c`` (plain C, fp64, one vector at a time), built into ``liboracle.so`` by
+``build()``; this module only marshals numpy arrays.
+
+Parity status of each function (what pins it) is listed in the repository's design notes;
+every function here is pinned by a test in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile tq_oracle.c (gcc, -O2, OpenMP, no fast-math) into liboracle.so."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-fno-fast-math", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = ctypes.CDLL(_LIB)
+    return _lib
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
+
+
+def _f64(a):
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _u8(a):
+    return np.ascontiguousarray(a, dtype=np.uint8)
+
+
+def threads() -> int:
+    """OpenMP threads the oracle uses (OMP_NUM_THREADS, else the process's CPU set)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env:
+        return int(env)
+    return len(os.sched_getaffinity(0))
+
+
+# ----------------------------------------------------------------------------- API
+def round_half(x) -> np.ndarray:
+    """Round to IEEE binary16 (ties to even), returned as fp64."""
+    lib = _load()
+    a = _f64(x).ravel()
+    out = np.empty_like(a)
+    lib.orc_round_half_array(ctypes.c_int64(a.size), _p(a), _p(out))
+    return out.reshape(np.shape(x))
+
+
+def codebook(d: int, bits: int, law: str = "beta"):
+    """Lloyd-Max codebook for one rotated coordinate: (centroids[L], boundaries[L-1],
+    normalised mse, iterations). law='beta' is the exact finite-d law, 'gauss' its limit."""
+    lib = _load()
+    nl = 1 << bits
+    c = np.zeros(nl)
+    t = np.zeros(nl - 1)
+    mse = ctypes.c_double()
+    it = ctypes.c_int()
+    st = lib.orc_codebook(d, bits, 0 if law == "beta" else 1, _p(c), _p(t), ctypes.byref(mse), ctypes.byref(it))
+    if st != 0:
+        raise RuntimeError(f"orc_codebook({d}, {bits}, {law}) -> {st}")
+    return c, t, mse.value, it.value
+
+
+def cell_mass(d: int, bits: int, t, law: str = "beta") -> np.ndarray:
+    lib = _load()
+    out = np.zeros(1 << bits)
+    lib.orc_cell_mass(d, bits, 0 if law == "beta" else 1, _p(_f64(t)), _p(out))
+    return out
+
+
+class Quantized:
+    """Unpacked quantizer output: idx [n,d] uint8, sbit [n,m] uint8, nhat/ghat (binary16 values
+    as fp64), the exact n and gamma, y [n,d] and z [n,m] for band checks, flags [n]."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+
+def quantize(x, pi, s, c, t, bits: int, qjl: bool, keep_yz: bool = True) -> Quantized:
+    lib = _load()
+    x = _f64(x)
+    nv, d = x.shape
+    pi = _f32(pi)
+    m = int(np.shape(s)[0]) if qjl else 0
+    s_ = _f32(s) if qjl else np.zeros(1, np.float32)
+    idx = np.zeros((nv, d), np.uint8)
+    sbit = np.zeros((nv, max(m, 1)), np.uint8)
+    nhat, ghat, nex, gex = (np.zeros(nv) for _ in range(4))
+    y = np.zeros((nv, d)) if keep_yz else None
+    z = np.zeros((nv, max(m, 1))) if (keep_yz and qjl) else None
+    flags = np.zeros(nv, np.int32)
+    st = lib.orc_quantize(ctypes.c_int64(nv), d, m, bits, int(qjl), _p(x), _p(pi), _p(s_),
+                          _p(_f64(c)), _p(_f64(t)), _p(idx), _p(sbit), _p(nhat), _p(ghat),
+                          _p(nex), _p(gex), _p(y), _p(z), _p(flags))
+    if st != 0:
+        raise RuntimeError(f"orc_quantize -> {st}")
+    return Quantized(idx=idx, sbit=sbit[:, :m], nhat=nhat, ghat=ghat, n_exact=nex, g_exact=gex,
+                     y=y, z=(z[:, :m] if z is not None else None), flags=flags)
+
+
+def logits(idx, sbit, nhat, ghat, pi, s, c, q, qjl: bool, scale: float = 1.0) -> np.ndarray:
+    """scale * n^ (<Pi q, c[idx]> + gamma^ sqrt(pi/2)/m <S q, s>) for every (query, key)."""
+    lib = _load()
+    idx = _u8(idx)
+    nk, d = idx.shape
+    m = int(np.shape(s)[0]) if qjl else 0
+    q = _f64(q).reshape(-1, d)
+    out = np.zeros((q.shape[0], nk))
+    st = lib.orc_logits(ctypes.c_int64(nk), d, m, 0, int(qjl), _p(idx),
+                        _p(_u8(sbit) if qjl else np.zeros(1, np.uint8)), _p(_f64(nhat)),
+                        _p(_f64(ghat) if qjl else np.zeros(1)), _p(_f32(pi)),
+                        _p(_f32(s) if qjl else np.zeros(1, np.float32)), _p(_f64(c)),
+                        ctypes.c_int64(q.shape[0]), _p(q), ctypes.c_double(scale), _p(out))
+    if st != 0:
+        raise RuntimeError(f"orc_logits -> {st}")
+    return out
+
+
+def exact_dot(keys, q, scale: float = 1.0) -> np.ndarray:
+    lib = _load()
+    keys = _f64(keys)
+    nk, d = keys.shape
+    q = _f64(q).reshape(-1, d)
+    out = np.zeros((q.shape[0], nk))
+    lib.orc_exact_dot(ctypes.c_int64(nk), d, _p(keys), ctypes.c_int64(q.shape[0]), _p(q),
+                      ctypes.c_double(scale), _p(out))
+    return out
+
+
+def reconstruct(idx, sbit, nhat, ghat, pi, s, c, qjl: bool) -> np.ndarray:
+    lib = _load()
+    idx = _u8(idx)
+    nv, d = idx.shape
+    m = int(np.shape(s)[0]) if qjl else 0
+    out = np.zeros((nv, d))
+    lib.orc_reconstruct(ctypes.c_int64(nv), d, m, 0, int(qjl), _p(idx),
+                        _p(_u8(sbit) if qjl else np.zeros(1, np.uint8)), _p(_f64(nhat)),
+                        _p(_f64(ghat) if qjl else np.zeros(1)), _p(_f32(pi)),
+                        _p(_f32(s) if qjl else np.zeros(1, np.float32)), _p(_f64(c)), _p(out))
+    return out
+
+
+def pv(idx, nhat, pi, c, P) -> np.ndarray:
+    """softmax(P[h]) . V^ for every head h, values reconstructed token by token."""
+    lib = _load()
+    idx = _u8(idx)
+    nt, d = idx.shape
+    P = _f32(P)
+    nh = P.shape[0]
+    out = np.zeros((nh, d))
+    st = lib.orc_pv(ctypes.c_int64(nt), d, 0, _p(idx), _p(_f64(nhat)), _p(_f32(pi)), _p(_f64(c)),
+                    nh, _p(P), _p(out))
+    if st != 0:
+        raise RuntimeError(f"orc_pv -> {st}")
+    return out
+
+
+def topk(idx, sbit, nhat, ghat, pi, s, c, q, k: int, qjl: bool = True):
+    lib = _load()
+    idx = _u8(idx)
+    ndb, d = idx.shape
+    m = int(np.shape(s)[0]) if qjl else 0
+    q = _f64(q).reshape(-1, d)
+    oi = np.zeros((q.shape[0], k), np.int64)
+    osc = np.zeros((q.shape[0], k))
+    st = lib.orc_topk(ctypes.c_int64(ndb), d, m, 0, int(qjl), _p(idx),
+                      _p(_u8(sbit) if qjl else np.zeros(1, np.uint8)), _p(_f64(nhat)),
+                      _p(_f64(ghat) if qjl else np.zeros(1)), _p(_f32(pi)),
+                      _p(_f32(s) if qjl else np.zeros(1, np.float32)), _p(_f64(c)),
+                      ctypes.c_int64(q.shape[0]), _p(q), k, _p(oi), _p(osc))
+    if st != 0:
+        raise RuntimeError(f"orc_topk -> {st}")
+    return oi, osc
+
+
+def exact_topk(xdb, q, k: int):
+    lib = _load()
+    xdb = _f32(xdb)
+    ndb, d = xdb.shape
+    q = _f64(q).reshape(-1, d)
+    oi = np.zeros((q.shape[0], k), np.int64)
+    osc = np.zeros((q.shape[0], k))
+    st = lib.orc_exact_topk(ctypes.c_int64(ndb), d, _p(xdb), ctypes.c_int64(q.shape[0]), _p(q), k,
+                            _p(oi), _p(osc))
+    if st != 0:
+        raise RuntimeError(f"orc_exact_topk -> {st}")
+    return oi, osc

@@ -1,0 +1,181 @@
+"""Pins for the oracle's quantizer (CPU only): rotation, nearest centroid, residual, QJL
+sketch and the statistics the pages state (kurtosis, cosine, unbiasedness)."""
+import itertools
+import math
+
+import numpy as np
+import pytest
+from scipy import stats
+
+import oracle
+import tq_inputs as ti
+from conftest import golden
+
+
+def test_rotation_is_orthogonal():
+    # the rotation is the Q factor of the QR of a Gaussian matrix (a2a-mcp.org, stage 1)
+    for d in (8, 128, 200):
+        p = ti.haar_rotation(d, 11)
+        assert np.max(np.abs(p.T @ p - np.eye(d))) < 1e-12
+        p32 = p.astype(np.float32).astype(np.float64)
+        assert np.max(np.abs(p32.T @ p32 - np.eye(d))) < 2e-7
+
+
+def test_rotation_gaussianises_outlier_data():
+    # ai-coding.wiselychen.com, TurboQuant+: kurtosis 900.4 -> 2.9 (Gaussian 3.0). A Haar
+    # rotation maps any fixed unit vector to a uniform point of the sphere, whose
+    # coordinates have kurtosis 3d/(d+2); pooled over independent rotations of one outlier
+    # key that is what the generator must give.
+    d = 128
+    g = golden("kurtosis.txt")
+    keys = ti.bf16_to_f64(ti.key_stream(2, 0, 0, 256, d))
+    u = keys / np.linalg.norm(keys, axis=1, keepdims=True)
+    assert stats.kurtosis(u.ravel(), fisher=False) > 10.0   # outlier channels: heavy tails
+    x = u[0]
+    y = np.concatenate([ti.haar_rotation(d, 7000 + k) @ x for k in range(400)]) * math.sqrt(d)
+    k_after = stats.kurtosis(y, fisher=False)
+    se = math.sqrt(24.0 / y.size)
+    assert abs(k_after - 3 * d / (d + 2)) < 3 * se
+    assert abs(k_after - g["kurt_after"]) < 0.1 and k_after < g["kurt_gauss"]
+
+
+def _codebook(d, bits):
+    c, t, _, _ = oracle.codebook(d, bits)
+    return c, t
+
+
+@pytest.mark.parametrize("d,bits", [(4, 2), (8, 3), (6, 1), (8, 4)])
+def test_nearest_centroid_exhaustive(d, bits):
+    # y_i -> argmin_k |y_i - c_k| over all levels (ties to the lower index), checked
+    # against brute force, with Pi = I so that y = u.
+    c, t = _codebook(d, bits)
+    rng = np.random.default_rng(d * 10 + bits)
+    x = rng.standard_normal((300, d))
+    q = oracle.quantize(x, np.eye(d), np.zeros((1, d)), c, t, bits, qjl=False)
+    u = x / np.linalg.norm(x, axis=1, keepdims=True)
+    brute = np.argmin(np.abs(u[:, :, None] - c[None, None, :]), axis=2)
+    assert np.array_equal(q.idx, brute)
+    if d <= 4:
+        # the product codebook: the per-coordinate choice is the vector argmin
+        grid = np.array(list(itertools.product(c, repeat=d)))
+        gidx = np.array(list(itertools.product(range(len(c)), repeat=d)))
+        best = np.argmin(((u[:, None, :] - grid[None]) ** 2).sum(-1), axis=1)
+        assert np.array_equal(q.idx, gidx[best])
+
+
+def test_boundary_ties_go_to_lower_cell():
+    # a coordinate exactly on a boundary takes the lower cell: idx = #{k : y > t_k}.
+    # x = (+-1/2, ...) has norm exactly 1, and the boundaries include -1/2, 0 and 1/2.
+    d = 4
+    c = np.array([-0.75, -0.25, 0.25, 0.75])
+    t = np.array([-0.5, 0.0, 0.5])
+    x = np.array([[0.5, -0.5, 0.5, -0.5], [0.0, 0.0, 0.0, 1.0]])
+    q = oracle.quantize(x, np.eye(d), np.zeros((1, d)), c, t, 2, qjl=False)
+    assert q.idx[0].tolist() == [2, 0, 2, 0]
+    assert q.idx[1].tolist() == [1, 1, 1, 3]
+    # and the real codebook's middle boundary is exactly 0
+    c, t = _codebook(8, 2)
+    q = oracle.quantize(np.eye(8)[:1], np.eye(8), np.zeros((1, 8)), c, t, 2, qjl=False)
+    assert q.idx[0, 1:].tolist() == [1] * 7
+
+
+def test_residual_sketch_and_norms():
+    d = m = 128
+    bits = 2
+    c, t = _codebook(d, bits)
+    pi = ti.haar_rotation(d, 5)
+    s = ti.gaussian_sketch(m, d, 6)
+    x = ti.c1_keys(64).astype(np.float64)
+    q = oracle.quantize(x, pi, s, c, t, bits, qjl=True)
+    n = np.linalg.norm(x, axis=1)
+    u = x / n[:, None]
+    pi32 = pi.astype(np.float32).astype(np.float64)
+    s32 = s.astype(np.float32).astype(np.float64)
+    assert np.allclose(q.y, u @ pi32.T, atol=1e-14)
+    r = u - c[q.idx] @ pi32
+    assert np.allclose(q.g_exact, np.linalg.norm(r, axis=1), rtol=1e-13)
+    # |r| = |y - c[idx]| since Pi is orthogonal (up to its fp32 rounding)
+    assert np.allclose(q.g_exact, np.linalg.norm(q.y - c[q.idx], axis=1), rtol=1e-6)
+    assert np.allclose(q.z, r @ s32.T, atol=1e-13)
+    assert np.array_equal(q.sbit, (q.z >= 0).astype(np.uint8))
+    assert np.array_equal(q.nhat, n.astype(np.float16).astype(np.float64))
+    assert np.array_equal(q.ghat, q.g_exact.astype(np.float16).astype(np.float64))
+    assert np.all(q.flags == 0)
+
+
+def test_range_flags_and_zero_vector():
+    d = 8
+    c, t = _codebook(d, 2)
+    x = np.zeros((3, d))
+    x[1, 0] = 70000.0
+    x[2, 3] = np.inf
+    q = oracle.quantize(x, np.eye(d), np.eye(d), c, t, 2, qjl=True)
+    assert q.nhat[0] == 0.0 and q.flags[0] == 0
+    assert q.flags[1] & 1 and q.flags[2] & 2
+    # the zero vector scores 0 against any query
+    lg = oracle.logits(q.idx[:1], q.sbit[:1], q.nhat[:1], q.ghat[:1], np.eye(d), np.eye(d), c,
+                       np.ones((1, d)), qjl=True)
+    assert lg[0, 0] == 0.0
+
+
+def test_cosine_three_bit():
+    # a2a-mcp.org, stage 2: cosine 0.983+ at 3 bits. For a Lloyd-Max quantizer the centroid
+    # condition gives E<u, x_mse> = E|x_mse|^2 = 1 - D, so the cosine is about sqrt(1 - D).
+    d, bits = 128, 3
+    c, t, mse, _ = oracle.codebook(d, bits)
+    pi = ti.haar_rotation(d, 21)
+    x = np.random.default_rng(3).standard_normal((3000, d))
+    q = oracle.quantize(x, pi, np.zeros((1, d)), c, t, bits, qjl=False)
+    u = x / np.linalg.norm(x, axis=1, keepdims=True)
+    xm = c[q.idx] @ pi.astype(np.float32).astype(np.float64)
+    cos = (u * xm).sum(1) / np.linalg.norm(xm, axis=1)
+    assert abs(cos.mean() - math.sqrt(1 - mse)) < 1e-3
+    assert round(cos.mean(), 3) >= golden("cosine_3bit.txt")["cos_3bit"]
+    # the MSE itself, measured: E|u - x_mse|^2 = D
+    assert abs(((u - xm) ** 2).sum(1).mean() / mse - 1) < 0.02
+
+
+def _estimator_draws(qjl_scale=1.0, K=4000):
+    """<y, x~> - <y, x> for one fixed unit x and query y over K independent sketches S."""
+    d = m = 64
+    bits = 2
+    c, t = _codebook(d, bits)
+    pi = ti.haar_rotation(d, 31)
+    rng = np.random.default_rng(32)
+    x = rng.standard_normal(d)
+    x /= np.linalg.norm(x)
+    # the MSE stage does not depend on S: find the residual first, then take a query with
+    # a sizeable component along it so that a biased correction shows clearly
+    q0 = oracle.quantize(x[None], pi, np.zeros((1, d)), c, t, bits, qjl=False)
+    r = x - c[q0.idx[0]] @ pi.astype(np.float32).astype(np.float64)
+    y = rng.standard_normal(d) + 4.0 * r / np.linalg.norm(r)
+    diffs = np.empty(K)
+    for k in range(K):
+        s = ti.gaussian_sketch(m, d, 100000 + k)
+        q = oracle.quantize(x[None], pi, s, c, t, bits, qjl=True)
+        # exact gamma and norm: the fp16 storage is not part of the unbiasedness claim
+        xt = oracle.reconstruct(q.idx, q.sbit, q.n_exact, q.g_exact, pi, s, c, qjl=True)[0]
+        xm = oracle.reconstruct(q.idx, q.sbit, q.n_exact, q.g_exact, pi, s, c, qjl=False)[0]
+        xt = xm + qjl_scale * (xt - xm)
+        diffs[k] = y @ xt - y @ x
+    return diffs, r, y, m
+
+
+def test_qjl_unbiased_with_closed_form_variance():
+    # blog.hotdry.top, QJL residual correction: E<y, x~> = <y, x>.
+    diffs, r, y, m = _estimator_draws()
+    K = diffs.size
+    sd = diffs.std(ddof=1)
+    assert abs(diffs.mean()) < 3 * sd / math.sqrt(K)
+    # Var = (1/m) [ (pi/2) |r|^2 |y|^2 - <y, r>^2 ]  (i.i.d. rows of S)
+    var = ((math.pi / 2) * (r @ r) * (y @ y) - (y @ r) ** 2) / m
+    lo = stats.chi2.ppf(0.0005, K - 1) / (K - 1)
+    hi = stats.chi2.ppf(0.9995, K - 1) / (K - 1)
+    assert lo * var < sd ** 2 < hi * var
+
+
+def test_dropping_the_sqrt_pi_over_2_factor_is_detected():
+    # ai-coding.wiselychen.com: a QJL correction without the exact factor is biased.
+    # Planted mistake: scale the correction by 1/sqrt(pi/2); the bias must exceed 10 sigma.
+    diffs, r, y, m = _estimator_draws(qjl_scale=1 / math.sqrt(math.pi / 2))
+    assert abs(diffs.mean()) > 10 * diffs.std(ddof=1) / math.sqrt(diffs.size)
