@@ -1,0 +1,34 @@
+// Derived operands of a codec: transposes of Pi and S, and M = S Pi^T (the sketch applied in
+// the rotated domain: S r = S Pi^T (y - c[idx]) because Pi^T Pi = I; blog.hotdry.top
+// "TurboQuant vector-search compression", section "QJL residual correction").
+#include "tq_device.cuh"
+
+__global__ void k_prepare(PrepParams p) {
+    const int64_t n_pi = (int64_t)p.D * p.D;
+    const int64_t n_s = (int64_t)p.D * p.Mp;
+    const int64_t total = n_pi + (p.qjl ? 2 * n_s : 0);
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        if (e < n_pi) {
+            int j = (int)(e / p.D), i = (int)(e % p.D);          // PiT[j][i] = Pi[i][j]
+            p.piT[e] = (i < p.d && j < p.d) ? p.pi[(int64_t)i * p.d + j] : 0.f;
+        } else if (e < n_pi + n_s) {
+            int64_t f = e - n_pi;
+            int j = (int)(f / p.Mp), k = (int)(f % p.Mp);        // ST[j][k] = S[k][j]
+            p.sT[f] = (j < p.d && k < p.m) ? p.s[(int64_t)k * p.d + j] : 0.f;
+        } else {
+            int64_t f = e - n_pi - n_s;
+            int i = (int)(f / p.Mp), k = (int)(f % p.Mp);        // MT[i][k] = sum_j S[k][j] Pi[i][j]
+            double acc = 0.0;
+            if (i < p.d && k < p.m)
+                for (int j = 0; j < p.d; ++j)
+                    acc += (double)p.s[(int64_t)k * p.d + j] * (double)p.pi[(int64_t)i * p.d + j];
+            p.mT[f] = (float)acc;
+        }
+    }
+}
+
+cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
+    k_prepare<<<296, 256, 0, st>>>(p);
+    return cudaGetLastError();
+}

@@ -1,0 +1,342 @@
+// C-ABI entry points of libtq: argument checks, codebook-derived constants, workspace
+// layout and kernel launches. Every entry point is declared and documented in include/tq.h.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+
+#include "tq.h"
+#include "tq_device.cuh"
+
+size_t tq_logits_prologue_smem(const TqDims& t, int g);
+
+namespace {
+
+constexpr int kNumSms = 148;
+
+size_t align_up(size_t v) { return (v + TQ_ALIGN - 1) / TQ_ALIGN * TQ_ALIGN; }
+
+bool aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+// shape checks shared by every call
+int check_codec(const tq_codec* c, bool need_prep) {
+    if (!c) return TQ_ERR_ARG;
+    if (c->d < 8 || c->d > TQ_MAX_D || c->d % 8) return TQ_ERR_UNSUPPORTED;
+    if (c->qjl != 0 && c->qjl != 1) return TQ_ERR_ARG;
+    if (c->qjl && (c->m < 8 || c->m > TQ_MAX_D || c->m % 8)) return TQ_ERR_UNSUPPORTED;
+    if (c->mse_bits < 1 || c->mse_bits > (c->qjl ? 3 : 4)) return TQ_ERR_UNSUPPORTED;
+    if (!c->pi || !c->centroids || (c->qjl && !c->s)) return TQ_ERR_ARG;
+    if (!aligned(c->pi, 4) || (c->qjl && !aligned(c->s, 4))) return TQ_ERR_ARG;
+    if (need_prep) {
+        if (!c->prep || !aligned(c->prep, 256)) return TQ_ERR_ARG;
+        if (c->prep_bytes < tq_prep_bytes(c)) return TQ_ERR_WORKSPACE;
+    }
+    return TQ_OK;
+}
+
+TqDims dims_of(const tq_codec* c) { return tq_dims(c->d, c->m, c->mse_bits, c->qjl); }
+
+// centroids (host, fp64) -> boundaries, fp32 copies, +-1 plane coefficients, binary16 table
+int codebook_consts(const tq_codec* c, TqCodebookConsts* k) {
+    std::memset(k, 0, sizeof(*k));
+    const int B = c->mse_bits, L = 1 << B;
+    const double* cc = c->centroids;
+    double mx = 0.0;
+    for (int i = 0; i < L; ++i) {
+        if (!std::isfinite(cc[i])) return TQ_ERR_ARG;
+        mx = std::fmax(mx, std::fabs(cc[i]));
+        if (i && !(cc[i] > cc[i - 1])) return TQ_ERR_ARG;
+    }
+    for (int i = 0; i < L; ++i)
+        if (std::fabs(cc[i] + cc[L - 1 - i]) > 1e-12 * mx) return TQ_ERR_ARG;  // symmetric
+    for (int i = 0; i + 1 < L; ++i) k->bounds[i] = (float)(0.5 * (cc[i] + cc[i + 1]));
+    for (int i = 0; i < L; ++i) {
+        k->cent[i] = (float)cc[i];
+        k->lut_half[i] = __half_as_ushort(__float2half_rn((float)cc[i]));
+    }
+    // Walsh coefficients a_S = 2^-B sum_idx c[idx] prod_{k in S} s_k(idx), s_k = 2 bit_k - 1,
+    // for the odd sets the estimator uses: {0}, {1}, {2}, {0,1,2}
+    const int sets[4] = {1, 2, 4, 7};
+    const int nplanes = B == 3 ? 4 : B;
+    double sum = 0.0;
+    for (int pl = 0; pl < nplanes; ++pl) {
+        double a = 0.0;
+        for (int idx = 0; idx < L; ++idx) {
+            double prod = 1.0;
+            for (int kb = 0; kb < B; ++kb)
+                if (sets[pl] >> kb & 1) prod *= (idx >> kb & 1) ? 1.0 : -1.0;
+            a += cc[idx] * prod;
+        }
+        a /= L;
+        k->plane_coef[pl] = (float)a;
+        sum += a;
+    }
+    k->plane_sum = (float)sum;
+    if (c->qjl) {  // the odd expansion must reproduce every centroid
+        for (int idx = 0; idx < L; ++idx) {
+            double v = 0.0;
+            for (int pl = 0; pl < nplanes; ++pl) {
+                double prod = 1.0;
+                for (int kb = 0; kb < B; ++kb)
+                    if (sets[pl] >> kb & 1) prod *= (idx >> kb & 1) ? 1.0 : -1.0;
+                v += k->plane_coef[pl] * prod;
+            }
+            if (std::fabs(v - cc[idx]) > 1e-6 * mx) return TQ_ERR_ARG;
+        }
+    }
+    return TQ_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+// workspace regions after the status word
+struct LogitsWs { size_t qfrag, qscale, total; };
+LogitsWs logits_ws(const TqDims& t, int64_t n_streams, int g) {
+    const int ntiles = g > 4 ? 2 : 1;
+    LogitsWs w;
+    size_t off = TQ_STATUS_BYTES;
+    w.qfrag = off; off = align_up(off + (size_t)n_streams * ntiles * t.nmg * 4 * 64 * 4);
+    w.qscale = off; off = align_up(off + (size_t)n_streams * ntiles * 4 * 16);
+    w.total = off;
+    return w;
+}
+
+struct PvWs { int nsplit, bps; size_t part, ml, total; };
+PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
+    PvWs w;
+    const int64_t nb = (n_tok + 31) / 32;
+    int64_t bps = (nb * n_streams + 4 * kNumSms - 1) / (4 * kNumSms);
+    if (bps < 8) bps = 8;
+    if (bps > nb) bps = nb;
+    if (bps < 1) bps = 1;
+    w.bps = (int)bps;
+    w.nsplit = (int)((nb + bps - 1) / bps);
+    size_t off = TQ_STATUS_BYTES;
+    w.part = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * t.D * 4);
+    w.ml = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * 8);
+    w.total = off;
+    return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tq_abi_version(void) { return 1; }
+
+const char* tq_status_string(int s) {
+    switch (s) {
+        case TQ_OK: return "ok";
+        case TQ_ERR_ARG: return "invalid argument";
+        case TQ_ERR_UNSUPPORTED: return "unsupported shape";
+        case TQ_ERR_CUDA: return "CUDA runtime error";
+        case TQ_ERR_RANGE: return "norm overflowed binary16 or input not finite";
+        case TQ_ERR_TIMEOUT: return "timeout";
+        case TQ_ERR_NOCONV: return "codebook did not converge";
+        case TQ_ERR_WORKSPACE: return "workspace or prepared buffer too small";
+    }
+    return "unknown status";
+}
+
+int tq_make_codebook(int d, int mse_bits, double* centroids, double* bounds, double* mse) {
+    if (!centroids || !bounds) return TQ_ERR_ARG;
+    if (d < 3 || d > 4096 || mse_bits < 1 || mse_bits > 8) return TQ_ERR_UNSUPPORTED;
+    const int r = tq_host_codebook(d, mse_bits, centroids, bounds, mse);
+    return r == 0 ? TQ_OK : (r == -6 ? TQ_ERR_NOCONV : TQ_ERR_ARG);
+}
+
+size_t tq_block_bytes(const tq_codec* c) {
+    if (check_codec(c, false) != TQ_OK) return 0;
+    return dims_of(c).block_bytes;
+}
+
+size_t tq_record_bytes(const tq_codec* c) { return tq_block_bytes(c) / 32; }
+
+size_t tq_packed_bytes(const tq_codec* c, int64_t n_streams, int64_t n_tok) {
+    if (n_streams < 0 || n_tok < 0) return 0;
+    return tq_block_bytes(c) * (size_t)n_streams * (size_t)((n_tok + 31) / 32);
+}
+
+size_t tq_prep_bytes(const tq_codec* c) {
+    if (check_codec(c, false) != TQ_OK) return 0;
+    return tq_prep_layout(dims_of(c)).total;
+}
+
+int tq_prepare(const tq_codec* c, void* stream) {
+    int st = check_codec(c, true);
+    if (st != TQ_OK) return st;
+    const TqDims t = dims_of(c);
+    const TqPrepLayout L = tq_prep_layout(t);
+    uint8_t* base = static_cast<uint8_t*>(c->prep);
+    PrepParams p;
+    p.pi = c->pi; p.s = c->s;
+    p.piT = reinterpret_cast<float*>(base + L.piT);
+    p.sT = reinterpret_cast<float*>(base + L.sT);
+    p.mT = reinterpret_cast<float*>(base + L.mT);
+    p.d = t.d; p.m = t.m; p.D = t.D; p.Mp = t.Mp; p.qjl = t.qjl;
+    return cuda_status(tq_launch_prepare(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t tq_workspace_bytes(const tq_codec* c, int op, int64_t a, int64_t b, int64_t cc) {
+    if (check_codec(c, false) != TQ_OK) return 0;
+    const TqDims t = dims_of(c);
+    switch (op) {
+        case TQ_OP_QUANTIZE:
+        case TQ_OP_DEQUANTIZE:
+            return TQ_STATUS_BYTES;
+        case TQ_OP_LOGITS:
+            if (a < 0 || b < 1 || cc < 1 || cc > 8) return 0;
+            return logits_ws(t, a * b, (int)cc).total;
+        case TQ_OP_PV:
+            if (a < 0 || b < 1 || cc < 1 || cc > 8) return 0;
+            return pv_ws(t, a, b, (int)cc).total;
+        case TQ_OP_TOPK:
+            return 0;
+    }
+    return 0;
+}
+
+int tq_reset_status(void* ws, void* stream) {
+    if (!ws) return TQ_ERR_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_get_status(void* ws, void* stream) {
+    if (!ws) return TQ_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    if (cudaMemcpyAsync(&word, ws, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
+    if (word) {
+        if (cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return TQ_ERR_CUDA;
+        if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
+    }
+    return (word & TQ_FLAG_RANGE) ? TQ_ERR_RANGE : TQ_OK;
+}
+
+int tq_quantize(const tq_codec* c, const void* x, tq_dtype dtype, int64_t n_streams, int64_t n_tok,
+                int64_t x_stream_stride, void* packed, void* ws, size_t ws_bytes, void* stream) {
+    int st = check_codec(c, true);
+    if (st != TQ_OK) return st;
+    if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_streams < 0 || n_tok < 0) return TQ_ERR_ARG;
+    if (n_streams == 0 || n_tok == 0) return TQ_OK;
+    if (!x || !packed || !ws) return TQ_ERR_ARG;
+    if (!aligned(packed, 16) || !aligned(x, dtype == TQ_F32 ? 4 : 2) || !aligned(ws, 4)) return TQ_ERR_ARG;
+    if (n_streams > 1 && x_stream_stride < n_tok * c->d) return TQ_ERR_ARG;
+    if (ws_bytes < TQ_STATUS_BYTES) return TQ_ERR_WORKSPACE;
+    const TqDims t = dims_of(c);
+    const TqPrepLayout L = tq_prep_layout(t);
+    QuantParams p;
+    p.x = x; p.dtype = dtype;
+    p.n_streams = n_streams; p.n_tok = n_tok; p.x_stride = x_stream_stride;
+    p.nb = (n_tok + 31) / 32;
+    if (p.n_streams * p.nb > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    p.packed = static_cast<uint8_t*>(packed);
+    p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
+    p.mT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.mT);
+    p.status = static_cast<uint32_t*>(ws);
+    p.t = t;
+    if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    return cuda_status(tq_launch_quantize(p, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+              tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
+              size_t ws_bytes, void* stream) {
+    int st = check_codec(c, true);
+    if (st != TQ_OK) return st;
+    if (!c->qjl) return TQ_ERR_ARG;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return TQ_ERR_UNSUPPORTED;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_seq == 0 || n_tok + n_tail == 0) return TQ_OK;
+    if (!q || !out || !ws || (n_tok > 0 && !packed) || (n_tail > 0 && !tail)) return TQ_ERR_ARG;
+    if ((n_tok > 0 && !aligned(packed, 16)) || !aligned(out, 4) || !aligned(ws, 256) ||
+        !aligned(q, q_dtype == TQ_F32 ? 4 : 2) || (n_tail > 0 && !aligned(tail, 2)))
+        return TQ_ERR_ARG;
+    if (!std::isfinite(scale)) return TQ_ERR_ARG;
+    const TqDims t = dims_of(c);
+    const int64_t n_streams = n_seq * n_kv;
+    const LogitsWs W = logits_ws(t, n_streams, g);
+    if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
+    const TqPrepLayout L = tq_prep_layout(t);
+    LogitsParams p;
+    p.packed = static_cast<const uint8_t*>(packed);
+    p.q = q; p.q_dtype = q_dtype;
+    p.tail = static_cast<const uint16_t*>(tail);
+    p.out = out;
+    p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
+    p.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
+    p.qfrag = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + W.qfrag);
+    p.qscale = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.qscale);
+    p.n_seq = n_seq; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
+    p.n_kv = n_kv; p.g = g; p.ntiles = g > 4 ? 2 : 1; p.n_tail = n_tail;
+    p.scale = scale;
+    p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
+    const int64_t work = n_streams * p.ntiles * p.nb;
+    int64_t bpt = work / (kNumSms * 16 * 2);
+    if (bpt < 2) bpt = 2;
+    if (bpt > 32) bpt = 32;
+    p.blocks_per_task = (int)bpt;
+    const int64_t tasks = n_streams * p.ntiles * ((p.nb + bpt - 1) / bpt);
+    if ((tasks + 3) / 4 > 0x7fffffffLL || n_streams > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    p.t = t;
+    if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    return cuda_status(tq_launch_logits(p, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int64_t n_tok, const float* P, int g,
+          float* out, void* ws, size_t ws_bytes, void* stream) {
+    int st = check_codec(c, true);
+    if (st != TQ_OK) return st;
+    if (c->qjl) return TQ_ERR_ARG;
+    if (g != 1 && g != 2 && g != 4 && g != 8) return TQ_ERR_UNSUPPORTED;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 1) return TQ_ERR_ARG;
+    if (n_seq == 0) return TQ_OK;
+    if (!packed_v || !P || !out || !ws) return TQ_ERR_ARG;
+    if (!aligned(packed_v, 16) || !aligned(P, 4) || !aligned(out, 4) || !aligned(ws, 256)) return TQ_ERR_ARG;
+    const TqDims t = dims_of(c);
+    const int64_t n_streams = n_seq * n_kv;
+    const PvWs W = pv_ws(t, n_streams, n_tok, g);
+    if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
+    PvParams p;
+    p.packed = static_cast<const uint8_t*>(packed_v);
+    p.P = P; p.out = out; p.pi = c->pi;
+    p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.part);
+    p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.ml);
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
+    p.g = g; p.nsplit = W.nsplit; p.blocks_per_split = W.bps;
+    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    p.t = t;
+    if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    return cuda_status(tq_launch_pv(p, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,
+            float* score, void* ws, size_t ws_bytes, void* stream) {
+    (void)c; (void)packed_db; (void)n_db; (void)q; (void)n_q; (void)k; (void)idx; (void)score; (void)ws;
+    (void)ws_bytes; (void)stream;
+    return TQ_ERR_UNSUPPORTED;
+}
+
+int tq_dequantize(const tq_codec* c, const void* packed, int64_t n_streams, int64_t n_tok, float* out, void* ws,
+                  size_t ws_bytes, void* stream) {
+    int st = check_codec(c, false);
+    if (st != TQ_OK) return st;
+    if (n_streams < 0 || n_tok < 0) return TQ_ERR_ARG;
+    if (n_streams == 0 || n_tok == 0) return TQ_OK;
+    if (!packed || !out || !aligned(packed, 16) || !aligned(out, 4)) return TQ_ERR_ARG;
+    (void)ws; (void)ws_bytes;
+    DequantParams p;
+    p.packed = static_cast<const uint8_t*>(packed);
+    p.out = out; p.pi = c->pi; p.s = c->s;
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
+    p.kappa = c->qjl ? (float)(std::sqrt(M_PI / 2.0) / c->m) : 0.f;
+    p.t = dims_of(c);
+    if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    return cuda_status(tq_launch_dequant(p, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

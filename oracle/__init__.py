@@ -104,7 +104,8 @@ class Quantized:
         self.__dict__.update(kw)
 
 
-def quantize(x, pi, s, c, t, bits: int, qjl: bool, keep_yz: bool = True) -> Quantized:
+def quantize(x, pi, s, c, t, bits: int, qjl: bool, keep_yz: bool = True, idx_in=None) -> Quantized:
+    """Quantize rows of x. With idx_in, the given indices replace the nearest-centroid step."""
     lib = _load()
     x = _f64(x)
     nv, d = x.shape
@@ -119,7 +120,8 @@ def quantize(x, pi, s, c, t, bits: int, qjl: bool, keep_yz: bool = True) -> Quan
     flags = np.zeros(nv, np.int32)
     st = lib.orc_quantize(ctypes.c_int64(nv), d, m, bits, int(qjl), _p(x), _p(pi), _p(s_),
                           _p(_f64(c)), _p(_f64(t)), _p(idx), _p(sbit), _p(nhat), _p(ghat),
-                          _p(nex), _p(gex), _p(y), _p(z), _p(flags))
+                          _p(nex), _p(gex), _p(y), _p(z), _p(flags),
+                          _p(_u8(idx_in).reshape(nv, d) if idx_in is not None else None))
     if st != 0:
         raise RuntimeError(f"orc_quantize -> {st}")
     return Quantized(idx=idx, sbit=sbit[:, :m], nhat=nhat, ghat=ghat, n_exact=nex, g_exact=gex,

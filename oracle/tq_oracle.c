@@ -248,11 +248,13 @@ int orc_cell_mass(int d, int B, int law, const double* t, double* mass) {
  *   stored n^ = half(n), gamma^ = half(gamma)
  * Optional outputs y (n x d) and z (n x m) let the tests find coordinates that lie within
  * a tolerance band of a decision boundary. flags[v] bit 0: n^ overflowed binary16,
- * bit 1: non-finite input.                                                               */
+ * bit 1: non-finite input. When idx_in is given, those indices replace the nearest-centroid
+ * step and the residual, gamma and signs follow from them (used to check the later steps
+ * of a vector whose index was decided differently inside the tolerance band).            */
 int orc_quantize(int64_t nv, int d, int m, int B, int qjl, const double* x, const float* pi,
                  const float* s, const double* c, const double* t, uint8_t* idx, uint8_t* sbit,
                  double* nhat, double* ghat, double* n_exact, double* g_exact, double* y_out,
-                 double* z_out, int32_t* flags) {
+                 double* z_out, int32_t* flags, const uint8_t* idx_in) {
     if (nv < 0 || d < 1 || d > 1024 || B < 1 || B > 8 || (qjl && (m < 1 || m > 1024))) return ORC_ERR_ARG;
     int nb = (1 << B) - 1;
 #pragma omp parallel for schedule(dynamic, 16)
@@ -275,7 +277,7 @@ int orc_quantize(int64_t nv, int d, int m, int B, int qjl, const double* x, cons
         for (int i = 0; i < d; ++i) {
             int k = 0;
             for (int b = 0; b < nb; ++b) k += y[i] > t[b];
-            idx[v * d + i] = (uint8_t)k;
+            idx[v * d + i] = idx_in ? idx_in[v * d + i] : (uint8_t)k;
             if (y_out) y_out[v * d + i] = y[i];
         }
         for (int j = 0; j < d; ++j) {

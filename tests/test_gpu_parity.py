@@ -1,0 +1,277 @@
+"""GPU parity of the CUDA hot path against the fp64 oracle (through the C ABI).
+
+Tolerances: indices and sign bits bit-exact except coordinates within 1e-5 of a decision
+boundary (at most 1e-4 of all coordinates may differ there); stored |x| and gamma within one
+binary16 ulp; logits |dl| / (scale |q| |x|) <= 1e-3; reconstructions |dx~|_inf / |x| <= 1e-3;
+P.V |do|_inf / sum_t w_t |v_t| <= 1e-3.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import tq_inputs as ti
+from gpu_helpers import (TOL, compare_codes, gpu_quantize, make_codec, to_dev_bf16, to_dev_f32, torch_cuda, tq,
+                         unpack)
+
+pytestmark = pytest.mark.gpu
+
+
+def _cb(d, B):
+    c, t, _, _ = oracle.codebook(d, B)
+    return c, t
+
+
+# ----------------------------------------------------------------------------- quantize
+def test_quantize_c1_tiny_keys():
+    cfg = ti.C1
+    d = m = 128
+    B = 2
+    pi, s = cfg.pi(), cfg.s()
+    x = ti.c1_keys()
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, st = gpu_quantize(codec, to_dev_f32(x), 1, x.shape[0])
+    assert st == tq().TQ_OK
+    idx, sbit, nhat, ghat = unpack(codec, packed, 1, x.shape[0])
+    c, t = _cb(d, B)
+    ref = oracle.quantize(x.astype(np.float64), pi, s, c, t, B, qjl=True)
+    nb, nm, na = compare_codes(idx[0], sbit[0], nhat[0], ghat[0], ref, t, x=x.astype(np.float64), pi=pi, s=s,
+                               c=c, t=t, B=B)
+    print(f"c1: {nb} coordinates in the band, {nm} differ, of {na}")
+
+
+@pytest.mark.parametrize("B", [1, 2, 3])
+def test_quantize_ragged_streams_bf16(B):
+    # 3 streams of 77 tokens with a stream stride larger than n_tok*d (a cache with room)
+    d = m = 128
+    pi, s = ti.haar_rotation(d, 71), ti.gaussian_sketch(m, d, 72)
+    n_tok, stride_tok = 77, 90
+    bits = np.concatenate([ti.key_stream(2, 0, h, stride_tok) for h in range(3)])
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, st = gpu_quantize(codec, to_dev_bf16(bits), 3, n_tok, stride_tok * d)
+    assert st == tq().TQ_OK
+    idx, sbit, nhat, ghat = unpack(codec, packed, 3, n_tok)
+    c, t = _cb(d, B)
+    x = ti.bf16_to_f64(bits).reshape(3, stride_tok, d)[:, :n_tok]
+    for h in range(3):
+        ref = oracle.quantize(x[h], pi, s, c, t, B, qjl=True)
+        compare_codes(idx[h], sbit[h], nhat[h], ghat[h], ref, t, x=x[h], pi=pi, s=s, c=c, t=t, B=B)
+    # unused records of the last block are zero
+    raw = packed.cpu().numpy()
+    from tq_format import unpack_keys
+    i2, s2, n2, g2 = unpack_keys(raw, d, m, B, 3, 96)
+    assert not i2[:, n_tok:].any() and not s2[:, n_tok:].any() and not n2[:, n_tok:].any()
+
+
+@pytest.mark.parametrize("B", [3, 4])
+def test_quantize_values(B):
+    d = 128
+    pi = ti.C3.pi()
+    bits = np.concatenate([ti.value_stream(h, 1000) for h in range(2)])
+    codec = make_codec(d, 0, B, False, pi, None)
+    packed, st = gpu_quantize(codec, to_dev_bf16(bits), 2, 1000)
+    assert st == tq().TQ_OK
+    idx, nhat = unpack(codec, packed, 2, 1000)
+    c, t = _cb(d, B)
+    x = ti.bf16_to_f64(bits).reshape(2, 1000, d)
+    for h in range(2):
+        ref = oracle.quantize(x[h], pi, None, c, t, B, qjl=False)
+        compare_codes(idx[h], None, nhat[h], None, ref, t, qjl=False)
+
+
+@pytest.mark.parametrize("B", [1, 3])
+def test_quantize_d200_vector_search(B):
+    d = m = 200
+    pi, s = ti.C5.pi(), ti.C5.s()
+    x = ti.c5_rows("db", 0, 3000)
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, st = gpu_quantize(codec, to_dev_f32(x), 1, 3000)
+    assert st == tq().TQ_OK
+    idx, sbit, nhat, ghat = unpack(codec, packed, 1, 3000)
+    c, t = _cb(d, B)
+    ref = oracle.quantize(x.astype(np.float64), pi, s, c, t, B, qjl=True)
+    compare_codes(idx[0], sbit[0], nhat[0], ghat[0], ref, t, x=x.astype(np.float64), pi=pi, s=s, c=c, t=t, B=B)
+
+
+def test_quantize_range_status_and_zero_vector():
+    d = m = 128
+    pi, s = ti.haar_rotation(d, 81), ti.gaussian_sketch(m, d, 82)
+    x = np.random.default_rng(0).standard_normal((40, d)).astype(np.float32)
+    x[3] = 0.0
+    x[7] *= 1e5                       # |x| ~ 1.1e6 > 65504
+    codec = make_codec(d, m, 2, True, pi, s)
+    packed, st = gpu_quantize(codec, to_dev_f32(x), 1, 40)
+    assert st == tq().TQ_ERR_RANGE
+    idx, sbit, nhat, ghat = unpack(codec, packed, 1, 40)
+    assert nhat[0, 3] == 0.0 and math.isinf(nhat[0, 7])
+    x[7] = 1.0
+    x[9, 5] = np.nan
+    packed, st = gpu_quantize(codec, to_dev_f32(x), 1, 40)
+    assert st == tq().TQ_ERR_RANGE
+    x[9, 5] = 0.0
+    packed, st = gpu_quantize(codec, to_dev_f32(x), 1, 40)
+    assert st == tq().TQ_OK
+
+
+# ----------------------------------------------------------------------------- logits
+def _logits_gpu(codec, packed, n_seq, n_kv, n_tok, q_dev, g, tail_dev, n_tail, scale):
+    torch = torch_cuda()
+    m = tq()
+    out = torch.full((n_seq, n_kv * g, n_tok + n_tail), float("nan"), dtype=torch.float32, device="cuda")
+    ws = m.workspace(codec.workspace_bytes(m.TQ_OP_LOGITS, n_seq, n_kv, g))
+    m.tq_logits(codec, packed, n_seq, n_kv, n_tok, q_dev, g, tail_dev, n_tail, scale, out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _check_logits(got, want, q, xnorm, scale):
+    err = np.abs(got - want) / (abs(scale) * np.linalg.norm(q, axis=-1)[:, None] * xnorm[None, :])
+    assert np.all(np.isfinite(got))
+    assert err.max() <= TOL, f"max normalised logit error {err.max():.3e}"
+    return err.max()
+
+
+def test_logits_c1_tiny():
+    cfg = ti.C1
+    d = m = 128
+    B = 2
+    pi, s = cfg.pi(), cfg.s()
+    x = ti.c1_keys()
+    q = ti.c1_queries()
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, _ = gpu_quantize(codec, to_dev_f32(x), 1, 4096)
+    # 8 queries as one sequence with 8 kv heads? No: one kv head, g = 8 query heads
+    got = _logits_gpu(codec, packed, 1, 1, 4096, to_dev_f32(q[None]), 8, None, 0, 1.0)[0]
+    idx, sbit, nhat, ghat = unpack(codec, packed, 1, 4096)
+    c, t = _cb(d, B)
+    want = oracle.logits(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, q.astype(np.float64), qjl=True)
+    _check_logits(got, want, q.astype(np.float64), np.linalg.norm(x.astype(np.float64), axis=1), 1.0)
+    # end to end against the oracle's own quantization (the codes agree outside the band)
+    ref = oracle.quantize(x.astype(np.float64), pi, s, c, t, B, qjl=True)
+    same = np.all(ref.idx == idx[0], axis=1) & np.all(ref.sbit == sbit[0], axis=1)
+    want2 = oracle.logits(ref.idx, ref.sbit, ref.nhat, ref.ghat, pi, s, c, q.astype(np.float64), qjl=True)
+    _check_logits(got[:, same], want2[:, same], q.astype(np.float64),
+                  np.linalg.norm(x.astype(np.float64), axis=1)[same], 1.0)
+    assert same.mean() > 0.99
+
+
+@pytest.mark.parametrize("B,g", [(1, 1), (2, 2), (3, 4), (2, 8), (3, 8)])
+def test_logits_gqa_ragged_with_tail(B, g):
+    d = m = 128
+    pi, s = ti.haar_rotation(d, 91), ti.gaussian_sketch(m, d, 92)
+    n_seq, n_kv, n_tok, n_tail = 2, 3, 301, 5
+    keys = np.stack([np.stack([ti.key_stream(4, sq, h, n_tok + n_tail) for h in range(n_kv)]) for sq in range(n_seq)])
+    comp = np.ascontiguousarray(keys[:, :, :n_tok])
+    tail = np.ascontiguousarray(keys[:, :, n_tok:])
+    qb = ti.decode_queries(9, n_seq, n_kv * g)
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(comp.reshape(-1, d)), n_seq * n_kv, n_tok)
+    scale = 1.0 / math.sqrt(d)
+    got = _logits_gpu(codec, packed, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, to_dev_bf16(tail), n_tail, scale)
+    idx, sbit, nhat, ghat = unpack(codec, packed, n_seq * n_kv, n_tok)
+    c, t = _cb(d, B)
+    q = ti.bf16_to_f64(qb)
+    kf = ti.bf16_to_f64(keys)
+    for sq in range(n_seq):
+        for h in range(n_kv):
+            st = sq * n_kv + h
+            qh = q[sq, h * g:(h + 1) * g]
+            want = oracle.logits(idx[st], sbit[st], nhat[st], ghat[st], pi, s, c, qh, qjl=True, scale=scale)
+            xn = np.linalg.norm(kf[sq, h, :n_tok], axis=1)
+            _check_logits(got[sq, h * g:(h + 1) * g, :n_tok], want, qh, xn, scale)
+            wt = oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)
+            _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1), scale)
+
+
+def test_logits_d200_codec():
+    d = m = 200
+    pi, s = ti.C5.pi(), ti.C5.s()
+    x = ti.c5_rows("db", 0, 700)
+    q = ti.c5_rows("q", 0, 4)
+    for B in (1, 3):
+        codec = make_codec(d, m, B, True, pi, s)
+        packed, _ = gpu_quantize(codec, to_dev_f32(x), 1, 700)
+        got = _logits_gpu(codec, packed, 1, 1, 700, to_dev_f32(q[None]), 4, None, 0, 1.0)[0]
+        idx, sbit, nhat, ghat = unpack(codec, packed, 1, 700)
+        c, t = _cb(d, B)
+        want = oracle.logits(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, q.astype(np.float64), qjl=True)
+        _check_logits(got, want, q.astype(np.float64), np.linalg.norm(x.astype(np.float64), axis=1), 1.0)
+
+
+# ----------------------------------------------------------------------------- P.V
+def _pv_gpu(codec, packed, n_seq, n_kv, n_tok, P_dev, g):
+    torch = torch_cuda()
+    m = tq()
+    out = torch.full((n_seq, n_kv * g, codec.c.d), float("nan"), dtype=torch.float32, device="cuda")
+    ws = m.workspace(codec.workspace_bytes(m.TQ_OP_PV, n_seq * n_kv, n_tok, g))
+    m.tq_pv(codec, packed, n_seq, n_kv, n_tok, P_dev, g, out, ws)
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _check_pv(got, want, P, nhat):
+    w = np.exp(P - P.max(axis=1, keepdims=True))
+    w /= w.sum(axis=1, keepdims=True)
+    denom = w @ nhat
+    err = np.max(np.abs(got - want), axis=1) / denom
+    assert np.all(np.isfinite(got))
+    assert err.max() <= TOL, f"max normalised P.V error {err.max():.3e}"
+    return err.max()
+
+
+@pytest.mark.parametrize("B,g,n_tok", [(3, 4, 5000), (4, 4, 4097), (2, 1, 100), (4, 8, 777), (1, 2, 64)])
+def test_pv(B, g, n_tok):
+    d = 128
+    pi = ti.C3.pi()
+    n_kv = 2
+    bits = np.concatenate([ti.value_stream(h, n_tok) for h in range(n_kv)])
+    codec = make_codec(d, 0, B, False, pi, None)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(bits), n_kv, n_tok)
+    P = ti.logits_p(n_kv * g, n_tok)
+    got = _pv_gpu(codec, packed, 1, n_kv, n_tok, to_dev_f32(P), g)[0]
+    idx, nhat = unpack(codec, packed, n_kv, n_tok)
+    c, t = _cb(d, B)
+    for h in range(n_kv):
+        Ph = P[h * g:(h + 1) * g]
+        want = oracle.pv(idx[h], nhat[h], pi, c, Ph)
+        _check_pv(got[h * g:(h + 1) * g], want, Ph.astype(np.float64), nhat[h])
+
+
+def test_pv_one_hot_and_uniform():
+    d, B, n_tok = 128, 3, 300
+    pi = ti.C3.pi()
+    bits = ti.value_stream(0, n_tok)
+    codec = make_codec(d, 0, B, False, pi, None)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(bits), 1, n_tok)
+    P = np.zeros((2, n_tok), np.float32)
+    P[1, 123] = 1e4
+    got = _pv_gpu(codec, packed, 1, 1, n_tok, to_dev_f32(P), 2)[0]
+    idx, nhat = unpack(codec, packed, 1, n_tok)
+    c, _ = _cb(d, B)
+    vh = oracle.reconstruct(idx[0], None, nhat[0], None, pi, None, c, qjl=False)
+    assert np.max(np.abs(got[0] - vh.mean(0))) <= TOL * nhat[0].mean()
+    assert np.max(np.abs(got[1] - vh[123])) <= TOL * nhat[0, 123]
+
+
+# ----------------------------------------------------------------------------- reconstruction
+@pytest.mark.parametrize("qjl,B", [(True, 2), (True, 3), (False, 4)])
+def test_dequantize_reconstruction(qjl, B):
+    d = m = 128
+    pi, s = ti.haar_rotation(d, 61), ti.gaussian_sketch(m, d, 62)
+    x = ti.c1_keys(500)
+    codec = make_codec(d, m, B, qjl, pi, s if qjl else None)
+    packed, _ = gpu_quantize(codec, to_dev_f32(x), 1, 500)
+    torch = torch_cuda()
+    out = torch.zeros((500, d), dtype=torch.float32, device="cuda")
+    tq().tq_dequantize(codec, packed, 1, 500, out)
+    got = out.cpu().numpy().astype(np.float64)
+    c, t = _cb(d, B)
+    if qjl:
+        idx, sbit, nhat, ghat = unpack(codec, packed, 1, 500)
+        want = oracle.reconstruct(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, qjl=True)
+    else:
+        idx, nhat = unpack(codec, packed, 1, 500)
+        want = oracle.reconstruct(idx[0], None, nhat[0], None, pi, None, c, qjl=False)
+    err = np.max(np.abs(got - want), axis=1) / np.linalg.norm(x.astype(np.float64), axis=1)
+    assert err.max() <= TOL
