@@ -1,0 +1,388 @@
+"""Benchmark of the TurboQuant KV-vector hot path on B200.
+
+Workload (default, "c4_batched_decode"): a batched decode step of a serving engine with a
+TurboQuant key cache, shaped like Llama-3.1-8B attention (8 kv-heads, head_dim 128, GQA 4):
+  * cache: 64 sequences x 8 kv-heads x 8192 tokens, keys at b = 3 (2-bit Lloyd-Max + 1-bit
+    QJL, m = 128), 52 B per key (218 MB packed);
+  * one step = tq_quantize of a 64 x 512-token append (262,144 bf16 vectors) followed by
+    tq_logits of 64 x 32 query heads (bf16) over the whole cache (4,194,304 keys).
+Synthetic data with the pages' laws: key norms 4-182x value norms, 4 outlier channels per
+kv-head scaled x20, queries N(0, 1); generated on the device from a seeded generator.
+
+One JSON line on rank 0. `value` = cache keys scanned per second by whole steps (the
+quantize of the append included); per-kernel times, the logits roofline and the quantize
+throughput are reported beside it. `--impl reference` times the fp64 CPU oracle on a
+bounded sample of the same step instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tq_logits keys/s & HBM GB/s (% of ~8 TB/s); tq_quantize vectors/s"
+N_SEQ, N_KV, N_TOK, G, D = 64, 8, 8192, 4, 128
+N_APPEND = 512
+MSE_BITS = 2  # b = 3 keys
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, \
+        "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- device workload
+def make_keys_device(torch, gen, n_streams, n_tok, heads_per_seq, d=D):
+    """Keys with the decode law on the device, bf16 [n_streams, n_tok, d]; stream = seq*8 + head."""
+    import tq_inputs as ti
+    out = torch.empty((n_streams, n_tok, d), dtype=torch.bfloat16, device="cuda")
+    mult = torch.ones((heads_per_seq, d), device="cuda")
+    for h in range(heads_per_seq):
+        mult[h, torch.as_tensor(ti.outlier_channels(4, h, d), device="cuda")] = 20.0
+    chunk = 64
+    lo, hi = math.log(4.0), math.log(182.0)
+    for s0 in range(0, n_streams, chunk):
+        s1 = min(n_streams, s0 + chunk)
+        heads = torch.arange(s0, s1, device="cuda") % heads_per_seq
+        g = torch.randn((s1 - s0, n_tok, d), generator=gen, device="cuda") * mult[heads][:, None, :]
+        v = torch.randn((s1 - s0, n_tok, d), generator=gen, device="cuda")
+        rho = torch.exp(lo + (hi - lo) * torch.rand((s1 - s0, n_tok, 1), generator=gen, device="cuda"))
+        k = g / g.norm(dim=-1, keepdim=True) * rho * v.norm(dim=-1, keepdim=True)
+        out[s0:s1] = k.to(torch.bfloat16)
+        del g, v, k
+    return out
+
+
+def run_gpu(args, world, rank, local):
+    import torch
+
+    import kv_cache_vector_03_b200 as tq
+    import tq_inputs as ti
+
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(20260000 + rank)
+    cfg = ti.C4
+    pi = torch.from_numpy(cfg.pi().astype(np.float32))
+    s = torch.from_numpy(cfg.s().astype(np.float32))
+    codec = tq.Codec(D, D, MSE_BITS, True, pi, s)
+    n_streams = N_SEQ * N_KV
+
+    # resident cache (quantized once, outside the timed region)
+    keys = make_keys_device(torch, gen, n_streams, N_TOK, N_KV)
+    cache = torch.empty(codec.packed_bytes(n_streams, N_TOK), dtype=torch.uint8, device="cuda")
+    wsq = tq.workspace(codec.workspace_bytes(tq.TQ_OP_QUANTIZE))
+    tq.tq_quantize(codec, keys, n_streams, N_TOK, N_TOK * D, cache, wsq)
+    del keys
+    append = make_keys_device(torch, gen, n_streams, N_APPEND, N_KV)
+    append_packed = torch.empty(codec.packed_bytes(n_streams, N_APPEND), dtype=torch.uint8, device="cuda")
+    q = torch.randn((N_SEQ, N_KV * G, D), generator=gen, device="cuda").to(torch.bfloat16)
+    out = torch.empty((N_SEQ, N_KV * G, N_TOK), dtype=torch.float32, device="cuda")
+    wsl = tq.workspace(codec.workspace_bytes(tq.TQ_OP_LOGITS, N_SEQ, N_KV, G))
+    scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    assert tq.tq_get_status(wsq) == tq.TQ_OK
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        tq.tq_quantize(codec, append, n_streams, N_APPEND, N_APPEND * D, append_packed, wsq, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        tq.tq_logits(codec, cache, N_SEQ, N_KV, N_TOK, q, G, None, 0, scale, out, wsl, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    total_ms = start.elapsed_time(stop)
+    t_quant = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+    t_logit = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+    ms_step = max_over_ranks(world, total_ms / args.steps)
+    t_quant = max_over_ranks(world, t_quant)
+    t_logit = max_over_ranks(world, t_logit)
+    clocks = clk.summary()
+
+    keys_per_step = n_streams * N_TOK
+    vec_per_step = n_streams * N_APPEND
+    rec = codec.record_bytes()
+    logit_bytes = keys_per_step * rec + N_SEQ * N_KV * G * N_TOK * 4 + N_SEQ * N_KV * G * D * 2
+    quant_bytes = vec_per_step * (D * 2 + rec)
+    logit_gbs = logit_bytes / (t_logit * 1e-3) / 1e9
+    quant_flops = vec_per_step * 2 * (2 * D * D)  # two d x d contractions per vector
+    quant_tf = quant_flops / (t_quant * 1e-3) / 1e12
+
+    # end to end through the public API: append + queries from pinned host memory in, logits out
+    h_append = torch.empty(append.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_append.copy_(append.cpu())
+    h_q = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_q.copy_(q.cpu())
+    h_out = torch.empty(out.shape, dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        append.copy_(h_append, non_blocking=True)
+        q.copy_(h_q, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(3, min(args.steps, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(world, start.elapsed_time(stop) / e_steps)
+    h2d = h_append.numel() * 2 + h_q.numel() * 2
+    d2h = h_out.numel() * 4
+
+    # kernels launched per step: quantize 1, logits 2 (prologue + stream)
+    launches_per_step = 3
+    dominant = "tq_logits" if t_logit >= t_quant else "tq_quantize"
+    logits_roof = {"kernel": "tq_logits (prologue + int8-MMA stream)", "bound": "hbm", "achieved": round(logit_gbs, 1),
+                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(logit_gbs / peaks["hbm_gbs"], 4),
+                   "traffic": None, "peak_kind": peak_kind,
+                   "algorithmic_bytes_per_launch": logit_bytes}
+    # fp32 FMA peak of the quantize kernel's CUDA-core path: 148 SMs x 128 FMA/clk x 2 flop x clock
+    fma_peak = 148 * 128 * 2 * (clocks["sm_mhz"] or peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    quant_roof = {"kernel": "tq_quantize (fp32 CUDA-core)", "bound": "alu", "achieved": round(quant_tf, 2),
+                  "peak": round(fma_peak, 1), "unit": "TFLOP/s", "frac": round(quant_tf / fma_peak, 4),
+                  "traffic": None, "algorithmic_flops_per_launch": quant_flops,
+                  "peak_kind": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x median SM clock"}
+    line = {
+        "metric": METRIC, "value": keys_per_step * world / (ms_step * 1e-3), "unit": "keys/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8 codes, int8/fp32 arithmetic",
+        "data": "synthetic (device-generated, pages' key law)",
+        "config": {"workload": "c4_batched_decode: 64 seq x 8 kv-heads x 8192 tok, d=128, b=3 keys; "
+                               "step = quantize 64x512x8 append + logits 64x32 q-heads",
+                   "seq_len": N_TOK, "n_seq_per_gpu": N_SEQ, "kv_heads": N_KV, "q_heads": N_KV * G, "head_dim": D,
+                   "key_bits": MSE_BITS + 1, "record_bytes": rec, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (packed cache 218 MB + 67 MB logits); no flush"},
+        "kernels": {
+            "tq_logits": {"ms": t_logit, "keys_per_s": keys_per_step / (t_logit * 1e-3), "GB_per_s": logit_gbs,
+                          "frac_of_8TBps": logit_gbs / 8000.0, "frac_of_measured_hbm": logit_gbs / peaks["hbm_gbs"]},
+            "tq_quantize": {"ms": t_quant, "vectors_per_s": vec_per_step / (t_quant * 1e-3),
+                            "GB_per_s": quant_bytes / (t_quant * 1e-3) / 1e9, "TFLOP_per_s": quant_tf}},
+        "roofline": logits_roof if dominant == "tq_logits" else quant_roof,
+        "roofline_other": quant_roof if dominant == "tq_logits" else logits_roof,
+        "e2e": {"value": keys_per_step * world / (e2e_ms * 1e-3), "unit": "keys/s", "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def oracle_sample():
+    """One sequence of the step (8 kv-heads x 8192 cached keys, 8 x 512 appended vectors,
+    32 query heads) with the cache already quantized by the oracle."""
+    import oracle
+    import tq_inputs as ti
+    cfg = ti.C4
+    pi, s = cfg.pi(), cfg.s()
+    c, t, _, _ = oracle.codebook(D, MSE_BITS)
+    n_tok = N_TOK
+    keys = [ti.bf16_to_f64(ti.key_stream(4, 0, h, n_tok)) for h in range(N_KV)]
+    cache = [oracle.quantize(k, pi, s, c, t, MSE_BITS, qjl=True, keep_yz=False) for k in keys]
+    app = [ti.bf16_to_f64(ti.key_stream(4, 1000, h, N_APPEND)) for h in range(N_KV)]
+    q = ti.bf16_to_f64(ti.decode_queries(4, 1, N_KV * G))[0]
+    return dict(oracle=oracle, pi=pi, s=s, c=c, t=t, cache=cache, app=app, q=q)
+
+
+def oracle_step(smp):
+    o = smp["oracle"]
+    for h in range(N_KV):
+        o.quantize(smp["app"][h], smp["pi"], smp["s"], smp["c"], smp["t"], MSE_BITS, qjl=True, keep_yz=False)
+        ch = smp["cache"][h]
+        o.logits(ch.idx, ch.sbit, ch.nhat, ch.ghat, smp["pi"], smp["s"], smp["c"], smp["q"][h * G:(h + 1) * G],
+                 qjl=True, scale=1.0 / math.sqrt(D))
+
+
+SAMPLE_DESC = ("1 of 64 sequences: oracle quantize of 8 x 512 appended vectors + oracle logits of 32 q-heads "
+               "over 8 x 8192 cached keys (cache quantized beforehand)")
+
+
+def cpu_baseline(min_seconds=10.0):
+    import oracle
+    smp = oracle_sample()
+    oracle_step(smp)
+    t0 = time.perf_counter()
+    n = 0
+    while n < 1 or time.perf_counter() - t0 < min_seconds:
+        oracle_step(smp)
+        n += 1
+    dt = (time.perf_counter() - t0) / n
+    return {"value": N_KV * N_TOK / dt, "unit": "keys/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": SAMPLE_DESC, "s_per_sample_step": dt}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    smp = oracle_sample()
+    for _ in range(args.warmup):
+        oracle_step(smp)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(smp)
+    dt = (time.perf_counter() - t0) / args.steps
+    v = N_KV * N_TOK / dt
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "keys/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (numpy, pages' key law)",
+            "config": {"workload": "c4_batched_decode (sampled: 1 of 64 sequences per step)", "seq_len": N_TOK,
+                       "kv_heads": N_KV, "q_heads": N_KV * G, "head_dim": D, "key_bits": MSE_BITS + 1},
+            "cpu_baseline": {"value": v, "unit": "keys/s", "cores": oracle.threads(), "kind": "oracle",
+                             "sample": SAMPLE_DESC},
+            "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_init() if args.impl == "tq" else (int(os.environ.get("WORLD_SIZE", "1")),
+                                                                 int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    line = run_gpu(args, world, rank, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -10,298 +10,455 @@
 // with s0 s1 s2 = 2 (b0 ^ b1 ^ b2) - 1. Hence
 //   <q', c[idx]> = sum_p sum_i (2 a_p q'_i) beta_{p,i} - (sum_p a_p) sum_i q'_i,
 //   <q'', s>     = 2 sum_j q''_j bit_j - sum_j q''_j,
-// two contractions of {0,1} bit planes against fixed vectors. Each is run on the int8
-// tensor cores: the planes become 0/1 bytes with one shift+and per 4 coordinates, and the
-// query side is a 16-bit fixed-point vector split into two int8 columns (hi, lo) of the
-// same MMA, so the int32 accumulation is exact.
+// two contractions of {0,1} bit planes against fixed vectors, run on the int8 tensor cores
+// (mma.sync m16n8k32, u8 x s8 -> s32). A bit becomes the byte 0 or 128 with one shift and
+// one and per four coordinates (A = 128 * bits); the query side is a 16-bit fixed-point
+// vector split into two int8 columns (hi, lo) of the same MMA, so accumulation is exact.
 //
-// Kernel 1 (prologue, one CTA per (sequence, kv-head)): q', q'', fixed-point fragments in
-// MMA order, per-head scales, and the exact logits of the full-precision tail.
-// Kernel 2 (stream): each warp owns one (stream, n-tile of 4 heads, run of blocks) task,
-// keeps the query fragments in registers and streams 32-key blocks with 16-byte loads.
+// Kernel 1 (prologue, a few (sequence, kv-head) streams per CTA): q', q'' for every query
+// head, fixed-point fragments in MMA order, per-head scales, exact logits of the tail.
+// Kernel 2 (stream, persistent): each warp walks a list of (stream, block range) tasks and
+// keeps a ring of 32-key blocks in shared memory filled by bulk copies (TMA engine,
+// mbarrier completion), prefetching across task boundaries.
+#include <algorithm>
+
 #include "tq_device.cuh"
 
 namespace {
 
 constexpr int kPrologueThreads = 256;
+constexpr int kStreamWarps = 8;
+constexpr uint32_t kWaitLimit = 1u << 22;
 
-// fragment index of (stream, ntile, mma plane group, chunk, lane, half)
 __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles, int nmg, int mg, int c,
                                            int lane, int h) {
     return ((((size_t)stream * ntiles + ntile) * nmg + mg) * 4 + c) * 64 + lane * 2 + h;
 }
 
+// Prologue. Per CTA: 8 consecutive query heads (rows s*g + h of q).
+//   1. register-tiled GEMM [8 x d] x [d x (D + Mp)] against (Pi^T | S^T), streamed through
+//      shared memory 32 rows at a time (the next chunk is loaded into registers while the
+//      current one is used); each thread owns 2 heads x 4 columns (x 2 for wide codecs):
+//      q' = Pi q and q'' = S q.
+//   2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
+//   3. every thread rounds (head, plane, coordinate) values and scatters their hi and lo
+//      bytes straight into MMA fragment order; per-head constants and the tail follow.
+constexpr int kPH = 8;    // heads per prologue CTA
+constexpr int kPK = 16;   // matrix rows per shared-memory chunk
+
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
     const TqDims& T = p.t;
-    const int D = T.D, Mp = T.Mp, d = T.d, G = p.g;
-    const int64_t stream = blockIdx.x;                 // seq * n_kv + kv
-    const int64_t seq = stream / p.n_kv;
-    const int kv = (int)(stream % p.n_kv);
-    extern __shared__ float sm[];
-    float* qs = sm;                    // [G][D] raw query
-    float* qp = qs + G * D;            // [G][D] Pi q
-    float* qpp = qp + G * D;           // [G][Mp] S q
-    int* iv = reinterpret_cast<int*>(qpp + G * Mp);   // [G][nplanes][D] + [G][Mp] fixed point
-    __shared__ float s_max[2][8];
-    __shared__ double s_sum[2][8];
-
-    const int np = T.nplanes_mma;
-    int* ivA = iv;
-    int* ivS = iv + G * np * D;
-
-    // query heads of this kv group
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int h = e / D, i = e % D;
-        const int64_t qh = seq * ((int64_t)p.n_kv * G) + (int64_t)kv * G + h;
-        qs[e] = i < d ? tq_load_elem(p.q, p.q_dtype, qh * d + i) : 0.f;
-    }
-    __syncthreads();
-    // q' = Pi q, q'' = S q (fp32 accumulate)
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int h = e / D, i = e % D;
-        float a = 0.f;
-        for (int j = 0; j < d; ++j) a = fmaf(__ldg(p.piT + (size_t)j * D + i), qs[h * D + j], a);
-        qp[e] = a;
-    }
-    for (int e = threadIdx.x; e < G * Mp; e += blockDim.x) {
-        const int h = e / Mp, k = e % Mp;
-        float a = 0.f;
-        for (int j = 0; j < d; ++j) a = fmaf(__ldg(p.sT + (size_t)j * Mp + k), qs[h * D + j], a);
-        qpp[e] = a;
-    }
-    __syncthreads();
-    // per-head max |q'| and |q''| (warp h handles head h; G <= 8 = warps per CTA)
-    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (wid < G) {
-        float ma = 0.f, ms = 0.f;
-        for (int i = lane; i < D; i += 32) ma = fmaxf(ma, fabsf(qp[wid * D + i]));
-        for (int k = lane; k < Mp; k += 32) ms = fmaxf(ms, fabsf(qpp[wid * Mp + k]));
-        ma = tq_warp_max(ma);
-        ms = tq_warp_max(ms);
-        if (lane == 0) { s_max[0][wid] = ma; s_max[1][wid] = ms; }
-    }
-    __syncthreads();
-    float amax = 0.f;
-    for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
-    // fixed point: v = round(value / delta), |v| <= 32000
-    for (int e = threadIdx.x; e < G * np * D; e += blockDim.x) {
-        const int h = e / (np * D), pl = (e / D) % np, i = e % D;
-        const float m0 = s_max[0][h] * amax;
-        const float delta = m0 > 0.f ? m0 / 32000.f : 1.f;
-        ivA[e] = __float2int_rn(2.f * p.cb.plane_coef[pl] * qp[h * D + i] / delta);
-    }
-    for (int e = threadIdx.x; e < G * Mp; e += blockDim.x) {
-        const int h = e / Mp;
-        const float m0 = s_max[1][h];
-        const float delta = m0 > 0.f ? m0 / 32000.f : 1.f;
-        ivS[e] = __float2int_rn(qpp[e] / delta);
-    }
-    __syncthreads();
-    if (wid < G) {
-        double sa = 0.0, ss = 0.0;
-        for (int e = lane; e < np * D; e += 32) sa += ivA[wid * np * D + e];
-        for (int k = lane; k < Mp; k += 32) ss += ivS[wid * Mp + k];
-        sa = tq_warp_sum_d(sa);
-        ss = tq_warp_sum_d(ss);
-        if (lane == 0) { s_sum[0][wid] = sa; s_sum[1][wid] = ss; }
-    }
-    __syncthreads();
-    // per-head scales: l = |x| (dA accA - KA + gamma kappa (2 dS accS - KS))
-    if (threadIdx.x < p.ntiles * 4) {
-        const int h = threadIdx.x;
-        float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (h < G) {
-            const float ma = s_max[0][h] * amax, ms = s_max[1][h];
-            const float dA = ma > 0.f ? ma / 32000.f : 1.f;
-            const float dS = ms > 0.f ? ms / 32000.f : 1.f;
-            sc = make_float4(dA, (float)(0.5 * dA * s_sum[0][h]), 2.f * dS, (float)(dS * s_sum[1][h]));
-        }
-        reinterpret_cast<float4*>(p.qscale)[stream * p.ntiles * 4 + h] = sc;
-    }
-    // fragments: lane (g, t), column g = (head g>>1, part g&1); register (mg, c, h) byte b holds
-    // coordinate 128 gr + 32 t + 2c + h + 8b of plane group mg
+    const int D = T.D, Mp = T.Mp, d = T.d, G = p.g, np = T.nplanes_mma, W = D + Mp;
+    const int n_heads = (int)(p.n_seq * p.n_kv * G);
+    const int h_base = blockIdx.x * kPH;
+    const int H = min(kPH, n_heads - h_base);
+    extern __shared__ __align__(16) float sm[];
+    float* qo = sm;                    // [8][W]: q' (0..D-1) then q'' (D..W-1)
+    float* qT = qo + kPH * W;          // [d rounded to 32][8] query, transposed
+    float* mt = qT + 256 * kPH;        // [kPK][W] rows of (Pi^T | S^T)
+    __shared__ float s_inv[2][kPH], s_step[2][kPH];
+    __shared__ int s_sum[2][kPH], s_fbase[kPH], s_gcol[kPH];
+    const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
     const int nmg = T.nmg;
-    const int total = p.ntiles * nmg * 4 * 64;
-    for (int e = threadIdx.x; e < total; e += blockDim.x) {
-        const int hh = e & 1, ln = (e >> 1) & 31, c = (e >> 6) & 3;
-        const int mg = (e >> 8) % nmg, nt = (e >> 8) / nmg;
-        const int g = ln >> 2, t = ln & 3;
-        const int head = nt * 4 + (g >> 1), part = g & 1;
-        uint32_t word = 0;
-        if (head < G) {
-            const bool is_code = mg < np * T.GD;
-            const int gr = is_code ? mg % T.GD : mg - np * T.GD;
-            const int pl = is_code ? mg / T.GD : 0;
+    const int frag_words = p.ntiles * nmg * 256;
+
+    // heads beyond g inside an n-tile keep zero fragments (only when g < 4)
+    if (G < 4) {
+        const int st0 = (h_base + G - 1) / G, st1 = (h_base + H) / G;
+        uint4* fz = reinterpret_cast<uint4*>(p.qfrag + (size_t)st0 * frag_words);
+        for (int e = tid; e < (st1 - st0) * frag_words / 4; e += blockDim.x) fz[e] = make_uint4(0, 0, 0, 0);
+    }
+    for (int e = tid; e < 256 * kPH; e += blockDim.x) {
+        const int j = e / kPH, h = e % kPH;
+        qT[e] = (h < H && j < d) ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
+    }
+    if (tid < kPH) {
+        const int gh = h_base + tid, stream = gh / G, head = gh % G;
+        s_fbase[tid] = (stream * p.ntiles + (head >> 2)) * nmg * 256;
+        s_gcol[tid] = 2 * (head & 3);
+        s_sum[0][tid] = s_sum[1][tid] = 0;
+    }
+
+    // 1. GEMM: thread (hp = tid / 64 -> heads 2hp, 2hp+1; cq = tid % 64 -> columns 4cq + 256r)
+    const int hp = tid >> 6, cq = tid & 63;
+    const int nr = (W + 255) / 256;
+    const int n4 = kPK * W / 4;        // float4 per chunk
+    float acc[2][2][4];
 #pragma unroll
-            for (int bb = 0; bb < 4; ++bb) {
-                const int i = 128 * gr + 32 * t + 2 * c + hh + 8 * bb;
-                const int v = is_code ? ivA[(head * np + pl) * D + i] : ivS[head * Mp + i];
-                const int hi = (v + 128) >> 8;
-                const int lo = v - 256 * hi;
-                word |= ((uint32_t)(part ? lo : hi) & 0xffu) << (8 * bb);
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) acc[r][a][b] = 0.f;
+    constexpr int kPre = kPK * 512 / 4 / kPrologueThreads;   // float4 per thread for the widest codec
+    static_assert(kPre * 4 * kPrologueThreads >= kPK * 512, "prefetch must cover a chunk");
+    float4 pre[kPre];   // next chunk
+    // float4 e = tid + k * 256 of a chunk sits at row (4e) / W, column (4e) % W; the first
+    // position is divided once, the others follow by stepping 1024 floats
+    int f_row0 = (4 * tid) / W, f_col0 = (4 * tid) % W;
+    auto fetch = [&](int j0) {
+        int jj = f_row0, o = f_col0;
+#pragma unroll
+        for (int k = 0; k < kPre; ++k) {
+            const int e = tid + k * kPrologueThreads;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            const int j = j0 + jj;
+            if (e < n4 && j < d)
+                v = o < D ? *reinterpret_cast<const float4*>(p.piT + (size_t)j * D + o)
+                          : *reinterpret_cast<const float4*>(p.sT + (size_t)j * Mp + (o - D));
+            pre[k] = v;
+            o += 4 * kPrologueThreads;
+            while (o >= W) { o -= W; ++jj; }
+        }
+    };
+    fetch(0);
+    for (int j0 = 0; j0 < d; j0 += kPK) {
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < kPre; ++k) {
+            const int e = tid + k * kPrologueThreads;
+            if (e < n4) reinterpret_cast<float4*>(mt)[e] = pre[k];
+        }
+        __syncthreads();
+        if (j0 + kPK < d) fetch(j0 + kPK);
+#pragma unroll 4
+        for (int jj = 0; jj < kPK; ++jj) {
+            const float2 a = reinterpret_cast<const float2*>(qT + (j0 + jj) * kPH)[hp];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (r < nr && 256 * r + 4 * cq < W) {
+                    const float4 b = reinterpret_cast<const float4*>(mt + jj * W + 256 * r)[cq];
+                    acc[r][0][0] = fmaf(a.x, b.x, acc[r][0][0]); acc[r][0][1] = fmaf(a.x, b.y, acc[r][0][1]);
+                    acc[r][0][2] = fmaf(a.x, b.z, acc[r][0][2]); acc[r][0][3] = fmaf(a.x, b.w, acc[r][0][3]);
+                    acc[r][1][0] = fmaf(a.y, b.x, acc[r][1][0]); acc[r][1][1] = fmaf(a.y, b.y, acc[r][1][1]);
+                    acc[r][1][2] = fmaf(a.y, b.z, acc[r][1][2]); acc[r][1][3] = fmaf(a.y, b.w, acc[r][1][3]);
+                }
             }
         }
-        p.qfrag[qf_index(stream, nt, p.ntiles, nmg, mg, c, ln, hh)] = word;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+        if (r < nr && 256 * r + 4 * cq < W)
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+                *reinterpret_cast<float4*>(qo + (2 * hp + x) * W + 256 * r + 4 * cq) =
+                    make_float4(acc[r][x][0], acc[r][x][1], acc[r][x][2], acc[r][x][3]);
+    __syncthreads();
+    // 2. fixed-point steps (one head per warp)
+    float amax = 0.f;
+    for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
+    if (wid < H) {
+        const int h = wid;
+        float ma = 0.f, ms = 0.f;
+        for (int i = lane; i < D; i += 32) ma = fmaxf(ma, fabsf(qo[h * W + i]));
+        for (int k = lane; k < Mp; k += 32) ms = fmaxf(ms, fabsf(qo[h * W + D + k]));
+        ma = tq_warp_max(ma) * amax;
+        ms = tq_warp_max(ms);
+        if (lane == 0) {
+            s_step[0][h] = ma > 0.f ? ma / 32000.f : 1.f;
+            s_step[1][h] = ms > 0.f ? ms / 32000.f : 1.f;
+            s_inv[0][h] = 1.f / s_step[0][h];
+            s_inv[1][h] = 1.f / s_step[1][h];
+        }
+    }
+    __syncthreads();
+    // 3. round and scatter. Thread -> (coordinate slot within 128, plane group); loops over
+    //    heads. Byte bb of register (mg, c, lane = 4 gcol + t, hh) holds coordinate
+    //    128 gr + 32 t + 2c + hh + 8 bb, column gcol = 2 (head % 4) + part.
+    uint8_t* fb = reinterpret_cast<uint8_t*>(p.qfrag);
+    const int w32 = tid & 127, t = w32 >> 5, sb = w32 & 31;
+    const int bb = sb >> 3, c = (sb & 7) >> 1, hh = sb & 1;
+    const int slot = c * 64 + 2 * t + hh;     // word offset inside (stream, ntile, mg) for lane 4*gcol + t
+    int sa_loc[kPH], ss_loc[kPH];
+#pragma unroll
+    for (int h = 0; h < kPH; ++h) { sa_loc[h] = 0; ss_loc[h] = 0; }
+    for (int mg = tid >> 7; mg < nmg; mg += kPrologueThreads / 128) {
+        const bool is_code = mg < np * T.GD;
+        const int gr = is_code ? mg % T.GD : mg - np * T.GD;
+        const int pl = is_code ? mg / T.GD : 0;
+        const float coef = is_code ? 2.f * p.cb.plane_coef[pl] : 1.f;
+        const int col = (is_code ? 0 : D) + 128 * gr + w32;
+        const int kind = is_code ? 0 : 1;
+#pragma unroll
+        for (int h = 0; h < kPH; ++h) {
+            if (h < H) {
+                const int v = __float2int_rn(coef * qo[h * W + col] * s_inv[kind][h]);
+                if (is_code) sa_loc[h] += v; else ss_loc[h] += v;
+                const int hi = (v + 128) >> 8, lo = v - 256 * hi;
+                const int w0 = s_fbase[h] + mg * 256 + slot + 8 * s_gcol[h];
+                fb[4 * w0 + bb] = (uint8_t)(hi & 0xff);
+                fb[4 * (w0 + 8) + bb] = (uint8_t)(lo & 0xff);   // lane + 4 -> word + 8
+            }
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < kPH; ++h) {
+        int a = sa_loc[h], b = ss_loc[h];
+        for (int o = 16; o > 0; o >>= 1) { a += __shfl_xor_sync(0xffffffffu, a, o); b += __shfl_xor_sync(0xffffffffu, b, o); }
+        if (lane == 0 && h < H) { atomicAdd(&s_sum[0][h], a); atomicAdd(&s_sum[1][h], b); }
+    }
+    __syncthreads();
+    // per-head scales, folding the 128 of the u8 bit bytes and the QJL factor kappa:
+    //   l = |x| (dA/128 accA - KA + gamma (kappa 2 dS/128 accS - kappa KS))
+    if (tid < H) {
+        const int gh = h_base + tid, stream = gh / G, head = gh % G;
+        const float dA = s_step[0][tid], dS = s_step[1][tid];
+        reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
+            make_float4(dA / 128.f, 0.5f * dA * (float)s_sum[0][tid], p.kappa * 2.f * dS / 128.f,
+                        p.kappa * dS * (float)s_sum[1][tid]);
     }
     // exact logits of the full-precision tail: scale <q, k>
     if (p.n_tail > 0) {
         const int64_t row = p.n_tok + p.n_tail;
-        for (int e = threadIdx.x; e < G * p.n_tail; e += blockDim.x) {
+        for (int e = tid; e < H * p.n_tail; e += blockDim.x) {
             const int h = e / p.n_tail, tt = e % p.n_tail;
+            const int64_t gh = h_base + h, stream = gh / G;
             const uint16_t* kp = p.tail + ((size_t)stream * p.n_tail + tt) * d;
             float a = 0.f;
-            for (int i = 0; i < d; ++i) a = fmaf(__uint_as_float((uint32_t)kp[i] << 16), qs[h * D + i], a);
-            const int64_t qh = seq * ((int64_t)p.n_kv * G) + (int64_t)kv * G + h;
-            p.out[qh * row + p.n_tok + tt] = p.scale * a;
+            for (int i = 0; i < d; ++i) a = fmaf(__uint_as_float((uint32_t)kp[i] << 16), qT[i * kPH + h], a);
+            p.out[gh * row + p.n_tok + tt] = p.scale * a;
         }
     }
 }
 
-// Stream kernel. NP = code planes in the estimator, GD/GM = 128-coordinate groups of the
-// code and sign planes, B = stored code planes.
-template <int B, int GD, int GM>
-__global__ void __launch_bounds__(128) k_logits_stream(LogitsParams p) {
+// Walks a warp's tasks: task k = first + k * step over (stream, chunk) pairs, chunk in
+// [0, tpt); no divisions after the first (step = step_s * tpt + step_c).
+struct TaskWalk {
+    int stream, chunk, blk, b1;
+    __device__ void open(const LogitsParams& p) {
+        blk = chunk * p.blocks_per_task;
+        b1 = min(blk + p.blocks_per_task, (int)p.nb);
+    }
+    __device__ void init(const LogitsParams& p, int first) {
+        stream = first / p.tpt;
+        chunk = first - stream * p.tpt;
+        if (valid(p)) open(p);
+    }
+    __device__ bool valid(const LogitsParams& p) const { return stream < p.n_streams32; }
+    __device__ void advance(const LogitsParams& p) {
+        if (++blk < b1) return;
+        chunk += p.step_c;
+        stream += p.step_s;
+        if (chunk >= p.tpt) { chunk -= p.tpt; ++stream; }
+        if (valid(p)) open(p);
+    }
+};
+
+// NP = estimator code planes, GD/GM = 128-coordinate groups of code / sign planes,
+// B = stored code planes, NT = n-tiles of 4 query heads, NS = ring stages per warp.
+template <int B, int GD, int GM, int NT, int NS>
+__global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParams p) {
     constexpr int NP = B == 3 ? 4 : B;
     constexpr int NPG = B * GD + GM;       // stored plane groups
     constexpr int NMG = NP * GD + GM;      // MMA plane groups
-    const TqDims& T = p.t;
-    const int lane = threadIdx.x & 31;
+    constexpr uint32_t BB = 512u * NPG + 128u;
+    // exact int32 combination of the hi/lo columns while 128 * 32000 * K < 2^31
+    constexpr bool kIntComb = NP * GD <= 4 && GM <= 4;
+    extern __shared__ __align__(128) uint8_t ring[];
+    __shared__ uint64_t bars[kStreamWarps][NS];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int64_t tasks_per_tile = (p.nb + p.blocks_per_task - 1) / p.blocks_per_task;
-    const int64_t task = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int64_t n_tasks = p.n_seq * p.n_kv * p.ntiles * tasks_per_tile;
-    if (task >= n_tasks) return;
-    const int64_t stream = task / (p.ntiles * tasks_per_tile);
-    const int ntile = (int)((task / tasks_per_tile) % p.ntiles);
-    const int64_t b0 = (task % tasks_per_tile) * p.blocks_per_task;
-    const int64_t b1 = min(b0 + p.blocks_per_task, p.nb);
+    uint8_t* my_ring = ring + (size_t)warp * NS * BB;
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[warp][s], 1);
+    tq_fence_mbar_init();
+    __syncwarp();
 
-    // query fragments and scales of this (stream, n-tile)
-    uint32_t qf[NMG][4][2];
-#pragma unroll
-    for (int mg = 0; mg < NMG; ++mg)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const uint2 v = *reinterpret_cast<const uint2*>(
-                p.qfrag + qf_index(stream, ntile, p.ntiles, NMG, mg, c, lane, 0));
-            qf[mg][c][0] = v.x;
-            qf[mg][c][1] = v.y;
+    const int first = blockIdx.x * kStreamWarps + warp;
+    TaskWalk prod, cons;
+    prod.init(p, first);
+    cons.init(p, first);
+    if (lane == 0) {
+        for (int s = 0; s < NS && prod.valid(p); ++s) {
+            tq_bulk_load(my_ring + s * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB, &bars[warp][s]);
+            prod.advance(p);
         }
-    const int head = ntile * 4 + t;
-    const bool head_ok = head < p.g;
-    const float4 sc = reinterpret_cast<const float4*>(p.qscale)[stream * p.ntiles * 4 + ntile * 4 + t];
-    const float kap = p.kappa, scale = p.scale;
-    const int64_t seq = stream / p.n_kv;
-    const int kv = (int)(stream % p.n_kv);
-    const int64_t row = p.n_tok + p.n_tail;
-    float* orow = p.out + (seq * ((int64_t)p.n_kv * p.g) + (int64_t)kv * p.g + head) * row;
+    }
 
-    const uint8_t* base = p.packed + (size_t)(stream * p.nb) * T.block_bytes;
-    uint4 cur[NPG + 1], nxt[NPG + 1];
-    auto load_block = [&](int64_t bi, uint4 (&dst)[NPG + 1]) {
-        const uint8_t* bp = base + (size_t)bi * T.block_bytes;
+    const float scale = p.scale;
+    const int64_t row = p.n_tok + p.n_tail;
+    uint32_t mul[7];   // 2^(7-s), s < 7, unknown to the compiler: the shifts issue as IMAD
 #pragma unroll
-        for (int pg = 0; pg < NPG; ++pg) dst[pg] = tq_ldg_stream(bp + (size_t)(pg * 32 + lane) * 16);
-        dst[NPG] = tq_ldg_stream(bp + (size_t)NPG * 512 + g * 16);
-    };
-    if (b0 < b1) load_block(b0, cur);
-#pragma unroll 1
-    for (int64_t bi = b0; bi < b1; ++bi) {
-        if (bi + 1 < b1) load_block(bi + 1, nxt);
+    for (int k = 0; k < 7; ++k) mul[k] = p.shl[k];
+    uint32_t qf[NT][NMG][4][2];
+    float4 sc[NT];
+    float* orow[NT];
+    bool hv[NT];
+    int cur_stream = -1;
+    uint32_t seq = 0;
+    bool ok = true;
+    while (cons.valid(p)) {
+        if (cons.stream != cur_stream) {
+            cur_stream = cons.stream;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                for (int mg = 0; mg < NMG; ++mg)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint2 v = *reinterpret_cast<const uint2*>(
+                            p.qfrag + qf_index(cur_stream, n, NT, NMG, mg, c, lane, 0));
+                        qf[n][mg][c][0] = v.x;
+                        qf[n][mg][c][1] = v.y;
+                    }
+                sc[n] = reinterpret_cast<const float4*>(p.qscale)[(size_t)cur_stream * NT * 4 + n * 4 + t];
+                hv[n] = n * 4 + t < p.g;
+                orow[n] = p.out + ((int64_t)cur_stream * p.g + (hv[n] ? n * 4 + t : 0)) * row;
+            }
+        }
+        const int stage = seq % NS;
+        ok = __all_sync(0xffffffffu, tq_mbar_wait(&bars[warp][stage], (seq / NS) & 1u, kWaitLimit));
+        if (!ok) break;
+        const uint8_t* bp = my_ring + stage * BB;
+        uint4 cur[NPG + 1];
+#pragma unroll
+        for (int pg = 0; pg < NPG; ++pg) cur[pg] = *reinterpret_cast<const uint4*>(bp + (pg * 32 + lane) * 16);
+        cur[NPG] = *reinterpret_cast<const uint4*>(bp + NPG * 512 + g * 16);
+        const bool full = (int64_t)(cons.blk + 1) * 32 <= p.n_tok;
+        const int n_valid = full ? 32 : (int)(p.n_tok - (int64_t)cons.blk * 32);
+        const int tok0 = cons.blk * 32 + g;
+
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            int accA[4] = {0, 0, 0, 0}, accS[4] = {0, 0, 0, 0};
+            int accA[NT][4], accS[NT][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) { accA[n][r] = 0; accS[n][r] = 0; }
 #pragma unroll
             for (int mg = 0; mg < NMG; ++mg) {
                 uint32_t w0, w1;  // words of rows g (u = 2mt) and g + 8 (u = 2mt + 1)
-                const uint32_t* cw = nullptr;
-                if (mg < NP * GD) {
-                    const int pl = mg / GD, gr = mg % GD;
-                    if (pl < B) {
-                        cw = reinterpret_cast<const uint32_t*>(&cur[pl * GD + gr]);
-                        w0 = cw[2 * mt];
-                        w1 = cw[2 * mt + 1];
-                    } else {  // b0 ^ b1 ^ b2
-                        const uint32_t* c0 = reinterpret_cast<const uint32_t*>(&cur[0 * GD + gr]);
-                        const uint32_t* c1 = reinterpret_cast<const uint32_t*>(&cur[1 * GD + gr]);
-                        const uint32_t* c2 = reinterpret_cast<const uint32_t*>(&cur[2 * GD + gr]);
-                        w0 = c0[2 * mt] ^ c1[2 * mt] ^ c2[2 * mt];
-                        w1 = c0[2 * mt + 1] ^ c1[2 * mt + 1] ^ c2[2 * mt + 1];
-                    }
+                if (mg < NP * GD && mg / GD == 3) {  // b0 ^ b1 ^ b2
+                    const int gr = mg % GD;
+                    const uint32_t* c0 = reinterpret_cast<const uint32_t*>(&cur[0 * GD + gr]);
+                    const uint32_t* c1 = reinterpret_cast<const uint32_t*>(&cur[1 * GD + gr]);
+                    const uint32_t* c2 = reinterpret_cast<const uint32_t*>(&cur[2 * GD + gr]);
+                    w0 = c0[2 * mt] ^ c1[2 * mt] ^ c2[2 * mt];
+                    w1 = c0[2 * mt + 1] ^ c1[2 * mt + 1] ^ c2[2 * mt + 1];
                 } else {
-                    cw = reinterpret_cast<const uint32_t*>(&cur[B * GD + (mg - NP * GD)]);
+                    const int pg = mg < NP * GD ? mg : B * GD + (mg - NP * GD);
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(&cur[pg]);
                     w0 = cw[2 * mt];
                     w1 = cw[2 * mt + 1];
                 }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint32_t a0 = (w0 >> (2 * c)) & 0x01010101u;
-                    const uint32_t a1 = (w1 >> (2 * c)) & 0x01010101u;
-                    const uint32_t a2 = (w0 >> (2 * c + 1)) & 0x01010101u;
-                    const uint32_t a3 = (w1 >> (2 * c + 1)) & 0x01010101u;
-                    if (mg < NP * GD) tq_imma(accA, a0, a1, a2, a3, qf[mg][c][0], qf[mg][c][1]);
-                    else tq_imma(accS, a0, a1, a2, a3, qf[mg][c][0], qf[mg][c][1]);
+                    // coordinate bit s (= 2c, 2c + 1) of each byte moved to bit 7: A byte = 128 * bit
+                    const uint32_t a0 = (w0 * mul[2 * c]) & 0x80808080u;
+                    const uint32_t a1 = (w1 * mul[2 * c]) & 0x80808080u;
+                    const uint32_t a2 = (c == 3 ? w0 : w0 * mul[(2 * c + 1) % 7]) & 0x80808080u;
+                    const uint32_t a3 = (c == 3 ? w1 : w1 * mul[(2 * c + 1) % 7]) & 0x80808080u;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        if (mg < NP * GD) tq_imma_u8(accA[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
+                        else tq_imma_u8(accS[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
+                    }
                 }
             }
-            // epilogue: thread (g, t) -> head t of the tile, rows g and g + 8
+            // epilogue: thread (g, t) -> head t of each n-tile, rows g and g + 8
             const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int u = 2 * mt + r;
-                const int64_t tok = bi * 32 + 8 * u + g;
                 const uint32_t nw = nrm[u];
-                const float nh = tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
-                const float va = (float)(256 * accA[2 * r] + accA[2 * r + 1]);
-                const float vs = (float)(256 * accS[2 * r] + accS[2 * r + 1]);
-                const float est = fmaf(sc.x, va, -sc.y) + gh * kap * fmaf(sc.z, vs, -sc.w);
-                if (head_ok && tok < p.n_tok) orow[tok] = scale * nh * est;
+                const float nh = scale * tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    float va, vs;
+                    if (kIntComb) {
+                        va = (float)(256 * accA[n][2 * r] + accA[n][2 * r + 1]);
+                        vs = (float)(256 * accS[n][2 * r] + accS[n][2 * r + 1]);
+                    } else {
+                        va = fmaf(256.f, (float)accA[n][2 * r], (float)accA[n][2 * r + 1]);
+                        vs = fmaf(256.f, (float)accS[n][2 * r], (float)accS[n][2 * r + 1]);
+                    }
+                    const float est = fmaf(sc[n].x, va, -sc[n].y) + gh * fmaf(sc[n].z, vs, -sc[n].w);
+                    if (hv[n] && (full || 8 * u + g < n_valid)) orow[n][tok0 + 8 * u] = nh * est;
+                }
             }
         }
-        if (bi + 1 < b1) {
-#pragma unroll
-            for (int i = 0; i <= NPG; ++i) cur[i] = nxt[i];
+        // the stage's data are consumed (all reads above fed the MMAs): refill it
+        __syncwarp();
+        if (lane == 0 && prod.valid(p)) {
+            tq_fence_proxy_async();
+            tq_bulk_load(my_ring + stage * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB,
+                         &bars[warp][stage]);
+            prod.advance(p);
         }
+        ++seq;
+        cons.advance(p);
+    }
+    if (!ok) {
+        // a wait ran out: record it, then give the outstanding copies a bounded time to land
+        if (lane == 0) {
+            tq_raise(p.status, TQ_FLAG_TIMEOUT);
+            for (int s = 0; s < NS; ++s) tq_mbar_wait(&bars[warp][(seq + s) % NS], ((seq + s) / NS) & 1u, kWaitLimit);
+        }
+        __syncwarp();
     }
 }
 
-template <int B, int GD, int GM>
-cudaError_t launch_stream(const LogitsParams& p, cudaStream_t st) {
-    const int64_t tpt = (p.nb + p.blocks_per_task - 1) / p.blocks_per_task;
-    const int64_t tasks = p.n_seq * p.n_kv * p.ntiles * tpt;
-    const int64_t ctas = (tasks + 3) / 4;
-    if (ctas > 0) k_logits_stream<B, GD, GM><<<(unsigned)ctas, 128, 0, st>>>(p);
+template <int B, int GD, int GM, int NT>
+cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
+    constexpr int NS = 4;
+    constexpr int NPG = B * GD + GM;
+    constexpr size_t BB = 512u * NPG + 128u;
+    const size_t smem = (size_t)kStreamWarps * NS * BB;
+    auto kern = k_logits_stream<B, GD, GM, NT, NS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStreamWarps * 32, smem)) != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    per_sm = std::max(per_sm, 1);
+    // tasks of a few blocks each, about eight per resident warp, so that the static
+    // round-robin over tasks balances; copies run ahead across task boundaries
+    LogitsParams p = p0;
+    const int64_t n_streams = p.n_seq * p.n_kv;
+    const int64_t warps = (int64_t)per_sm * sms * kStreamWarps;
+    int64_t bpt = (n_streams * p.nb) / (warps * 8);
+    bpt = std::min<int64_t>(std::max<int64_t>(bpt, 1), 64);
+    p.blocks_per_task = (int)bpt;
+    p.tpt = (int)((p.nb + bpt - 1) / bpt);
+    p.n_tasks = n_streams * p.tpt;
+    p.n_streams32 = (int)n_streams;
+    const int64_t grid = std::min<int64_t>((p.n_tasks + kStreamWarps - 1) / kStreamWarps, (int64_t)per_sm * sms);
+    const int64_t step = grid * kStreamWarps;
+    p.step_s = (int)(step / p.tpt);
+    p.step_c = (int)(step % p.tpt);
+    if (grid > 0) kern<<<(unsigned)grid, kStreamWarps * 32, smem, st>>>(p);
     return cudaGetLastError();
+}
+
+template <int B, int GD, int GM>
+cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
+    return p.ntiles == 1 ? launch_stream<B, GD, GM, 1>(p, st) : launch_stream<B, GD, GM, 2>(p, st);
 }
 
 }  // namespace
 
-size_t tq_logits_prologue_smem(const TqDims& t, int g) {
-    return (size_t)g * (2 * t.D + t.Mp) * 4 + (size_t)g * (t.nplanes_mma * t.D + t.Mp) * 4;
+size_t tq_logits_prologue_smem(const TqDims& t, int) {
+    return ((size_t)kPH * (t.D + t.Mp) + (size_t)256 * kPH + (size_t)kPK * (t.D + t.Mp)) * 4;
 }
 
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st) {
-    const size_t smem = tq_logits_prologue_smem(p.t, p.g);
+    const size_t smem = tq_logits_prologue_smem(p.t, 0);
     cudaError_t e = cudaFuncSetAttribute(k_logits_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_logits_prologue<<<(unsigned)(p.n_seq * p.n_kv), kPrologueThreads, smem, st>>>(p);
+    const int64_t n_heads = p.n_seq * p.n_kv * p.g;
+    k_logits_prologue<<<(unsigned)((n_heads + kPH - 1) / kPH), kPrologueThreads, smem, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.nb == 0) return cudaSuccess;
     const int B = p.t.B, GD = p.t.GD, GM = p.t.GM;
-    if (GD == 1 && GM == 1) {
-        if (B == 1) return launch_stream<1, 1, 1>(p, st);
-        if (B == 2) return launch_stream<2, 1, 1>(p, st);
-        if (B == 3) return launch_stream<3, 1, 1>(p, st);
-    } else if (GD == 2 && GM == 2) {
-        if (B == 1) return launch_stream<1, 2, 2>(p, st);
-        if (B == 2) return launch_stream<2, 2, 2>(p, st);
-        if (B == 3) return launch_stream<3, 2, 2>(p, st);
-    } else if (GD == 1 && GM == 2) {
-        if (B == 1) return launch_stream<1, 1, 2>(p, st);
-        if (B == 2) return launch_stream<2, 1, 2>(p, st);
-        if (B == 3) return launch_stream<3, 1, 2>(p, st);
-    } else if (GD == 2 && GM == 1) {
-        if (B == 1) return launch_stream<1, 2, 1>(p, st);
-        if (B == 2) return launch_stream<2, 2, 1>(p, st);
-        if (B == 3) return launch_stream<3, 2, 1>(p, st);
-    }
+#define TQ_LOGITS_CASE(b, gd, gm) \
+    if (B == b && GD == gd && GM == gm) return launch_nt<b, gd, gm>(p, st);
+    TQ_LOGITS_CASE(1, 1, 1) TQ_LOGITS_CASE(2, 1, 1) TQ_LOGITS_CASE(3, 1, 1)
+    TQ_LOGITS_CASE(1, 2, 2) TQ_LOGITS_CASE(2, 2, 2) TQ_LOGITS_CASE(3, 2, 2)
+    TQ_LOGITS_CASE(1, 1, 2) TQ_LOGITS_CASE(2, 1, 2) TQ_LOGITS_CASE(3, 1, 2)
+    TQ_LOGITS_CASE(1, 2, 1) TQ_LOGITS_CASE(2, 2, 1) TQ_LOGITS_CASE(3, 2, 1)
+#undef TQ_LOGITS_CASE
     return cudaErrorInvalidValue;
 }

@@ -3,6 +3,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 
@@ -212,6 +213,7 @@ int tq_get_status(void* ws, void* stream) {
         if (cudaMemsetAsync(ws, 0, 4, st) != cudaSuccess) return TQ_ERR_CUDA;
         if (cudaStreamSynchronize(st) != cudaSuccess) return TQ_ERR_CUDA;
     }
+    if (word & TQ_FLAG_TIMEOUT) return TQ_ERR_TIMEOUT;
     return (word & TQ_FLAG_RANGE) ? TQ_ERR_RANGE : TQ_OK;
 }
 
@@ -275,13 +277,15 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.n_kv = n_kv; p.g = g; p.ntiles = g > 4 ? 2 : 1; p.n_tail = n_tail;
     p.scale = scale;
     p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
-    const int64_t work = n_streams * p.ntiles * p.nb;
-    int64_t bpt = work / (kNumSms * 16 * 2);
-    if (bpt < 2) bpt = 2;
-    if (bpt > 32) bpt = 32;
-    p.blocks_per_task = (int)bpt;
-    const int64_t tasks = n_streams * p.ntiles * ((p.nb + bpt - 1) / bpt);
-    if ((tasks + 3) / 4 > 0x7fffffffLL || n_streams > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    p.status = static_cast<uint32_t*>(ws);
+    // streams per prologue CTA: about one CTA per SM, at most 32 query heads per CTA
+    int64_t spc = n_streams / kNumSms;
+    spc = std::max<int64_t>(1, std::min<int64_t>(spc, 16 / g));
+    p.streams_per_cta = (int)spc;
+    p.blocks_per_task = 1;
+    p.n_tasks = 0;
+    for (int k = 0; k < 8; ++k) p.shl[k] = 1u << (7 - k);
+    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_logits(p, static_cast<cudaStream_t>(stream)));

@@ -37,6 +37,52 @@ TQ_DEVICE float tq_warp_max(float v) {
     return v;
 }
 
+// int8 tensor-core MMA, 16x8x32, s32 accumulate (legacy warp-level path): A u8, B s8
+TQ_DEVICE void tq_imma_u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                          uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// ---------------------------------------------------------------------- mbarrier + bulk copy
+// One-dimensional bulk copies global -> shared through the TMA engine, completion tracked
+// by a shared-memory mbarrier (transaction bytes). Waits are bounded: a wait that does not
+// complete within `limit` polls returns false and the caller records TQ_FLAG_TIMEOUT.
+TQ_DEVICE uint32_t tq_smem_addr(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+TQ_DEVICE void tq_mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(tq_smem_addr(bar)), "r"(count));
+}
+TQ_DEVICE void tq_fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+TQ_DEVICE void tq_fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+TQ_DEVICE void tq_bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tq_smem_addr(bar)), "r"(bytes)
+                 : "memory");
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+            tq_smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(tq_smem_addr(bar))
+        : "memory");
+}
+
+TQ_DEVICE bool tq_mbar_wait(uint64_t* bar, uint32_t phase, uint32_t limit) {
+    const uint32_t a = tq_smem_addr(bar);
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(a), "r"(phase)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
 // int8 tensor-core MMA, 16x8x32, s32 accumulate (legacy warp-level path)
 TQ_DEVICE void tq_imma(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                        uint32_t b1) {
@@ -97,11 +143,14 @@ struct LogitsParams {
     const float* piT;
     const float* sT;
     uint32_t* qfrag;       // [stream][ntile][nmg][4][32][2]
-    float* qscale;         // [stream][ntile*4][4]: dA, KA, 2dS, KS
-    int64_t n_seq, n_tok, nb;
+    float* qscale;         // [stream][ntile*4][4]: dA/128, KA, 2dS/128, KS
+    uint32_t* status;
+    int64_t n_seq, n_tok, nb, n_tasks;
     int n_kv, g, ntiles, n_tail;
     float scale, kappa;
-    int blocks_per_task;
+    int blocks_per_task, streams_per_cta;
+    int tpt, n_streams32, step_s, step_c;   // task walk: tasks per stream, stride in (stream, chunk)
+    uint32_t shl[8];       // 2^(7-s): runtime multipliers that move bit s of each byte to bit 7
     TqDims t;
     TqCodebookConsts cb;
 };

@@ -32,6 +32,7 @@
 
 // status word bits (device, first word of the workspace)
 #define TQ_FLAG_RANGE 1u
+#define TQ_FLAG_TIMEOUT 2u
 
 struct TqDims {
     int d, m, B, qjl;
