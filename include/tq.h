@@ -157,6 +157,26 @@ int tq_pv(const tq_codec* codec, const void* packed_v, int64_t n_seq, int n_kv, 
 int tq_topk(const tq_codec* codec, const void* packed_db, int64_t n_db, const float* q,
             int64_t n_q, int k, int64_t* idx, float* score, void* ws, size_t ws_bytes, void* stream);
 
+/* tq_logits without a caller workspace, for callers that cannot allocate device memory:
+ * code inside a host framework whose pool owns all device memory, plugins that may only use
+ * the buffers they are given, latency-critical loops under a no-allocation policy. The pages
+ * have no counterpart: this is a deployment convenience, not part of the method.
+ *   Arguments and results are those of tq_logits, minus ws / ws_bytes.
+ *   Scratch: a fixed TQ_NOALLOC_SCRATCH_BYTES (4 MiB) array in device memory, held by every
+ *   GPU that loads the library until the process exits. A request whose
+ *   tq_workspace_bytes(codec, TQ_OP_LOGITS, n_seq, n_kv, g) exceeds it returns
+ *   TQ_ERR_WORKSPACE and enqueues nothing.
+ *   The first call on a device resolves the array's device address (cudaGetSymbolAddress,
+ *   with that device current): make that first call before any stream capture.
+ *   Every call on a device shares the array: calls whose GPU work may overlap (other
+ *   streams, other threads) race and must be serialised by the caller. Each call clears
+ *   the status word first; data-dependent faults are not reported by this variant.
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine.        */
+#define TQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+int tq_logits_noalloc(const tq_codec* codec, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok,
+                      const void* q, tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale,
+                      float* out, void* stream);
+
 /* Diagnostic reconstruction (not on the hot path): x~ = |x|(Pi^T c[idx] + gamma
  * sqrt(pi/2)/m S^T s) for keys, |x| Pi^T c[idx] for values (blog.hotdry.top, "QJL residual
  * correction"). out: device fp32 [n_streams, n_tok, d].                                  */

@@ -26,7 +26,8 @@ TQ_F32, TQ_BF16 = 0, 1
 TQ_OP_QUANTIZE, TQ_OP_LOGITS, TQ_OP_PV, TQ_OP_TOPK, TQ_OP_DEQUANTIZE = 0, 1, 2, 3, 4
 EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_bytes", "tq_prep_bytes",
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
-            "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version"]
+            "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",
+            "tq_logits_noalloc"]
 
 
 class tq_codec(ctypes.Structure):
@@ -47,6 +48,7 @@ _sig = {
     "tq_workspace_bytes": (_SZ, [_CP, _I, _I64, _I64, _I64]),
     "tq_quantize": (_I, [_CP, _P, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_logits": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _P]),
+    "tq_logits_noalloc": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P]),
     "tq_pv": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "tq_dequantize": (_I, [_CP, _P, _I64, _I64, _P, _P, _SZ, _P]),
@@ -156,6 +158,13 @@ def tq_logits(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_tail, scal
     return _check("tq_logits", lib.tq_logits(codec.ref, _ptr(packed), n_seq, n_kv, n_tok, _ptr(q), _dtype(q), g,
                                              _ptr(tail), n_tail, scale, _ptr(out), _ptr(ws), ws.numel(),
                                              _stream(stream)))
+
+
+def tq_logits_noalloc(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_tail, scale, out, stream=None):
+    """tq_logits with the library's fixed device scratch instead of a caller workspace."""
+    return _check("tq_logits_noalloc", lib.tq_logits_noalloc(codec.ref, _ptr(packed), n_seq, n_kv, n_tok, _ptr(q),
+                                                             _dtype(q), g, _ptr(tail), n_tail, scale, _ptr(out),
+                                                             _stream(stream)))
 
 
 def tq_pv(codec: Codec, packed_v, n_seq, n_kv, n_tok, P, g, out, ws, stream=None):
