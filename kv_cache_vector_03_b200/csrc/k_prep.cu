@@ -3,6 +3,33 @@
 // "TurboQuant vector-search compression", section "QJL residual correction").
 #include "tq_device.cuh"
 
+__device__ void split_half(double v, uint16_t* hi, uint16_t* lo) {
+    const __half h = __double2half(v);
+    *hi = __half_as_ushort(h);
+    *lo = __half_as_ushort(__double2half(v - (double)__half2float(h)));
+}
+
+// fp16 hi/lo pairs of 256 Pi (row = output coordinate i, column = input j) and 256 M
+__global__ void k_prepare_split(PrepParams p) {
+    const int64_t n_pi = (int64_t)p.D * p.D, n_m = p.qjl ? (int64_t)p.Mp * p.D : 0;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n_pi + n_m;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        if (e < n_pi) {
+            const int i = (int)(e / p.D), j = (int)(e % p.D);
+            const double v = (i < p.d && j < p.d) ? 256.0 * (double)p.pi[(int64_t)i * p.d + j] : 0.0;
+            split_half(v, p.pih + e, p.pil + e);
+        } else {
+            const int64_t f = e - n_pi;
+            const int k = (int)(f / p.D), i = (int)(f % p.D);  // M[k][i] = sum_j S[k][j] Pi[i][j]
+            double acc = 0.0;
+            if (k < p.m && i < p.d)
+                for (int j = 0; j < p.d; ++j)
+                    acc += (double)p.s[(int64_t)k * p.d + j] * (double)p.pi[(int64_t)i * p.d + j];
+            split_half(256.0 * acc, p.mh + f, p.ml + f);
+        }
+    }
+}
+
 __global__ void k_prepare(PrepParams p) {
     const int64_t n_pi = (int64_t)p.D * p.D;
     const int64_t n_s = (int64_t)p.D * p.Mp;
@@ -30,5 +57,8 @@ __global__ void k_prepare(PrepParams p) {
 
 cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
     k_prepare<<<296, 256, 0, st>>>(p);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    k_prepare_split<<<296, 256, 0, st>>>(p);
     return cudaGetLastError();
 }

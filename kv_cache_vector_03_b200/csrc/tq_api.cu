@@ -175,6 +175,10 @@ int tq_prepare(const tq_codec* c, void* stream) {
     p.piT = reinterpret_cast<float*>(base + L.piT);
     p.sT = reinterpret_cast<float*>(base + L.sT);
     p.mT = reinterpret_cast<float*>(base + L.mT);
+    p.pih = reinterpret_cast<uint16_t*>(base + L.pih);
+    p.pil = reinterpret_cast<uint16_t*>(base + L.pil);
+    p.mh = reinterpret_cast<uint16_t*>(base + L.mh);
+    p.ml = reinterpret_cast<uint16_t*>(base + L.ml);
     p.d = t.d; p.m = t.m; p.D = t.D; p.Mp = t.Mp; p.qjl = t.qjl;
     return cuda_status(tq_launch_prepare(p, static_cast<cudaStream_t>(stream)));
 }
@@ -238,7 +242,12 @@ int tq_quantize(const tq_codec* c, const void* x, tq_dtype dtype, int64_t n_stre
     p.packed = static_cast<uint8_t*>(packed);
     p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
     p.mT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.mT);
+    p.pih = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pih);
+    p.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
+    p.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
+    p.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
     p.status = static_cast<uint32_t*>(ws);
+    p.vec_ok = aligned(x, dtype == TQ_F32 ? 16 : 8) && x_stream_stride % 4 == 0 && c->d % 4 == 0;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_quantize(p, static_cast<cudaStream_t>(stream)));

@@ -119,6 +119,7 @@ struct PrepParams {
     float* piT;
     float* sT;
     float* mT;
+    uint16_t *pih, *pil, *mh, *ml;
     int d, m, D, Mp, qjl;
 };
 
@@ -129,7 +130,9 @@ struct QuantParams {
     uint8_t* packed;
     const float* piT;
     const float* mT;
+    const uint16_t *pih, *pil, *mh, *ml;
     uint32_t* status;
+    int vec_ok;            // rows can be read 4 elements at a time (alignment of x, stride, d)
     TqDims t;
     TqCodebookConsts cb;
 };

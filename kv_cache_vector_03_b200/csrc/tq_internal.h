@@ -63,10 +63,12 @@ static inline TqDims tq_dims(int d, int m, int B, int qjl) {
 
 // Prepared (derived) operands, laid out in the caller's prep buffer:
 //   header (256 B) | PiT fp32 [D][D] | ST fp32 [D][Mp] | MT fp32 [D][Mp]
+//   | Pi_hi, Pi_lo fp16 [D][D] | M_hi, M_lo fp16 [Mp][D]     (tensor-core quantize)
 // PiT[j][i] = Pi[i][j], ST[j][k] = S[k][j], MT[i][k] = M[k][i] with M = S Pi^T, all zero
-// outside the d x d / m x d corners.
+// outside the d x d / m x d corners. The fp16 pairs hold 256 Pi and 256 M split as
+// hi = half(v), lo = half(v - hi), row-major (row = output coordinate).
 struct TqPrepLayout {
-    size_t hdr, piT, sT, mT, total;
+    size_t hdr, piT, sT, mT, pih, pil, mh, ml, total;
 };
 
 static inline TqPrepLayout tq_prep_layout(const TqDims& t) {
@@ -76,6 +78,10 @@ static inline TqPrepLayout tq_prep_layout(const TqDims& t) {
     L.piT = off; off += (size_t)t.D * t.D * 4;
     L.sT = off; off += t.qjl ? (size_t)t.D * t.Mp * 4 : 0;
     L.mT = off; off += t.qjl ? (size_t)t.D * t.Mp * 4 : 0;
+    L.pih = off; off += (size_t)t.D * t.D * 2;
+    L.pil = off; off += (size_t)t.D * t.D * 2;
+    L.mh = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
+    L.ml = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
     L.total = off;
     return L;
 }
