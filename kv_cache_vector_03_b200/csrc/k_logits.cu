@@ -70,7 +70,8 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     }
     for (int e = tid; e < 256 * kPH; e += blockDim.x) {
         const int j = e / kPH, h = e % kPH;
-        qT[e] = (h < H && j < d) ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
+        const bool ok = h < H && j < d && (int64_t)(h_base + h) < p.n_heads_valid;
+        qT[e] = ok ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
     }
     if (tid < kPH) {
         const int gh = h_base + tid, stream = gh / G, head = gh % G;
@@ -442,6 +443,15 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 
 size_t tq_logits_prologue_smem(const TqDims& t, int) {
     return ((size_t)kPH * (t.D + t.Mp) + (size_t)256 * kPH + (size_t)kPK * (t.D + t.Mp)) * 4;
+}
+
+cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
+    const size_t smem = tq_logits_prologue_smem(p.t, 0);
+    cudaError_t e = cudaFuncSetAttribute(k_logits_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t n_heads = p.n_seq * p.n_kv * p.g;
+    k_logits_prologue<<<(unsigned)((n_heads + kPH - 1) / kPH), kPrologueThreads, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st) {

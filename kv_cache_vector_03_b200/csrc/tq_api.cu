@@ -103,6 +103,25 @@ LogitsWs logits_ws(const TqDims& t, int64_t n_streams, int g) {
     return w;
 }
 
+struct TopkWs { int nsplit, bps, n_groups; size_t qfrag, qscale, psc, pix, total; };
+TopkWs topk_ws(const TqDims& t, int64_t n_q, int64_t n_db, int k) {
+    TopkWs w;
+    const int64_t nb = (n_db + 31) / 32;
+    w.n_groups = (int)((n_q + 3) / 4);
+    const int64_t qgroups = (w.n_groups + 7) / 8;
+    int64_t ns = (4 * kNumSms + qgroups - 1) / qgroups;
+    ns = std::max<int64_t>(1, std::min<int64_t>(ns, nb));
+    w.bps = (int)((nb + ns - 1) / ns);
+    w.nsplit = (int)((nb + w.bps - 1) / w.bps);
+    size_t off = TQ_STATUS_BYTES;
+    w.qfrag = off; off = align_up(off + (size_t)w.n_groups * t.nmg * 4 * 64 * 4);
+    w.qscale = off; off = align_up(off + (size_t)w.n_groups * 4 * 16);
+    w.psc = off; off = align_up(off + (size_t)n_q * w.nsplit * k * 4);
+    w.pix = off; off = align_up(off + (size_t)n_q * w.nsplit * k * 4);
+    w.total = off;
+    return w;
+}
+
 struct PvWs { int nsplit, bps; size_t part, ml, total; };
 PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
     PvWs w;
@@ -197,7 +216,8 @@ size_t tq_workspace_bytes(const tq_codec* c, int op, int64_t a, int64_t b, int64
             if (a < 0 || b < 1 || cc < 1 || cc > 8) return 0;
             return pv_ws(t, a, b, (int)cc).total;
         case TQ_OP_TOPK:
-            return 0;
+            if (!c->qjl || a < 1 || b < 1 || cc < 1 || cc > 32 || cc > b) return 0;
+            return topk_ws(t, a, b, (int)cc).total;
     }
     return 0;
 }
@@ -293,6 +313,7 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.streams_per_cta = (int)spc;
     p.blocks_per_task = 1;
     p.n_tasks = 0;
+    p.n_heads_valid = n_streams * g;
     for (int k = 0; k < 8; ++k) p.shl[k] = 1u << (7 - k);
     if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
     p.t = t;
@@ -329,9 +350,51 @@ int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int6
 
 int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,
             float* score, void* ws, size_t ws_bytes, void* stream) {
-    (void)c; (void)packed_db; (void)n_db; (void)q; (void)n_q; (void)k; (void)idx; (void)score; (void)ws;
-    (void)ws_bytes; (void)stream;
-    return TQ_ERR_UNSUPPORTED;
+    int st = check_codec(c, true);
+    if (st != TQ_OK) return st;
+    if (!c->qjl) return TQ_ERR_ARG;
+    if (n_q < 0 || n_db < 1 || n_db > 0x7fffffffLL || k < 1 || k > 32 || k > n_db) return TQ_ERR_ARG;
+    if (n_q == 0) return TQ_OK;
+    if (!packed_db || !q || !idx || !score || !ws) return TQ_ERR_ARG;
+    if (!aligned(packed_db, 16) || !aligned(q, 4) || !aligned(idx, 8) || !aligned(score, 4) || !aligned(ws, 256))
+        return TQ_ERR_ARG;
+    const TqDims t = dims_of(c);
+    const TopkWs W = topk_ws(t, n_q, n_db, k);
+    if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
+    if ((int64_t)((W.n_groups + 7) / 8) * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    const TqPrepLayout L = tq_prep_layout(t);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    // queries rotated once: groups of 4 queries are the heads of one prologue stream
+    LogitsParams lp;
+    std::memset(&lp, 0, sizeof(lp));
+    lp.q = q; lp.q_dtype = TQ_F32;
+    lp.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
+    lp.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
+    lp.qfrag = reinterpret_cast<uint32_t*>(wsb + W.qfrag);
+    lp.qscale = reinterpret_cast<float*>(wsb + W.qscale);
+    lp.status = static_cast<uint32_t*>(ws);
+    lp.n_seq = 1; lp.n_kv = W.n_groups; lp.g = 4; lp.ntiles = 1; lp.n_tok = 0; lp.nb = 0; lp.n_tail = 0;
+    lp.scale = 1.f;
+    lp.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
+    lp.n_heads_valid = n_q;
+    lp.t = t;
+    if ((st = codebook_consts(c, &lp.cb)) != TQ_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (tq_launch_logits_prologue(lp, cs) != cudaSuccess) return TQ_ERR_CUDA;
+    TopkParams p;
+    p.packed = static_cast<const uint8_t*>(packed_db);
+    p.qfrag = lp.qfrag;
+    p.qscale = lp.qscale;
+    p.part_score = reinterpret_cast<float*>(wsb + W.psc);
+    p.part_idx = reinterpret_cast<int*>(wsb + W.pix);
+    p.out_idx = idx;
+    p.out_score = score;
+    p.status = static_cast<uint32_t*>(ws);
+    p.n_db = n_db; p.nb = (n_db + 31) / 32; p.n_q = n_q;
+    p.k = k; p.nsplit = W.nsplit; p.blocks_per_split = W.bps; p.n_groups = W.n_groups;
+    for (int s2 = 0; s2 < 8; ++s2) p.shl[s2] = 1u << (7 - s2);
+    p.t = t;
+    return cuda_status(tq_launch_topk(p, cs));
 }
 
 int tq_dequantize(const tq_codec* c, const void* packed, int64_t n_streams, int64_t n_tok, float* out, void* ws,

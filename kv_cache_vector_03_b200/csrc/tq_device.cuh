@@ -153,6 +153,7 @@ struct LogitsParams {
     float scale, kappa;
     int blocks_per_task, streams_per_cta;
     int tpt, n_streams32, step_s, step_c;   // task walk: tasks per stream, stride in (stream, chunk)
+    int64_t n_heads_valid;                   // query rows that exist (later heads read as zero)
     uint32_t shl[8];       // 2^(7-s): runtime multipliers that move bit s of each byte to bit 7
     TqDims t;
     TqCodebookConsts cb;
@@ -169,6 +170,21 @@ struct PvParams {
     int g, nsplit, blocks_per_split;
     TqDims t;
     TqCodebookConsts cb;
+};
+
+struct TopkParams {
+    const uint8_t* packed;      // one stream of n_db key records
+    const uint32_t* qfrag;      // [group of 4 queries][1][nmg][4][32][2] (prologue output)
+    const float* qscale;        // [group][4][4]
+    float* part_score;          // [n_q][nsplit][k]
+    int* part_idx;              // [n_q][nsplit][k]
+    int64_t* out_idx;
+    float* out_score;
+    uint32_t* status;
+    int64_t n_db, nb, n_q;
+    int k, nsplit, blocks_per_split, n_groups;
+    uint32_t shl[8];
+    TqDims t;
 };
 
 struct DequantParams {
@@ -188,3 +204,5 @@ cudaError_t tq_launch_quantize(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st);
 cudaError_t tq_launch_dequant(const DequantParams& p, cudaStream_t st);
+cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
+cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
