@@ -266,6 +266,7 @@ def run_gpu(args, world, rank, local):
                   "peak": round(fma_peak, 1), "unit": "TFLOP/s", "frac": round(quant_tf / fma_peak, 4),
                   "traffic": None, "algorithmic_flops_per_launch": quant_flops,
                   "peak_kind": "derived: 148 SMs x 128 fp32 FMA/clk x 2 x median SM clock"}
+    also = {} if args.no_extras else extra_workloads(torch, tq, ti, gen, peaks)
     line = {
         "metric": METRIC, "value": keys_per_step * world / (ms_step * 1e-3), "unit": "keys/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -287,8 +288,101 @@ def run_gpu(args, world, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
+        "also": also,
     }
     return line
+
+
+def time_calls(torch, fn, n_iter, n_warm=3):
+    """Mean device time of fn(i) over n_iter calls (CUDA events on the current stream)."""
+    for i in range(n_warm):
+        fn(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(n_iter):
+        fn(i)
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n_iter
+
+
+def extra_workloads(torch, tq, ti, gen, peaks):
+    """The other workloads of the hot path, each timed on its own (device time per call).
+    Inputs that fit in L2 are rotated over enough copies to exceed it."""
+    out = {}
+    d = 128
+    # c2: Llama-3.1-8B-shaped decode, 8 kv-heads x 32768 tokens (32640 packed + 128 bf16), 32 q-heads
+    n_kv, n_all, n_tail = 8, 32768, 128
+    n_tok = n_all - n_tail
+    for b in (4, 3):
+        cfg = ti.C2
+        codec = tq.Codec(d, d, b - 1, True, torch.from_numpy(cfg.pi().astype(np.float32)),
+                         torch.from_numpy(cfg.s().astype(np.float32)))
+        keys = make_keys_device(torch, gen, n_kv, n_all, n_kv)
+        copies = 12
+        packs = []
+        for _ in range(copies):
+            pk = torch.empty(codec.packed_bytes(n_kv, n_tok), dtype=torch.uint8, device="cuda")
+            tq.tq_quantize(codec, keys, n_kv, n_tok, n_all * d, pk, tq.workspace(256))
+            packs.append(pk)
+        tail = keys[:, n_tok:].contiguous()
+        q = torch.randn((1, n_kv * 4, d), generator=gen, device="cuda").to(torch.bfloat16)
+        lo = torch.empty((1, n_kv * 4, n_all), dtype=torch.float32, device="cuda")
+        ws = tq.workspace(codec.workspace_bytes(tq.TQ_OP_LOGITS, 1, n_kv, 4))
+        ms = time_calls(torch, lambda i: tq.tq_logits(codec, packs[i % copies], 1, n_kv, n_tok, q, 4, tail, n_tail,
+                                                      1.0 / math.sqrt(d), lo, ws), 240)
+        byts = n_kv * n_tok * codec.record_bytes() + n_kv * n_tail * d * 2 + lo.numel() * 4
+        out[f"c2_llama8b_decode_logits_b{b}"] = {
+            "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "l2": f"{copies} rotating copies of the packed cache"}
+        del keys, packs
+    # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
+    n_kv, n_tok, g = 8, 131072, 4
+    vals = torch.randn((n_kv, n_tok, d), generator=gen, device="cuda").to(torch.bfloat16)
+    P = [2.0 * torch.randn((1, n_kv * g, n_tok), generator=gen, device="cuda") for _ in range(2)]
+    for B in (3, 4):
+        codec = tq.Codec(d, 0, B, False, torch.from_numpy(ti.C3.pi().astype(np.float32)), None)
+        copies = 4
+        packs = []
+        for _ in range(copies):
+            pk = torch.empty(codec.packed_bytes(n_kv, n_tok), dtype=torch.uint8, device="cuda")
+            tq.tq_quantize(codec, vals, n_kv, n_tok, n_tok * d, pk, tq.workspace(256))
+            packs.append(pk)
+        o = torch.empty((1, n_kv * g, d), dtype=torch.float32, device="cuda")
+        ws = tq.workspace(codec.workspace_bytes(tq.TQ_OP_PV, n_kv, n_tok, g))
+        ms = time_calls(torch, lambda i: tq.tq_pv(codec, packs[i % copies], 1, n_kv, n_tok, P[i % 2], g, o, ws), 60)
+        byts = n_kv * n_tok * codec.record_bytes() + P[0].numel() * 4
+        out[f"c3_values_128k_pv_{B}bit"] = {
+            "ms": ms, "tokens_per_s": n_kv * n_tok / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "l2": f"{copies} rotating copies of the packed values, 2 of P"}
+        del packs
+    del vals, P
+    # c5: vector search, 1M x d=200 database (anisotropic, unit rows), 10,000 queries, top-10
+    dd, n_db, n_q = 200, 1_000_000, 10_000
+    sig = torch.from_numpy(ti.c5_scales(dd).astype(np.float32)).cuda()
+    for b in (2, 4):
+        codec = tq.Codec(dd, dd, b - 1, True, torch.from_numpy(ti.C5.pi().astype(np.float32)),
+                         torch.from_numpy(ti.C5.s().astype(np.float32)))
+        db = torch.randn((n_db, dd), generator=gen, device="cuda") * sig
+        db /= db.norm(dim=1, keepdim=True)
+        qs = torch.randn((n_q, dd), generator=gen, device="cuda") * sig
+        qs /= qs.norm(dim=1, keepdim=True)
+        pk = torch.empty(codec.packed_bytes(1, n_db), dtype=torch.uint8, device="cuda")
+        wq = tq.workspace(256)
+        tq_ms = time_calls(torch, lambda i: tq.tq_quantize(codec, db, 1, n_db, n_db * dd, pk, wq), 3, 1)
+        idx = torch.empty((n_q, 10), dtype=torch.int64, device="cuda")
+        sc = torch.empty((n_q, 10), dtype=torch.float32, device="cuda")
+        ws = tq.workspace(codec.workspace_bytes(tq.TQ_OP_TOPK, n_q, n_db, 10))
+        ms = time_calls(torch, lambda i: tq.tq_topk(codec, pk, n_db, qs, n_q, 10, idx, sc, ws), 3, 1)
+        out[f"c5_vector_search_b{b}"] = {
+            "topk_ms": ms, "queries_per_s": n_q / (ms * 1e-3), "pairs_per_s": n_q * n_db / (ms * 1e-3),
+            "quantize_ms": tq_ms, "quantize_vectors_per_s": n_db / (tq_ms * 1e-3)}
+        del db, qs, pk
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -364,6 +458,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the c2/c3/c5 side measurements")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

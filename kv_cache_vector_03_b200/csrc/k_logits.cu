@@ -406,15 +406,10 @@ cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
     constexpr size_t BB = 512u * NPG + 128u;
     const size_t smem = (size_t)kStreamWarps * NS * BB;
     auto kern = k_logits_stream<B, GD, GM, NT, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static TqLaunchCache cache;
+    int sms = 0, per_sm = 0;
+    cudaError_t e = tq_kernel_setup(kern, kStreamWarps * 32, smem, cache, &sms, &per_sm);
     if (e != cudaSuccess) return e;
-    int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kStreamWarps * 32, smem)) != cudaSuccess)
-        return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    per_sm = std::max(per_sm, 1);
     // tasks of a few blocks each, about eight per resident warp, so that the static
     // round-robin over tasks balances; copies run ahead across task boundaries
     LogitsParams p = p0;
@@ -445,9 +440,13 @@ size_t tq_logits_prologue_smem(const TqDims& t, int) {
     return ((size_t)kPH * (t.D + t.Mp) + (size_t)256 * kPH + (size_t)kPK * (t.D + t.Mp)) * 4;
 }
 
+// largest prologue shared memory over the supported codecs (D = Mp = 256)
+constexpr size_t kPrologueMaxSmem = ((size_t)kPH * 512 + (size_t)256 * kPH + (size_t)kPK * 512) * 4;
+
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     const size_t smem = tq_logits_prologue_smem(p.t, 0);
-    cudaError_t e = cudaFuncSetAttribute(k_logits_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(k_logits_prologue, kPrologueThreads, kPrologueMaxSmem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t n_heads = p.n_seq * p.n_kv * p.g;
     k_logits_prologue<<<(unsigned)((n_heads + kPH - 1) / kPH), kPrologueThreads, smem, st>>>(p);
@@ -455,12 +454,8 @@ cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
 }
 
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st) {
-    const size_t smem = tq_logits_prologue_smem(p.t, 0);
-    cudaError_t e = cudaFuncSetAttribute(k_logits_prologue, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = tq_launch_logits_prologue(p, st);
     if (e != cudaSuccess) return e;
-    const int64_t n_heads = p.n_seq * p.n_kv * p.g;
-    k_logits_prologue<<<(unsigned)((n_heads + kPH - 1) / kPH), kPrologueThreads, smem, st>>>(p);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.nb == 0) return cudaSuccess;
     const int B = p.t.B, GD = p.t.GD, GM = p.t.GM;
 #define TQ_LOGITS_CASE(b, gd, gm) \

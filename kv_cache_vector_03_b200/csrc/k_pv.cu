@@ -188,7 +188,8 @@ template <int B, int KT, int NT>
 cudaError_t launch_split(const PvParams& p, cudaStream_t st) {
     const size_t smem = (size_t)(1 << (2 * B)) * 32 * 4;
     auto kern = k_pv_split<B, KT, NT>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, 128, smem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)(p.n_streams * p.nsplit), 128, smem, st>>>(p);
     return cudaGetLastError();

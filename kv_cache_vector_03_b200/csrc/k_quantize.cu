@@ -547,7 +547,8 @@ template <int KD, int KM, int B>
 cudaError_t launch(const QuantParams& p, cudaStream_t st) {
     const size_t smem_bytes = (size_t)32 * KD * 32 * 4 + (size_t)32 * KD * 32;
     auto kern = k_quantize_f32<KD, KM, B>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, 128, smem_bytes, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t nblocks = p.n_streams * p.nb;
     kern<<<(unsigned)nblocks, 128, smem_bytes, st>>>(p);
@@ -581,11 +582,10 @@ template <bool kF32, int B>
 cudaError_t launch_mma(const QuantParams& p, cudaStream_t st) {
     const size_t smem = 6 * (size_t)mma16::kMatBytes + 128 * 128;
     auto kern = k_quantize_mma<kF32, B>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static TqLaunchCache cache;
+    int sms = 0;
+    cudaError_t e = tq_kernel_setup(kern, 256, smem, cache, &sms, nullptr);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int64_t tiles = (p.n_streams * p.nb + 3) / 4;
     const int64_t grid = std::min<int64_t>(tiles, sms);
     if (grid > 0) kern<<<(unsigned)grid, 256, smem, st>>>(p);

@@ -254,7 +254,8 @@ cudaError_t launch_scan(const TopkParams& p, cudaStream_t st) {
     constexpr size_t BB = 512u * (B * GD + GM) + 128u;
     const size_t smem = NS * BB + (size_t)kWarps * 4 * kList * 8;
     auto kern = k_topk_scan<B, GD, GM, NS>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, kWarps * 32, smem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t qgroups = (p.n_groups + kWarps - 1) / kWarps;
     kern<<<(unsigned)(qgroups * p.nsplit), kWarps * 32, smem, st>>>(p);

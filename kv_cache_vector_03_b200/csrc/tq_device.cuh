@@ -6,7 +6,48 @@
 
 #include "tq_internal.h"
 
+#include <atomic>
+#include <mutex>
+
 #define TQ_DEVICE __device__ __forceinline__
+
+// Per-device launch facts of one kernel, established on its first launch on a device: the
+// dynamic shared-memory opt-in (cudaFuncSetAttribute), the SM count and the CTAs that fit
+// on one SM. Later launches read them without any CUDA API call.
+struct TqLaunchCache {
+    static constexpr int kDevices = 64;
+    int sms[kDevices];
+    int per_sm[kDevices];
+    std::atomic<bool> done[kDevices];
+    std::mutex mu;
+};
+
+template <typename Kernel>
+inline cudaError_t tq_kernel_setup(Kernel kern, int threads, size_t max_smem, TqLaunchCache& c, int* sms,
+                                   int* per_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= TqLaunchCache::kDevices) return cudaErrorInvalidDevice;
+    if (!c.done[dev].load(std::memory_order_acquire)) {
+        std::lock_guard<std::mutex> guard(c.mu);
+        if (!c.done[dev].load(std::memory_order_relaxed)) {
+            if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)max_smem)) !=
+                cudaSuccess)
+                return e;
+            int n = 0, occ = 0;
+            if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+            if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, threads, max_smem)) != cudaSuccess)
+                return e;
+            c.sms[dev] = n;
+            c.per_sm[dev] = occ > 0 ? occ : 1;
+            c.done[dev].store(true, std::memory_order_release);
+        }
+    }
+    if (sms) *sms = c.sms[dev];
+    if (per_sm) *per_sm = c.per_sm[dev];
+    return cudaSuccess;
+}
 
 TQ_DEVICE uint32_t tq_half_bits(float v) { return (uint32_t)__half_as_ushort(__float2half_rn(v)); }
 TQ_DEVICE float tq_half_val(uint32_t bits) { return __half2float(__ushort_as_half((unsigned short)bits)); }
