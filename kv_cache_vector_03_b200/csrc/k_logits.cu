@@ -35,30 +35,73 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
     return ((((size_t)stream * ntiles + ntile) * nmg + mg) * 4 + c) * 64 + lane * 2 + h;
 }
 
-// Prologue. Per CTA: 8 consecutive query heads (rows s*g + h of q).
-//   1. register-tiled GEMM [8 x d] x [d x (D + Mp)] against (Pi^T | S^T), streamed through
-//      shared memory 32 rows at a time (the next chunk is loaded into registers while the
-//      current one is used); each thread owns 2 heads x 4 columns (x 2 for wide codecs):
-//      q' = Pi q and q'' = S q.
-//   2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
-//   3. every thread rounds (head, plane, coordinate) values and scatters their hi and lo
-//      bytes straight into MMA fragment order; per-head constants and the tail follow.
-constexpr int kPH = 8;    // heads per prologue CTA
-constexpr int kPK = 16;   // matrix rows per shared-memory chunk
+// Prologue. Grid (ceil(heads / 8), 1 + ceil(n_tail / 32)); each CTA owns 8 consecutive query
+// heads (rows s*g + h of q).
+//   y = 0: 1. q' = Pi q and q'' = S q as one [8 x d] x [d x (D + Mp)] product against
+//             (Pi^T | S^T). Thread (row half, head quad, column quad) keeps 4 heads x 4 columns
+//             (x 2 for wide codecs) and reads the matrix rows from global memory, where every
+//             CTA finds them in L1 / L2; the two row halves are added in shared memory.
+//          2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
+//          3. one thread per fragment word: it rounds its four coordinates, packs their hi and
+//             lo bytes into two words and stores them; warp sums give the per-head constants.
+//   y > 0: exact logits of 32 tail tokens for the 8 heads, one warp per token.
+constexpr int kPH = 8;         // heads per prologue CTA
+constexpr int kTailTok = 32;   // tail tokens per tail CTA
 
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
+    // the kernel that consumes the fragments may launch now; it waits for this grid's
+    // completion before it reads them
+    tq_pdl_launch_dependents();
     const TqDims& T = p.t;
     const int D = T.D, Mp = T.Mp, d = T.d, G = p.g, np = T.nplanes_mma, W = D + Mp;
     const int n_heads = (int)(p.n_seq * p.n_kv * G);
     const int h_base = blockIdx.x * kPH;
     const int H = min(kPH, n_heads - h_base);
     extern __shared__ __align__(16) float sm[];
-    float* qo = sm;                    // [8][W]: q' (0..D-1) then q'' (D..W-1)
-    float* qT = qo + kPH * W;          // [d rounded to 32][8] query, transposed
-    float* mt = qT + 256 * kPH;        // [kPK][W] rows of (Pi^T | S^T)
-    __shared__ float s_inv[2][kPH], s_step[2][kPH];
-    __shared__ int s_sum[2][kPH], s_fbase[kPH], s_gcol[kPH];
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
+
+    if (blockIdx.y > 0) {
+        // exact logits of the full-precision tail: scale <q, k>
+        float* qh = sm;   // [8][d]
+        for (int e = tid; e < kPH * d; e += blockDim.x) {
+            const int h = e / d, j = e - h * d;
+            qh[e] = h < H ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
+        }
+        __syncthreads();
+        const int64_t row = p.n_tok + p.n_tail;
+        for (int tk = wid; tk < kTailTok; tk += kPrologueThreads / 32) {
+            const int tt = (blockIdx.y - 1) * kTailTok + tk;
+            if (tt >= p.n_tail) break;
+            int64_t cur = -1;
+            float kv[8];   // coordinates lane + 32 i of the key (d <= 256)
+            for (int h = 0; h < H; ++h) {
+                const int64_t gh = h_base + h, stream = gh / G;
+                if (stream != cur) {
+                    cur = stream;
+                    const uint16_t* kp = p.tail + ((size_t)stream * p.n_tail + tt) * d;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int j = lane + 32 * i;
+                        kv[i] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
+                    }
+                }
+                float a = 0.f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int j = lane + 32 * i;
+                    if (j < d) a = fmaf(kv[i], qh[h * d + j], a);
+                }
+                a = tq_warp_sum(a);
+                if (lane == 0) p.out[gh * row + p.n_tok + tt] = p.scale * a;
+            }
+        }
+        return;
+    }
+
+    float* qT = sm;                    // [256][8] query, transposed (rows >= d are zero)
+    float* qo = qT + 256 * kPH;        // [8][W]: q' (0..D-1) then q'' (D..W-1)
+    __shared__ float s_inv[2][kPH], s_step[2][kPH];
+    __shared__ int s_sum[2][kPH];
     const int nmg = T.nmg;
     const int frag_words = p.ntiles * nmg * 256;
 
@@ -73,78 +116,73 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         const bool ok = h < H && j < d && (int64_t)(h_base + h) < p.n_heads_valid;
         qT[e] = ok ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
     }
-    if (tid < kPH) {
-        const int gh = h_base + tid, stream = gh / G, head = gh % G;
-        s_fbase[tid] = (stream * p.ntiles + (head >> 2)) * nmg * 256;
-        s_gcol[tid] = 2 * (head & 3);
-        s_sum[0][tid] = s_sum[1][tid] = 0;
-    }
+    if (tid < 2 * kPH) s_sum[tid / kPH][tid % kPH] = 0;
+    __syncthreads();
 
-    // 1. GEMM: thread (hp = tid / 64 -> heads 2hp, 2hp+1; cq = tid % 64 -> columns 4cq + 256r)
-    const int hp = tid >> 6, cq = tid & 63;
-    const int nr = (W + 255) / 256;
-    const int n4 = kPK * W / 4;        // float4 per chunk
-    float acc[2][2][4];
+    // 1. product. Thread -> ks (rows j of half ks), hq (heads 4hq .. 4hq + 3), cq (columns
+    //    4cq + 256r). Column c < D is row c of Pi (PiT[j][c]); c >= D is row c - D of S.
+    {
+        const int ks = tid >> 7, hq = (tid >> 6) & 1, cq = tid & 63;
+        const float* bp[2];
+        int bs[2];
+        bool bv[2];
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int b = 0; b < 4; ++b) acc[r][a][b] = 0.f;
-    constexpr int kPre = kPK * 512 / 4 / kPrologueThreads;   // float4 per thread for the widest codec
-    static_assert(kPre * 4 * kPrologueThreads >= kPK * 512, "prefetch must cover a chunk");
-    float4 pre[kPre];   // next chunk
-    // float4 e = tid + k * 256 of a chunk sits at row (4e) / W, column (4e) % W; the first
-    // position is divided once, the others follow by stepping 1024 floats
-    int f_row0 = (4 * tid) / W, f_col0 = (4 * tid) % W;
-    auto fetch = [&](int j0) {
-        int jj = f_row0, o = f_col0;
-#pragma unroll
-        for (int k = 0; k < kPre; ++k) {
-            const int e = tid + k * kPrologueThreads;
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            const int j = j0 + jj;
-            if (e < n4 && j < d)
-                v = o < D ? *reinterpret_cast<const float4*>(p.piT + (size_t)j * D + o)
-                          : *reinterpret_cast<const float4*>(p.sT + (size_t)j * Mp + (o - D));
-            pre[k] = v;
-            o += 4 * kPrologueThreads;
-            while (o >= W) { o -= W; ++jj; }
+        for (int r = 0; r < 2; ++r) {
+            const int col = 256 * r + 4 * cq;
+            bv[r] = col < W;
+            bp[r] = col < D ? p.piT + col : p.sT + (col - D);
+            bs[r] = col < D ? D : Mp;
         }
-    };
-    fetch(0);
-    for (int j0 = 0; j0 < d; j0 += kPK) {
-        __syncthreads();
+        float acc[2][4][4];
 #pragma unroll
-        for (int k = 0; k < kPre; ++k) {
-            const int e = tid + k * kPrologueThreads;
-            if (e < n4) reinterpret_cast<float4*>(mt)[e] = pre[k];
-        }
-        __syncthreads();
-        if (j0 + kPK < d) fetch(j0 + kPK);
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) acc[r][x][y] = 0.f;
+        const int jh = (d + 1) >> 1, j0 = ks * jh, j1 = min(d, j0 + jh);
 #pragma unroll 4
-        for (int jj = 0; jj < kPK; ++jj) {
-            const float2 a = reinterpret_cast<const float2*>(qT + (j0 + jj) * kPH)[hp];
+        for (int j = j0; j < j1; ++j) {
+            const float4 a = *reinterpret_cast<const float4*>(qT + j * kPH + 4 * hq);
+            const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
-                if (r < nr && 256 * r + 4 * cq < W) {
-                    const float4 b = reinterpret_cast<const float4*>(mt + jj * W + 256 * r)[cq];
-                    acc[r][0][0] = fmaf(a.x, b.x, acc[r][0][0]); acc[r][0][1] = fmaf(a.x, b.y, acc[r][0][1]);
-                    acc[r][0][2] = fmaf(a.x, b.z, acc[r][0][2]); acc[r][0][3] = fmaf(a.x, b.w, acc[r][0][3]);
-                    acc[r][1][0] = fmaf(a.y, b.x, acc[r][1][0]); acc[r][1][1] = fmaf(a.y, b.y, acc[r][1][1]);
-                    acc[r][1][2] = fmaf(a.y, b.z, acc[r][1][2]); acc[r][1][3] = fmaf(a.y, b.w, acc[r][1][3]);
+                if (!bv[r]) continue;
+                const float4 b = __ldg(reinterpret_cast<const float4*>(bp[r] + (size_t)j * bs[r]));
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    acc[r][x][0] = fmaf(av[x], b.x, acc[r][x][0]);
+                    acc[r][x][1] = fmaf(av[x], b.y, acc[r][x][1]);
+                    acc[r][x][2] = fmaf(av[x], b.z, acc[r][x][2]);
+                    acc[r][x][3] = fmaf(av[x], b.w, acc[r][x][3]);
                 }
             }
         }
+        // the second row half parks its sums in qo; the first adds its own
+        if (ks == 1) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                if (bv[r])
+#pragma unroll
+                    for (int x = 0; x < 4; ++x)
+                        *reinterpret_cast<float4*>(qo + (4 * hq + x) * W + 256 * r + 4 * cq) =
+                            make_float4(acc[r][x][0], acc[r][x][1], acc[r][x][2], acc[r][x][3]);
+        }
+        __syncthreads();
+        if (ks == 0) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+                if (bv[r])
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) {
+                        float4* o = reinterpret_cast<float4*>(qo + (4 * hq + x) * W + 256 * r + 4 * cq);
+                        const float4 v = *o;
+                        *o = make_float4(v.x + acc[r][x][0], v.y + acc[r][x][1], v.z + acc[r][x][2],
+                                         v.w + acc[r][x][3]);
+                    }
+        }
+        __syncthreads();
     }
-#pragma unroll
-    for (int r = 0; r < 2; ++r)
-        if (r < nr && 256 * r + 4 * cq < W)
-#pragma unroll
-            for (int x = 0; x < 2; ++x)
-                *reinterpret_cast<float4*>(qo + (2 * hp + x) * W + 256 * r + 4 * cq) =
-                    make_float4(acc[r][x][0], acc[r][x][1], acc[r][x][2], acc[r][x][3]);
-    __syncthreads();
     // 2. fixed-point steps (one head per warp)
     float amax = 0.f;
     for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
@@ -163,40 +201,38 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         }
     }
     __syncthreads();
-    // 3. round and scatter. Thread -> (coordinate slot within 128, plane group); loops over
-    //    heads. Byte bb of register (mg, c, lane = 4 gcol + t, hh) holds coordinate
-    //    128 gr + 32 t + 2c + hh + 8 bb, column gcol = 2 (head % 4) + part.
-    uint8_t* fb = reinterpret_cast<uint8_t*>(p.qfrag);
-    const int w32 = tid & 127, t = w32 >> 5, sb = w32 & 31;
-    const int bb = sb >> 3, c = (sb & 7) >> 1, hh = sb & 1;
-    const int slot = c * 64 + 2 * t + hh;     // word offset inside (stream, ntile, mg) for lane 4*gcol + t
-    int sa_loc[kPH], ss_loc[kPH];
-#pragma unroll
-    for (int h = 0; h < kPH; ++h) { sa_loc[h] = 0; ss_loc[h] = 0; }
-    for (int mg = tid >> 7; mg < nmg; mg += kPrologueThreads / 128) {
+    // 3. fragment words. Item e -> head h, plane group mg, chunk c, slot t, register hh; byte bb
+    //    of the word is coordinate 128 gr + 32 t + 2c + hh + 8 bb, in column 2 (head % 4) (hi)
+    //    or 2 (head % 4) + 1 (lo) of n-tile head / 4. A warp's 32 items share h and mg.
+    const int per_head = 32 * nmg;
+    for (int e = tid; e < kPH * per_head; e += blockDim.x) {
+        const int h = e / per_head, w = e - h * per_head;
+        const int mg = w >> 5, c = (w >> 3) & 3, t = (w >> 1) & 3, hh = w & 1;
         const bool is_code = mg < np * T.GD;
-        const int gr = is_code ? mg % T.GD : mg - np * T.GD;
-        const int pl = is_code ? mg / T.GD : 0;
-        const float coef = is_code ? 2.f * p.cb.plane_coef[pl] : 1.f;
-        const int col = (is_code ? 0 : D) + 128 * gr + w32;
-        const int kind = is_code ? 0 : 1;
+        int sum = 0;
+        if (h < H) {
+            const int gr = is_code ? mg % T.GD : mg - np * T.GD;
+            const float coef = is_code ? 2.f * p.cb.plane_coef[mg / T.GD] : 1.f;
+            const float inv = coef * s_inv[is_code ? 0 : 1][h];
+            const float* src = qo + h * W + (is_code ? 0 : D) + 128 * gr + 32 * t + 2 * c + hh;
+            uint32_t whi = 0, wlo = 0;
 #pragma unroll
-        for (int h = 0; h < kPH; ++h) {
-            if (h < H) {
-                const int v = __float2int_rn(coef * qo[h * W + col] * s_inv[kind][h]);
-                if (is_code) sa_loc[h] += v; else ss_loc[h] += v;
+            for (int bb = 0; bb < 4; ++bb) {
+                const int v = __float2int_rn(src[8 * bb] * inv);
+                sum += v;
                 const int hi = (v + 128) >> 8, lo = v - 256 * hi;
-                const int w0 = s_fbase[h] + mg * 256 + slot + 8 * s_gcol[h];
-                fb[4 * w0 + bb] = (uint8_t)(hi & 0xff);
-                fb[4 * (w0 + 8) + bb] = (uint8_t)(lo & 0xff);   // lane + 4 -> word + 8
+                whi |= (uint32_t)(hi & 0xff) << (8 * bb);
+                wlo |= (uint32_t)(lo & 0xff) << (8 * bb);
             }
+            const int gh = h_base + h, stream = gh / G, head = gh - stream * G;
+            const size_t wi = ((size_t)stream * p.ntiles + (head >> 2)) * nmg * 256 + mg * 256 + c * 64 +
+                              16 * (head & 3) + 2 * t + hh;
+            p.qfrag[wi] = whi;
+            p.qfrag[wi + 8] = wlo;   // lane + 4 (column lo) -> word + 8
         }
-    }
 #pragma unroll
-    for (int h = 0; h < kPH; ++h) {
-        int a = sa_loc[h], b = ss_loc[h];
-        for (int o = 16; o > 0; o >>= 1) { a += __shfl_xor_sync(0xffffffffu, a, o); b += __shfl_xor_sync(0xffffffffu, b, o); }
-        if (lane == 0 && h < H) { atomicAdd(&s_sum[0][h], a); atomicAdd(&s_sum[1][h], b); }
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (lane == 0 && h < H) atomicAdd(&s_sum[is_code ? 0 : 1][h], sum);
     }
     __syncthreads();
     // per-head scales, folding the 128 of the u8 bit bytes and the QJL factor kappa:
@@ -207,18 +243,6 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
             make_float4(dA / 128.f, 0.5f * dA * (float)s_sum[0][tid], p.kappa * 2.f * dS / 128.f,
                         p.kappa * dS * (float)s_sum[1][tid]);
-    }
-    // exact logits of the full-precision tail: scale <q, k>
-    if (p.n_tail > 0) {
-        const int64_t row = p.n_tok + p.n_tail;
-        for (int e = tid; e < H * p.n_tail; e += blockDim.x) {
-            const int h = e / p.n_tail, tt = e % p.n_tail;
-            const int64_t gh = h_base + h, stream = gh / G;
-            const uint16_t* kp = p.tail + ((size_t)stream * p.n_tail + tt) * d;
-            float a = 0.f;
-            for (int i = 0; i < d; ++i) a = fmaf(__uint_as_float((uint32_t)kp[i] << 16), qT[i * kPH + h], a);
-            p.out[gh * row + p.n_tok + tt] = p.scale * a;
-        }
     }
 }
 
@@ -276,11 +300,10 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
         }
     }
 
+    // the copies above read only keys; the query fragments come from the prologue
+    tq_pdl_wait();
     const float scale = p.scale;
     const int64_t row = p.n_tok + p.n_tail;
-    uint32_t mul[7];   // 2^(7-s), s < 7, unknown to the compiler: the shifts issue as IMAD
-#pragma unroll
-    for (int k = 0; k < 7; ++k) mul[k] = p.shl[k];
     uint32_t qf[NT][NMG][4][2];
     float4 sc[NT];
     float* orow[NT];
@@ -342,19 +365,13 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
                     w0 = cw[2 * mt];
                     w1 = cw[2 * mt + 1];
                 }
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    // coordinate bit s (= 2c, 2c + 1) of each byte moved to bit 7: A byte = 128 * bit
-                    const uint32_t a0 = (w0 * mul[2 * c]) & 0x80808080u;
-                    const uint32_t a1 = (w1 * mul[2 * c]) & 0x80808080u;
-                    const uint32_t a2 = (c == 3 ? w0 : w0 * mul[(2 * c + 1) % 7]) & 0x80808080u;
-                    const uint32_t a3 = (c == 3 ? w1 : w1 * mul[(2 * c + 1) % 7]) & 0x80808080u;
+                tq_expand_planes(w0, w1, [&](int c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
                         if (mg < NP * GD) tq_imma_u8(accA[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
                         else tq_imma_u8(accS[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
                     }
-                }
+                });
             }
             // epilogue: thread (g, t) -> head t of each n-tile, rows g and g + 8
             const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
@@ -425,8 +442,8 @@ cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
     const int64_t step = grid * kStreamWarps;
     p.step_s = (int)(step / p.tpt);
     p.step_c = (int)(step % p.tpt);
-    if (grid > 0) kern<<<(unsigned)grid, kStreamWarps * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    if (grid == 0) return cudaSuccess;
+    return tq_launch_pdl(kern, dim3((unsigned)grid), dim3(kStreamWarps * 32), smem, st, p);
 }
 
 template <int B, int GD, int GM>
@@ -437,11 +454,11 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 }  // namespace
 
 size_t tq_logits_prologue_smem(const TqDims& t, int) {
-    return ((size_t)kPH * (t.D + t.Mp) + (size_t)256 * kPH + (size_t)kPK * (t.D + t.Mp)) * 4;
+    return ((size_t)256 * kPH + (size_t)kPH * (t.D + t.Mp)) * 4;
 }
 
 // largest prologue shared memory over the supported codecs (D = Mp = 256)
-constexpr size_t kPrologueMaxSmem = ((size_t)kPH * 512 + (size_t)256 * kPH + (size_t)kPK * 512) * 4;
+constexpr size_t kPrologueMaxSmem = ((size_t)256 * kPH + (size_t)kPH * 512) * 4;
 
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     const size_t smem = tq_logits_prologue_smem(p.t, 0);
@@ -449,7 +466,8 @@ cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     cudaError_t e = tq_kernel_setup(k_logits_prologue, kPrologueThreads, kPrologueMaxSmem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t n_heads = p.n_seq * p.n_kv * p.g;
-    k_logits_prologue<<<(unsigned)((n_heads + kPH - 1) / kPH), kPrologueThreads, smem, st>>>(p);
+    const dim3 grid((unsigned)((n_heads + kPH - 1) / kPH), 1u + (unsigned)((p.n_tail + kTailTok - 1) / kTailTok));
+    k_logits_prologue<<<grid, kPrologueThreads, smem, st>>>(p);
     return cudaGetLastError();
 }
 

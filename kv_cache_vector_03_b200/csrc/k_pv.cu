@@ -4,28 +4,51 @@
 //   o_h = sum_t w_t |v_t| Pi^T c[idx_t] = Pi^T ( sum_t w_t |v_t| c[idx_t] )
 // so the weighted sum is accumulated in the rotated domain and rotated back once.
 //
-// Kernel 1 (split): one CTA of 4 warps per (stream, token range). The range's softmax
-// maximum is found first; then each 32-token block is dequantized straight into fp16 MMA
-// A fragments (rows = coordinates, K = tokens) through a per-lane shared-memory table that
-// maps a 2B-bit field (two tokens' codes of one coordinate) to a half2 of centroids, and
-// multiplied on the tensor cores by B = weights exp(P - m) |v| split into fp16 hi + lo
-// columns. Partial sums, maxima and softmax denominators go to the workspace.
+// Kernel 1 (split): one CTA of 4 warps per (stream, block range); warp w takes blocks
+// w, w + 4, ... of the range. Each warp keeps a ring of NS stages in shared memory: the packed
+// 32-token block arrives by a bulk copy (TMA engine, mbarrier completion) and its P values by
+// 4-byte asynchronous copies. Per block and head the warp updates a running maximum (online
+// softmax: a new maximum rescales the accumulators), computes one exp per (head, token) and
+// stages the weights exp(P - m) |v| as fp16 hi + lo columns. The codes are dequantized
+// straight into fp16 MMA A fragments (rows = coordinates, K = tokens) through a per-lane
+// table that maps a 2B-bit field (two tokens' codes of one coordinate) to a half2 of
+// centroids, and multiplied on the tensor cores. The 4 warps meet at the CTA's maximum;
+// partial sums, maxima and denominators go to the workspace.
 // Kernel 2 (merge): one CTA per query head combines the partials (log-sum-exp rescale) and
 // rotates by Pi^T.
 #include "tq_device.cuh"
 
 namespace {
 
+constexpr int kPvWarps = 4;
+constexpr int kPvNS = 4;              // ring stages per warp
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kWCol = 20;             // words per staged weight column (16 used; 20 spreads the banks)
+
+template <int B, int KT, int NT>
+constexpr size_t pv_smem_bytes() {
+    return (size_t)(1 << (2 * B)) * 128 + (size_t)kPvWarps * kPvNS * (512 * (KT * B / 8) + 64) +
+           (size_t)kPvWarps * kPvNS * 4 * NT * 32 * 4;
+}
+
 template <int B, int KT, int NT>  // KT = D/16 coordinate tiles, NT = n-tiles of 4 heads
-__global__ void __launch_bounds__(128) k_pv_split(PvParams p) {
+__global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
+    constexpr int NS = kPvNS;
     constexpr int E = 1 << (2 * B);          // table entries
     constexpr int CH = KT * B / 8;           // 16-byte chunks per lane per block (D*B/128)
     constexpr int NW = 4 * CH;               // 32-bit words per lane per block
-    extern __shared__ uint32_t lut[];        // [E][32]
-    __shared__ float s_acc[8][KT * 16];
-    __shared__ float s_m[8], s_l[8];
+    constexpr uint32_t SEC_A = 512u * CH;    // codes; 32 fp16 norms follow
+    constexpr uint32_t BBYTES = SEC_A + 64u;
+    constexpr int HP = 4 * NT;               // heads, padded to whole n-tiles
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);                              // [E][32]
+    uint8_t* ring = smem + (size_t)E * 128;                                          // [warp][NS][BBYTES]
+    float* pring = reinterpret_cast<float*>(ring + (size_t)kPvWarps * NS * BBYTES);  // [warp][NS][HP][32]
+    __shared__ uint32_t wst[kPvWarps][2 * HP][kWCol];   // column 2h (hi) / 2h + 1 (lo): token pairs
+    __shared__ float s_acc[HP][KT * 16];
+    __shared__ float s_m[kPvWarps][HP], s_l[HP];
+    __shared__ uint64_t bars[kPvWarps][NS];
 
-    const TqDims& T = p.t;
     const int G = p.g;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -33,22 +56,38 @@ __global__ void __launch_bounds__(128) k_pv_split(PvParams p) {
     const int split = blockIdx.x % p.nsplit;
     const int64_t b0 = (int64_t)split * p.blocks_per_split;
     const int64_t b1 = min(b0 + p.blocks_per_split, p.nb);
-    const int64_t t0 = b0 * 32, t1 = min(b1 * 32, p.n_tok);
     const float* Pst = p.P + (size_t)stream * G * p.n_tok;
+    const uint8_t* sbase = p.packed + (size_t)stream * p.nb * BBYTES;
 
     for (int e = threadIdx.x; e < E * 32; e += blockDim.x) {
         const int ent = e >> 5;
         lut[e] = p.cb.lut_half[ent & ((1 << B) - 1)] | (p.cb.lut_half[ent >> B] << 16);
     }
-    for (int e = threadIdx.x; e < 8 * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
-    // pass 1: per-head maximum over the range
-    for (int h = w; h < G; h += 4) {
-        float mx = -INFINITY;
-        for (int64_t tok = t0 + lane; tok < t1; tok += 32) mx = fmaxf(mx, Pst[(size_t)h * p.n_tok + tok]);
-        mx = tq_warp_max(mx);
-        if (lane == 0) { s_m[h] = mx; s_l[h] = 0.f; }
-    }
+    for (int e = threadIdx.x; e < HP * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
+    if (threadIdx.x < HP) s_l[threadIdx.x] = 0.f;
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[w][s], 1);
+    tq_fence_mbar_init();
     __syncthreads();
+
+    uint8_t* my_ring = ring + (size_t)w * NS * BBYTES;
+    float* my_p = pring + (size_t)w * NS * HP * 32;
+    const int64_t first = b0 + w;
+    const int nmine = first < b1 ? (int)((b1 - first + kPvWarps - 1) / kPvWarps) : 0;
+    // block k of this warp (first + 4k) into stage k % NS; every lane commits one copy group
+    auto issue = [&](int k) {
+        if (k < nmine) {
+            const int s = k % NS;
+            const int64_t bi = first + (int64_t)kPvWarps * k;
+            if (lane == 0) tq_bulk_load(my_ring + s * BBYTES, sbase + (size_t)bi * BBYTES, BBYTES, &bars[w][s]);
+            const int64_t tok = bi * 32 + lane;
+            const bool in = tok < p.n_tok;
+            for (int h = 0; h < G; ++h)
+                tq_cp_async4(my_p + (s * HP + h) * 32 + lane, in ? Pst + (size_t)h * p.n_tok + tok : p.P, in ? 4u : 0u);
+        }
+        tq_cp_async_commit();
+    };
+    for (int k = 0; k < NS; ++k) issue(k);
 
     float acc[KT][NT][4];
 #pragma unroll
@@ -57,67 +96,81 @@ __global__ void __launch_bounds__(128) k_pv_split(PvParams p) {
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int r = 0; r < 4; ++r) acc[k][n][r] = 0.f;
-    float lsum[NT];
+    float m_run[HP], lsum[HP];   // m_run is the same in every lane; lsum holds the lane's tokens
 #pragma unroll
-    for (int n = 0; n < NT; ++n) lsum[n] = 0.f;
-    float mh[NT];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const int head = n * 4 + (g >> 1);
-        mh[n] = head < G ? s_m[head] : 0.f;
-    }
+    for (int h = 0; h < HP; ++h) { m_run[h] = -INFINITY; lsum[h] = 0.f; }
 
-    const uint8_t* sbase = p.packed + (size_t)stream * p.nb * T.block_bytes;
-    const uint32_t sec_a = T.sec_a;
-#pragma unroll 1
-    for (int64_t bi = b0 + w; bi < b1; bi += 4) {
-        const uint8_t* bp = sbase + (size_t)bi * T.block_bytes;
-        uint32_t W[NW + 1];
+    bool ok = true;
+    int k = 0;
+    for (; k < nmine; ++k) {
+        const int s = k % NS;
+        tq_cp_async_wait<NS - 1>();   // this lane's P copies of block k have landed
+        ok = __all_sync(0xffffffffu, tq_mbar_wait(&bars[w][s], (uint32_t)(k / NS) & 1u, kWaitLimit));
+        if (!ok) break;
+        __syncwarp();                 // and those of the other lanes are visible
+        const uint8_t* bp = my_ring + s * BBYTES;
+        const int64_t tok = (first + (int64_t)kPvWarps * k) * 32 + lane;
+        const bool in = tok < p.n_tok;
+        const float nrm = tq_half_val(reinterpret_cast<const uint16_t*>(bp + SEC_A)[lane]);
+        // online maximum and weights of this lane's token, one head at a time
+        float fac[HP];
+        bool grew = false;
 #pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            const uint4 v = tq_ldg_stream(bp + (size_t)(c * 32 + lane) * 16);
-            W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
+        for (int h = 0; h < HP; ++h) {
+            fac[h] = 1.f;
+            if (h < G) {
+                const float pv = in ? my_p[(s * HP + h) * 32 + lane] : -INFINITY;
+                const float bm = tq_warp_max(pv);
+                if (bm > m_run[h]) {
+                    fac[h] = __expf(m_run[h] - bm);   // 0 while the running maximum is -inf
+                    m_run[h] = bm;
+                    grew = true;
+                }
+                const float ex = m_run[h] > -INFINITY ? __expf(pv - m_run[h]) : 0.f;
+                lsum[h] = fmaf(lsum[h], fac[h], ex);
+                const float wt = ex * nrm;
+                const __half hi = __float2half_rn(wt);
+                reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = hi;
+                reinterpret_cast<__half*>(&wst[w][2 * h + 1][0])[lane] = __float2half_rn(wt - __half2float(hi));
+            }
         }
-        W[NW] = 0u;
-        const uint16_t* nrm = reinterpret_cast<const uint16_t*>(bp + sec_a);
-        // weights for the 8 tokens this thread feeds: chunk c, pair (2t, 2t+1) and (8+2t, 9+2t)
+        if (grew) {
+            // accumulator columns 2t, 2t + 1 of n-tile n belong to head 4n + t
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const float f = t == 0 ? fac[4 * n] : t == 1 ? fac[4 * n + 1] : t == 2 ? fac[4 * n + 2] : fac[4 * n + 3];
+#pragma unroll
+                for (int kk = 0; kk < KT; ++kk)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[kk][n][r] *= f;
+            }
+        }
+        __syncwarp();
+        // B fragments: column g of n-tile n (head 4n + g/2, hi or lo), tokens 16c + 8hv + 2t, +1
         uint32_t bw[NT][2][2];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int head = n * 4 + (g >> 1);
-            const bool part_lo = g & 1;
+        for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    uint32_t packed2 = 0;
+                for (int hv = 0; hv < 2; ++hv) bw[n][c][hv] = wst[w][8 * n + g][8 * c + 4 * hv + t];
+        uint32_t W[NW + 1];
 #pragma unroll
-                    for (int e2 = 0; e2 < 2; ++e2) {
-                        const int tb = 16 * c + 8 * hv + 2 * t + e2;
-                        const int64_t tok = bi * 32 + tb;
-                        float wt = 0.f;
-                        if (head < G && tok < p.n_tok) {
-                            const float ex = __expf(Pst[(size_t)head * p.n_tok + tok] - mh[n]);
-                            if (!part_lo) lsum[n] += ex;
-                            wt = ex * tq_half_val(nrm[tb]);
-                        }
-                        const __half hi = __float2half_rn(wt);
-                        const __half val = part_lo ? __float2half_rn(wt - __half2float(hi)) : hi;
-                        packed2 |= (uint32_t)__half_as_ushort(val) << (16 * e2);
-                    }
-                    bw[n][c][hv] = packed2;
-                }
+        for (int c = 0; c < CH; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(bp + (c * 32 + lane) * 16);
+            W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
         }
+        W[NW] = 0u;
         // A fragments: field (a, pp) at bit (4a + pp) * 2B of the lane string
 #pragma unroll
-        for (int k = 0; k < KT; ++k)
+        for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
                 uint32_t a[4];
 #pragma unroll
                 for (int r = 0; r < 4; ++r) {
-                    // r: 0 -> (a=2k, pp=2c), 1 -> (2k+1, 2c), 2 -> (2k, 2c+1), 3 -> (2k+1, 2c+1)
-                    const int f = 4 * (2 * k + (r & 1)) + 2 * c + (r >> 1);
+                    // r: 0 -> (a=2kk, pp=2c), 1 -> (2kk+1, 2c), 2 -> (2kk, 2c+1), 3 -> (2kk+1, 2c+1)
+                    const int f = 4 * (2 * kk + (r & 1)) + 2 * c + (r >> 1);
                     const int bit = f * 2 * B;
                     const int wi = bit >> 5, sh = bit & 31;
                     uint32_t fld = sh == 0 ? W[wi] : __funnelshift_r(W[wi], W[wi + 1], sh);
@@ -125,73 +178,163 @@ __global__ void __launch_bounds__(128) k_pv_split(PvParams p) {
                     a[r] = lut[fld * 32 + lane];
                 }
 #pragma unroll
-                for (int n = 0; n < NT; ++n) tq_hmma(acc[k][n], a[0], a[1], a[2], a[3], bw[n][c][0], bw[n][c][1]);
+                for (int n = 0; n < NT; ++n) tq_hmma(acc[kk][n], a[0], a[1], a[2], a[3], bw[n][c][0], bw[n][c][1]);
             }
+        // the stage is consumed: refill it with block k + NS
+        __syncwarp();
+        if (lane == 0) tq_fence_proxy_async();
+        issue(k + NS);
     }
-    // combine hi + lo columns and the 4 warps
+    tq_cp_async_wait<0>();
+    if (!ok) {
+        // a wait ran out: record it and give the copies in flight a bounded time to land
+        if (lane == 0) {
+            tq_raise(p.status, TQ_FLAG_TIMEOUT);
+            for (int j = k; j < min(k + NS, nmine); ++j)
+                tq_mbar_wait(&bars[w][j % NS], (uint32_t)(j / NS) & 1u, kWaitLimit);
+        }
+        __syncwarp();
+    }
+    // the CTA's maximum per head; each warp's sums are rescaled to it
+    if (lane == 0)
+#pragma unroll
+        for (int h = 0; h < HP; ++h) s_m[w][h] = m_run[h];
+    __syncthreads();
+    float scl[HP];
+#pragma unroll
+    for (int h = 0; h < HP; ++h) {
+        float M = s_m[0][h];
+#pragma unroll
+        for (int v = 1; v < kPvWarps; ++v) M = fmaxf(M, s_m[v][h]);
+        scl[h] = m_run[h] > -INFINITY ? __expf(m_run[h] - M) : 0.f;
+    }
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int head = n * 4 + t;
+        const float f = t == 0 ? scl[4 * n] : t == 1 ? scl[4 * n + 1] : t == 2 ? scl[4 * n + 2] : scl[4 * n + 3];
         if (head < G) {
 #pragma unroll
-            for (int k = 0; k < KT; ++k) {
-                atomicAdd(&s_acc[head][16 * k + g], acc[k][n][0] + acc[k][n][1]);
-                atomicAdd(&s_acc[head][16 * k + 8 + g], acc[k][n][2] + acc[k][n][3]);
+            for (int kk = 0; kk < KT; ++kk) {
+                atomicAdd(&s_acc[head][16 * kk + g], f * (acc[kk][n][0] + acc[kk][n][1]));
+                atomicAdd(&s_acc[head][16 * kk + 8 + g], f * (acc[kk][n][2] + acc[kk][n][3]));
             }
         }
-        float ls = lsum[n];
-        // lanes 8h + t (t = 0..3) hold the exps of head n*4 + h
-        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-        const int hh = n * 4 + (g >> 1);
-        if ((lane & 7) == 0 && hh < G) atomicAdd(&s_l[hh], ls);
+    }
+#pragma unroll
+    for (int h = 0; h < HP; ++h) {
+        if (h < G) {
+            const float ls = tq_warp_sum(lsum[h]) * scl[h];
+            if (lane == 0) atomicAdd(&s_l[h], ls);
+        }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < G * T.D; e += blockDim.x) {
-        const int h = e / T.D, i = e % T.D;
-        p.part[(((size_t)stream * G + h) * p.nsplit + split) * T.D + i] = s_acc[h][i];
+    const int D = KT * 16;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, i = e % D;
+        p.part[(((size_t)stream * G + h) * p.nsplit + split) * D + i] = s_acc[h][i];
     }
     if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = s_m[0][h];
+        for (int v = 1; v < kPvWarps; ++v) M = fmaxf(M, s_m[v][h]);
         float2* ml = reinterpret_cast<float2*>(p.part_ml);
-        ml[((size_t)stream * G + threadIdx.x) * p.nsplit + split] = make_float2(s_m[threadIdx.x], s_l[threadIdx.x]);
+        ml[((size_t)stream * G + h) * p.nsplit + split] = make_float2(M, s_l[h]);
     }
 }
 
-__global__ void __launch_bounds__(256) k_pv_merge(PvParams p) {
-    const TqDims& T = p.t;
-    const int64_t hq = blockIdx.x;  // stream * g + head
-    __shared__ float s_o[TQ_MAX_D];
-    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * p.nsplit;
-    float M = -INFINITY;
-    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, ml[s].x);
-    for (int i = threadIdx.x; i < T.D; i += blockDim.x) {
-        float acc = 0.f, den = 0.f;
-        for (int s = 0; s < p.nsplit; ++s) {
-            const float2 v = ml[s];
-            if (v.y > 0.f) {
-                const float f = __expf(v.x - M);
-                acc += f * p.part[((size_t)hq * p.nsplit + s) * T.D + i];
-                den += f * v.y;
-            }
-        }
-        s_o[i] = acc / den;
+// One CTA per query head: o = sum_s e^{m_s - M} part_s / sum_s e^{m_s - M} l_s, then Pi^T o.
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
+    const int D = p.t.D, d = p.t.d, ns = p.nsplit;
+    const int64_t hq = blockIdx.x;   // stream * g + head
+    extern __shared__ float msm[];
+    float* fs = msm;                     // [ns] split weights e^{m_s - M}, padded to 4 floats
+    float* red = fs + ((ns + 3) & ~3);   // [1024], 16-byte aligned: [groups][D] partial sums, later [2][256]
+    float* s_o = red + 1024;             // [256]
+    __shared__ float s_w[kMergeThreads / 32];
+    __shared__ float s_M, s_den;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
+
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += kMergeThreads) {
+        const float2 v = ml[s];
+        if (v.y > 0.f) mx = fmaxf(mx, v.x);
+    }
+    mx = tq_warp_max(mx);
+    if (lane == 0) s_w[wid] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        float M = s_w[0];
+        for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, s_w[i]);
+        s_M = M;
     }
     __syncthreads();
-    for (int j = threadIdx.x; j < T.d; j += blockDim.x) {
-        float o = 0.f;
-        for (int i = 0; i < T.d; ++i) o = fmaf(__ldg(p.pi + (size_t)i * T.d + j), s_o[i], o);
-        p.out[(size_t)hq * T.d + j] = o;
+    const float M = s_M;
+    float den = 0.f;
+    for (int s = tid; s < ns; s += kMergeThreads) {
+        const float2 v = ml[s];
+        const float f = v.y > 0.f ? __expf(v.x - M) : 0.f;
+        fs[s] = f;
+        den = fmaf(f, v.y, den);
     }
+    den = tq_warp_sum(den);
+    __syncthreads();   // s_w reused
+    if (lane == 0) s_w[wid] = den;
+    __syncthreads();
+    if (tid == 0) {
+        float v = 0.f;
+        for (int i = 0; i < kMergeThreads / 32; ++i) v += s_w[i];
+        s_den = v;
+    }
+    // weighted sum over splits: thread (group, column quad)
+    const int nq = D / 4, ngrp = kMergeThreads / nq;
+    const int grp = tid / nq, qd = tid % nq;
+    const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = grp; s < ns; s += ngrp) {
+        const float f = fs[s];
+        if (f != 0.f) {
+            const float4 v = src[(size_t)s * nq];
+            a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
+        }
+    }
+    reinterpret_cast<float4*>(red)[grp * nq + qd] = a;
+    __syncthreads();
+    const float inv = 1.f / s_den;
+    for (int i = tid; i < D; i += kMergeThreads) {
+        float v = 0.f;
+        for (int q = 0; q < ngrp; ++q) v += red[q * D + i];
+        s_o[i] = v * inv;
+    }
+    __syncthreads();
+    // out[j] = sum_i Pi[i][j] o_i: thread (j = tid % 128 + 128 r, row half ih)
+    const int ih = tid >> 7, jl = tid & 127, half = (d + 1) >> 1;
+    const int i0 = ih * half, i1 = min(d, i0 + half);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int j = jl + 128 * r;
+        float o = 0.f;
+        if (j < d) {
+#pragma unroll 16
+            for (int i = i0; i < i1; ++i) o = fmaf(__ldg(p.pi + (size_t)i * d + j), s_o[i], o);
+        }
+        red[ih * 256 + j] = o;
+    }
+    __syncthreads();
+    for (int j = tid; j < d; j += kMergeThreads) p.out[(size_t)hq * d + j] = red[j] + red[256 + j];
 }
 
 template <int B, int KT, int NT>
 cudaError_t launch_split(const PvParams& p, cudaStream_t st) {
-    const size_t smem = (size_t)(1 << (2 * B)) * 32 * 4;
+    constexpr size_t smem = pv_smem_bytes<B, KT, NT>();
     auto kern = k_pv_split<B, KT, NT>;
     static TqLaunchCache cache;
-    cudaError_t e = tq_kernel_setup(kern, 128, smem, cache, nullptr, nullptr);
+    cudaError_t e = tq_kernel_setup(kern, kPvWarps * 32, smem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
-    kern<<<(unsigned)(p.n_streams * p.nsplit), 128, smem, st>>>(p);
+    kern<<<(unsigned)(p.n_streams * p.nsplit), kPvWarps * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -206,6 +349,8 @@ cudaError_t launch_b(const PvParams& p, cudaStream_t st) {
     return cudaErrorInvalidValue;
 }
 
+size_t pv_merge_smem(int nsplit) { return (((size_t)nsplit + 3) / 4 * 4 + 1024 + 256) * 4; }
+
 }  // namespace
 
 cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
@@ -215,6 +360,8 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
     else if (p.t.D == 256) e = nt == 1 ? launch_b<16, 1>(p, st) : launch_b<16, 2>(p, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
-    k_pv_merge<<<(unsigned)(p.n_streams * p.g), 256, 0, st>>>(p);
+    const size_t msmem = pv_merge_smem(p.nsplit);
+    if (msmem > 48 * 1024) return cudaErrorInvalidValue;
+    k_pv_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, msmem, st>>>(p);
     return cudaGetLastError();
 }

@@ -112,9 +112,6 @@ __global__ void __launch_bounds__(kWarps * 32) k_topk_scan(TopkParams p) {
             }
         sc = reinterpret_cast<const float4*>(p.qscale)[(size_t)group * 4 + t];
     }
-    uint32_t mul[7];
-#pragma unroll
-    for (int k = 0; k < 7; ++k) mul[k] = p.shl[k];
     float tau = -INFINITY;   // threshold of query t of this warp
     float* my_sc = lsc + (warp * 4) * kList;
     int* my_ix = lix + (warp * 4) * kList;
@@ -150,15 +147,10 @@ __global__ void __launch_bounds__(kWarps * 32) k_topk_scan(TopkParams p) {
                         w0 = cw[2 * mt];
                         w1 = cw[2 * mt + 1];
                     }
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const uint32_t a0 = (w0 * mul[2 * c]) & 0x80808080u;
-                        const uint32_t a1 = (w1 * mul[2 * c]) & 0x80808080u;
-                        const uint32_t a2 = (c == 3 ? w0 : w0 * mul[(2 * c + 1) % 7]) & 0x80808080u;
-                        const uint32_t a3 = (c == 3 ? w1 : w1 * mul[(2 * c + 1) % 7]) & 0x80808080u;
+                    tq_expand_planes(w0, w1, [&](int c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
                         if (mg < NP * GD) tq_imma_u8(accA, a0, a1, a2, a3, qf[mg][c][0], qf[mg][c][1]);
                         else tq_imma_u8(accS, a0, a1, a2, a3, qf[mg][c][0], qf[mg][c][1]);
-                    }
+                    });
                 }
                 const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
 #pragma unroll

@@ -307,15 +307,12 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.scale = scale;
     p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.status = static_cast<uint32_t*>(ws);
-    // streams per prologue CTA: about one CTA per SM, at most 32 query heads per CTA
-    int64_t spc = n_streams / kNumSms;
-    spc = std::max<int64_t>(1, std::min<int64_t>(spc, 16 / g));
-    p.streams_per_cta = (int)spc;
     p.blocks_per_task = 1;
     p.n_tasks = 0;
     p.n_heads_valid = n_streams * g;
-    for (int k = 0; k < 8; ++k) p.shl[k] = 1u << (7 - k);
-    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
+    // the tail runs on a second grid dimension of 32-token CTAs (at most 65535)
+    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 32 * 65534)
+        return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_logits(p, static_cast<cudaStream_t>(stream)));
@@ -338,6 +335,7 @@ int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int6
     PvParams p;
     p.packed = static_cast<const uint8_t*>(packed_v);
     p.P = P; p.out = out; p.pi = c->pi;
+    p.status = static_cast<uint32_t*>(ws);
     p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.part);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.ml);
     p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
@@ -392,7 +390,6 @@ int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float*
     p.status = static_cast<uint32_t*>(ws);
     p.n_db = n_db; p.nb = (n_db + 31) / 32; p.n_q = n_q;
     p.k = k; p.nsplit = W.nsplit; p.blocks_per_split = W.bps; p.n_groups = W.n_groups;
-    for (int s2 = 0; s2 < 8; ++s2) p.shl[s2] = 1u << (7 - s2);
     p.t = t;
     return cuda_status(tq_launch_topk(p, cs));
 }

@@ -61,6 +61,31 @@ TQ_DEVICE void tq_raise(uint32_t* status, uint32_t flag) {
     if (status) atomicOr(status, flag);
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization may
+// start once every CTA of the kernel before it has called launch_dependents (or exited); its
+// wait returns when that kernel has completed and its writes are visible. Without the launch
+// attribute both are no-ops.
+TQ_DEVICE void tq_pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+TQ_DEVICE void tq_pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launches kern<<<grid, block, smem, st>>>(args...) as a programmatic dependent of the
+// previous kernel on st.
+template <typename... KArgs, typename... Args>
+inline cudaError_t tq_launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                 Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // warp-wide reductions
 TQ_DEVICE float tq_warp_sum(float v) {
 #pragma unroll
@@ -79,6 +104,37 @@ TQ_DEVICE float tq_warp_max(float v) {
 }
 
 // int8 tensor-core MMA, 16x8x32, s32 accumulate (legacy warp-level path): A u8, B s8
+// x + x as an integer add. On sm_100 a 32-bit add issues at the full rate, while shifts,
+// IMAD and LOP3 issue at half of it, so the byte-bit moves below are built from adds.
+TQ_DEVICE uint32_t tq_dbl(uint32_t x) {
+    uint32_t y;
+    asm("add.u32 %0, %1, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+// Bit planes to u8 MMA operands. Bit s of every byte of a packed word is one coordinate;
+// a left shift by 7 - s moves it to bit 7, and the mask leaves the byte 0 or 128. For the
+// words w0 (row g) and w1 (row g + 8) of one k-chunk this yields, for c = 3 .. 0,
+//   a0, a1 <- bit 2c and a2, a3 <- bit 2c + 1,
+// the A fragment of chunk c; f(c, a0, a1, a2, a3) consumes it. Shifts 0 .. 7 are reached by
+// doubling, one add per step.
+template <typename F>
+TQ_DEVICE void tq_expand_planes(uint32_t w0, uint32_t w1, F&& f) {
+    uint32_t x0 = w0, x1 = w1;
+#pragma unroll
+    for (int c = 3; c >= 0; --c) {
+        const uint32_t a2 = x0 & 0x80808080u, a3 = x1 & 0x80808080u;   // shift 6 - 2c: bit 2c + 1
+        x0 = tq_dbl(x0);
+        x1 = tq_dbl(x1);
+        const uint32_t a0 = x0 & 0x80808080u, a1 = x1 & 0x80808080u;   // shift 7 - 2c: bit 2c
+        if (c > 0) {
+            x0 = tq_dbl(x0);
+            x1 = tq_dbl(x1);
+        }
+        f(c, a0, a1, a2, a3);
+    }
+}
+
 TQ_DEVICE void tq_imma_u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                           uint32_t b1) {
     asm volatile(
@@ -145,6 +201,17 @@ TQ_DEVICE void tq_hmma(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uin
 }
 
 // 16-byte streaming load of data read once (does not allocate in L1)
+// 4-byte asynchronous copy global -> shared (zero-filled when src_bytes = 0, which reads
+// nothing), grouped per thread by commit / wait_group.
+TQ_DEVICE void tq_cp_async4(void* dst_smem, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(tq_smem_addr(dst_smem)), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+TQ_DEVICE void tq_cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+TQ_DEVICE void tq_cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory"); }
+
 TQ_DEVICE uint4 tq_ldg_stream(const void* p) {
     uint4 v;
     asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
@@ -192,10 +259,9 @@ struct LogitsParams {
     int64_t n_seq, n_tok, nb, n_tasks;
     int n_kv, g, ntiles, n_tail;
     float scale, kappa;
-    int blocks_per_task, streams_per_cta;
+    int blocks_per_task;
     int tpt, n_streams32, step_s, step_c;   // task walk: tasks per stream, stride in (stream, chunk)
     int64_t n_heads_valid;                   // query rows that exist (later heads read as zero)
-    uint32_t shl[8];       // 2^(7-s): runtime multipliers that move bit s of each byte to bit 7
     TqDims t;
     TqCodebookConsts cb;
 };
@@ -205,6 +271,7 @@ struct PvParams {
     const float* P;
     float* out;
     const float* pi;
+    uint32_t* status;
     float* part;           // [stream*g heads][nsplit][D]
     float* part_ml;        // [stream*g heads][nsplit][2]: max, sum
     int64_t n_streams, n_tok, nb;
@@ -224,7 +291,6 @@ struct TopkParams {
     uint32_t* status;
     int64_t n_db, nb, n_q;
     int k, nsplit, blocks_per_split, n_groups;
-    uint32_t shl[8];
     TqDims t;
 };
 
