@@ -11,12 +11,14 @@
 //   <q', c[idx]> = sum_p sum_i (2 a_p q'_i) beta_{p,i} - (sum_p a_p) sum_i q'_i,
 //   <q'', s>     = 2 sum_j q''_j bit_j - sum_j q''_j,
 // two contractions of {0,1} bit planes against fixed vectors, run on the int8 tensor cores
-// (mma.sync m16n8k32, u8 x s8 -> s32). A bit becomes the byte 0 or 128 with one shift and
-// one and per four coordinates (A = 128 * bits); the query side is a 16-bit fixed-point
-// vector split into two int8 columns (hi, lo) of the same MMA, so accumulation is exact.
+// (mma.sync m16n8k32, u8 x s8 -> s32). A bit s of a packed byte is masked in place (one
+// and per four coordinates, plus one shift per word for s < 4) and leaves the byte 0 or
+// 2^(s mod 4 + 4); the query side is a fixed-point vector (|v| <= 4000, about 12 bits) whose
+// entries carry the factor 2^(3 - s mod 4), so every product is 128 * bit * v. Each entry
+// is split into two int8 columns (hi, lo) of the same MMA, so accumulation is exact.
 //
-// Kernel 1 (prologue, a few (sequence, kv-head) streams per CTA): q', q'' for every query
-// head, fixed-point fragments in MMA order, per-head scales, exact logits of the tail.
+// Kernel 1 (prologue, 8 query heads per CTA): q', q'' for every query head, fixed-point
+// fragments in MMA order, per-head scales, exact logits of the tail.
 // Kernel 2 (stream, persistent): each warp walks a list of (stream, block range) tasks and
 // keeps a ring of 32-key blocks in shared memory filled by bulk copies (TMA engine,
 // mbarrier completion), prefetching across task boundaries.
@@ -35,7 +37,7 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
     return ((((size_t)stream * ntiles + ntile) * nmg + mg) * 4 + c) * 64 + lane * 2 + h;
 }
 
-// Prologue. Grid (ceil(heads / 8), 1 + ceil(n_tail / 32)); each CTA owns 8 consecutive query
+// Prologue. Grid (ceil(heads / 8), 1 + ceil(n_tail / 8)); each CTA owns 8 consecutive query
 // heads (rows s*g + h of q).
 //   y = 0: 1. q' = Pi q and q'' = S q as one [8 x d] x [d x (D + Mp)] product against
 //             (Pi^T | S^T). Thread (row half, head quad, column quad) keeps 4 heads x 4 columns
@@ -44,9 +46,11 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
 //          2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
 //          3. one thread per fragment word: it rounds its four coordinates, packs their hi and
 //             lo bytes into two words and stores them; warp sums give the per-head constants.
-//   y > 0: exact logits of 32 tail tokens for the 8 heads, one warp per token.
+//   y > 0: exact logits of 8 tail tokens for the 8 heads, one warp per token.
 constexpr int kPH = 8;         // heads per prologue CTA
-constexpr int kTailTok = 32;   // tail tokens per tail CTA
+// matrix rows per bulk-copied chunk: 32 KB stages at most
+__host__ __device__ constexpr int prologue_rows(int W) { return W <= 256 ? 32 : 16; }
+constexpr int kTailTok = 8;    // tail tokens per tail CTA (one per warp)
 
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
     // the kernel that consumes the fragments may launch now; it waits for this grid's
@@ -61,30 +65,28 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
 
     if (blockIdx.y > 0) {
-        // exact logits of the full-precision tail: scale <q, k>
+        // exact logits of the full-precision tail, scale <q, k>: warp w takes token
+        // 8 (y - 1) + w and the key rows of the CTA's streams (one for g >= 8, up to 8 for g = 1)
         float* qh = sm;   // [8][d]
         for (int e = tid; e < kPH * d; e += blockDim.x) {
             const int h = e / d, j = e - h * d;
             qh[e] = h < H ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
         }
         __syncthreads();
+        const int tt = (blockIdx.y - 1) * kTailTok + wid;
+        if (tt >= p.n_tail) return;
         const int64_t row = p.n_tok + p.n_tail;
-        for (int tk = wid; tk < kTailTok; tk += kPrologueThreads / 32) {
-            const int tt = (blockIdx.y - 1) * kTailTok + tk;
-            if (tt >= p.n_tail) break;
-            int64_t cur = -1;
+        const int s0 = h_base / G, s1 = (h_base + H - 1) / G;
+        for (int st = s0; st <= s1; ++st) {
+            const uint16_t* kp = p.tail + ((size_t)st * p.n_tail + tt) * d;
             float kv[8];   // coordinates lane + 32 i of the key (d <= 256)
-            for (int h = 0; h < H; ++h) {
-                const int64_t gh = h_base + h, stream = gh / G;
-                if (stream != cur) {
-                    cur = stream;
-                    const uint16_t* kp = p.tail + ((size_t)stream * p.n_tail + tt) * d;
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const int j = lane + 32 * i;
-                        kv[i] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
-                    }
-                }
+            for (int i = 0; i < 8; ++i) {
+                const int j = lane + 32 * i;
+                kv[i] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
+            }
+            const int h0 = max(st * G - h_base, 0), h1 = min((st + 1) * G - h_base, H);
+            for (int h = h0; h < h1; ++h) {
                 float a = 0.f;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -92,7 +94,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                     if (j < d) a = fmaf(kv[i], qh[h * d + j], a);
                 }
                 a = tq_warp_sum(a);
-                if (lane == 0) p.out[gh * row + p.n_tok + tt] = p.scale * a;
+                if (lane == 0) p.out[(int64_t)(h_base + h) * row + p.n_tok + tt] = p.scale * a;
             }
         }
         return;
@@ -102,7 +104,13 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     float* qo = qT + 256 * kPH;        // [8][W]: q' (0..D-1) then q'' (D..W-1)
     __shared__ float s_inv[2][kPH], s_step[2][kPH];
     __shared__ int s_sum[2][kPH];
+    __shared__ uint64_t s_bar[2];   // matrix chunk stages (two bulk copies each)
     const int nmg = T.nmg;
+    if (tid == 0) {
+        tq_mbar_init(&s_bar[0], 2);
+        tq_mbar_init(&s_bar[1], 2);
+        tq_fence_mbar_init();
+    }
     const int frag_words = p.ntiles * nmg * 256;
 
     // heads beyond g inside an n-tile keep zero fragments (only when g < 4)
@@ -119,20 +127,32 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     if (tid < 2 * kPH) s_sum[tid / kPH][tid % kPH] = 0;
     __syncthreads();
 
-    // 1. product. Thread -> ks (rows j of half ks), hq (heads 4hq .. 4hq + 3), cq (columns
-    //    4cq + 256r). Column c < D is row c of Pi (PiT[j][c]); c >= D is row c - D of S.
+    // 1. product. Rows of (Pi^T | S^T) arrive in chunks of R rows by bulk copies into two
+    //    shared-memory stages ([R][D] rows of Pi^T, then [R][Mp] rows of S^T). Thread -> ks
+    //    (half ks of a chunk's rows), hq (heads 4hq .. 4hq + 3), cq (columns 4cq + 256r).
     {
+        const int R = prologue_rows(W), nchunk = (d + R - 1) / R;
+        float* stg = qo + kPH * W;
+        auto load_chunk = [&](int c) {   // one thread
+            const int j0 = c * R, rows = min(R, d - j0);
+            float* dst = stg + (size_t)(c & 1) * R * W;
+            tq_bulk_load(dst, p.piT + (size_t)j0 * D, (uint32_t)(rows * D * 4), &s_bar[c & 1]);
+            tq_bulk_load(dst + R * D, p.sT + (size_t)j0 * Mp, (uint32_t)(rows * Mp * 4), &s_bar[c & 1]);
+        };
+        if (tid == 0) {
+            load_chunk(0);
+            if (nchunk > 1) load_chunk(1);
+        }
         const int ks = tid >> 7, hq = (tid >> 6) & 1, cq = tid & 63;
-        const float* bp[2];
-        int bs[2];
+        int off[2];
         bool bv[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int col = 256 * r + 4 * cq;
             bv[r] = col < W;
-            bp[r] = col < D ? p.piT + col : p.sT + (col - D);
-            bs[r] = col < D ? D : Mp;
+            off[r] = col < D ? col : R * D + (col - D);
         }
+        const int rs[2] = {D, Mp};
         float acc[2][4][4];
 #pragma unroll
         for (int r = 0; r < 2; ++r)
@@ -140,23 +160,47 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             for (int x = 0; x < 4; ++x)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) acc[r][x][y] = 0.f;
-        const int jh = (d + 1) >> 1, j0 = ks * jh, j1 = min(d, j0 + jh);
+        bool ok = true;
+        int c = 0;
+        for (; c < nchunk; ++c) {
+            ok = __syncthreads_and(ok && tq_mbar_wait(&s_bar[c & 1], (uint32_t)(c >> 1) & 1u, kWaitLimit));
+            if (!ok) break;
+            const int j0 = c * R, rows = min(R, d - j0), half = (rows + 1) >> 1;
+            const int jj0 = ks * half, jj1 = min(rows, jj0 + half);
+            const float* st = stg + (size_t)(c & 1) * R * W;
 #pragma unroll 4
-        for (int j = j0; j < j1; ++j) {
-            const float4 a = *reinterpret_cast<const float4*>(qT + j * kPH + 4 * hq);
-            const float av[4] = {a.x, a.y, a.z, a.w};
+            for (int jj = jj0; jj < jj1; ++jj) {
+                const float4 a = *reinterpret_cast<const float4*>(qT + (j0 + jj) * kPH + 4 * hq);
+                const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                if (!bv[r]) continue;
-                const float4 b = __ldg(reinterpret_cast<const float4*>(bp[r] + (size_t)j * bs[r]));
+                for (int r = 0; r < 2; ++r) {
+                    if (!bv[r]) continue;
+                    const int colr = 256 * r + 4 * cq;
+                    const float4 b = *reinterpret_cast<const float4*>(st + off[r] + jj * (colr < D ? rs[0] : rs[1]));
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    acc[r][x][0] = fmaf(av[x], b.x, acc[r][x][0]);
-                    acc[r][x][1] = fmaf(av[x], b.y, acc[r][x][1]);
-                    acc[r][x][2] = fmaf(av[x], b.z, acc[r][x][2]);
-                    acc[r][x][3] = fmaf(av[x], b.w, acc[r][x][3]);
+                    for (int x = 0; x < 4; ++x) {
+                        acc[r][x][0] = fmaf(av[x], b.x, acc[r][x][0]);
+                        acc[r][x][1] = fmaf(av[x], b.y, acc[r][x][1]);
+                        acc[r][x][2] = fmaf(av[x], b.z, acc[r][x][2]);
+                        acc[r][x][3] = fmaf(av[x], b.w, acc[r][x][3]);
+                    }
                 }
             }
+            __syncthreads();   // stage c & 1 is consumed
+            if (tid == 0 && c + 2 < nchunk) {
+                tq_fence_proxy_async();
+                load_chunk(c + 2);
+            }
+        }
+        if (!ok) {
+            // a copy did not land in time: record it, give the copies in flight a bounded
+            // time, and leave the fragments unwritten
+            if (tid == 0) {
+                tq_raise(p.status, TQ_FLAG_TIMEOUT);
+                for (int k = c; k < min(c + 2, nchunk); ++k)
+                    tq_mbar_wait(&s_bar[k & 1], (uint32_t)(k >> 1) & 1u, kWaitLimit);
+            }
+            return;
         }
         // the second row half parks its sums in qo; the first adds its own
         if (ks == 1) {
@@ -194,8 +238,8 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         ma = tq_warp_max(ma) * amax;
         ms = tq_warp_max(ms);
         if (lane == 0) {
-            s_step[0][h] = ma > 0.f ? ma / 32000.f : 1.f;
-            s_step[1][h] = ms > 0.f ? ms / 32000.f : 1.f;
+            s_step[0][h] = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
+            s_step[1][h] = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
             s_inv[0][h] = 1.f / s_step[0][h];
             s_inv[1][h] = 1.f / s_step[1][h];
         }
@@ -216,11 +260,13 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             const float inv = coef * s_inv[is_code ? 0 : 1][h];
             const float* src = qo + h * W + (is_code ? 0 : D) + 128 * gr + 32 * t + 2 * c + hh;
             uint32_t whi = 0, wlo = 0;
+            // bit s = 2c + hh of the key bytes meets this register: factor 2^(3 - s mod 4)
+            const int f = 8 >> ((2 * c + hh) & 3);
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
                 const int v = __float2int_rn(src[8 * bb] * inv);
                 sum += v;
-                const int hi = (v + 128) >> 8, lo = v - 256 * hi;
+                const int vf = v * f, hi = (vf + 128) >> 8, lo = vf - 256 * hi;
                 whi |= (uint32_t)(hi & 0xff) << (8 * bb);
                 wlo |= (uint32_t)(lo & 0xff) << (8 * bb);
             }
@@ -277,7 +323,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     constexpr int NPG = B * GD + GM;       // stored plane groups
     constexpr int NMG = NP * GD + GM;      // MMA plane groups
     constexpr uint32_t BB = 512u * NPG + 128u;
-    // exact int32 combination of the hi/lo columns while 128 * 32000 * K < 2^31
+    // exact int32 combination of the hi/lo columns while 128 * 8 kTqQueryMax * K < 2^31
     constexpr bool kIntComb = NP * GD <= 4 && GM <= 4;
     extern __shared__ __align__(128) uint8_t ring[];
     __shared__ uint64_t bars[kStreamWarps][NS];
@@ -454,11 +500,12 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 }  // namespace
 
 size_t tq_logits_prologue_smem(const TqDims& t, int) {
-    return ((size_t)256 * kPH + (size_t)kPH * (t.D + t.Mp)) * 4;
+    const int W = t.D + t.Mp;
+    return ((size_t)256 * kPH + (size_t)kPH * W + (size_t)2 * prologue_rows(W) * W) * 4;
 }
 
 // largest prologue shared memory over the supported codecs (D = Mp = 256)
-constexpr size_t kPrologueMaxSmem = ((size_t)256 * kPH + (size_t)kPH * 512) * 4;
+constexpr size_t kPrologueMaxSmem = ((size_t)256 * kPH + (size_t)kPH * 512 + (size_t)2 * 16 * 512) * 4;
 
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     const size_t smem = tq_logits_prologue_smem(p.t, 0);

@@ -96,9 +96,12 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int r = 0; r < 4; ++r) acc[k][n][r] = 0.f;
-    float m_run[HP], lsum[HP];   // m_run is the same in every lane; lsum holds the lane's tokens
+    // m_run (the same in every lane) and ml2 = m_run log2(e); lsum holds the lane's tokens
+    float m_run[HP], ml2[HP], lsum[HP];
 #pragma unroll
-    for (int h = 0; h < HP; ++h) { m_run[h] = -INFINITY; lsum[h] = 0.f; }
+    for (int h = 0; h < HP; ++h) { m_run[h] = -INFINITY; ml2[h] = -INFINITY; lsum[h] = 0.f; }
+    constexpr float kLog2e = 1.4426950408889634f;
+    const uint32_t lane4 = (uint32_t)lane * 4u;
 
     bool ok = true;
     int k = 0;
@@ -113,21 +116,25 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
         const bool in = tok < p.n_tok;
         const float nrm = tq_half_val(reinterpret_cast<const uint16_t*>(bp + SEC_A)[lane]);
         // online maximum and weights of this lane's token, one head at a time
-        float fac[HP];
+        float myf[NT];   // rescale factor of this thread's accumulator head 4n + t
+#pragma unroll
+        for (int n = 0; n < NT; ++n) myf[n] = 1.f;
         bool grew = false;
 #pragma unroll
         for (int h = 0; h < HP; ++h) {
-            fac[h] = 1.f;
             if (h < G) {
                 const float pv = in ? my_p[(s * HP + h) * 32 + lane] : -INFINITY;
-                const float bm = tq_warp_max(pv);
-                if (bm > m_run[h]) {
-                    fac[h] = __expf(m_run[h] - bm);   // 0 while the running maximum is -inf
+                if (__any_sync(0xffffffffu, pv > m_run[h])) {
+                    const float bm = tq_warp_max(pv);
+                    const float fac = tq_exp2((m_run[h] - bm) * kLog2e);   // 0 while the maximum was -inf
+                    if ((h & 3) == t) myf[h >> 2] = fac;
+                    lsum[h] *= fac;
                     m_run[h] = bm;
+                    ml2[h] = bm * kLog2e;
                     grew = true;
                 }
-                const float ex = m_run[h] > -INFINITY ? __expf(pv - m_run[h]) : 0.f;
-                lsum[h] = fmaf(lsum[h], fac[h], ex);
+                const float ex = m_run[h] > -INFINITY ? tq_exp2(fmaf(pv, kLog2e, -ml2[h])) : 0.f;
+                lsum[h] += ex;
                 const float wt = ex * nrm;
                 const __half hi = __float2half_rn(wt);
                 reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = hi;
@@ -137,13 +144,11 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
         if (grew) {
             // accumulator columns 2t, 2t + 1 of n-tile n belong to head 4n + t
 #pragma unroll
-            for (int n = 0; n < NT; ++n) {
-                const float f = t == 0 ? fac[4 * n] : t == 1 ? fac[4 * n + 1] : t == 2 ? fac[4 * n + 2] : fac[4 * n + 3];
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) acc[kk][n][r] *= f;
-            }
+                    for (int r = 0; r < 4; ++r) acc[kk][n][r] *= myf[n];
         }
         __syncwarp();
         // B fragments: column g of n-tile n (head 4n + g/2, hi or lo), tokens 16c + 8hv + 2t, +1
@@ -173,9 +178,11 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
                     const int f = 4 * (2 * kk + (r & 1)) + 2 * c + (r >> 1);
                     const int bit = f * 2 * B;
                     const int wi = bit >> 5, sh = bit & 31;
-                    uint32_t fld = sh == 0 ? W[wi] : __funnelshift_r(W[wi], W[wi + 1], sh);
-                    fld &= (uint32_t)(E - 1);
-                    a[r] = lut[fld * 32 + lane];
+                    // the field lands at bits 7.., i.e. already times the 128-byte entry stride
+                    // (fields start below bit 7 only when they lie inside one word)
+                    const uint32_t x = sh >= 7 ? __funnelshift_r(W[wi], W[wi + 1], sh - 7) : W[wi] << (7 - sh);
+                    const uint32_t off = (x & ((uint32_t)(E - 1) << 7)) | lane4;
+                    a[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(lut) + off);
                 }
 #pragma unroll
                 for (int n = 0; n < NT; ++n) tq_hmma(acc[kk][n], a[0], a[1], a[2], a[3], bw[n][c][0], bw[n][c][1]);
@@ -200,18 +207,19 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
 #pragma unroll
         for (int h = 0; h < HP; ++h) s_m[w][h] = m_run[h];
     __syncthreads();
-    float scl[HP];
+    float scl[HP], mys[NT];
 #pragma unroll
     for (int h = 0; h < HP; ++h) {
         float M = s_m[0][h];
 #pragma unroll
         for (int v = 1; v < kPvWarps; ++v) M = fmaxf(M, s_m[v][h]);
         scl[h] = m_run[h] > -INFINITY ? __expf(m_run[h] - M) : 0.f;
+        if ((h & 3) == t) mys[h >> 2] = scl[h];
     }
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int head = n * 4 + t;
-        const float f = t == 0 ? scl[4 * n] : t == 1 ? scl[4 * n + 1] : t == 2 ? scl[4 * n + 2] : scl[4 * n + 3];
+        const float f = mys[n];
         if (head < G) {
 #pragma unroll
             for (int kk = 0; kk < KT; ++kk) {

@@ -310,8 +310,8 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.blocks_per_task = 1;
     p.n_tasks = 0;
     p.n_heads_valid = n_streams * g;
-    // the tail runs on a second grid dimension of 32-token CTAs (at most 65535)
-    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 32 * 65534)
+    // the tail runs on a second grid dimension of 8-token CTAs (at most 65535)
+    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 8 * 65534)
         return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;

@@ -86,6 +86,13 @@ inline cudaError_t tq_launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, 
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error about 2^-22)
+TQ_DEVICE float tq_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // warp-wide reductions
 TQ_DEVICE float tq_warp_sum(float v) {
 #pragma unroll
@@ -104,35 +111,24 @@ TQ_DEVICE float tq_warp_max(float v) {
 }
 
 // int8 tensor-core MMA, 16x8x32, s32 accumulate (legacy warp-level path): A u8, B s8
-// x + x as an integer add. On sm_100 a 32-bit add issues at the full rate, while shifts,
-// IMAD and LOP3 issue at half of it, so the byte-bit moves below are built from adds.
-TQ_DEVICE uint32_t tq_dbl(uint32_t x) {
-    uint32_t y;
-    asm("add.u32 %0, %1, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
+// Bit planes to u8 MMA operands. Bit s of every byte of a packed word is one coordinate.
+// Masking it in place leaves the byte 0 or 2^s; bits 4..7 are masked in the word itself and
+// bits 0..3 in the word shifted left by 4, where they sit at 4..7. The weight 2^(s mod 4 + 4)
+// this leaves on the A byte is compensated on the query side, whose fixed-point values carry
+// the factor 2^(3 - s mod 4) (at most 8 x kTqQueryMax, inside the int16 hi/lo range), so
+// every product is 128 * bit * query value. For the words w0 (row g) and w1 (row g + 8) of
+// one k-chunk this yields, for c = 3 .. 0, a0, a1 <- bit 2c and a2, a3 <- bit 2c + 1, the A
+// fragment of chunk c; f(c, a0, a1, a2, a3) consumes it. One shift and one mask per register
+// pair of the old shift-then-mask form is saved.
+constexpr int kTqQueryMax = 4000;   // |query fixed-point value| before the 2^(3 - s mod 4) factor
 
-// Bit planes to u8 MMA operands. Bit s of every byte of a packed word is one coordinate;
-// a left shift by 7 - s moves it to bit 7, and the mask leaves the byte 0 or 128. For the
-// words w0 (row g) and w1 (row g + 8) of one k-chunk this yields, for c = 3 .. 0,
-//   a0, a1 <- bit 2c and a2, a3 <- bit 2c + 1,
-// the A fragment of chunk c; f(c, a0, a1, a2, a3) consumes it. Shifts 0 .. 7 are reached by
-// doubling, one add per step.
 template <typename F>
 TQ_DEVICE void tq_expand_planes(uint32_t w0, uint32_t w1, F&& f) {
-    uint32_t x0 = w0, x1 = w1;
-#pragma unroll
-    for (int c = 3; c >= 0; --c) {
-        const uint32_t a2 = x0 & 0x80808080u, a3 = x1 & 0x80808080u;   // shift 6 - 2c: bit 2c + 1
-        x0 = tq_dbl(x0);
-        x1 = tq_dbl(x1);
-        const uint32_t a0 = x0 & 0x80808080u, a1 = x1 & 0x80808080u;   // shift 7 - 2c: bit 2c
-        if (c > 0) {
-            x0 = tq_dbl(x0);
-            x1 = tq_dbl(x1);
-        }
-        f(c, a0, a1, a2, a3);
-    }
+    const uint32_t u0 = w0 << 4, u1 = w1 << 4;
+    f(3, w0 & 0x40404040u, w1 & 0x40404040u, w0 & 0x80808080u, w1 & 0x80808080u);
+    f(2, w0 & 0x10101010u, w1 & 0x10101010u, w0 & 0x20202020u, w1 & 0x20202020u);
+    f(1, u0 & 0x40404040u, u1 & 0x40404040u, u0 & 0x80808080u, u1 & 0x80808080u);
+    f(0, u0 & 0x10101010u, u1 & 0x10101010u, u0 & 0x20202020u, u1 & 0x20202020u);
 }
 
 TQ_DEVICE void tq_imma_u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
