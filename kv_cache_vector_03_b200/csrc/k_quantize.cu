@@ -593,7 +593,8 @@ cudaError_t launch_mma(const QuantParams& p, cudaStream_t st) {
 }
 
 cudaError_t tq_launch_quantize(const QuantParams& p, cudaStream_t st) {
-    if (p.t.D == 128 && (p.t.Mp == 128 || !p.t.qjl)) {
+    if (p.t.D == 128 && (p.t.Mp == 128 || !p.t.qjl)) return tq_launch_quantize_tc(p, st);
+    if (false) {
         const bool f32 = p.dtype == 0;
         switch (p.t.B) {
             case 1: return f32 ? launch_mma<true, 1>(p, st) : launch_mma<false, 1>(p, st);

@@ -1,0 +1,432 @@
+// tq_quantize for d <= 128 on the fifth-generation tensor cores (tcgen05.mma with TMEM
+// accumulators): rotate, nearest Lloyd-Max centroid, residual, QJL sign sketch, pack
+// (blog.hotdry.top "TurboQuant vector-search compression", sections "Random rotation and
+// scalar quantization" and "QJL residual correction"; a2a-mcp.org "What is TurboQuant",
+// stage 1).
+//
+// One persistent CTA of 8 warps per SM walks tiles of 128 vectors (4 blocks of 32).
+//   A. Each warp loads 16 rows (the next tile's rows are fetched into registers while the
+//      current tile is in the tensor cores), forms |x|, scales each row by a power of two
+//      and writes it as fp16 hi (and lo for fp32 input) into the A operand, laid out in
+//      shared memory in the canonical K-major 128-byte-swizzled form.
+//   B. One thread issues Y = X (256 Pi)^T as 128 x 128 x 16 MMAs over the split operands
+//      (X_hi Pi_hi + X_hi Pi_lo [+ X_lo Pi_hi]); fp32 accumulation in TMEM columns 0..127.
+//   C. Thread (warp, lane) owns TMEM lane 32 (warp % 4) + lane = one vector and half of its
+//      columns: y, idx = #{k : y > t_k}, r = y - c[idx], gamma^2, code-plane words; the
+//      residual goes back into the A operand as fp16 hi and lo (scaled by 2^12).
+//   D. Z = R (256 M)^T with M = S Pi^T (three split passes) into TMEM columns 128..255; the
+//      sign bits are z >= 0. Planes, norms and gamma are stored in the key block format.
+// Values (qjl = 0) stop after C: the codes go through shared memory into the value block's
+// two-token fields.
+#include "tq_device.cuh"
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr uint32_t kMat = 32768;             // one 128 x 128 fp16 operand
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kTmemCols = 256;
+
+// Byte offset of 16-byte chunk kc (8 fp16 of columns 8kc..8kc+7) of row r in a 128 x 128
+// fp16 operand: two K-blocks of 64 columns, each [128 rows][128 B] in atoms of 8 rows
+// (1024 B), the chunk index XOR (row mod 8) (128-byte swizzle). Operands start 1024-aligned.
+__device__ __forceinline__ uint32_t sw128(int r, int kc) {
+    return (uint32_t)((kc >> 3) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + (((kc & 7) ^ (r & 7)) << 4));
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B, fp32 D, both K-major, M = 128, N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t ad, uint64_t bd, uint32_t accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n}\n" ::"r"(tmem_d),
+        "l"(ad), "l"(bd), "r"(accumulate), "r"(kIdesc));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     tq_smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
+}
+
+// hi / lo fp16 pairs of four values
+__device__ __forceinline__ void split4(const float (&a)[4], uint2& h, uint2& l) {
+    h = make_uint2(pack_half2(a[0], a[1]), pack_half2(a[2], a[3]));
+    const __half2 h0 = *reinterpret_cast<const __half2*>(&h.x), h1 = *reinterpret_cast<const __half2*>(&h.y);
+    l = make_uint2(pack_half2(a[0] - __low2float(h0), a[1] - __high2float(h0)),
+                   pack_half2(a[2] - __low2float(h1), a[3] - __high2float(h1)));
+}
+
+template <bool kF32>
+struct RowRegs;
+template <>
+struct RowRegs<false> { uint2 v[16]; };   // 4 bf16 per lane and row
+template <>
+struct RowRegs<true> { float4 v[16]; };   // 4 fp32 per lane and row
+
+template <bool kF32, int B>
+__global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
+    constexpr int L = 1 << B;
+    extern __shared__ uint8_t qraw[];
+    __shared__ float s_inv[128], s_norm[128], s_g2[2][128], s_cent[16];
+    __shared__ int s_bad[128], s_valid[128];
+    __shared__ uint64_t s_bar;
+    __shared__ uint32_t s_tmem;
+
+    const TqDims& T = p.t;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = T.d;
+    const bool qjl = T.qjl != 0;
+    const int64_t total_blocks = p.n_streams * p.nb;
+    const int64_t n_tiles = (total_blocks + 3) / 4;
+
+    // operand area, 1024-byte aligned: Pi_hi Pi_lo [M_hi M_lo] X_hi X_lo [codes]
+    const uint32_t raw = tq_smem_addr(qraw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* sm = qraw + pad;
+    const uint32_t sb = raw + pad;
+    const uint32_t oXH = qjl ? 4 * kMat : 2 * kMat, oXL = oXH + kMat, oCS = oXL + kMat;
+
+    {   // resident B operands: rows = output coordinate (N), columns = K
+        const int nmat = qjl ? 4 : 2;
+        const uint16_t* srcs[4] = {p.pih, p.pil, p.mh, p.ml};
+        for (int e = tid; e < nmat * 128 * 16; e += kThreads) {
+            const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
+            const uint4 v = *reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8);
+            *reinterpret_cast<uint4*>(sm + m * kMat + sw128(row, ch)) = v;
+        }
+    }
+    if (tid < L) s_cent[tid] = p.cb.cent[tid];
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tq_smem_addr(&s_tmem)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    if (tid == 0) {
+        tq_mbar_init(&s_bar, 1);
+        tq_fence_mbar_init();
+    }
+    tq_fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    uint32_t n_commit = 0;
+
+    // rows 16 warp .. 16 warp + 15 of a tile lie in one block
+    auto load_rows = [&](int64_t tile, RowRegs<kF32>& rg) {
+        const int64_t gb = tile * 4 + (warp >> 1);
+        const int64_t s = gb / p.nb, tok0 = (gb % p.nb) * 32 + 16 * (warp & 1);
+        const bool blk = gb < total_blocks;
+        const int64_t base0 = s * p.x_stride + tok0 * d + 4 * lane;
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            const bool in = blk && tok0 + rr < p.n_tok && 4 * lane < d;
+            const int64_t base = base0 + (int64_t)rr * d;
+            if constexpr (kF32) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (in) {
+                    const float* xp = static_cast<const float*>(p.x) + base;
+                    if (p.vec_ok) v = __ldg(reinterpret_cast<const float4*>(xp));
+                    else v = make_float4(xp[0], xp[1], xp[2], xp[3]);
+                }
+                rg.v[rr] = v;
+            } else {
+                uint2 v = make_uint2(0u, 0u);
+                if (in) {
+                    const uint16_t* xp = static_cast<const uint16_t*>(p.x) + base;
+                    if (p.vec_ok) v = __ldg(reinterpret_cast<const uint2*>(xp));
+                    else v = make_uint2((uint32_t)xp[0] | ((uint32_t)xp[1] << 16), (uint32_t)xp[2] | ((uint32_t)xp[3] << 16));
+                }
+                rg.v[rr] = v;
+            }
+        }
+    };
+
+    RowRegs<kF32> rg;
+    if ((int64_t)blockIdx.x < n_tiles) load_rows(blockIdx.x, rg);
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
+        // ---- A. rows -> norms, power-of-two scale, fp16 A operand
+        {
+            const int64_t gb = tile * 4 + (warp >> 1);
+            const int64_t tok0 = (gb % p.nb) * 32 + 16 * (warp & 1);
+            const bool blk = gb < total_blocks;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int row = 16 * warp + rr;
+                float x[4];
+                if constexpr (kF32) {
+                    x[0] = rg.v[rr].x; x[1] = rg.v[rr].y; x[2] = rg.v[rr].z; x[3] = rg.v[rr].w;
+                } else {
+                    x[0] = __uint_as_float(rg.v[rr].x << 16); x[1] = __uint_as_float(rg.v[rr].x & 0xffff0000u);
+                    x[2] = __uint_as_float(rg.v[rr].y << 16); x[3] = __uint_as_float(rg.v[rr].y & 0xffff0000u);
+                }
+                float ss = 0.f, mx = 0.f;
+                int bad = 0;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    ss = fmaf(x[k], x[k], ss);
+                    mx = fmaxf(mx, fabsf(x[k]));
+                    bad |= !isfinite(x[k]);
+                }
+                ss = tq_warp_sum(ss);
+                mx = tq_warp_max(mx);
+                bad = __any_sync(0xffffffffu, bad);
+                // 2^ex with max * 2^ex in [2^14, 2^15), from the exponent field of the max
+                int ex = 0;
+                if (mx > 0.f && isfinite(mx)) ex = min(max(14 - (((__float_as_int(mx) >> 23) & 0xff) - 127), -126), 126);
+                const float sc2 = __int_as_float((127 + ex) << 23);
+                float a[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) a[k] = x[k] * sc2;
+                uint2 h, l;
+                split4(a, h, l);
+                const uint32_t off = sw128(row, lane >> 1) + (lane & 1) * 8;
+                *reinterpret_cast<uint2*>(sm + oXH + off) = h;
+                if (kF32) *reinterpret_cast<uint2*>(sm + oXL + off) = l;
+                if (lane == 0) {
+                    const bool valid = blk && tok0 + rr < p.n_tok;
+                    const float n = sqrtf(ss);
+                    s_norm[row] = valid ? n : 0.f;
+                    s_inv[row] = n > 0.f ? 1.f / (n * 256.f * sc2) : 0.f;
+                    s_bad[row] = valid && bad;
+                    s_valid[row] = valid;
+                }
+            }
+        }
+        // the next tile's rows stream in while this one is in the tensor cores
+        if (tile + gridDim.x < n_tiles) load_rows(tile + gridDim.x, rg);
+
+        // ---- B. Y = X Pi^T (scaled), TMEM columns 0..127
+        tq_fence_proxy_async();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr int np = kF32 ? 3 : 2;
+#pragma unroll
+            for (int ps = 0; ps < np; ++ps) {
+                const uint32_t oa = ps == 2 ? oXL : oXH, ob = ps == 1 ? kMat : 0u;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const uint32_t ko = (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u;
+                    umma_f16(tmem, umma_desc(sb + oa + ko), umma_desc(sb + ob + ko), (ps | k) != 0);
+                }
+            }
+            umma_commit(&s_bar);
+        }
+        ok = __syncthreads_and(tq_mbar_wait(&s_bar, n_commit & 1u, kWaitLimit));
+        ++n_commit;
+        if (!ok) break;
+        tc_fence_after();
+
+        // ---- C. codes, residual, gamma; thread -> vector row r, columns 64 hc .. 64 hc + 63
+        const int r = 32 * (warp & 3) + lane, hc = warp >> 2;
+        const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+        const float inv = s_inv[r];
+        const bool rvalid = s_valid[r] != 0;
+        const int64_t gb = tile * 4 + (r >> 5);
+        const int vb = r & 31, u = vb >> 3, gq = vb & 7;
+        uint8_t* blk = p.packed + (size_t)gb * T.block_bytes;
+        uint32_t cw[B][2];
+#pragma unroll
+        for (int pl = 0; pl < B; ++pl) cw[pl][0] = cw[pl][1] = 0u;
+        float g2 = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float y[16];
+            tmem_ld16(tl + 64 * hc + 16 * q, y);
+            float rv[16];
+            uint32_t cb4[4] = {0u, 0u, 0u, 0u};   // codes as bytes (values)
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int i = 64 * hc + 16 * q + e;
+                const float yy = y[e] * inv;
+                int c = 0;
+#pragma unroll
+                for (int k = 0; k < L - 1; ++k) c += yy > p.cb.bounds[k];
+                float rr = yy - s_cent[c];
+                if (i >= d || !rvalid) { c = 0; rr = 0.f; }
+                g2 = fmaf(rr, rr, g2);
+                rv[e] = rr * 4096.f;
+#pragma unroll
+                for (int pl = 0; pl < B; ++pl) cw[pl][(16 * q + e) >> 5] |= (uint32_t)((c >> pl) & 1) << ((16 * q + e) & 31);
+                cb4[e >> 2] |= (uint32_t)c << (8 * (e & 3));
+            }
+            if (qjl) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint2 h0, l0, h1, l1;
+                    const float a0[4] = {rv[8 * hh], rv[8 * hh + 1], rv[8 * hh + 2], rv[8 * hh + 3]};
+                    const float a1[4] = {rv[8 * hh + 4], rv[8 * hh + 5], rv[8 * hh + 6], rv[8 * hh + 7]};
+                    split4(a0, h0, l0);
+                    split4(a1, h1, l1);
+                    const uint32_t off = sw128(r, 8 * hc + 2 * q + hh);
+                    *reinterpret_cast<uint4*>(sm + oXH + off) = make_uint4(h0.x, h0.y, h1.x, h1.y);
+                    *reinterpret_cast<uint4*>(sm + oXL + off) = make_uint4(l0.x, l0.y, l1.x, l1.y);
+                }
+            } else {
+                *reinterpret_cast<uint4*>(sm + oCS + r * 128 + 64 * hc + 16 * q) = make_uint4(cb4[0], cb4[1], cb4[2], cb4[3]);
+            }
+        }
+        s_g2[hc][r] = g2;
+        if (qjl && gb < total_blocks) {
+            // word w (coordinates 32w .. 32w + 31) of plane pl of vector 8u + gq
+#pragma unroll
+            for (int pl = 0; pl < B; ++pl)
+#pragma unroll
+                for (int w2 = 0; w2 < 2; ++w2)
+                    reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + 2 * hc + w2) * 4 + u] = cw[pl][w2];
+        }
+
+        if (qjl) {
+            // ---- D. Z = R M^T (scaled), TMEM columns 128..255; signs, norms
+            tq_fence_proxy_async();
+            tc_fence_before();
+            __syncthreads();
+            if (tid == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ps = 0; ps < 3; ++ps) {
+                    const uint32_t oa = ps == 2 ? oXL : oXH, ob = ps == 1 ? 3 * kMat : 2 * kMat;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t ko = (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u;
+                        umma_f16(tmem + 128, umma_desc(sb + oa + ko), umma_desc(sb + ob + ko), (ps | k) != 0);
+                    }
+                }
+                umma_commit(&s_bar);
+            }
+            ok = __syncthreads_and(tq_mbar_wait(&s_bar, n_commit & 1u, kWaitLimit));
+            ++n_commit;
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sw[2] = {0u, 0u};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float z[16];
+                tmem_ld16(tl + 128 + 64 * hc + 16 * q, z);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int j = 64 * hc + 16 * q + e;
+                    const bool bit = rvalid && j < T.m && z[e] >= 0.f;
+                    sw[(16 * q + e) >> 5] |= (uint32_t)bit << ((16 * q + e) & 31);
+                }
+            }
+            if (gb < total_blocks) {
+#pragma unroll
+                for (int w2 = 0; w2 < 2; ++w2)
+                    reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + 2 * hc + w2) * 4 + u] = sw[w2];
+                if (hc == 0) {
+                    const uint32_t nh = rvalid ? tq_half_bits(s_norm[r]) : 0u;
+                    const uint32_t gh = rvalid ? tq_half_bits(sqrtf(s_g2[0][r] + s_g2[1][r])) : 0u;
+                    if (rvalid && (s_bad[r] || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
+                    reinterpret_cast<uint32_t*>(blk + T.sec_a)[gq * 4 + u] = nh | (gh << 16);
+                }
+            }
+        } else {
+            // value layout: norms, then each lane string of the tile's blocks from the codes
+            __syncthreads();
+            if (tid < 128) {
+                const int row = tid;
+                const int64_t gbr = tile * 4 + (row >> 5);
+                if (gbr < total_blocks) {
+                    const uint32_t nh = s_valid[row] ? tq_half_bits(s_norm[row]) : 0u;
+                    if (s_valid[row] && (s_bad[row] || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
+                    reinterpret_cast<uint16_t*>(p.packed + (size_t)gbr * T.block_bytes + T.sec_a)[row & 31] = (uint16_t)nh;
+                }
+            }
+            const uint8_t* CS = sm + oCS;
+            constexpr int fb = 2 * B, words = 128 * B / 32;
+            for (int e = tid; e < 4 * 32 * words; e += kThreads) {
+                const int bl = e / (32 * words), rem = e % (32 * words);
+                const int64_t gbw = tile * 4 + bl;
+                if (gbw >= total_blocks) continue;
+                const int ln = rem % 32, wd = rem / 32;
+                const int gq2 = ln >> 2, tq = ln & 3;
+                uint32_t val = 0;
+                const int f0 = (32 * wd) / fb, f1 = (32 * wd + 31) / fb;
+                for (int f = f0; f <= f1; ++f) {
+                    const int a = f >> 2, pp = f & 3;
+                    const int i = 8 * a + gq2;
+                    const int tau = 16 * (pp >> 1) + 8 * (pp & 1) + 2 * tq;
+                    const uint8_t* crow = CS + (bl * 32) * 128;
+                    const uint32_t F = (uint32_t)crow[tau * 128 + i] | ((uint32_t)crow[(tau + 1) * 128 + i] << B);
+                    const int pos = f * fb - 32 * wd;
+                    val |= pos >= 0 ? (F << pos) : (F >> (-pos));
+                }
+                reinterpret_cast<uint32_t*>(p.packed + (size_t)gbw * T.block_bytes)[((wd >> 2) * 32 + ln) * 4 + (wd & 3)] = val;
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
+    if (!ok) {
+        // an MMA did not complete in time: record it and give it a bounded time to finish
+        if (tid == 0) {
+            tq_raise(p.status, TQ_FLAG_TIMEOUT);
+            tq_mbar_wait(&s_bar, (n_commit - 1) & 1u, kWaitLimit);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols));
+    }
+}
+
+template <bool kF32, int B>
+cudaError_t launch_tc(const QuantParams& p, cudaStream_t st) {
+    const size_t smem = (size_t)(p.t.qjl ? 6 : 5) * kMat + 1024;
+    auto kern = k_quantize_tc<kF32, B>;
+    static TqLaunchCache cache;
+    int sms = 0;
+    cudaError_t e = tq_kernel_setup(kern, kThreads, (size_t)6 * kMat + 1024, cache, &sms, nullptr);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (p.n_streams * p.nb + 3) / 4;
+    const int64_t grid = std::min<int64_t>(tiles, sms);
+    if (grid > 0) kern<<<(unsigned)grid, kThreads, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// d <= 128 with m <= 128 (or no sketch)
+cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st) {
+    const bool f32 = p.dtype == 0;
+    switch (p.t.B) {
+        case 1: return f32 ? launch_tc<true, 1>(p, st) : launch_tc<false, 1>(p, st);
+        case 2: return f32 ? launch_tc<true, 2>(p, st) : launch_tc<false, 2>(p, st);
+        case 3: return f32 ? launch_tc<true, 3>(p, st) : launch_tc<false, 3>(p, st);
+        case 4: return f32 ? launch_tc<true, 4>(p, st) : launch_tc<false, 4>(p, st);
+    }
+    return cudaErrorInvalidValue;
+}

@@ -308,4 +308,5 @@ cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st);
 cudaError_t tq_launch_dequant(const DequantParams& p, cudaStream_t st);
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
+cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
