@@ -4,16 +4,17 @@
 // scalar quantization" and "QJL residual correction"; a2a-mcp.org "What is TurboQuant",
 // stage 1).
 //
-// One persistent CTA of 8 warps per SM walks tiles of 128 vectors (4 blocks of 32).
-//   A. Each warp loads 16 rows (the next tile's rows are fetched into registers while the
-//      current tile is in the tensor cores), forms |x|, scales each row by a power of two
-//      and writes it as fp16 hi (and lo for fp32 input) into the A operand, laid out in
-//      shared memory in the canonical K-major 128-byte-swizzled form.
+// One persistent CTA of 16 warps per SM walks tiles of 128 vectors (4 blocks of 32).
+//   A. Each warp loads 8 rows (the next tile's rows are fetched into registers while the
+//      current tile is in the tensor cores), forms |x| by a transposed warp reduction, scales
+//      each row by a power of two and writes it as fp16 hi (and lo for fp32 input) into the
+//      A operand, laid out in shared memory in the canonical K-major 128-byte-swizzled form.
 //   B. One thread issues Y = X (256 Pi)^T as 128 x 128 x 16 MMAs over the split operands
 //      (X_hi Pi_hi + X_hi Pi_lo [+ X_lo Pi_hi]); fp32 accumulation in TMEM columns 0..127.
-//   C. Thread (warp, lane) owns TMEM lane 32 (warp % 4) + lane = one vector and half of its
-//      columns: y, idx = #{k : y > t_k}, r = y - c[idx], gamma^2, code-plane words; the
-//      residual goes back into the A operand as fp16 hi and lo (scaled by 2^12).
+//   C. Thread (warp, lane) owns TMEM lane 32 (warp % 4) + lane = one vector and a quarter of
+//      its columns (32 coordinates = one word of each plane): y, idx = #{k : y > t_k},
+//      r = y - c[idx], gamma^2, code-plane words; the residual goes back into the A operand
+//      as fp16 hi and lo (scaled by 2^12).
 //   D. Z = R (256 M)^T with M = S Pi^T (three split passes) into TMEM columns 128..255; the
 //      sign bits are z >= 0. Planes, norms and gamma are stored in the key block format.
 // Values (qjl = 0) stop after C: the codes go through shared memory into the value block's
@@ -22,7 +23,7 @@
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr uint32_t kMat = 32768;             // one 128 x 128 fp16 operand
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr uint32_t kTmemCols = 256;
@@ -82,18 +83,23 @@ __device__ __forceinline__ void split4(const float (&a)[4], uint2& h, uint2& l) 
                    pack_half2(a[2] - __low2float(h1), a[3] - __high2float(h1)));
 }
 
+constexpr int kRowsPerWarp = 8;   // 16 warps x 8 rows = one 128-vector tile
+
 template <bool kF32>
 struct RowRegs;
 template <>
-struct RowRegs<false> { uint2 v[16]; };   // 4 bf16 per lane and row
+struct RowRegs<false> { uint2 v[kRowsPerWarp]; };   // 4 bf16 per lane and row
 template <>
-struct RowRegs<true> { float4 v[16]; };   // 4 fp32 per lane and row
+struct RowRegs<true> { float4 v[kRowsPerWarp]; };   // 4 fp32 per lane and row
 
-template <bool kF32, int B>
+// bits e < n of a 32-bit word, n clamped to [0, 32]
+__device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? ~0u : n <= 0 ? 0u : (1u << n) - 1u; }
+
+template <bool kF32, int B, bool QJL>
 __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
     constexpr int L = 1 << B;
     extern __shared__ uint8_t qraw[];
-    __shared__ float s_inv[128], s_norm[128], s_g2[2][128], s_cent[16];
+    __shared__ float s_inv[128], s_norm[128], s_sc[128], s_g2[4][128], s_cent[16];
     __shared__ int s_bad[128], s_valid[128];
     __shared__ uint64_t s_bar;
     __shared__ uint32_t s_tmem;
@@ -101,7 +107,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
     const TqDims& T = p.t;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d = T.d;
-    const bool qjl = T.qjl != 0;
     const int64_t total_blocks = p.n_streams * p.nb;
     const int64_t n_tiles = (total_blocks + 3) / 4;
 
@@ -110,14 +115,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* sm = qraw + pad;
     const uint32_t sb = raw + pad;
-    const uint32_t oXH = qjl ? 4 * kMat : 2 * kMat, oXL = oXH + kMat, oCS = oXL + kMat;
+    constexpr uint32_t oXH = QJL ? 4 * kMat : 2 * kMat, oXL = oXH + kMat, oCS = oXL + kMat;
 
     {   // resident B operands: rows = output coordinate (N), columns = K
-        const int nmat = qjl ? 4 : 2;
-        const uint16_t* srcs[4] = {p.pih, p.pil, p.mh, p.ml};
+        constexpr int nmat = QJL ? 4 : 2;
         for (int e = tid; e < nmat * 128 * 16; e += kThreads) {
             const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
-            const uint4 v = *reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8);
+            const uint16_t* src = m == 0 ? p.pih : m == 1 ? p.pil : m == 2 ? p.mh : p.ml;
+            const uint4 v = *reinterpret_cast<const uint4*>(src + row * 128 + ch * 8);
             *reinterpret_cast<uint4*>(sm + m * kMat + sw128(row, ch)) = v;
         }
     }
@@ -137,15 +142,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
     tc_fence_after();
     const uint32_t tmem = s_tmem;
     uint32_t n_commit = 0;
+    // coordinates >= d read y = 0 (zero rows of Pi): their residual -c[idx(0)] is taken
+    // back out of gamma^2 below
+    float c0 = 0.f;
+    {
+        int i0 = 0;
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) i0 += 0.f > p.cb.bounds[k];
+        c0 = s_cent[i0];
+    }
 
-    // rows 16 warp .. 16 warp + 15 of a tile lie in one block
+    // rows 8 warp .. 8 warp + 7 of a tile lie in one block
     auto load_rows = [&](int64_t tile, RowRegs<kF32>& rg) {
-        const int64_t gb = tile * 4 + (warp >> 1);
-        const int64_t s = gb / p.nb, tok0 = (gb % p.nb) * 32 + 16 * (warp & 1);
+        const int64_t gb = tile * 4 + (warp >> 2);
+        const int64_t s = gb / p.nb, tok0 = (gb % p.nb) * 32 + kRowsPerWarp * (warp & 3);
         const bool blk = gb < total_blocks;
         const int64_t base0 = s * p.x_stride + tok0 * d + 4 * lane;
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
+        for (int rr = 0; rr < kRowsPerWarp; ++rr) {
             const bool in = blk && tok0 + rr < p.n_tok && 4 * lane < d;
             const int64_t base = base0 + (int64_t)rr * d;
             if constexpr (kF32) {
@@ -167,57 +181,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
             }
         }
     };
+    // one thread waits for the MMAs; the others wait at the barrier
+    auto mma_done = [&]() -> bool {
+        bool w = true;
+        if (tid == 0) w = tq_mbar_wait(&s_bar, n_commit & 1u, kWaitLimit);
+        ++n_commit;
+        return __syncthreads_and(w) != 0;
+    };
 
     RowRegs<kF32> rg;
     if ((int64_t)blockIdx.x < n_tiles) load_rows(blockIdx.x, rg);
     bool ok = true;
     for (int64_t tile = blockIdx.x; tile < n_tiles; tile += gridDim.x) {
-        // ---- A. rows -> norms, power-of-two scale, fp16 A operand
+        // ---- A. rows -> norms (transposed warp reduction), power-of-two scale, fp16 A operand
         {
-            const int64_t gb = tile * 4 + (warp >> 1);
-            const int64_t tok0 = (gb % p.nb) * 32 + 16 * (warp & 1);
-            const bool blk = gb < total_blocks;
+            float x[kRowsPerWarp][4], v[kRowsPerWarp];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                const int row = 16 * warp + rr;
-                float x[4];
+            for (int rr = 0; rr < kRowsPerWarp; ++rr) {
                 if constexpr (kF32) {
-                    x[0] = rg.v[rr].x; x[1] = rg.v[rr].y; x[2] = rg.v[rr].z; x[3] = rg.v[rr].w;
+                    x[rr][0] = rg.v[rr].x; x[rr][1] = rg.v[rr].y; x[rr][2] = rg.v[rr].z; x[rr][3] = rg.v[rr].w;
                 } else {
-                    x[0] = __uint_as_float(rg.v[rr].x << 16); x[1] = __uint_as_float(rg.v[rr].x & 0xffff0000u);
-                    x[2] = __uint_as_float(rg.v[rr].y << 16); x[3] = __uint_as_float(rg.v[rr].y & 0xffff0000u);
+                    x[rr][0] = __uint_as_float(rg.v[rr].x << 16); x[rr][1] = __uint_as_float(rg.v[rr].x & 0xffff0000u);
+                    x[rr][2] = __uint_as_float(rg.v[rr].y << 16); x[rr][3] = __uint_as_float(rg.v[rr].y & 0xffff0000u);
                 }
-                float ss = 0.f, mx = 0.f;
-                int bad = 0;
+                v[rr] = fmaf(x[rr][0], x[rr][0], fmaf(x[rr][1], x[rr][1], fmaf(x[rr][2], x[rr][2], x[rr][3] * x[rr][3])));
+            }
+            // after the xor-16, -8, -4 exchanges lane l holds row (l >> 2) & 7 summed over 8 lanes
+            float a4[4], a2[2], a1;
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    ss = fmaf(x[k], x[k], ss);
-                    mx = fmaxf(mx, fabsf(x[k]));
-                    bad |= !isfinite(x[k]);
-                }
-                ss = tq_warp_sum(ss);
-                mx = tq_warp_max(mx);
-                bad = __any_sync(0xffffffffu, bad);
-                // 2^ex with max * 2^ex in [2^14, 2^15), from the exponent field of the max
+            for (int k = 0; k < 4; ++k) {
+                const bool hi = lane & 16;
+                a4[k] = (hi ? v[k + 4] : v[k]) + __shfl_xor_sync(0xffffffffu, hi ? v[k] : v[k + 4], 16);
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const bool hi = lane & 8;
+                a2[k] = (hi ? a4[k + 2] : a4[k]) + __shfl_xor_sync(0xffffffffu, hi ? a4[k] : a4[k + 2], 8);
+            }
+            {
+                const bool hi = lane & 4;
+                a1 = (hi ? a2[1] : a2[0]) + __shfl_xor_sync(0xffffffffu, hi ? a2[0] : a2[1], 4);
+            }
+            a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+            a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+            const int64_t gb = tile * 4 + (warp >> 2);
+            const int64_t tok0 = (gb % p.nb) * 32 + kRowsPerWarp * (warp & 3);
+            if ((lane & 3) == 0) {
+                const int rr = (lane >> 2) & 7, row = kRowsPerWarp * warp + rr;
+                const bool valid = gb < total_blocks && tok0 + rr < p.n_tok;
+                const float n = sqrtf(a1);
+                // 2^ex with |x| 2^ex in [2^14, 2^15): every element then fits binary16
                 int ex = 0;
-                if (mx > 0.f && isfinite(mx)) ex = min(max(14 - (((__float_as_int(mx) >> 23) & 0xff) - 127), -126), 126);
+                if (n > 0.f && isfinite(n)) ex = min(max(14 - (((__float_as_int(n) >> 23) & 0xff) - 127), -126), 126);
                 const float sc2 = __int_as_float((127 + ex) << 23);
+                s_sc[row] = sc2;
+                s_norm[row] = valid ? n : 0.f;
+                s_inv[row] = n > 0.f ? 1.f / (n * 256.f * sc2) : 0.f;
+                s_bad[row] = valid && !isfinite(n);
+                s_valid[row] = valid;
+            }
+            __syncwarp();
+#pragma unroll
+            for (int rr = 0; rr < kRowsPerWarp; ++rr) {
+                const int row = kRowsPerWarp * warp + rr;
+                const float sc2 = s_sc[row];
                 float a[4];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) a[k] = x[k] * sc2;
+                for (int k = 0; k < 4; ++k) a[k] = x[rr][k] * sc2;
                 uint2 h, l;
                 split4(a, h, l);
                 const uint32_t off = sw128(row, lane >> 1) + (lane & 1) * 8;
                 *reinterpret_cast<uint2*>(sm + oXH + off) = h;
                 if (kF32) *reinterpret_cast<uint2*>(sm + oXL + off) = l;
-                if (lane == 0) {
-                    const bool valid = blk && tok0 + rr < p.n_tok;
-                    const float n = sqrtf(ss);
-                    s_norm[row] = valid ? n : 0.f;
-                    s_inv[row] = n > 0.f ? 1.f / (n * 256.f * sc2) : 0.f;
-                    s_bad[row] = valid && bad;
-                    s_valid[row] = valid;
-                }
             }
         }
         // the next tile's rows stream in while this one is in the tensor cores
@@ -241,45 +276,45 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
             }
             umma_commit(&s_bar);
         }
-        ok = __syncthreads_and(tq_mbar_wait(&s_bar, n_commit & 1u, kWaitLimit));
-        ++n_commit;
+        ok = mma_done();
         if (!ok) break;
         tc_fence_after();
 
-        // ---- C. codes, residual, gamma; thread -> vector row r, columns 64 hc .. 64 hc + 63
-        const int r = 32 * (warp & 3) + lane, hc = warp >> 2;
+        // ---- C. codes, residual, gamma; thread -> vector row r, columns 32 qc .. 32 qc + 31
+        const int r = 32 * (warp & 3) + lane, qc = warp >> 2;
         const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
         const float inv = s_inv[r];
         const bool rvalid = s_valid[r] != 0;
         const int64_t gb = tile * 4 + (r >> 5);
         const int vb = r & 31, u = vb >> 3, gq = vb & 7;
         uint8_t* blk = p.packed + (size_t)gb * T.block_bytes;
-        uint32_t cw[B][2];
+        uint32_t cw[B];
 #pragma unroll
-        for (int pl = 0; pl < B; ++pl) cw[pl][0] = cw[pl][1] = 0u;
+        for (int pl = 0; pl < B; ++pl) cw[pl] = 0u;
         float g2 = 0.f;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             float y[16];
-            tmem_ld16(tl + 64 * hc + 16 * q, y);
+            tmem_ld16(tl + 32 * qc + 16 * q, y);
             float rv[16];
-            uint32_t cb4[4] = {0u, 0u, 0u, 0u};   // codes as bytes (values)
+            uint32_t cb4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-                const int i = 64 * hc + 16 * q + e;
                 const float yy = y[e] * inv;
                 int c = 0;
 #pragma unroll
                 for (int k = 0; k < L - 1; ++k) c += yy > p.cb.bounds[k];
-                float rr = yy - s_cent[c];
-                if (i >= d || !rvalid) { c = 0; rr = 0.f; }
+                const float rr = yy - s_cent[c];
                 g2 = fmaf(rr, rr, g2);
-                rv[e] = rr * 4096.f;
+                if (QJL) {
+                    rv[e] = rr * 4096.f;
 #pragma unroll
-                for (int pl = 0; pl < B; ++pl) cw[pl][(16 * q + e) >> 5] |= (uint32_t)((c >> pl) & 1) << ((16 * q + e) & 31);
-                cb4[e >> 2] |= (uint32_t)c << (8 * (e & 3));
+                    for (int pl = 0; pl < B; ++pl) cw[pl] |= (uint32_t)((c >> pl) & 1) << (16 * q + e);
+                } else {
+                    cb4[e >> 2] |= (uint32_t)c << (8 * (e & 3));
+                }
             }
-            if (qjl) {
+            if (QJL) {
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint2 h0, l0, h1, l1;
@@ -287,25 +322,25 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
                     const float a1[4] = {rv[8 * hh + 4], rv[8 * hh + 5], rv[8 * hh + 6], rv[8 * hh + 7]};
                     split4(a0, h0, l0);
                     split4(a1, h1, l1);
-                    const uint32_t off = sw128(r, 8 * hc + 2 * q + hh);
+                    const uint32_t off = sw128(r, 4 * qc + 2 * q + hh);
                     *reinterpret_cast<uint4*>(sm + oXH + off) = make_uint4(h0.x, h0.y, h1.x, h1.y);
                     *reinterpret_cast<uint4*>(sm + oXL + off) = make_uint4(l0.x, l0.y, l1.x, l1.y);
                 }
             } else {
-                *reinterpret_cast<uint4*>(sm + oCS + r * 128 + 64 * hc + 16 * q) = make_uint4(cb4[0], cb4[1], cb4[2], cb4[3]);
+                *reinterpret_cast<uint4*>(sm + oCS + r * 128 + 32 * qc + 16 * q) = make_uint4(cb4[0], cb4[1], cb4[2], cb4[3]);
             }
         }
-        s_g2[hc][r] = g2;
-        if (qjl && gb < total_blocks) {
-            // word w (coordinates 32w .. 32w + 31) of plane pl of vector 8u + gq
+        // coordinates >= d: codes 0, residual out of gamma^2
+        const int nfake = min(32, max(0, 32 * qc + 32 - d));
+        s_g2[qc][r] = g2 - (float)nfake * c0 * c0;
+        if (QJL && gb < total_blocks) {
+            const uint32_t keep = rvalid ? low_bits(d - 32 * qc) : 0u;
 #pragma unroll
             for (int pl = 0; pl < B; ++pl)
-#pragma unroll
-                for (int w2 = 0; w2 < 2; ++w2)
-                    reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + 2 * hc + w2) * 4 + u] = cw[pl][w2];
+                reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + qc) * 4 + u] = cw[pl] & keep;
         }
 
-        if (qjl) {
+        if constexpr (QJL) {
             // ---- D. Z = R M^T (scaled), TMEM columns 128..255; signs, norms
             tq_fence_proxy_async();
             tc_fence_before();
@@ -323,29 +358,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
                 }
                 umma_commit(&s_bar);
             }
-            ok = __syncthreads_and(tq_mbar_wait(&s_bar, n_commit & 1u, kWaitLimit));
-            ++n_commit;
+            ok = mma_done();
             if (!ok) break;
             tc_fence_after();
-            uint32_t sw[2] = {0u, 0u};
+            uint32_t sw = 0u;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 float z[16];
-                tmem_ld16(tl + 128 + 64 * hc + 16 * q, z);
+                tmem_ld16(tl + 128 + 32 * qc + 16 * q, z);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int j = 64 * hc + 16 * q + e;
-                    const bool bit = rvalid && j < T.m && z[e] >= 0.f;
-                    sw[(16 * q + e) >> 5] |= (uint32_t)bit << ((16 * q + e) & 31);
-                }
+                for (int e = 0; e < 16; ++e) sw |= (uint32_t)(z[e] >= 0.f) << (16 * q + e);
             }
             if (gb < total_blocks) {
-#pragma unroll
-                for (int w2 = 0; w2 < 2; ++w2)
-                    reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + 2 * hc + w2) * 4 + u] = sw[w2];
-                if (hc == 0) {
+                reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + qc) * 4 + u] =
+                    rvalid ? sw & low_bits(T.m - 32 * qc) : 0u;
+                if (qc == 0) {
                     const uint32_t nh = rvalid ? tq_half_bits(s_norm[r]) : 0u;
-                    const uint32_t gh = rvalid ? tq_half_bits(sqrtf(s_g2[0][r] + s_g2[1][r])) : 0u;
+                    const float gam = sqrtf(fmaxf(s_g2[0][r] + s_g2[1][r] + s_g2[2][r] + s_g2[3][r], 0.f));
+                    const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
                     if (rvalid && (s_bad[r] || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
                     reinterpret_cast<uint32_t*>(blk + T.sec_a)[gq * 4 + u] = nh | (gh << 16);
                 }
@@ -377,7 +407,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
                     const int i = 8 * a + gq2;
                     const int tau = 16 * (pp >> 1) + 8 * (pp & 1) + 2 * tq;
                     const uint8_t* crow = CS + (bl * 32) * 128;
-                    const uint32_t F = (uint32_t)crow[tau * 128 + i] | ((uint32_t)crow[(tau + 1) * 128 + i] << B);
+                    uint32_t F = 0;
+                    if (i < d && s_valid[bl * 32 + tau]) F |= (uint32_t)crow[tau * 128 + i];
+                    if (i < d && s_valid[bl * 32 + tau + 1]) F |= (uint32_t)crow[(tau + 1) * 128 + i] << B;
                     const int pos = f * fb - 32 * wd;
                     val |= pos >= 0 ? (F << pos) : (F >> (-pos));
                 }
@@ -403,13 +435,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
     }
 }
 
-template <bool kF32, int B>
+template <bool kF32, int B, bool QJL>
 cudaError_t launch_tc(const QuantParams& p, cudaStream_t st) {
-    const size_t smem = (size_t)(p.t.qjl ? 6 : 5) * kMat + 1024;
-    auto kern = k_quantize_tc<kF32, B>;
+    const size_t smem = (size_t)(QJL ? 6 : 5) * kMat + 1024;
+    auto kern = k_quantize_tc<kF32, B, QJL>;
     static TqLaunchCache cache;
     int sms = 0;
-    cudaError_t e = tq_kernel_setup(kern, kThreads, (size_t)6 * kMat + 1024, cache, &sms, nullptr);
+    cudaError_t e = tq_kernel_setup(kern, kThreads, smem, cache, &sms, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t tiles = (p.n_streams * p.nb + 3) / 4;
     const int64_t grid = std::min<int64_t>(tiles, sms);
@@ -417,16 +449,22 @@ cudaError_t launch_tc(const QuantParams& p, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+template <bool kF32, bool QJL>
+cudaError_t launch_b(const QuantParams& p, cudaStream_t st) {
+    switch (p.t.B) {
+        case 1: return launch_tc<kF32, 1, QJL>(p, st);
+        case 2: return launch_tc<kF32, 2, QJL>(p, st);
+        case 3: return launch_tc<kF32, 3, QJL>(p, st);
+        case 4: if constexpr (!QJL) return launch_tc<kF32, 4, QJL>(p, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 // d <= 128 with m <= 128 (or no sketch)
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st) {
     const bool f32 = p.dtype == 0;
-    switch (p.t.B) {
-        case 1: return f32 ? launch_tc<true, 1>(p, st) : launch_tc<false, 1>(p, st);
-        case 2: return f32 ? launch_tc<true, 2>(p, st) : launch_tc<false, 2>(p, st);
-        case 3: return f32 ? launch_tc<true, 3>(p, st) : launch_tc<false, 3>(p, st);
-        case 4: return f32 ? launch_tc<true, 4>(p, st) : launch_tc<false, 4>(p, st);
-    }
-    return cudaErrorInvalidValue;
+    if (p.t.qjl) return f32 ? launch_b<true, true>(p, st) : launch_b<false, true>(p, st);
+    return f32 ? launch_b<true, false>(p, st) : launch_b<false, false>(p, st);
 }
