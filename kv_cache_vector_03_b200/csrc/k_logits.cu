@@ -292,26 +292,24 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     }
 }
 
-// Walks a warp's tasks: task k = first + k * step over (stream, chunk) pairs, chunk in
-// [0, tpt); no divisions after the first (step = step_s * tpt + step_c).
-struct TaskWalk {
-    int stream, chunk, blk, b1;
-    __device__ void open(const LogitsParams& p) {
-        blk = chunk * p.blocks_per_task;
-        b1 = min(blk + p.blocks_per_task, (int)p.nb);
+// Walks a warp's contiguous range of the flattened (stream, block) index: every warp gets
+// the same number of blocks (+-1) and changes stream (reloading its query fragments) at most
+// a few times; no divisions after the first.
+struct FlatWalk {
+    int64_t left;   // blocks still to visit
+    int stream, blk;
+    __device__ void init(const LogitsParams& p, int64_t b0, int64_t b1) {
+        left = b1 - b0;
+        stream = (int)(b0 / p.nb);
+        blk = (int)(b0 - (int64_t)stream * p.nb);
     }
-    __device__ void init(const LogitsParams& p, int first) {
-        stream = first / p.tpt;
-        chunk = first - stream * p.tpt;
-        if (valid(p)) open(p);
-    }
-    __device__ bool valid(const LogitsParams& p) const { return stream < p.n_streams32; }
+    __device__ bool valid() const { return left > 0; }
     __device__ void advance(const LogitsParams& p) {
-        if (++blk < b1) return;
-        chunk += p.step_c;
-        stream += p.step_s;
-        if (chunk >= p.tpt) { chunk -= p.tpt; ++stream; }
-        if (valid(p)) open(p);
+        --left;
+        if (++blk == (int)p.nb) {
+            blk = 0;
+            ++stream;
+        }
     }
 };
 
@@ -335,12 +333,13 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     tq_fence_mbar_init();
     __syncwarp();
 
-    const int first = blockIdx.x * kStreamWarps + warp;
-    TaskWalk prod, cons;
-    prod.init(p, first);
-    cons.init(p, first);
+    const int64_t n_blocks = p.n_seq * p.n_kv * p.nb, n_warps = (int64_t)gridDim.x * kStreamWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kStreamWarps + warp;
+    FlatWalk prod, cons;
+    prod.init(p, gw * n_blocks / n_warps, (gw + 1) * n_blocks / n_warps);
+    cons = prod;
     if (lane == 0) {
-        for (int s = 0; s < NS && prod.valid(p); ++s) {
+        for (int s = 0; s < NS && prod.valid(); ++s) {
             tq_bulk_load(my_ring + s * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB, &bars[warp][s]);
             prod.advance(p);
         }
@@ -357,7 +356,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     int cur_stream = -1;
     uint32_t seq = 0;
     bool ok = true;
-    while (cons.valid(p)) {
+    while (cons.valid()) {
         if (cons.stream != cur_stream) {
             cur_stream = cons.stream;
 #pragma unroll
@@ -443,7 +442,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
         }
         // the stage's data are consumed (all reads above fed the MMAs): refill it
         __syncwarp();
-        if (lane == 0 && prod.valid(p)) {
+        if (lane == 0 && prod.valid()) {
             tq_fence_proxy_async();
             tq_bulk_load(my_ring + stage * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB,
                          &bars[warp][stage]);
@@ -473,21 +472,10 @@ cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
     int sms = 0, per_sm = 0;
     cudaError_t e = tq_kernel_setup(kern, kStreamWarps * 32, smem, cache, &sms, &per_sm);
     if (e != cudaSuccess) return e;
-    // tasks of a few blocks each, about eight per resident warp, so that the static
-    // round-robin over tasks balances; copies run ahead across task boundaries
-    LogitsParams p = p0;
-    const int64_t n_streams = p.n_seq * p.n_kv;
-    const int64_t warps = (int64_t)per_sm * sms * kStreamWarps;
-    int64_t bpt = (n_streams * p.nb) / (warps * 8);
-    bpt = std::min<int64_t>(std::max<int64_t>(bpt, 1), 64);
-    p.blocks_per_task = (int)bpt;
-    p.tpt = (int)((p.nb + bpt - 1) / bpt);
-    p.n_tasks = n_streams * p.tpt;
-    p.n_streams32 = (int)n_streams;
-    const int64_t grid = std::min<int64_t>((p.n_tasks + kStreamWarps - 1) / kStreamWarps, (int64_t)per_sm * sms);
-    const int64_t step = grid * kStreamWarps;
-    p.step_s = (int)(step / p.tpt);
-    p.step_c = (int)(step % p.tpt);
+    // persistent: as many CTAs as fit, each warp a contiguous equal share of the blocks
+    const LogitsParams& p = p0;
+    const int64_t n_blocks = p.n_seq * p.n_kv * p.nb;
+    const int64_t grid = std::min<int64_t>((n_blocks + kStreamWarps - 1) / kStreamWarps, (int64_t)per_sm * sms);
     if (grid == 0) return cudaSuccess;
     return tq_launch_pdl(kern, dim3((unsigned)grid), dim3(kStreamWarps * 32), smem, st, p);
 }

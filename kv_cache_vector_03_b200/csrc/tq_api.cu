@@ -307,8 +307,6 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.scale = scale;
     p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.status = static_cast<uint32_t*>(ws);
-    p.blocks_per_task = 1;
-    p.n_tasks = 0;
     p.n_heads_valid = n_streams * g;
     // the tail runs on a second grid dimension of 8-token CTAs (at most 65535)
     if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 8 * 65534)

@@ -252,11 +252,9 @@ struct LogitsParams {
     uint32_t* qfrag;       // [stream][ntile][nmg][4][32][2]
     float* qscale;         // [stream][ntile*4][4]: dA/128, KA, 2dS/128, KS
     uint32_t* status;
-    int64_t n_seq, n_tok, nb, n_tasks;
+    int64_t n_seq, n_tok, nb;
     int n_kv, g, ntiles, n_tail;
     float scale, kappa;
-    int blocks_per_task;
-    int tpt, n_streams32, step_s, step_c;   // task walk: tasks per stream, stride in (stream, chunk)
     int64_t n_heads_valid;                   // query rows that exist (later heads read as zero)
     TqDims t;
     TqCodebookConsts cb;
