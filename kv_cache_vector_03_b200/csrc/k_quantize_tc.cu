@@ -71,16 +71,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-    return (uint32_t)__half_as_ushort(__float2half_rn(lo)) | ((uint32_t)__half_as_ushort(__float2half_rn(hi)) << 16);
-}
-
-// hi / lo fp16 pairs of four values
+// hi / lo fp16 pairs of four values (packed conversions: one instruction per pair)
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<const uint32_t*>(&h); }
 __device__ __forceinline__ void split4(const float (&a)[4], uint2& h, uint2& l) {
-    h = make_uint2(pack_half2(a[0], a[1]), pack_half2(a[2], a[3]));
-    const __half2 h0 = *reinterpret_cast<const __half2*>(&h.x), h1 = *reinterpret_cast<const __half2*>(&h.y);
-    l = make_uint2(pack_half2(a[0] - __low2float(h0), a[1] - __high2float(h0)),
-                   pack_half2(a[2] - __low2float(h1), a[3] - __high2float(h1)));
+    const __half2 h0 = __floats2half2_rn(a[0], a[1]), h1 = __floats2half2_rn(a[2], a[3]);
+    const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+    h = make_uint2(h2bits(h0), h2bits(h1));
+    l = make_uint2(h2bits(__floats2half2_rn(a[0] - f0.x, a[1] - f0.y)), h2bits(__floats2half2_rn(a[2] - f1.x, a[3] - f1.y)));
+}
+// hi only (values exactly representable, e.g. scaled bf16)
+__device__ __forceinline__ uint2 half4(const float (&a)[4]) {
+    return make_uint2(h2bits(__floats2half2_rn(a[0], a[1])), h2bits(__floats2half2_rn(a[2], a[3])));
 }
 
 constexpr int kRowsPerWarp = 8;   // 16 warps x 8 rows = one 128-vector tile
@@ -248,11 +249,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_quantize_tc(QuantParams p) {
                 float a[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) a[k] = x[rr][k] * sc2;
-                uint2 h, l;
-                split4(a, h, l);
                 const uint32_t off = sw128(row, lane >> 1) + (lane & 1) * 8;
-                *reinterpret_cast<uint2*>(sm + oXH + off) = h;
-                if (kF32) *reinterpret_cast<uint2*>(sm + oXL + off) = l;
+                if constexpr (kF32) {
+                    uint2 h, l;
+                    split4(a, h, l);
+                    *reinterpret_cast<uint2*>(sm + oXH + off) = h;
+                    *reinterpret_cast<uint2*>(sm + oXL + off) = l;
+                } else {
+                    // a scaled bf16 value is exact in binary16 (8 significant bits)
+                    *reinterpret_cast<uint2*>(sm + oXH + off) = half4(a);
+                }
             }
         }
         // the next tile's rows stream in while this one is in the tensor cores
