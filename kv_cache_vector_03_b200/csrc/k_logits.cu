@@ -286,9 +286,11 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     if (tid < H) {
         const int gh = h_base + tid, stream = gh / G, head = gh % G;
         const float dA = s_step[0][tid], dS = s_step[1][tid];
+        // the attention scale is folded in as well
+        const float sa = p.scale;
         reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
-            make_float4(dA / 128.f, 0.5f * dA * (float)s_sum[0][tid], p.kappa * 2.f * dS / 128.f,
-                        p.kappa * dS * (float)s_sum[1][tid]);
+            make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)s_sum[0][tid], sa * p.kappa * 2.f * dS / 128.f,
+                        sa * p.kappa * dS * (float)s_sum[1][tid]);
     }
 }
 
@@ -347,7 +349,6 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
 
     // the copies above read only keys; the query fragments come from the prologue
     tq_pdl_wait();
-    const float scale = p.scale;
     const int64_t row = p.n_tok + p.n_tail;
     uint32_t qf[NT][NMG][4][2];
     float4 sc[NT];
@@ -389,11 +390,8 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
 
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
-            int accA[NT][4], accS[NT][4];
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int r = 0; r < 4; ++r) { accA[n][r] = 0; accS[n][r] = 0; }
+            // code planes accumulate in two chains (chunks c odd / even), the sign plane in one
+            int accA[NT][4], accA2[NT][4], accS[NT][4];
 #pragma unroll
             for (int mg = 0; mg < NMG; ++mg) {
                 uint32_t w0, w1;  // words of rows g (u = 2mt) and g + 8 (u = 2mt + 1)
@@ -413,18 +411,29 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
                 tq_expand_planes(w0, w1, [&](int c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
 #pragma unroll
                     for (int n = 0; n < NT; ++n) {
-                        if (mg < NP * GD) tq_imma_u8(accA[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
-                        else tq_imma_u8(accS[n], a0, a1, a2, a3, qf[n][mg][c][0], qf[n][mg][c][1]);
+                        const uint32_t b0 = qf[n][mg][c][0], b1 = qf[n][mg][c][1];
+                        if (mg < NP * GD) {
+                            int(&acc)[4] = (c & 1) ? accA[n] : accA2[n];
+                            if (mg == 0 && c >= 2) tq_imma_u8_z(acc, a0, a1, a2, a3, b0, b1);   // first of its chain
+                            else tq_imma_u8(acc, a0, a1, a2, a3, b0, b1);
+                        } else {
+                            if (mg == NP * GD && c == 3) tq_imma_u8_z(accS[n], a0, a1, a2, a3, b0, b1);
+                            else tq_imma_u8(accS[n], a0, a1, a2, a3, b0, b1);
+                        }
                     }
                 });
             }
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int r = 0; r < 4; ++r) accA[n][r] += accA2[n][r];
             // epilogue: thread (g, t) -> head t of each n-tile, rows g and g + 8
             const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int u = 2 * mt + r;
                 const uint32_t nw = nrm[u];
-                const float nh = scale * tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
+                const float nh = tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
 #pragma unroll
                 for (int n = 0; n < NT; ++n) {
                     float va, vs;

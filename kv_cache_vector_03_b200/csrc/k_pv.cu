@@ -74,16 +74,21 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
     float* my_p = pring + (size_t)w * NS * HP * 32;
     const int64_t first = b0 + w;
     const int nmine = first < b1 ? (int)((b1 - first + kPvWarps - 1) / kPvWarps) : 0;
-    // block k of this warp (first + 4k) into stage k % NS; every lane commits one copy group
+    // block k of this warp (first + 4k) into stage k % NS; every lane commits one copy group.
+    // The lane's P pointer (head 0, token 32 (first + 4k) + lane) advances by 128 tokens a block.
+    const float* pk = Pst + first * 32 + lane;
+    const uint8_t* vk = sbase + (size_t)first * BBYTES;
     auto issue = [&](int k) {
         if (k < nmine) {
             const int s = k % NS;
-            const int64_t bi = first + (int64_t)kPvWarps * k;
-            if (lane == 0) tq_bulk_load(my_ring + s * BBYTES, sbase + (size_t)bi * BBYTES, BBYTES, &bars[w][s]);
-            const int64_t tok = bi * 32 + lane;
-            const bool in = tok < p.n_tok;
-            for (int h = 0; h < G; ++h)
-                tq_cp_async4(my_p + (s * HP + h) * 32 + lane, in ? Pst + (size_t)h * p.n_tok + tok : p.P, in ? 4u : 0u);
+            if (lane == 0) tq_bulk_load(my_ring + s * BBYTES, vk, BBYTES, &bars[w][s]);
+            const bool in = (first + (int64_t)kPvWarps * k) * 32 + lane < p.n_tok;
+            float* dst = my_p + s * HP * 32 + lane;
+#pragma unroll
+            for (int h = 0; h < HP; ++h)
+                if (h < G) tq_cp_async4(dst + h * 32, in ? pk + (size_t)h * p.n_tok : p.P, in ? 4u : 0u);
+            pk += 32 * kPvWarps;
+            vk += (size_t)kPvWarps * BBYTES;
         }
         tq_cp_async_commit();
     };
@@ -120,8 +125,10 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
 #pragma unroll
         for (int n = 0; n < NT; ++n) myf[n] = 1.f;
         bool grew = false;
+        float wt[HP];
 #pragma unroll
         for (int h = 0; h < HP; ++h) {
+            wt[h] = 0.f;
             if (h < G) {
                 const float pv = in ? my_p[(s * HP + h) * 32 + lane] : -INFINITY;
                 if (__any_sync(0xffffffffu, pv > m_run[h])) {
@@ -135,10 +142,22 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
                 }
                 const float ex = m_run[h] > -INFINITY ? tq_exp2(fmaf(pv, kLog2e, -ml2[h])) : 0.f;
                 lsum[h] += ex;
-                const float wt = ex * nrm;
-                const __half hi = __float2half_rn(wt);
-                reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = hi;
-                reinterpret_cast<__half*>(&wst[w][2 * h + 1][0])[lane] = __float2half_rn(wt - __half2float(hi));
+                wt[h] = ex * nrm;
+            }
+        }
+        // fp16 hi / lo of the weights, two heads per packed conversion
+#pragma unroll
+        for (int h = 0; h < HP; h += 2) {
+            if (h < G) {
+                const __half2 hi = __floats2half2_rn(wt[h], wt[h + 1]);
+                const float2 hf = __half22float2(hi);
+                const __half2 lo = __floats2half2_rn(wt[h] - hf.x, wt[h + 1] - hf.y);
+                reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = __low2half(hi);
+                reinterpret_cast<__half*>(&wst[w][2 * h + 1][0])[lane] = __low2half(lo);
+                if (h + 1 < G) {
+                    reinterpret_cast<__half*>(&wst[w][2 * h + 2][0])[lane] = __high2half(hi);
+                    reinterpret_cast<__half*>(&wst[w][2 * h + 3][0])[lane] = __high2half(lo);
+                }
             }
         }
         if (grew) {

@@ -140,6 +140,16 @@ TQ_DEVICE void tq_imma_u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, ui
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
+// the same MMA with a zero accumulator input (starts a chain without initialising registers)
+TQ_DEVICE void tq_imma_u8_z(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                            uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%10,%10,%10,%10};\n"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
+}
+
 // ---------------------------------------------------------------------- mbarrier + bulk copy
 // One-dimensional bulk copies global -> shared through the TMA engine, completion tracked
 // by a shared-memory mbarrier (transaction bytes). Waits are bounded: a wait that does not
