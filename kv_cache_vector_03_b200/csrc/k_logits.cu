@@ -52,6 +52,7 @@ constexpr int kPH = 8;         // heads per prologue CTA
 __host__ __device__ constexpr int prologue_rows(int W) { return W <= 256 ? 32 : 16; }
 constexpr int kTailTok = 8;    // tail tokens per tail CTA (one per warp)
 
+template <int NR>   // 256-column groups of (Pi^T | S^T): 1 for D + Mp <= 256, else 2
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
     // the kernel that consumes the fragments may launch now; it waits for this grid's
     // completion before it reads them
@@ -144,18 +145,18 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             if (nchunk > 1) load_chunk(1);
         }
         const int ks = tid >> 7, hq = (tid >> 6) & 1, cq = tid & 63;
-        int off[2];
-        bool bv[2];
+        int off[NR], rstr[NR];
+        bool bv[NR];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
+        for (int r = 0; r < NR; ++r) {
             const int col = 256 * r + 4 * cq;
             bv[r] = col < W;
             off[r] = col < D ? col : R * D + (col - D);
+            rstr[r] = col < D ? D : Mp;
         }
-        const int rs[2] = {D, Mp};
-        float acc[2][4][4];
+        float acc[NR][4][4];
 #pragma unroll
-        for (int r = 0; r < 2; ++r)
+        for (int r = 0; r < NR; ++r)
 #pragma unroll
             for (int x = 0; x < 4; ++x)
 #pragma unroll
@@ -173,10 +174,9 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                 const float4 a = *reinterpret_cast<const float4*>(qT + (j0 + jj) * kPH + 4 * hq);
                 const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    if (!bv[r]) continue;
-                    const int colr = 256 * r + 4 * cq;
-                    const float4 b = *reinterpret_cast<const float4*>(st + off[r] + jj * (colr < D ? rs[0] : rs[1]));
+                for (int r = 0; r < NR; ++r) {
+                    if (NR > 1 && !bv[r]) continue;
+                    const float4 b = *reinterpret_cast<const float4*>(st + off[r] + jj * rstr[r]);
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
                         acc[r][x][0] = fmaf(av[x], b.x, acc[r][x][0]);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         // the second row half parks its sums in qo; the first adds its own
         if (ks == 1) {
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+            for (int r = 0; r < NR; ++r)
                 if (bv[r])
 #pragma unroll
                     for (int x = 0; x < 4; ++x)
@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         __syncthreads();
         if (ks == 0) {
 #pragma unroll
-            for (int r = 0; r < 2; ++r)
+            for (int r = 0; r < NR; ++r)
                 if (bv[r])
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
@@ -506,12 +506,14 @@ constexpr size_t kPrologueMaxSmem = ((size_t)256 * kPH + (size_t)kPH * 512 + (si
 
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     const size_t smem = tq_logits_prologue_smem(p.t, 0);
-    static TqLaunchCache cache;
-    cudaError_t e = tq_kernel_setup(k_logits_prologue, kPrologueThreads, kPrologueMaxSmem, cache, nullptr, nullptr);
+    const bool wide = p.t.D + p.t.Mp > 256;
+    auto kern = wide ? k_logits_prologue<2> : k_logits_prologue<1>;
+    static TqLaunchCache cache1, cache2;
+    cudaError_t e = tq_kernel_setup(kern, kPrologueThreads, kPrologueMaxSmem, wide ? cache2 : cache1, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     const int64_t n_heads = p.n_seq * p.n_kv * p.g;
     const dim3 grid((unsigned)((n_heads + kPH - 1) / kPH), 1u + (unsigned)((p.n_tail + kTailTok - 1) / kTailTok));
-    k_logits_prologue<<<grid, kPrologueThreads, smem, st>>>(p);
+    kern<<<grid, kPrologueThreads, smem, st>>>(p);
     return cudaGetLastError();
 }
 
