@@ -79,40 +79,66 @@ def max_over_ranks(world, v):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs. Sampling
+    starts (first line received) before the caller's timed region; only samples stamped inside
+    [mark_start, mark_end] (plus one sampling period on each side) are summarised."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 50
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append((time.time(), ln))
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.PERIOD_MS)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        deadline = time.time() + 5.0
+        while not self.lines and time.time() < deadline:
+            time.sleep(0.01)
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+        # at least two periods of samples after the work ends
+        time.sleep(2 * self.PERIOD_MS / 1000.0)
+
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            self.reader.join(timeout=5)
 
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
+        pad = self.PERIOD_MS / 1000.0
+        for ts, ln in self.lines:
+            if self.t0 is not None and not (self.t0 - pad <= ts <= (self.t1 or ts) + pad):
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -201,11 +227,13 @@ def run_gpu(args, world, rank, local):
     with ClockSampler(local) as clk:
         barrier(world)
         torch.cuda.synchronize()
+        clk.mark_start()
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
         stop.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
         barrier(world)
     total_ms = start.elapsed_time(stop)
     t_quant = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
@@ -253,22 +281,25 @@ def run_gpu(args, world, rank, local):
     h2d = h_append.numel() * 2 + h_q.numel() * 2
     d2h = h_out.numel() * 4
 
+    # DRAM bytes (read + write) per launch of these kernels on this workload, from one ncu
+    # capture each (profiles/k_quantize_tc_c4_append.md, profiles/k_logits_stream_c4.md)
+    ncu_traffic = {"tq_quantize": 67.30e6 + 1.37e6, "tq_logits": 0.70e6 + 220.82e6 + 46.15e6}
     # kernels launched per step: quantize 1, logits 2 (prologue + stream)
     launches_per_step = 3
     dominant = "tq_logits" if t_logit >= t_quant else "tq_quantize"
     logits_roof = {"kernel": "tq_logits (prologue + int8-MMA stream)", "bound": "hbm", "achieved": round(logit_gbs, 1),
                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(logit_gbs / peaks["hbm_gbs"], 4),
-                   "traffic": None, "peak_kind": peak_kind,
+                   "traffic": ncu_traffic["tq_logits"], "peak_kind": peak_kind,
                    "algorithmic_bytes_per_launch": logit_bytes}
     # the d = 128 quantize runs its two contractions on fp16 tensor cores, split into hi/lo
     # passes for fp32-equivalent precision (2 passes for Pi x with bf16 input, 3 for M r):
     # measured against the bf16 (= fp16) dense peak, with and without the split passes
     tpeak = peaks["bf16_tflops"]
     passes = 2.5
-    quant_roof = {"kernel": "tq_quantize (fp16 tensor-core split, mma.sync)", "bound": "tensor",
+    quant_roof = {"kernel": "tq_quantize (fp16 tensor-core split, tcgen05.mma)", "bound": "tensor",
                   "achieved": round(quant_tf, 2), "peak": tpeak, "unit": "TFLOP/s",
                   "frac": round(quant_tf / tpeak, 4), "frac_with_split_passes": round(passes * quant_tf / tpeak, 4),
-                  "traffic": None, "algorithmic_flops_per_launch": quant_flops,
+                  "traffic": ncu_traffic["tq_quantize"], "algorithmic_flops_per_launch": quant_flops,
                   "peak_kind": peak_kind + " (bf16 burst)"}
     also = {} if args.no_extras else extra_workloads(torch, tq, ti, gen, peaks)
     line = {
@@ -311,6 +342,28 @@ def time_calls(torch, fn, n_iter, n_warm=3):
     return a.elapsed_time(b) / n_iter
 
 
+def time_graph(torch, fn, n_calls, n_replays=20):
+    """Mean device time per call of fn(0) .. fn(n_calls - 1) captured once in a CUDA graph and
+    replayed n_replays times (host launch overhead amortised, as in a captured decode loop)."""
+    for i in range(n_calls):   # first calls (one-time launch setup) outside the capture
+        fn(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(n_calls):
+            fn(i)
+    graph.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(n_replays):
+        graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del graph
+    return a.elapsed_time(b) / (n_replays * n_calls)
+
+
 def extra_workloads(torch, tq, ti, gen, peaks):
     """The other workloads of the hot path, each timed on its own (device time per call).
     Inputs that fit in L2 are rotated over enough copies to exceed it."""
@@ -334,13 +387,13 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         q = torch.randn((1, n_kv * 4, d), generator=gen, device="cuda").to(torch.bfloat16)
         lo = torch.empty((1, n_kv * 4, n_all), dtype=torch.float32, device="cuda")
         ws = tq.workspace(codec.workspace_bytes(tq.TQ_OP_LOGITS, 1, n_kv, 4))
-        ms = time_calls(torch, lambda i: tq.tq_logits(codec, packs[i % copies], 1, n_kv, n_tok, q, 4, tail, n_tail,
-                                                      1.0 / math.sqrt(d), lo, ws), 240)
+        ms = time_graph(torch, lambda i: tq.tq_logits(codec, packs[i % copies], 1, n_kv, n_tok, q, 4, tail, n_tail,
+                                                      1.0 / math.sqrt(d), lo, ws), copies)
         byts = n_kv * n_tok * codec.record_bytes() + n_kv * n_tail * d * 2 + lo.numel() * 4
         out[f"c2_llama8b_decode_logits_b{b}"] = {
             "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "l2": f"{copies} rotating copies of the packed cache"}
+            "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA-graph replays of 12 calls"}
         del keys, packs
     # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
     n_kv, n_tok, g = 8, 131072, 4
@@ -356,12 +409,12 @@ def extra_workloads(torch, tq, ti, gen, peaks):
             packs.append(pk)
         o = torch.empty((1, n_kv * g, d), dtype=torch.float32, device="cuda")
         ws = tq.workspace(codec.workspace_bytes(tq.TQ_OP_PV, n_kv, n_tok, g))
-        ms = time_calls(torch, lambda i: tq.tq_pv(codec, packs[i % copies], 1, n_kv, n_tok, P[i % 2], g, o, ws), 60)
+        ms = time_graph(torch, lambda i: tq.tq_pv(codec, packs[i % copies], 1, n_kv, n_tok, P[i % 2], g, o, ws), copies)
         byts = n_kv * n_tok * codec.record_bytes() + P[0].numel() * 4
         out[f"c3_values_128k_pv_{B}bit"] = {
             "ms": ms, "tokens_per_s": n_kv * n_tok / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "l2": f"{copies} rotating copies of the packed values, 2 of P"}
+            "l2": f"{copies} rotating copies of the packed values, 2 of P", "timing": "CUDA-graph replays of 4 calls"}
         del packs
     del vals, P
     # c5: vector search, 1M x d=200 database (anisotropic, unit rows), 10,000 queries, top-10
@@ -458,7 +511,7 @@ def run_reference(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")

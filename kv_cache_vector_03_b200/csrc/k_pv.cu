@@ -320,13 +320,13 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
     const int grp = tid / nq, qd = tid % nq;
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+    // every split wrote its partial (zeros where it saw no weight), so the loads need no guard
+    // and can all be in flight at once
+#pragma unroll 8
     for (int s = grp; s < ns; s += ngrp) {
         const float f = fs[s];
-        if (f != 0.f) {
-            const float4 v = src[(size_t)s * nq];
-            a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
-        }
+        const float4 v = src[(size_t)s * nq];
+        a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
     }
     reinterpret_cast<float4*>(red)[grp * nq + qd] = a;
     __syncthreads();
@@ -337,21 +337,26 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
         s_o[i] = v * inv;
     }
     __syncthreads();
-    // out[j] = sum_i Pi[i][j] o_i: thread (j = tid % 128 + 128 r, row half ih)
-    const int ih = tid >> 7, jl = tid & 127, half = (d + 1) >> 1;
-    const int i0 = ih * half, i1 = min(d, i0 + half);
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-        const int j = jl + 128 * r;
-        float o = 0.f;
-        if (j < d) {
+    // out[j] = sum_i Pi[i][j] o_i = <row j of Pi^T, o> (its columns i >= d are zero): pair
+    // (j, half), 16-byte loads of the row; the block-uniform trip count keeps warps whole for
+    // the shuffle that joins the halves (neighbouring lanes)
+    const int hl = D / 2;
+    for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
+        const int e = e0 + tid, j = e >> 1, hf = e & 1;
+        const bool valid = e < 2 * d;
+        float acc = 0.f;
+        if (valid) {
+            const float4* rowp = reinterpret_cast<const float4*>(p.piT + (size_t)j * D + hf * hl);
+            const float4* op = reinterpret_cast<const float4*>(s_o + hf * hl);
 #pragma unroll 16
-            for (int i = i0; i < i1; ++i) o = fmaf(__ldg(p.pi + (size_t)i * d + j), s_o[i], o);
+            for (int k = 0; k < hl / 4; ++k) {
+                const float4 w = __ldg(rowp + k), o = op[k];
+                acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
+            }
         }
-        red[ih * 256 + j] = o;
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (valid && hf == 0) p.out[(size_t)hq * d + j] = acc;
     }
-    __syncthreads();
-    for (int j = tid; j < d; j += kMergeThreads) p.out[(size_t)hq * d + j] = red[j] + red[256 + j];
 }
 
 template <int B, int KT, int NT>

@@ -332,7 +332,8 @@ int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int6
     if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
     PvParams p;
     p.packed = static_cast<const uint8_t*>(packed_v);
-    p.P = P; p.out = out; p.pi = c->pi;
+    p.P = P; p.out = out;
+    p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + tq_prep_layout(t).piT);
     p.status = static_cast<uint32_t*>(ws);
     p.part = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.part);
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.ml);

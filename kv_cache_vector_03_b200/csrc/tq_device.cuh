@@ -274,7 +274,7 @@ struct PvParams {
     const uint8_t* packed;
     const float* P;
     float* out;
-    const float* pi;
+    const float* piT;      // prepared Pi^T, fp32 [D][D] (row j = column j of Pi), 256-byte aligned
     uint32_t* status;
     float* part;           // [stream*g heads][nsplit][D]
     float* part_ml;        // [stream*g heads][nsplit][2]: max, sum
