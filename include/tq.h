@@ -129,7 +129,7 @@ int tq_quantize(const tq_codec* codec, const void* x, tq_dtype dtype, int64_t n_
  *   g        query heads per kv-head, 1, 2, 4 or 8.
  *   tail     device bf16 [n_seq, n_kv, n_tail, d] full-precision recent keys (blog.hotdry.top,
  *            "engineering configuration list": the most recent 128-256 tokens stay at full
- *            precision), or NULL with n_tail = 0. n_tail <= 524272, else
+ *            precision), or NULL with n_tail = 0. n_tail <= 1048544, else
  *            TQ_ERR_UNSUPPORTED.
  *   out      device fp32 [n_seq, n_kv * g, n_tok + n_tail]: the n_tok compressed-key logits
  *            scale * |x|(<Pi q, c[idx]> + gamma sqrt(pi/2)/m <S q, s>) followed by the n_tail

@@ -28,7 +28,7 @@
 
 namespace {
 
-constexpr int kPrologueThreads = 256;
+constexpr int kPrologueThreads = 512;
 constexpr int kStreamWarps = 8;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -37,22 +37,25 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
     return ((((size_t)stream * ntiles + ntile) * nmg + mg) * 4 + c) * 64 + lane * 2 + h;
 }
 
-// Prologue. Grid (ceil(heads / 8), 1 + ceil(n_tail / 8)); each CTA owns 8 consecutive query
-// heads (rows s*g + h of q).
-//   y = 0: 1. q' = Pi q and q'' = S q as one [8 x d] x [d x (D + Mp)] product against
-//             (Pi^T | S^T). Thread (row half, head quad, column quad) keeps 4 heads x 4 columns
-//             (x 2 for wide codecs) and reads the matrix rows from global memory, where every
-//             CTA finds them in L1 / L2; the two row halves are added in shared memory.
+// Prologue. Grid (ceil(heads / HPC), 1 + ceil(n_tail / 16)), 512 threads; each CTA owns HPC
+// (4, 8 or 16) consecutive query heads (rows s*g + h of q), chosen so that about one CTA per
+// SM covers all heads: the kernel is latency-bound and every CTA pays one matrix load.
+//   y = 0: 1. q' = Pi q and q'' = S q as one [HPC x d] x [d x (D + Mp)] product against
+//             (Pi^T | S^T), whose rows arrive by bulk copies of 32 KB: all four chunks at once
+//             for D + Mp <= 256 (each used as it lands), else 16-row chunks in two stages. Thread (row slice, head quad,
+//             column quad) keeps 4 heads x 4 columns (x 2 for wide codecs); the row slices are
+//             added in shared memory.
 //          2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
 //          3. one thread per fragment word: it rounds its four coordinates, packs their hi and
 //             lo bytes into two words and stores them; warp sums give the per-head constants.
-//   y > 0: exact logits of 8 tail tokens for the 8 heads, one warp per token.
-constexpr int kPH = 8;         // heads per prologue CTA
-// matrix rows per bulk-copied chunk: 32 KB stages at most
+//   y > 0: exact logits of 16 tail tokens for the CTA's heads, one warp per token.
+constexpr int kTailTok = 16;   // tail tokens per tail CTA (one per warp)
+// matrix rows per bulk-copied chunk (32 KB) and stages: 256-wide codecs hold all four chunks
+// at once (issued together, consumed as they land), wider ones cycle two stages
 __host__ __device__ constexpr int prologue_rows(int W) { return W <= 256 ? 32 : 16; }
-constexpr int kTailTok = 8;    // tail tokens per tail CTA (one per warp)
+__host__ __device__ constexpr int prologue_stages(int W) { return W <= 256 ? 4 : 2; }
 
-template <int NR>   // 256-column groups of (Pi^T | S^T): 1 for D + Mp <= 256, else 2
+template <int NR, int HPC>   // NR: 256-column groups of (Pi^T | S^T); HPC: heads per CTA
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
     // the kernel that consumes the fragments may launch now; it waits for this grid's
     // completion before it reads them
@@ -60,16 +63,16 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     const TqDims& T = p.t;
     const int D = T.D, Mp = T.Mp, d = T.d, G = p.g, np = T.nplanes_mma, W = D + Mp;
     const int n_heads = (int)(p.n_seq * p.n_kv * G);
-    const int h_base = blockIdx.x * kPH;
-    const int H = min(kPH, n_heads - h_base);
+    const int h_base = blockIdx.x * HPC;
+    const int H = min(HPC, n_heads - h_base);
     extern __shared__ __align__(16) float sm[];
     const int tid = threadIdx.x, wid = tid >> 5, lane = tid & 31;
 
     if (blockIdx.y > 0) {
         // exact logits of the full-precision tail, scale <q, k>: warp w takes token
-        // 8 (y - 1) + w and the key rows of the CTA's streams (one for g >= 8, up to 8 for g = 1)
-        float* qh = sm;   // [8][d]
-        for (int e = tid; e < kPH * d; e += blockDim.x) {
+        // 16 (y - 1) + w and the key rows of the CTA's streams
+        float* qh = sm;   // [HPC][d]
+        for (int e = tid; e < HPC * d; e += blockDim.x) {
             const int h = e / d, j = e - h * d;
             qh[e] = h < H ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
         }
@@ -101,15 +104,14 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         return;
     }
 
-    float* qT = sm;                    // [256][8] query, transposed (rows >= d are zero)
-    float* qo = qT + 256 * kPH;        // [8][W]: q' (0..D-1) then q'' (D..W-1)
-    __shared__ float s_inv[2][kPH], s_step[2][kPH];
-    __shared__ int s_sum[2][kPH];
-    __shared__ uint64_t s_bar[2];   // matrix chunk stages (two bulk copies each)
+    float* qT = sm;                    // [256][HPC] query, transposed (rows >= d are zero)
+    float* qo = qT + 256 * HPC;        // [HPC][W]: q' (0..D-1) then q'' (D..W-1)
+    __shared__ float s_inv[2][HPC], s_step[2][HPC];
+    __shared__ int s_sum[2][HPC];
+    __shared__ uint64_t s_bar[4];   // matrix chunk stages (two bulk copies each)
     const int nmg = T.nmg;
     if (tid == 0) {
-        tq_mbar_init(&s_bar[0], 2);
-        tq_mbar_init(&s_bar[1], 2);
+        for (int k = 0; k < 4; ++k) tq_mbar_init(&s_bar[k], 2);
         tq_fence_mbar_init();
     }
     const int frag_words = p.ntiles * nmg * 256;
@@ -120,31 +122,30 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         uint4* fz = reinterpret_cast<uint4*>(p.qfrag + (size_t)st0 * frag_words);
         for (int e = tid; e < (st1 - st0) * frag_words / 4; e += blockDim.x) fz[e] = make_uint4(0, 0, 0, 0);
     }
-    for (int e = tid; e < 256 * kPH; e += blockDim.x) {
-        const int j = e / kPH, h = e % kPH;
+    for (int e = tid; e < 256 * HPC; e += blockDim.x) {
+        const int j = e / HPC, h = e % HPC;
         const bool ok = h < H && j < d && (int64_t)(h_base + h) < p.n_heads_valid;
         qT[e] = ok ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
     }
-    if (tid < 2 * kPH) s_sum[tid / kPH][tid % kPH] = 0;
+    for (int e = tid; e < HPC * W; e += blockDim.x) qo[e] = 0.f;
+    if (tid < 2 * HPC) s_sum[tid / HPC][tid % HPC] = 0;
     __syncthreads();
 
-    // 1. product. Rows of (Pi^T | S^T) arrive in chunks of R rows by bulk copies into two
-    //    shared-memory stages ([R][D] rows of Pi^T, then [R][Mp] rows of S^T). Thread -> ks
-    //    (half ks of a chunk's rows), hq (heads 4hq .. 4hq + 3), cq (columns 4cq + 256r).
+    // 1. product. Thread -> ks (row slice ks of KS), hq (heads 4hq .. 4hq + 3), cq (columns
+    //    4cq + 256r). A chunk holds [R][D] rows of Pi^T, then [R][Mp] rows of S^T.
     {
-        const int R = prologue_rows(W), nchunk = (d + R - 1) / R;
-        float* stg = qo + kPH * W;
+        constexpr int NHQ = HPC / 4, KS = kPrologueThreads / (64 * NHQ);
+        const int R = prologue_rows(W), NST = prologue_stages(W), nchunk = (d + R - 1) / R;
+        float* stg = qo + HPC * W;
         auto load_chunk = [&](int c) {   // one thread
             const int j0 = c * R, rows = min(R, d - j0);
-            float* dst = stg + (size_t)(c & 1) * R * W;
-            tq_bulk_load(dst, p.piT + (size_t)j0 * D, (uint32_t)(rows * D * 4), &s_bar[c & 1]);
-            tq_bulk_load(dst + R * D, p.sT + (size_t)j0 * Mp, (uint32_t)(rows * Mp * 4), &s_bar[c & 1]);
+            float* dst = stg + (size_t)(c % NST) * R * W;
+            tq_bulk_load(dst, p.piT + (size_t)j0 * D, (uint32_t)(rows * D * 4), &s_bar[c % NST]);
+            tq_bulk_load(dst + R * D, p.sT + (size_t)j0 * Mp, (uint32_t)(rows * Mp * 4), &s_bar[c % NST]);
         };
-        if (tid == 0) {
-            load_chunk(0);
-            if (nchunk > 1) load_chunk(1);
-        }
-        const int ks = tid >> 7, hq = (tid >> 6) & 1, cq = tid & 63;
+        if (tid == 0)
+            for (int c = 0; c < min(nchunk, NST); ++c) load_chunk(c);
+        const int cq = tid & 63, hq = (tid >> 6) % NHQ, ks = tid / (64 * NHQ);
         int off[NR], rstr[NR];
         bool bv[NR];
 #pragma unroll
@@ -164,14 +165,16 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         bool ok = true;
         int c = 0;
         for (; c < nchunk; ++c) {
-            ok = __syncthreads_and(ok && tq_mbar_wait(&s_bar[c & 1], (uint32_t)(c >> 1) & 1u, kWaitLimit));
+            const int stg_i = c % NST;
+            const uint32_t parity = (uint32_t)(c / NST) & 1u;
+            ok = __syncthreads_and(ok && tq_mbar_wait(&s_bar[stg_i], parity, kWaitLimit));
             if (!ok) break;
-            const int j0 = c * R, rows = min(R, d - j0), half = (rows + 1) >> 1;
-            const int jj0 = ks * half, jj1 = min(rows, jj0 + half);
-            const float* st = stg + (size_t)(c & 1) * R * W;
+            const int j0 = c * R, rows = min(R, d - j0), slice = (rows + KS - 1) / KS;
+            const int jj0 = ks * slice, jj1 = min(rows, jj0 + slice);
+            const float* st = stg + (size_t)stg_i * R * W;
 #pragma unroll 4
             for (int jj = jj0; jj < jj1; ++jj) {
-                const float4 a = *reinterpret_cast<const float4*>(qT + (j0 + jj) * kPH + 4 * hq);
+                const float4 a = *reinterpret_cast<const float4*>(qT + (j0 + jj) * HPC + 4 * hq);
                 const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
                 for (int r = 0; r < NR; ++r) {
@@ -186,10 +189,12 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                     }
                 }
             }
-            __syncthreads();   // stage c & 1 is consumed
-            if (tid == 0 && c + 2 < nchunk) {
-                tq_fence_proxy_async();
-                load_chunk(c + 2);
+            if (c + NST < nchunk) {
+                __syncthreads();   // stage c % NST is consumed
+                if (tid == 0) {
+                    tq_fence_proxy_async();
+                    load_chunk(c + NST);
+                }
             }
         }
         if (!ok) {
@@ -197,34 +202,19 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             // time, and leave the fragments unwritten
             if (tid == 0) {
                 tq_raise(p.status, TQ_FLAG_TIMEOUT);
-                for (int k = c; k < min(c + 2, nchunk); ++k)
-                    tq_mbar_wait(&s_bar[k & 1], (uint32_t)(k >> 1) & 1u, kWaitLimit);
+                for (int k = c; k < min(c + NST, nchunk); ++k)
+                    tq_mbar_wait(&s_bar[k % NST], (uint32_t)(k / NST) & 1u, kWaitLimit);
             }
             return;
         }
-        // the second row half parks its sums in qo; the first adds its own
-        if (ks == 1) {
+        // the row slices meet in qo
 #pragma unroll
-            for (int r = 0; r < NR; ++r)
-                if (bv[r])
+        for (int r = 0; r < NR; ++r)
+            if (bv[r])
 #pragma unroll
-                    for (int x = 0; x < 4; ++x)
-                        *reinterpret_cast<float4*>(qo + (4 * hq + x) * W + 256 * r + 4 * cq) =
-                            make_float4(acc[r][x][0], acc[r][x][1], acc[r][x][2], acc[r][x][3]);
-        }
-        __syncthreads();
-        if (ks == 0) {
+                for (int x = 0; x < 4; ++x)
 #pragma unroll
-            for (int r = 0; r < NR; ++r)
-                if (bv[r])
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        float4* o = reinterpret_cast<float4*>(qo + (4 * hq + x) * W + 256 * r + 4 * cq);
-                        const float4 v = *o;
-                        *o = make_float4(v.x + acc[r][x][0], v.y + acc[r][x][1], v.z + acc[r][x][2],
-                                         v.w + acc[r][x][3]);
-                    }
-        }
+                    for (int y = 0; y < 4; ++y) atomicAdd(qo + (4 * hq + x) * W + 256 * r + 4 * cq + y, acc[r][x][y]);
         __syncthreads();
     }
     // 2. fixed-point steps (one head per warp)
@@ -249,7 +239,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     //    of the word is coordinate 128 gr + 32 t + 2c + hh + 8 bb, in column 2 (head % 4) (hi)
     //    or 2 (head % 4) + 1 (lo) of n-tile head / 4. A warp's 32 items share h and mg.
     const int per_head = 32 * nmg;
-    for (int e = tid; e < kPH * per_head; e += blockDim.x) {
+    for (int e = tid; e < HPC * per_head; e += blockDim.x) {
         const int h = e / per_head, w = e - h * per_head;
         const int mg = w >> 5, c = (w >> 3) & 3, t = (w >> 1) & 3, hh = w & 1;
         const bool is_code = mg < np * T.GD;
@@ -496,25 +486,39 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 
 }  // namespace
 
-size_t tq_logits_prologue_smem(const TqDims& t, int) {
+// heads per prologue CTA: about one CTA per SM
+static int prologue_hpc(int64_t n_heads) { return n_heads <= 148 * 4 ? 4 : n_heads <= 148 * 8 ? 8 : 16; }
+
+size_t tq_logits_prologue_smem(const TqDims& t, int hpc) {
     const int W = t.D + t.Mp;
-    return ((size_t)256 * kPH + (size_t)kPH * W + (size_t)2 * prologue_rows(W) * W) * 4;
+    return ((size_t)256 * hpc + (size_t)hpc * W + (size_t)prologue_stages(W) * prologue_rows(W) * W) * 4;
 }
 
-// largest prologue shared memory over the supported codecs (D = Mp = 256)
-constexpr size_t kPrologueMaxSmem = ((size_t)256 * kPH + (size_t)kPH * 512 + (size_t)2 * 16 * 512) * 4;
+// largest prologue shared memory over the supported codecs and head counts
+constexpr size_t kPrologueSmemWide = ((size_t)256 * 16 + (size_t)16 * 512 + (size_t)2 * 16 * 512) * 4;
+constexpr size_t kPrologueSmemNarrow = ((size_t)256 * 16 + (size_t)16 * 256 + (size_t)4 * 32 * 256) * 4;
+constexpr size_t kPrologueMaxSmem = kPrologueSmemWide > kPrologueSmemNarrow ? kPrologueSmemWide : kPrologueSmemNarrow;
 
-cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
-    const size_t smem = tq_logits_prologue_smem(p.t, 0);
-    const bool wide = p.t.D + p.t.Mp > 256;
-    auto kern = wide ? k_logits_prologue<2> : k_logits_prologue<1>;
-    static TqLaunchCache cache1, cache2;
-    cudaError_t e = tq_kernel_setup(kern, kPrologueThreads, kPrologueMaxSmem, wide ? cache2 : cache1, nullptr, nullptr);
+template <int NR, int HPC>
+cudaError_t launch_prologue(const LogitsParams& p, int64_t n_heads, cudaStream_t st) {
+    const size_t smem = tq_logits_prologue_smem(p.t, HPC);
+    auto kern = k_logits_prologue<NR, HPC>;
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, kPrologueThreads, kPrologueMaxSmem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
-    const int64_t n_heads = p.n_seq * p.n_kv * p.g;
-    const dim3 grid((unsigned)((n_heads + kPH - 1) / kPH), 1u + (unsigned)((p.n_tail + kTailTok - 1) / kTailTok));
+    const dim3 grid((unsigned)((n_heads + HPC - 1) / HPC), 1u + (unsigned)((p.n_tail + kTailTok - 1) / kTailTok));
     kern<<<grid, kPrologueThreads, smem, st>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
+    const int64_t n_heads = p.n_seq * p.n_kv * p.g;
+    const bool wide = p.t.D + p.t.Mp > 256;
+    switch (prologue_hpc(n_heads)) {
+        case 4: return wide ? launch_prologue<2, 4>(p, n_heads, st) : launch_prologue<1, 4>(p, n_heads, st);
+        case 8: return wide ? launch_prologue<2, 8>(p, n_heads, st) : launch_prologue<1, 8>(p, n_heads, st);
+        default: return wide ? launch_prologue<2, 16>(p, n_heads, st) : launch_prologue<1, 16>(p, n_heads, st);
+    }
 }
 
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st) {

@@ -10,7 +10,6 @@
 #include "tq.h"
 #include "tq_device.cuh"
 
-size_t tq_logits_prologue_smem(const TqDims& t, int g);
 
 namespace {
 
@@ -308,8 +307,8 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.status = static_cast<uint32_t*>(ws);
     p.n_heads_valid = n_streams * g;
-    // the tail runs on a second grid dimension of 8-token CTAs (at most 65535)
-    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 8 * 65534)
+    // the tail runs on a second grid dimension of 16-token CTAs (at most 65535)
+    if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 16 * 65534)
         return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
