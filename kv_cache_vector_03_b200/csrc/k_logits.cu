@@ -104,8 +104,10 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         return;
     }
 
-    float* qT = sm;                    // [256][HPC] query, transposed (rows >= d are zero)
-    float* qo = qT + 256 * HPC;        // [HPC][W]: q' (0..D-1) then q'' (D..W-1)
+    // FFMA path (wide codecs): qT [256][HPC] query transposed, then qo [HPC][W].
+    // MMA path (D + Mp = 256): qo [16][256], then the operand tiles.
+    float* qT = sm;
+    float* qo = NR == 1 ? sm : qT + 256 * HPC;   // q' (0..D-1) then q'' (D..W-1)
     __shared__ float s_inv[2][HPC], s_step[2][HPC];
     __shared__ int s_sum[2][HPC];
     __shared__ uint64_t s_bar[4];   // matrix chunk stages (two bulk copies each)
@@ -122,13 +124,113 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         uint4* fz = reinterpret_cast<uint4*>(p.qfrag + (size_t)st0 * frag_words);
         for (int e = tid; e < (st1 - st0) * frag_words / 4; e += blockDim.x) fz[e] = make_uint4(0, 0, 0, 0);
     }
+    if (tid < 2 * HPC) s_sum[tid / HPC][tid % HPC] = 0;
+    if constexpr (NR == 1) {
+        // 1. product on the fp16 tensor cores (mma.sync m16n8k16, hi/lo split passes):
+        //    q' = Pi q (A = queries, 16 rows, B = 256 Pi), then q'' = M q' = S q (B = 256 M,
+        //    M = S Pi^T). Warp w owns output columns 8w .. 8w + 7 of both products.
+        uint8_t* at = reinterpret_cast<uint8_t*>(sm + 16 * 256);   // A hi, A lo [16][256 B]
+        uint8_t* bt = at + 2 * 16 * 256;                            // Pi hi, Pi lo, M hi, M lo [128][256 B]
+        __shared__ float s_qsc[16];
+        const uint32_t sat = tq_smem_addr(at), sbt = tq_smem_addr(bt);
+        {   // B tiles, swizzled rows
+            const uint16_t* srcs[4] = {p.pih, p.pil, p.mh, p.ml};
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint4 v[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int e = tid + kPrologueThreads * (8 * half + k);
+                    const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
+                    v[k] = __ldg(reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8));
+                }
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int e = tid + kPrologueThreads * (8 * half + k);
+                    const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
+                    *reinterpret_cast<uint4*>(bt + m * 32768 + tq_swz256(row, ch)) = v[k];
+                }
+            }
+        }
+        // A rows: warp w = head w; lane l holds coordinates 4l .. 4l + 3, scaled per row by a power
+        // of two (max in [2^14, 2^15)) and split into binary16 hi + lo
+        auto put_row = [&](int row, const float (&x)[4], float scale_of_max) {
+            float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+            mx = tq_warp_max(mx);
+            int ex = 0;
+            if (mx > 0.f && isfinite(mx)) ex = min(max(14 - (((__float_as_int(mx) >> 23) & 0xff) - 127), -126), 126);
+            const float sc = __int_as_float((127 + ex) << 23);
+            const __half2 h0 = __floats2half2_rn(x[0] * sc, x[1] * sc), h1 = __floats2half2_rn(x[2] * sc, x[3] * sc);
+            const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+            const __half2 l0 = __floats2half2_rn(x[0] * sc - f0.x, x[1] * sc - f0.y);
+            const __half2 l1 = __floats2half2_rn(x[2] * sc - f1.x, x[3] * sc - f1.y);
+            const uint32_t off = tq_swz256(row, lane >> 1) + (lane & 1) * 8;
+            *reinterpret_cast<uint2*>(at + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&h0),
+                                                            *reinterpret_cast<const uint32_t*>(&h1));
+            *reinterpret_cast<uint2*>(at + 4096 + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&l0),
+                                                                   *reinterpret_cast<const uint32_t*>(&l1));
+            if (lane == 0) s_qsc[row] = scale_of_max / sc;
+        };
+        {
+            const int h = wid;   // 16 warps, 16 rows
+            const bool ok = h < H && (int64_t)(h_base + h) < p.n_heads_valid;
+            float x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * lane + k;
+                x[k] = ok && j < d ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
+            }
+            put_row(h, x, 1.f / 256.f);
+        }
+        __syncthreads();
+        // one 16 x 8 output tile per warp over K = 128: A hi/lo x B hi/lo (three passes)
+        const int mi = lane >> 3, r8 = lane & 7;
+        const int a_row = (mi & 1) * 8 + r8, a_chk = mi >> 1;
+        const int b_row = 8 * wid + r8, b_chk = mi & 1;
+        const int g = lane >> 2, t = lane & 3;
+        auto tile = [&](int bm, float (&acc)[4]) {   // bm: 0 = Pi, 2 = M
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll
+            for (int kc = 0; kc < 8; ++kc) {
+                uint32_t ah[4], al[4], bh[2], bl[2];
+                tq_ldsm_x4(sat + tq_swz256(a_row, 2 * kc + a_chk), ah[0], ah[1], ah[2], ah[3]);
+                tq_ldsm_x4(sat + 4096 + tq_swz256(a_row, 2 * kc + a_chk), al[0], al[1], al[2], al[3]);
+                tq_ldsm_x2(sbt + bm * 32768 + tq_swz256(b_row, 2 * kc + b_chk), bh[0], bh[1]);
+                tq_ldsm_x2(sbt + (bm + 1) * 32768 + tq_swz256(b_row, 2 * kc + b_chk), bl[0], bl[1]);
+                tq_hmma(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                tq_hmma(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                tq_hmma(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
+            }
+        };
+        float acc[4];
+        tile(0, acc);   // q' columns 8w + 2t, +1 of rows g, g + 8
+        qo[g * 256 + 8 * wid + 2 * t] = acc[0] * s_qsc[g];
+        qo[g * 256 + 8 * wid + 2 * t + 1] = acc[1] * s_qsc[g];
+        qo[(g + 8) * 256 + 8 * wid + 2 * t] = acc[2] * s_qsc[g + 8];
+        qo[(g + 8) * 256 + 8 * wid + 2 * t + 1] = acc[3] * s_qsc[g + 8];
+        __syncthreads();
+        {
+            const int h = wid;
+            float x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) x[k] = qo[h * 256 + 4 * lane + k];
+            __syncwarp();
+            put_row(h, x, 1.f / 256.f);   // A <- q'
+        }
+        __syncthreads();
+        tile(2, acc);   // q'' = M q'
+        qo[g * 256 + 128 + 8 * wid + 2 * t] = acc[0] * s_qsc[g];
+        qo[g * 256 + 128 + 8 * wid + 2 * t + 1] = acc[1] * s_qsc[g];
+        qo[(g + 8) * 256 + 128 + 8 * wid + 2 * t] = acc[2] * s_qsc[g + 8];
+        qo[(g + 8) * 256 + 128 + 8 * wid + 2 * t + 1] = acc[3] * s_qsc[g + 8];
+        __syncthreads();
+    } else {
     for (int e = tid; e < 256 * HPC; e += blockDim.x) {
         const int j = e / HPC, h = e % HPC;
         const bool ok = h < H && j < d && (int64_t)(h_base + h) < p.n_heads_valid;
         qT[e] = ok ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
     }
     for (int e = tid; e < HPC * W; e += blockDim.x) qo[e] = 0.f;
-    if (tid < 2 * HPC) s_sum[tid / HPC][tid % HPC] = 0;
     __syncthreads();
 
     // 1. product. Thread -> ks (row slice ks of KS), hq (heads 4hq .. 4hq + 3), cq (columns
@@ -216,6 +318,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
 #pragma unroll
                     for (int y = 0; y < 4; ++y) atomicAdd(qo + (4 * hq + x) * W + 256 * r + 4 * cq + y, acc[r][x][y]);
         __syncthreads();
+    }
     }
     // 2. fixed-point steps (one head per warp)
     float amax = 0.f;
@@ -489,15 +592,18 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 // heads per prologue CTA: about one CTA per SM
 static int prologue_hpc(int64_t n_heads) { return n_heads <= 148 * 4 ? 4 : n_heads <= 148 * 8 ? 8 : 16; }
 
+// MMA path (D + Mp = 256): qo [16][256] fp32 + A hi/lo [16][256 B] + four [128][256 B] B tiles
+constexpr size_t kPrologueSmemMma = (size_t)16 * 256 * 4 + 2 * 16 * 256 + 4 * 128 * 256;
+
 size_t tq_logits_prologue_smem(const TqDims& t, int hpc) {
     const int W = t.D + t.Mp;
+    if (W <= 256) return kPrologueSmemMma;
     return ((size_t)256 * hpc + (size_t)hpc * W + (size_t)prologue_stages(W) * prologue_rows(W) * W) * 4;
 }
 
 // largest prologue shared memory over the supported codecs and head counts
 constexpr size_t kPrologueSmemWide = ((size_t)256 * 16 + (size_t)16 * 512 + (size_t)2 * 16 * 512) * 4;
-constexpr size_t kPrologueSmemNarrow = ((size_t)256 * 16 + (size_t)16 * 256 + (size_t)4 * 32 * 256) * 4;
-constexpr size_t kPrologueMaxSmem = kPrologueSmemWide > kPrologueSmemNarrow ? kPrologueSmemWide : kPrologueSmemNarrow;
+constexpr size_t kPrologueMaxSmem = kPrologueSmemWide > kPrologueSmemMma ? kPrologueSmemWide : kPrologueSmemMma;
 
 template <int NR, int HPC>
 cudaError_t launch_prologue(const LogitsParams& p, int64_t n_heads, cudaStream_t st) {

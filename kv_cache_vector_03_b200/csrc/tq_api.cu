@@ -299,6 +299,10 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.out = out;
     p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
     p.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
+    p.pih = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pih);
+    p.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
+    p.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
+    p.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
     p.qfrag = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + W.qfrag);
     p.qscale = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.qscale);
     p.n_seq = n_seq; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
@@ -366,6 +370,10 @@ int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float*
     lp.q = q; lp.q_dtype = TQ_F32;
     lp.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
     lp.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
+    lp.pih = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pih);
+    lp.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
+    lp.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
+    lp.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
     lp.qfrag = reinterpret_cast<uint32_t*>(wsb + W.qfrag);
     lp.qscale = reinterpret_cast<float*>(wsb + W.qscale);
     lp.status = static_cast<uint32_t*>(ws);

@@ -150,6 +150,19 @@ TQ_DEVICE void tq_imma_u8_z(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, 
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(0));
 }
 
+// ldmatrix: four / two 8x8 b16 matrices from shared memory (row addresses from lanes 0-31 / 0-15)
+TQ_DEVICE void tq_ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+TQ_DEVICE void tq_ldsm_x2(uint32_t addr, uint32_t& r0, uint32_t& r1) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// byte offset of 16-byte chunk `chunk` of row `row` in rows of 256 bytes, XOR-swizzled by
+// row mod 8 so that ldmatrix reads of 8 rows hit distinct banks
+TQ_DEVICE uint32_t tq_swz256(int row, int chunk) { return (uint32_t)(row * 256 + ((chunk ^ (row & 7)) << 4)); }
+
 // ---------------------------------------------------------------------- mbarrier + bulk copy
 // One-dimensional bulk copies global -> shared through the TMA engine, completion tracked
 // by a shared-memory mbarrier (transaction bytes). Waits are bounded: a wait that does not
@@ -259,6 +272,7 @@ struct LogitsParams {
     float* out;
     const float* piT;
     const float* sT;
+    const uint16_t *pih, *pil, *mh, *ml;   // fp16 hi/lo of 256 Pi and 256 M (row = output)
     uint32_t* qfrag;       // [stream][ntile][nmg][4][32][2]
     float* qscale;         // [stream][ntile*4][4]: dA/128, KA, 2dS/128, KS
     uint32_t* status;
