@@ -184,6 +184,36 @@ def test_logits_gqa_ragged_with_tail(B, g):
             _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1), scale)
 
 
+@pytest.mark.parametrize("n_seq,n_kv,g,n_tail", [(40, 4, 4, 20), (25, 8, 8, 33)])
+def test_logits_many_heads(n_seq, n_kv, g, n_tail):
+    """640 / 1600 query heads: the prologue takes 8 / 16 heads per CTA; tails of 20 / 33 tokens
+    span two / three tail CTAs."""
+    d = m = 128
+    B = 2
+    pi, s = ti.haar_rotation(d, 93), ti.gaussian_sketch(m, d, 94)
+    n_tok = 70
+    keys = np.stack([np.stack([ti.key_stream(4, sq, h, n_tok + n_tail) for h in range(n_kv)]) for sq in range(n_seq)])
+    comp = np.ascontiguousarray(keys[:, :, :n_tok])
+    tail = np.ascontiguousarray(keys[:, :, n_tok:])
+    qb = ti.decode_queries(11, n_seq, n_kv * g)
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(comp.reshape(-1, d)), n_seq * n_kv, n_tok)
+    scale = 1.0 / math.sqrt(d)
+    got = _logits_gpu(codec, packed, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, to_dev_bf16(tail), n_tail, scale)
+    idx, sbit, nhat, ghat = unpack(codec, packed, n_seq * n_kv, n_tok)
+    c, t = _cb(d, B)
+    q = ti.bf16_to_f64(qb)
+    kf = ti.bf16_to_f64(keys)
+    for sq in range(0, n_seq, 7):
+        for h in range(n_kv):
+            st = sq * n_kv + h
+            qh = q[sq, h * g:(h + 1) * g]
+            want = oracle.logits(idx[st], sbit[st], nhat[st], ghat[st], pi, s, c, qh, qjl=True, scale=scale)
+            _check_logits(got[sq, h * g:(h + 1) * g, :n_tok], want, qh, np.linalg.norm(kf[sq, h, :n_tok], axis=1), scale)
+            wt = oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)
+            _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1), scale)
+
+
 def test_logits_d200_codec():
     d = m = 200
     pi, s = ti.C5.pi(), ti.C5.s()
