@@ -45,7 +45,7 @@ typedef enum {
     TQ_ERR_UNSUPPORTED = -2,  /* valid request outside the supported shapes */
     TQ_ERR_CUDA = -3,         /* a CUDA runtime call failed */
     TQ_ERR_RANGE = -4,        /* (status word) a norm overflowed binary16 or an input was not finite */
-    TQ_ERR_TIMEOUT = -5,      /* reserved: no call waits on another block */
+    TQ_ERR_TIMEOUT = -5,      /* (status word) a bounded wait for a bulk copy ran out */
     TQ_ERR_NOCONV = -6,       /* codebook iteration did not converge */
     TQ_ERR_WORKSPACE = -7     /* workspace or prepared buffer too small / not prepared */
 } tq_status;
@@ -144,9 +144,35 @@ int tq_logits(const tq_codec* codec, const void* packed, int64_t n_seq, int n_kv
  *   packed_v device value cache (qjl = 0): n_seq * n_kv streams of n_tok vectors.
  *   P        device fp32 [n_seq, n_kv * g, n_tok] attention logits (before softmax).
  *   out      device fp32 [n_seq, n_kv * g, d].
- *   ws       tq_workspace_bytes(codec, TQ_OP_PV, n_seq * n_kv * g, n_tok, 0) bytes.         */
+ *   ws       tq_workspace_bytes(codec, TQ_OP_PV, n_seq * n_kv, n_tok, g) bytes.             */
 int tq_pv(const tq_codec* codec, const void* packed_v, int64_t n_seq, int n_kv, int64_t n_tok,
           const float* P, int g, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Decode attention in one pass over compressed keys and values:
+ *   out_h = sum_t softmax_t(l_h) v_t,  l_h,t = scale <q_h, k_t>
+ * with the logits of tq_logits (estimator on the packed keys, exact on the bf16 tail) and
+ * the values of tq_pv (MSE codes, rotated back once), the logits never written to memory
+ * (a2a-mcp.org "What is TurboQuant": scores computed straight from the indices in a fused
+ * kernel; blog.hotdry.top, "engineering configuration list": recent tokens at full precision).
+ *   kcodec   key codec, qjl = 1, d <= 128 and m <= 128.
+ *   vcodec   value codec, qjl = 0, the same d; both prepared.
+ *   packed_k device key cache of n_seq * n_kv streams of n_tok tokens (tq_quantize layout).
+ *   packed_v device value cache, the same streams and tokens.
+ *   q        device [n_seq, n_kv * g, d], fp32 or bf16; query head j reads kv-head j / g.
+ *   g        query heads per kv-head, 1, 2 or 4 (else TQ_ERR_UNSUPPORTED).
+ *   tail_k, tail_v  device bf16 [n_seq, n_kv, n_tail, d] recent keys and values, the
+ *            tokens that follow the compressed ones; NULL with n_tail = 0.
+ *            n_tail <= TQ_ATTN_MAX_TAIL, else TQ_ERR_UNSUPPORTED.
+ *   out      device fp32 [n_seq, n_kv * g, d].
+ *   ws       tq_attention_workspace_bytes(kcodec, vcodec, n_seq, n_kv, n_tok, g, n_tail) bytes,
+ *            256-byte aligned. n_tok + n_tail = 0 is TQ_ERR_ARG (a softmax over no tokens). */
+#define TQ_ATTN_MAX_TAIL 8192
+size_t tq_attention_workspace_bytes(const tq_codec* kcodec, const tq_codec* vcodec, int64_t n_seq, int n_kv,
+                                    int64_t n_tok, int g, int n_tail);
+int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* packed_k, const void* packed_v,
+                 int64_t n_seq, int n_kv, int64_t n_tok, const void* q, tq_dtype q_dtype, int g,
+                 const void* tail_k, const void* tail_v, int n_tail, float scale, float* out, void* ws,
+                 size_t ws_bytes, void* stream);
 
 /* Top-k inner-product search over a packed database (a2a-mcp.org, benchmark section:
  * GloVe d=200 recall; scores are the same estimator as tq_logits with scale 1).

@@ -3,7 +3,7 @@
 Argument marshalling only: every function forwards torch device pointers and sizes to the
 C ABI in include/tq.h; all arithmetic runs in the CUDA library. PyTorch provides device
 memory and streams. Importing this package fails loudly if libtq.so has not been built
-(run ``python -m kv_cache_vector_03_b200.build`` or ``__graft_entry__.build()``).
+(run ``python kv_cache_vector_03_b200/build.py`` or ``__graft_entry__.build()``).
 """
 from __future__ import annotations
 
@@ -16,7 +16,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libtq.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libtq.so is missing at {LIB_PATH}: build it with kv_cache_vector_03_b200.build")
+    raise ImportError(f"libtq.so is missing at {LIB_PATH}: build it with python kv_cache_vector_03_b200/build.py")
 
 lib = ctypes.CDLL(LIB_PATH)
 
@@ -27,7 +27,7 @@ TQ_OP_QUANTIZE, TQ_OP_LOGITS, TQ_OP_PV, TQ_OP_TOPK, TQ_OP_DEQUANTIZE = 0, 1, 2, 
 EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_bytes", "tq_prep_bytes",
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
             "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",
-            "tq_logits_noalloc"]
+            "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes"]
 
 
 class tq_codec(ctypes.Structure):
@@ -50,6 +50,8 @@ _sig = {
     "tq_logits": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _P]),
     "tq_logits_noalloc": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P]),
     "tq_pv": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _P, _P, _SZ, _P]),
+    "tq_attention_workspace_bytes": (_SZ, [_CP, _CP, _I64, _I, _I64, _I, _I]),
+    "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "tq_dequantize": (_I, [_CP, _P, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_reset_status": (_I, [_P, _P]),
@@ -170,6 +172,17 @@ def tq_logits_noalloc(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_ta
 def tq_pv(codec: Codec, packed_v, n_seq, n_kv, n_tok, P, g, out, ws, stream=None):
     return _check("tq_pv", lib.tq_pv(codec.ref, _ptr(packed_v), n_seq, n_kv, n_tok, _ptr(P), g, _ptr(out), _ptr(ws),
                                      ws.numel(), _stream(stream)))
+
+
+def tq_attention_workspace_bytes(kcodec: Codec, vcodec: Codec, n_seq, n_kv, n_tok, g, n_tail):
+    return lib.tq_attention_workspace_bytes(kcodec.ref, vcodec.ref, n_seq, n_kv, n_tok, g, n_tail)
+
+
+def tq_attention(kcodec: Codec, vcodec: Codec, packed_k, packed_v, n_seq, n_kv, n_tok, q, g, tail_k, tail_v, n_tail,
+                 scale, out, ws, stream=None):
+    return _check("tq_attention", lib.tq_attention(kcodec.ref, vcodec.ref, _ptr(packed_k), _ptr(packed_v), n_seq, n_kv,
+                                                   n_tok, _ptr(q), _dtype(q), g, _ptr(tail_k), _ptr(tail_v), n_tail,
+                                                   scale, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=None):

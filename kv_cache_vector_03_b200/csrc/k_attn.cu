@@ -1,0 +1,422 @@
+// tq_attention: decode attention softmax(scale q . K) . V in one pass over compressed keys
+// and values (a2a-mcp.org "What is TurboQuant", the fused-kernel note: scores straight from the
+// indices with the query rotated once; friday-blog-bgf.pages.dev "TurboQuant deep dive II",
+// section 1, step 1: values keep the rotation + scalar quantizer; blog.hotdry.top "TurboQuant
+// vector-search compression", engineering configuration list: the most recent tokens stay at
+// full precision).
+//
+// The logits never leave the SM. Kernel 1 is the logits prologue (query fragments, exact tail
+// logits). Kernel 2 (split): one CTA of 4 warps per (stream, block range); per 32-token block
+// a warp receives the key block and the value block in one ring stage (two bulk copies, one
+// mbarrier), computes the 32 x 4 logits on the int8 tensor cores (bit planes, as tq_logits),
+// keeps a running maximum and sum per head (online softmax), turns exp(l - m) |v| into fp16
+// hi + lo MMA columns and accumulates the values, decoded through per-lane half2 tables, on the
+// fp16 tensor cores (as tq_pv). Kernel 3 (merge): one CTA per query head combines the ranges
+// (log-sum-exp), rotates the value sum by Pi^T once and adds the exact tail.
+#include <algorithm>
+
+#include "tq_device.cuh"
+
+namespace {
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnNS = 3;             // ring stages per warp (key + value block each)
+constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr int kWCol = 20;              // words per staged weight column (16 used)
+
+template <int BK, int BV>
+constexpr uint32_t attn_stage_bytes() {
+    return (512u * (BK + 1) + 128u) + (512u * BV + 64u);   // key block (d = m = 128) + value block
+}
+template <int BK, int BV>
+constexpr size_t attn_smem() {
+    return (size_t)(1 << (2 * BV)) * 128 + (size_t)kAttnWarps * kAttnNS * attn_stage_bytes<BK, BV>();
+}
+
+__device__ __forceinline__ size_t qf_word(int64_t stream, int nmg, int mg, int c, int lane) {
+    return (((size_t)stream * nmg + mg) * 4 + c) * 64 + lane * 2;
+}
+
+template <int BK, int BV>   // key MSE bits (1..3), value bits (1..4); d <= 128, m <= 128, g <= 4
+__global__ void __launch_bounds__(kAttnWarps * 32) k_attn_split(AttnParams p) {
+    constexpr int NS = kAttnNS;
+    constexpr int NP = BK == 3 ? 4 : BK;   // estimator code planes
+    constexpr int NPG = BK + 1;            // stored key plane groups (one 128-coordinate group each)
+    constexpr int NMG = NP + 1;            // MMA plane groups
+    constexpr uint32_t BBK = 512u * NPG + 128u;
+    constexpr int KT = 8, CH = KT * BV / 8, NW = 4 * CH;
+    constexpr uint32_t SEC_AV = 512u * CH;
+    constexpr uint32_t STG = attn_stage_bytes<BK, BV>();
+    constexpr int E = 1 << (2 * BV);
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);        // [E][32]
+    uint8_t* ring = smem + (size_t)E * 128;                    // [warp][NS][STG]
+    __shared__ uint32_t wst[kAttnWarps][8][kWCol];             // column 2 head + part: token pairs
+    __shared__ float s_acc[4][KT * 16];
+    __shared__ float s_m[kAttnWarps][4], s_l[kAttnWarps][4];
+    __shared__ uint64_t bars[kAttnWarps][NS];
+
+    const int G = p.g;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;   // MMA fragment coordinates; t is this thread's head
+    const int64_t stream = blockIdx.x / p.nsplit;
+    const int split = blockIdx.x % p.nsplit;
+    const int64_t b0 = (int64_t)split * p.blocks_per_split;
+    const int64_t b1 = min(b0 + p.blocks_per_split, p.nb);
+
+    for (int e = threadIdx.x; e < E * 32; e += blockDim.x) {
+        const int ent = e >> 5;
+        lut[e] = p.cbv.lut_half[ent & ((1 << BV) - 1)] | (p.cbv.lut_half[ent >> BV] << 16);
+    }
+    for (int e = threadIdx.x; e < 4 * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[w][s], 2);
+    tq_fence_mbar_init();
+    __syncthreads();
+
+    uint8_t* my_ring = ring + (size_t)w * NS * STG;
+    const int64_t first = b0 + w;
+    const int nmine = first < b1 ? (int)((b1 - first + kAttnWarps - 1) / kAttnWarps) : 0;
+    const uint8_t* kk = p.packed_k + ((size_t)stream * p.nb + first) * BBK;
+    const uint8_t* vk = p.packed_v + ((size_t)stream * p.nb + first) * p.tv.block_bytes;
+    auto issue = [&](int k) {
+        if (k < nmine && lane == 0) {
+            const int s = k % NS;
+            tq_bulk_load(my_ring + s * STG, kk, BBK, &bars[w][s]);
+            tq_bulk_load(my_ring + s * STG + BBK, vk, (uint32_t)p.tv.block_bytes, &bars[w][s]);
+        }
+        if (k < nmine) {
+            kk += (size_t)kAttnWarps * BBK;
+            vk += (size_t)kAttnWarps * p.tv.block_bytes;
+        }
+    };
+    for (int k = 0; k < NS; ++k) issue(k);
+
+    // the copies above read only the caches; the query fragments come from the prologue
+    tq_pdl_wait();
+    uint32_t qf[NMG][4][2];
+#pragma unroll
+    for (int mg = 0; mg < NMG; ++mg)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const uint2 v = *reinterpret_cast<const uint2*>(p.qfrag + qf_word(stream, NMG, mg, c, lane));
+            qf[mg][c][0] = v.x;
+            qf[mg][c][1] = v.y;
+        }
+    const float4 sc = reinterpret_cast<const float4*>(p.qscale)[(size_t)stream * 4 + t];
+    const bool hv = t < G;
+    constexpr float kLog2e = 1.4426950408889634f;
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+
+    float acc[KT][4];
+#pragma unroll
+    for (int i = 0; i < KT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    float m_run = -INFINITY, lsum = 0.f;   // head t: the same m in the 8 lanes of the head
+
+    bool ok = true;
+    int k = 0;
+    for (; k < nmine; ++k) {
+        const int s = k % NS;
+        ok = __all_sync(0xffffffffu, tq_mbar_wait(&bars[w][s], (uint32_t)(k / NS) & 1u, kWaitLimit));
+        if (!ok) break;
+        const uint8_t* kb = my_ring + s * STG;
+        const uint8_t* vb = kb + BBK;
+        const int64_t blk = first + (int64_t)kAttnWarps * k;
+
+        // ---- logits of the 32 keys for head t: keys 8u + g, u = 0..3
+        uint4 cur[NPG + 1];
+#pragma unroll
+        for (int pg = 0; pg < NPG; ++pg) cur[pg] = *reinterpret_cast<const uint4*>(kb + (pg * 32 + lane) * 16);
+        cur[NPG] = *reinterpret_cast<const uint4*>(kb + NPG * 512 + g * 16);
+        const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
+        float l[4];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            int accA[4], accA2[4], accS[4];
+#pragma unroll
+            for (int mg = 0; mg < NMG; ++mg) {
+                uint32_t w0, w1;
+                if (mg < NP && mg == 3) {   // b0 ^ b1 ^ b2
+                    const uint32_t* c0 = reinterpret_cast<const uint32_t*>(&cur[0]);
+                    const uint32_t* c1 = reinterpret_cast<const uint32_t*>(&cur[1]);
+                    const uint32_t* c2 = reinterpret_cast<const uint32_t*>(&cur[2]);
+                    w0 = c0[2 * mt] ^ c1[2 * mt] ^ c2[2 * mt];
+                    w1 = c0[2 * mt + 1] ^ c1[2 * mt + 1] ^ c2[2 * mt + 1];
+                } else {
+                    const int pg = mg < NP ? mg : BK;
+                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(&cur[pg]);
+                    w0 = cw[2 * mt];
+                    w1 = cw[2 * mt + 1];
+                }
+                tq_expand_planes(w0, w1, [&](int c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+                    const uint32_t q0 = qf[mg][c][0], q1 = qf[mg][c][1];
+                    if (mg < NP) {
+                        int(&a)[4] = (c & 1) ? accA : accA2;
+                        if (mg == 0 && c >= 2) tq_imma_u8_z(a, a0, a1, a2, a3, q0, q1);
+                        else tq_imma_u8(a, a0, a1, a2, a3, q0, q1);
+                    } else {
+                        if (c == 3) tq_imma_u8_z(accS, a0, a1, a2, a3, q0, q1);
+                        else tq_imma_u8(accS, a0, a1, a2, a3, q0, q1);
+                    }
+                });
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) accA[r] += accA2[r];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int u = 2 * mt + r;
+                const uint32_t nw = nrm[u];
+                const float nh = tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
+                const float va = (float)(256 * accA[2 * r] + accA[2 * r + 1]);
+                const float vs = (float)(256 * accS[2 * r] + accS[2 * r + 1]);
+                const float est = fmaf(sc.x, va, -sc.y) + gh * fmaf(sc.z, vs, -sc.w);
+                const bool in = hv && blk * 32 + 8 * u + g < p.n_tok;
+                l[u] = in ? nh * est : -INFINITY;
+            }
+        }
+        // ---- online softmax of head t over this block
+        float bm = fmaxf(fmaxf(l[0], l[1]), fmaxf(l[2], l[3]));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+        if (bm > m_run) {
+            const float fac = tq_exp2((m_run - bm) * kLog2e);   // 0 while the maximum was -inf
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+                acc[i][0] *= fac; acc[i][1] *= fac; acc[i][2] *= fac; acc[i][3] *= fac;
+            }
+            lsum *= fac;
+            m_run = bm;
+        }
+        const float ml2 = m_run * kLog2e;
+        const uint16_t* vn = reinterpret_cast<const uint16_t*>(vb + SEC_AV);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int tok = 8 * u + g;
+            const float e = m_run > -INFINITY ? tq_exp2(fmaf(l[u], kLog2e, -ml2)) : 0.f;
+            lsum += e;
+            const float wt = e * tq_half_val(vn[tok]);
+            const __half hi = __float2half_rn(wt);
+            reinterpret_cast<__half*>(&wst[w][2 * t][0])[tok] = hi;
+            reinterpret_cast<__half*>(&wst[w][2 * t + 1][0])[tok] = __float2half_rn(wt - __half2float(hi));
+        }
+        __syncwarp();
+        // ---- values: B fragments (column g = head g/2, hi / lo) and table-decoded A fragments
+        uint32_t bw[2][2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int hv2 = 0; hv2 < 2; ++hv2) bw[c][hv2] = wst[w][g][8 * c + 4 * hv2 + t];
+        uint32_t W[NW + 1];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(vb + (c * 32 + lane) * 16);
+            W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
+        }
+        W[NW] = 0u;
+#pragma unroll
+        for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+                uint32_t a[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int f = 4 * (2 * kt + (r & 1)) + 2 * c + (r >> 1);
+                    const int bit = f * 2 * BV;
+                    const int wi = bit >> 5, sh = bit & 31;
+                    const uint32_t x = sh >= 7 ? __funnelshift_r(W[wi], W[wi + 1], sh - 7) : W[wi] << (7 - sh);
+                    const uint32_t off = (x & ((uint32_t)(E - 1) << 7)) | lane4;
+                    a[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(lut) + off);
+                }
+                tq_hmma(acc[kt], a[0], a[1], a[2], a[3], bw[c][0], bw[c][1]);
+            }
+        // the stage is consumed: refill it
+        __syncwarp();
+        if (lane == 0) tq_fence_proxy_async();
+        issue(k + NS);
+    }
+    if (!ok) {
+        if (lane == 0) {
+            tq_raise(p.status, TQ_FLAG_TIMEOUT);
+            for (int j = k; j < min(k + NS, nmine); ++j)
+                tq_mbar_wait(&bars[w][j % NS], (uint32_t)(j / NS) & 1u, kWaitLimit);
+        }
+        __syncwarp();
+    }
+    // the 8 lanes of head t hold parts of its sum
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 4);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 8);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 16);
+    if (g == 0) { s_m[w][t] = m_run; s_l[w][t] = lsum; }
+    __syncthreads();
+    float M = s_m[0][t];
+#pragma unroll
+    for (int v = 1; v < kAttnWarps; ++v) M = fmaxf(M, s_m[v][t]);
+    const float f = m_run > -INFINITY ? tq_exp2((m_run - M) * kLog2e) : 0.f;
+    if (hv) {
+#pragma unroll
+        for (int kt = 0; kt < KT; ++kt) {
+            atomicAdd(&s_acc[t][16 * kt + g], f * (acc[kt][0] + acc[kt][1]));
+            atomicAdd(&s_acc[t][16 * kt + 8 + g], f * (acc[kt][2] + acc[kt][3]));
+        }
+    }
+    __syncthreads();
+    const int D = KT * 16;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, i = e % D;
+        p.part[(((size_t)stream * G + h) * p.nsplit + split) * D + i] = s_acc[h][i];
+    }
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float Mh = s_m[0][h], L = 0.f;
+        for (int v = 1; v < kAttnWarps; ++v) Mh = fmaxf(Mh, s_m[v][h]);
+        for (int v = 0; v < kAttnWarps; ++v)
+            if (s_m[v][h] > -INFINITY) L += s_l[v][h] * tq_exp2((s_m[v][h] - Mh) * kLog2e);
+        reinterpret_cast<float2*>(p.part_ml)[((size_t)stream * G + h) * p.nsplit + split] = make_float2(Mh, L);
+    }
+}
+
+// One CTA per query head: the ranges and the exact tail under one maximum M,
+//   out = (Pi^T sum_s e^{m_s - M} part_s + sum_t e^{l_t - M} v_t) / (sum_s e^{m_s - M} l_s + sum_t e^{l_t - M}).
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
+    const int D = p.tv.D, d = p.tv.d, ns = p.nsplit, nt = p.n_tail;
+    const int64_t hq = blockIdx.x;   // stream * g + head
+    const int64_t stream = hq / p.g;
+    extern __shared__ float msm[];
+    float* fs = msm;                       // [ns] split weights, padded to 4 floats
+    float* ft = fs + ((ns + 3) & ~3);      // [n_tail] tail weights, padded to 4 floats
+    float* red = ft + ((nt + 3) & ~3);     // [1024] partial sums, 16-byte aligned
+    float* s_o = red + 1024;               // [256]
+    __shared__ float s_w[kMergeThreads / 32];
+    __shared__ float s_M, s_den;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
+    const float* tl = p.tail_logit + (size_t)hq * nt;
+
+    float mx = -INFINITY;
+    for (int s = tid; s < ns; s += kMergeThreads) {
+        const float2 v = ml[s];
+        if (v.y > 0.f) mx = fmaxf(mx, v.x);
+    }
+    for (int j = tid; j < nt; j += kMergeThreads) mx = fmaxf(mx, tl[j]);
+    mx = tq_warp_max(mx);
+    if (lane == 0) s_w[wid] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        float M = s_w[0];
+        for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, s_w[i]);
+        s_M = M;
+    }
+    __syncthreads();
+    const float M = s_M;
+    float den = 0.f;
+    for (int s = tid; s < ns; s += kMergeThreads) {
+        const float2 v = ml[s];
+        const float f = v.y > 0.f ? __expf(v.x - M) : 0.f;
+        fs[s] = f;
+        den = fmaf(f, v.y, den);
+    }
+    for (int j = tid; j < nt; j += kMergeThreads) {
+        const float f = __expf(tl[j] - M);
+        ft[j] = f;
+        den += f;
+    }
+    den = tq_warp_sum(den);
+    __syncthreads();
+    if (lane == 0) s_w[wid] = den;
+    __syncthreads();
+    if (tid == 0) {
+        float v = 0.f;
+        for (int i = 0; i < kMergeThreads / 32; ++i) v += s_w[i];
+        s_den = v;
+    }
+    // rotated-domain sum over the ranges: thread (group, column quad)
+    const int nq = D / 4, ngrp = kMergeThreads / nq;
+    const int grp = tid / nq, qd = tid % nq;
+    const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+    for (int s = grp; s < ns; s += ngrp) {
+        const float f = fs[s];
+        const float4 v = src[(size_t)s * nq];
+        a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
+    }
+    reinterpret_cast<float4*>(red)[grp * nq + qd] = a;
+    __syncthreads();
+    for (int i = tid; i < D; i += kMergeThreads) {
+        float v = 0.f;
+        for (int q = 0; q < ngrp; ++q) v += red[q * D + i];
+        s_o[i] = v;
+    }
+    __syncthreads();
+    const float inv = 1.f / s_den;
+    // out[j] = (<row j of Pi^T, o> + sum_t f_t v_t[j]) / den: pair (j, half) as in tq_pv's merge
+    const int hl = D / 2;
+    const uint16_t* tv = p.tail_v + (size_t)stream * nt * d;
+    for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
+        const int e = e0 + tid, j = e >> 1, hf = e & 1;
+        const bool valid = e < 2 * d;
+        float acc = 0.f;
+        if (valid) {
+            const float4* rowp = reinterpret_cast<const float4*>(p.piT_v + (size_t)j * D + hf * hl);
+            const float4* op = reinterpret_cast<const float4*>(s_o + hf * hl);
+#pragma unroll 16
+            for (int k = 0; k < hl / 4; ++k) {
+                const float4 w = __ldg(rowp + k), o = op[k];
+                acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
+            }
+            // the tail: the two halves of the pair take alternate tokens
+            for (int tt = hf; tt < nt; tt += 2)
+                acc = fmaf(ft[tt], __uint_as_float((uint32_t)tv[(size_t)tt * d + j] << 16), acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (valid && hf == 0) p.out[(size_t)hq * d + j] = acc * inv;
+    }
+}
+
+template <int BK, int BV>
+cudaError_t launch_split(const AttnParams& p, cudaStream_t st) {
+    constexpr size_t smem = attn_smem<BK, BV>();
+    if (p.tk.block_bytes != 512u * (BK + 1) + 128u || p.tv.block_bytes != 512u * BV + 64u) return cudaErrorInvalidValue;
+    auto kern = k_attn_split<BK, BV>;
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, kAttnWarps * 32, smem, cache, nullptr, nullptr);
+    if (e != cudaSuccess) return e;
+    return tq_launch_pdl(kern, dim3((unsigned)(p.n_streams * p.nsplit)), dim3(kAttnWarps * 32), smem, st, p);
+}
+
+template <int BK>
+cudaError_t launch_bv(const AttnParams& p, cudaStream_t st) {
+    switch (p.tv.B) {
+        case 1: return launch_split<BK, 1>(p, st);
+        case 2: return launch_split<BK, 2>(p, st);
+        case 3: return launch_split<BK, 3>(p, st);
+        case 4: return launch_split<BK, 4>(p, st);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+size_t tq_attn_merge_smem(int nsplit, int n_tail) {
+    return (((size_t)nsplit + 3) / 4 * 4 + ((size_t)n_tail + 3) / 4 * 4 + 1024 + 256) * 4;
+}
+
+cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
+    if (p.tk.D != 128 || p.tk.Mp != 128 || p.tv.D != 128 || p.g < 1 || p.g > 4) return cudaErrorInvalidValue;
+    if (p.nsplit > 0) {   // no compressed tokens: the merge sees only the tail
+        cudaError_t e = cudaErrorInvalidValue;
+        switch (p.tk.B) {
+            case 1: e = launch_bv<1>(p, st); break;
+            case 2: e = launch_bv<2>(p, st); break;
+            case 3: e = launch_bv<3>(p, st); break;
+        }
+        if (e != cudaSuccess) return e;
+    }
+    const size_t msmem = tq_attn_merge_smem(p.nsplit, p.n_tail);
+    if (msmem > 48 * 1024) return cudaErrorInvalidValue;
+    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, msmem, st>>>(p);
+    return cudaGetLastError();
+}

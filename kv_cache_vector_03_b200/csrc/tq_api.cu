@@ -138,6 +138,36 @@ PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
     return w;
 }
 
+// fused attention: the logits prologue's fragments, the exact tail logits, split partials.
+// One CTA per (stream, range) at about two resident CTAs per SM; ranges of at least 4 blocks.
+struct AttnWs { int nsplit, bps; LogitsWs lg; size_t tl, part, ml, total; };
+AttnWs attn_ws(const TqDims& tk, int64_t n_streams, int64_t n_tok, int g, int n_tail) {
+    AttnWs w;
+    w.lg = logits_ws(tk, n_streams, g);
+    const int64_t nb = (n_tok + 31) / 32;
+    int64_t bps = (nb * n_streams + 2 * kNumSms - 1) / (2 * kNumSms);
+    bps = std::max<int64_t>(4, bps);
+    bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
+    w.bps = (int)bps;
+    w.nsplit = (int)((nb + bps - 1) / bps);
+    size_t off = w.lg.total;
+    w.tl = off; off = align_up(off + (size_t)n_streams * g * n_tail * 4);
+    w.part = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * 128 * 4);
+    w.ml = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * 8);
+    w.total = off;
+    return w;
+}
+
+// key codec (qjl = 1, d and m <= 128) and value codec (qjl = 0, the same d) of tq_attention
+int check_attention_codecs(const tq_codec* kc, const tq_codec* vc) {
+    int st = check_codec(kc, true);
+    if (st != TQ_OK) return st;
+    if ((st = check_codec(vc, true)) != TQ_OK) return st;
+    if (!kc->qjl || vc->qjl || kc->d != vc->d) return TQ_ERR_ARG;
+    if (kc->d > 128 || kc->m > 128) return TQ_ERR_UNSUPPORTED;
+    return TQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -346,6 +376,88 @@ int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int6
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_pv(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t tq_attention_workspace_bytes(const tq_codec* kcodec, const tq_codec* vcodec, int64_t n_seq, int n_kv,
+                                    int64_t n_tok, int g, int n_tail) {
+    if (check_attention_codecs(kcodec, vcodec) != TQ_OK) return 0;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0 || g < 1 || g > 4) return 0;
+    return attn_ws(dims_of(kcodec), n_seq * n_kv, n_tok, g, n_tail).total;
+}
+
+int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* packed_k, const void* packed_v,
+                 int64_t n_seq, int n_kv, int64_t n_tok, const void* q, tq_dtype q_dtype, int g, const void* tail_k,
+                 const void* tail_v, int n_tail, float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+    int st = check_attention_codecs(kcodec, vcodec);
+    if (st != TQ_OK) return st;
+    if (g != 1 && g != 2 && g != 4) return TQ_ERR_UNSUPPORTED;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_seq == 0) return TQ_OK;
+    if (n_tok + n_tail == 0) return TQ_ERR_ARG;   // softmax over no tokens
+    if (n_tail > TQ_ATTN_MAX_TAIL) return TQ_ERR_UNSUPPORTED;
+    if (!q || !out || !ws || (n_tok > 0 && (!packed_k || !packed_v)) || (n_tail > 0 && (!tail_k || !tail_v)))
+        return TQ_ERR_ARG;
+    if ((n_tok > 0 && (!aligned(packed_k, 16) || !aligned(packed_v, 16))) || !aligned(out, 4) ||
+        !aligned(ws, 256) || !aligned(q, q_dtype == TQ_F32 ? 4 : 2) ||
+        (n_tail > 0 && (!aligned(tail_k, 2) || !aligned(tail_v, 2))))
+        return TQ_ERR_ARG;
+    if (!std::isfinite(scale)) return TQ_ERR_ARG;
+    const TqDims tk = dims_of(kcodec), tv = dims_of(vcodec);
+    const int64_t n_streams = n_seq * n_kv;
+    if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
+    const AttnWs W = attn_ws(tk, n_streams, n_tok, g, n_tail);
+    if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
+    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    const uint8_t* kprep = static_cast<const uint8_t*>(kcodec->prep);
+    const TqPrepLayout L = tq_prep_layout(tk);
+
+    // 1. query fragments and exact tail logits: the logits prologue with no compressed tokens
+    LogitsParams lp;
+    lp.packed = nullptr;
+    lp.q = q; lp.q_dtype = q_dtype;
+    lp.tail = static_cast<const uint16_t*>(tail_k);
+    lp.out = reinterpret_cast<float*>(wsb + W.tl);
+    lp.piT = reinterpret_cast<const float*>(kprep + L.piT);
+    lp.sT = reinterpret_cast<const float*>(kprep + L.sT);
+    lp.pih = reinterpret_cast<const uint16_t*>(kprep + L.pih);
+    lp.pil = reinterpret_cast<const uint16_t*>(kprep + L.pil);
+    lp.mh = reinterpret_cast<const uint16_t*>(kprep + L.mh);
+    lp.ml = reinterpret_cast<const uint16_t*>(kprep + L.ml);
+    lp.qfrag = reinterpret_cast<uint32_t*>(wsb + W.lg.qfrag);
+    lp.qscale = reinterpret_cast<float*>(wsb + W.lg.qscale);
+    lp.status = static_cast<uint32_t*>(ws);
+    lp.n_seq = n_seq; lp.n_tok = 0; lp.nb = 0;
+    lp.n_kv = n_kv; lp.g = g; lp.ntiles = 1; lp.n_tail = n_tail;
+    lp.scale = scale;
+    lp.kappa = (float)(std::sqrt(M_PI / 2.0) / kcodec->m);
+    lp.n_heads_valid = n_streams * g;
+    lp.t = tk;
+    if ((st = codebook_consts(kcodec, &lp.cb)) != TQ_OK) return st;
+
+    // 2. + 3. split pass over the compressed keys and values, merge with the tail
+    AttnParams p;
+    p.packed_k = static_cast<const uint8_t*>(packed_k);
+    p.packed_v = static_cast<const uint8_t*>(packed_v);
+    p.qfrag = lp.qfrag;
+    p.qscale = lp.qscale;
+    p.tail_logit = lp.out;
+    p.tail_v = static_cast<const uint16_t*>(tail_v);
+    p.piT_v = reinterpret_cast<const float*>(static_cast<const uint8_t*>(vcodec->prep) + tq_prep_layout(tv).piT);
+    p.out = out;
+    p.part = reinterpret_cast<float*>(wsb + W.part);
+    p.part_ml = reinterpret_cast<float*>(wsb + W.ml);
+    p.status = static_cast<uint32_t*>(ws);
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
+    p.g = g; p.nsplit = p.nb > 0 ? W.nsplit : 0; p.blocks_per_split = W.bps; p.n_tail = n_tail;
+    p.tk = tk; p.tv = tv;
+    if ((st = codebook_consts(vcodec, &p.cbv)) != TQ_OK) return st;
+
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    cudaError_t e = tq_launch_logits_prologue(lp, cs);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    return cuda_status(tq_launch_attention(p, cs));
 }
 
 int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,

@@ -312,6 +312,24 @@ struct TopkParams {
     TqDims t;
 };
 
+struct AttnParams {
+    const uint8_t* packed_k;      // key blocks (qjl = 1), d <= 128, m <= 128
+    const uint8_t* packed_v;      // value blocks (qjl = 0), same d
+    const uint32_t* qfrag;        // query fragments of the key codec (logits prologue)
+    const float* qscale;          // per-head constants (attention scale folded in)
+    const float* tail_logit;      // [stream * g + head][n_tail] exact tail logits (prologue)
+    const uint16_t* tail_v;       // bf16 [stream][n_tail][d] full-precision recent values
+    const float* piT_v;           // prepared Pi^T of the value codec, fp32 [D][D]
+    float* out;                   // fp32 [stream * g + head][d]
+    float* part;                  // [stream * g + head][nsplit][D] rotated-domain partial sums
+    float* part_ml;               // [stream * g + head][nsplit][2]: max, sum of weights
+    uint32_t* status;
+    int64_t n_streams, n_tok, nb;
+    int g, nsplit, blocks_per_split, n_tail;
+    TqDims tk, tv;
+    TqCodebookConsts cbv;         // value codebook (binary16 decode table)
+};
+
 struct DequantParams {
     const uint8_t* packed;
     float* out;
@@ -331,4 +349,5 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st);
 cudaError_t tq_launch_dequant(const DequantParams& p, cudaStream_t st);
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st);
+cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);

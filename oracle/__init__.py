@@ -185,6 +185,31 @@ def pv(idx, nhat, pi, c, P) -> np.ndarray:
     return out
 
 
+def attention(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale: float,
+              tail_k=None, tail_v=None) -> np.ndarray:
+    """Decode attention of the query heads q [nh, d] of one kv stream, in fp64:
+    softmax over [estimated logits of the compressed keys, exact logits of the tail keys]
+    times [reconstructed compressed values, tail values] (a2a-mcp.org "What is TurboQuant":
+    scores from the codes, the weighted sum over the dequantized values; blog.hotdry.top
+    "TurboQuant vector-search compression", engineering configuration list: the recent
+    tokens kept at full precision). Either part may be empty (None or zero tokens)."""
+    q = _f64(q)
+    q = q.reshape(-1, q.shape[-1])
+    lgs, vals = [], []
+    if k_idx is not None and len(k_idx):
+        lgs.append(logits(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, q, qjl=True, scale=scale))
+        vals.append(reconstruct(v_idx, None, v_nhat, None, pi_v, None, c_v, qjl=False))
+    if tail_k is not None and len(tail_k):
+        lgs.append(exact_dot(tail_k, q, scale))
+        vals.append(_f64(tail_v))
+    if not lgs:
+        raise ValueError("attention over no tokens")
+    lg = np.concatenate(lgs, axis=1)
+    w = np.exp(lg - lg.max(axis=1, keepdims=True))
+    w /= w.sum(axis=1, keepdims=True)
+    return w @ np.concatenate(vals, axis=0)
+
+
 def topk(idx, sbit, nhat, ghat, pi, s, c, q, k: int, qjl: bool = True):
     lib = _load()
     idx = _u8(idx)

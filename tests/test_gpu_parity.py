@@ -284,6 +284,123 @@ def test_pv_one_hot_and_uniform():
     assert np.max(np.abs(got[1] - vh[123])) <= TOL * nhat[0, 123]
 
 
+# ----------------------------------------------------------------------------- fused attention
+def _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale):
+    torch = torch_cuda()
+    m = tq()
+    out = torch.full((n_seq, n_kv * g, kc.c.d), float("nan"), dtype=torch.float32, device="cuda")
+    ws = m.workspace(m.tq_attention_workspace_bytes(kc, vc, n_seq, n_kv, n_tok, g, n_tail))
+    m.tq_attention(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale, out, ws)
+    torch.cuda.synchronize()
+    assert m.tq_get_status(ws) == m.TQ_OK
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _normal_stream(seed, seq, head, n):
+    """N(0, I) vectors as bf16 bits [n, 128] (the value law, drawn under another seed)."""
+    return ti.value_stream(head, n, cfg_id=seed * 1000 + seq)
+
+
+@pytest.mark.parametrize("Bk,Bv,g,n_seq,n_kv,n_tok,n_tail,law,qs", [
+    (2, 3, 4, 2, 3, 301, 5, "normal", 1.0),      # several streams, ragged last block
+    (3, 4, 4, 1, 2, 5000, 128, "normal", 1.0),   # many ranges per stream, a 128-token tail
+    (1, 2, 1, 1, 2, 64, 0, "normal", 1.0),       # no tail
+    (2, 4, 2, 1, 2, 0, 33, "normal", 1.0),       # tail only
+    (3, 3, 4, 1, 1, 1000, 1, "normal", 8.0),     # peaked softmax: the running maximum moves
+    (2, 1, 4, 3, 1, 33, 7, "normal", 1.0),       # 1-bit values, a block of one valid token
+    (3, 4, 4, 1, 2, 3000, 128, "c2", 1.0),       # the decode key law (outlier channels, long keys)
+])
+def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
+    """softmax(scale q . K) . V against the oracle composition on the same codes.
+
+    Bound, from the step tolerances: a logit error of at most dl moves every softmax weight by
+    a factor within exp(+-2 dl), so |do| <= (expm1(2 dl) + TOL) sum_t w_t |v_t| with the P.V
+    tolerance TOL. dl is the logit error tq_logits makes on the same codes and queries (the
+    fused kernel evaluates the same fragments with the same arithmetic); it is itself held to
+    the logits tolerance."""
+    d = m = 128
+    pik, sk, piv = ti.haar_rotation(d, 95), ti.gaussian_sketch(m, d, 96), ti.haar_rotation(d, 97)
+    n = n_tok + n_tail
+    if law == "c2":
+        keys = np.stack([np.stack([ti.key_stream(4, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    else:
+        keys = np.stack([np.stack([_normal_stream(51, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    vals = np.stack([np.stack([_normal_stream(61, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    kc = make_codec(d, m, Bk, True, pik, sk)
+    vc = make_codec(d, 0, Bv, False, piv, None)
+    S = n_seq * n_kv
+    pk = pvv = None
+    if n_tok:
+        pk, _ = gpu_quantize(kc, to_dev_bf16(np.ascontiguousarray(keys[:, :, :n_tok]).reshape(-1, d)), S, n_tok)
+        pvv, _ = gpu_quantize(vc, to_dev_bf16(np.ascontiguousarray(vals[:, :, :n_tok]).reshape(-1, d)), S, n_tok)
+    tk = to_dev_bf16(np.ascontiguousarray(keys[:, :, n_tok:])) if n_tail else None
+    tv = to_dev_bf16(np.ascontiguousarray(vals[:, :, n_tok:])) if n_tail else None
+    qb = ti.decode_queries(12, n_seq, n_kv * g)
+    scale = qs / math.sqrt(d)
+    got = _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)
+    lg = _logits_gpu(kc, pk, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)
+    if n_tok:
+        kidx, ksb, knh, kgh = unpack(kc, pk, S, n_tok)
+        vidx, vnh = unpack(vc, pvv, S, n_tok)
+    c_k, _ = _cb(d, Bk)
+    c_v, _ = _cb(d, Bv)
+    q = ti.bf16_to_f64(qb)
+    kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
+    worst = 0.0
+    for sq in range(n_seq):
+        for h in range(n_kv):
+            st = sq * n_kv + h
+            qh = q[sq, h * g:(h + 1) * g]
+            if n_tok:
+                a = dict(k_idx=kidx[st], k_sbit=ksb[st], k_nhat=knh[st], k_ghat=kgh[st], pi_k=pik, s_k=sk, c_k=c_k,
+                         v_idx=vidx[st], v_nhat=vnh[st], pi_v=piv, c_v=c_v)
+                lo = oracle.logits(kidx[st], ksb[st], knh[st], kgh[st], pik, sk, c_k, qh, qjl=True, scale=scale)
+                vn = vnh[st]
+            else:
+                a = dict(k_idx=None, k_sbit=None, k_nhat=None, k_ghat=None, pi_k=None, s_k=None, c_k=None,
+                         v_idx=None, v_nhat=None, pi_v=None, c_v=None)
+                lo, vn = np.zeros((g, 0)), np.zeros(0)
+            tkh, tvh = (kf[sq, h, n_tok:], vf[sq, h, n_tok:]) if n_tail else (None, None)
+            want = oracle.attention(**a, q=qh, scale=scale, tail_k=tkh, tail_v=tvh)
+            L = np.concatenate([lo, oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)], axis=1)
+            w = np.exp(L - L.max(axis=1, keepdims=True))
+            w /= w.sum(axis=1, keepdims=True)
+            vnorm = np.concatenate([vn, np.linalg.norm(vf[sq, h, n_tok:], axis=1)])
+            xn = np.linalg.norm(kf[sq, h], axis=1)
+            dl_norm = np.abs(lg[sq, h * g:(h + 1) * g] - L) / (scale * np.linalg.norm(qh, axis=1)[:, None] * xn)
+            assert dl_norm.max() <= TOL
+            dl = np.abs(lg[sq, h * g:(h + 1) * g] - L).max(axis=1)
+            err = np.max(np.abs(got[sq, h * g:(h + 1) * g] - want), axis=1) / (w @ vnorm)
+            assert np.all(np.isfinite(got[sq, h * g:(h + 1) * g]))
+            bound = TOL + np.expm1(2 * dl) + 1e-5
+            assert np.all(err <= bound), f"stream {st}: normalised error {err} above {bound}"
+            worst = max(worst, float(err.max()))
+    return worst
+
+
+def test_attention_rejects_unsupported():
+    torch = torch_cuda()
+    m = tq()
+    d = 128
+    kc = make_codec(d, d, 2, True, ti.haar_rotation(d, 1), ti.gaussian_sketch(d, d, 2))
+    vc = make_codec(d, 0, 3, False, ti.haar_rotation(d, 3), None)
+    q = torch.zeros((1, 8, d), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((1, 8, d), dtype=torch.float32, device="cuda")
+    pk = torch.zeros(kc.packed_bytes(1, 64), dtype=torch.uint8, device="cuda")
+    pv_ = torch.zeros(vc.packed_bytes(1, 64), dtype=torch.uint8, device="cuda")
+    ws = m.workspace(1 << 20)
+    with pytest.raises(m.TQError) as e:   # g = 8 is outside the fused kernel's head tile
+        m.tq_attention(kc, vc, pk, pv_, 1, 1, 64, q, 8, None, None, 0, 1.0, out, ws)
+    assert e.value.status == m.TQ_ERR_UNSUPPORTED
+    with pytest.raises(m.TQError) as e:   # a softmax over no tokens
+        m.tq_attention(kc, vc, pk, pv_, 1, 1, 0, q, 4, None, None, 0, 1.0, out, ws)
+    assert e.value.status == m.TQ_ERR_ARG
+    with pytest.raises(m.TQError) as e:   # key and value codecs swapped
+        m.tq_attention(vc, kc, pk, pv_, 1, 1, 64, q, 4, None, None, 0, 1.0, out, ws)
+    assert e.value.status == m.TQ_ERR_ARG
+    assert m.tq_attention_workspace_bytes(kc, vc, 1, 1, 64, 8, 0) == 0
+
+
 # ----------------------------------------------------------------------------- reconstruction
 @pytest.mark.parametrize("qjl,B", [(True, 2), (True, 3), (False, 4)])
 def test_dequantize_reconstruction(qjl, B):

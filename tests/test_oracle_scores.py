@@ -95,6 +95,58 @@ def test_pv_special_cases_and_rotate_once():
     assert np.allclose(o[0], acc @ pi.astype(np.float32).astype(np.float64), rtol=1e-11, atol=1e-12)
 
 
+def _attention_setup(nt=200, n_tail=7, d=64, seed=20):
+    c_k, t_k, _, _ = oracle.codebook(d, 2)
+    c_v, t_v, _, _ = oracle.codebook(d, 3)
+    pi_k, s_k = ti.haar_rotation(d, seed), ti.gaussian_sketch(d, d, seed + 1)
+    pi_v = ti.haar_rotation(d, seed + 2)
+    rng = np.random.default_rng(seed + 3)
+    keys = rng.standard_normal((nt + n_tail, d)) * np.exp(rng.uniform(0, 2, nt + n_tail))[:, None]
+    vals = rng.standard_normal((nt + n_tail, d))
+    kq = oracle.quantize(keys[:nt], pi_k, s_k, c_k, t_k, 2, qjl=True)
+    vq = oracle.quantize(vals[:nt], pi_v, None, c_v, t_v, 3, qjl=False)
+    return dict(k_idx=kq.idx, k_sbit=kq.sbit, k_nhat=kq.nhat, k_ghat=kq.ghat, pi_k=pi_k, s_k=s_k, c_k=c_k,
+                v_idx=vq.idx, v_nhat=vq.nhat, pi_v=pi_v, c_v=c_v), keys, vals
+
+
+def test_attention_composes_logits_and_pv():
+    # no tail: the fused result is P.V of the estimated logits (two separately pinned functions)
+    a, keys, vals = _attention_setup(n_tail=0)
+    qs = np.random.default_rng(21).standard_normal((4, 64))
+    o = oracle.attention(**a, q=qs, scale=0.125)
+    P = oracle.logits(a["k_idx"], a["k_sbit"], a["k_nhat"], a["k_ghat"], a["pi_k"], a["s_k"], a["c_k"], qs,
+                      qjl=True, scale=0.125)
+    want = oracle.pv(a["v_idx"], a["v_nhat"], a["pi_v"], a["c_v"], P)
+    assert np.allclose(o, want, rtol=1e-5, atol=1e-6 * np.abs(want).max())
+
+
+def test_attention_uniform_and_one_hot_tail():
+    a, keys, vals = _attention_setup()
+    nt, d = 200, 64
+    vh = oracle.reconstruct(a["v_idx"], None, a["v_nhat"], None, a["pi_v"], None, a["c_v"], qjl=False)
+    allv = np.concatenate([vh, vals[nt:]])
+    # q = 0: every logit is 0 -> the mean over compressed and tail values together
+    o = oracle.attention(**a, q=np.zeros((1, d)), scale=1.0, tail_k=keys[nt:], tail_v=vals[nt:])
+    assert np.allclose(o[0], allv.mean(0), rtol=1e-12, atol=1e-12)
+    # a tail key far longer than every other, the query along it: all weight on that token
+    tk = keys[nt:].copy()
+    tk[3] = 1e3 * np.abs(keys).max() * tk[3] / np.linalg.norm(tk[3])
+    o = oracle.attention(**a, q=(tk[3] / np.linalg.norm(tk[3]))[None], scale=1.0, tail_k=tk, tail_v=vals[nt:])
+    assert np.allclose(o[0], vals[nt + 3], rtol=1e-12, atol=1e-12)
+    # tail only and compressed only are the two halves of the same softmax
+    qs = np.random.default_rng(22).standard_normal((2, d)) * 0.1
+    full = oracle.attention(**a, q=qs, scale=1.0, tail_k=keys[nt:], tail_v=vals[nt:])
+    none = {k: None for k in a}
+    only_tail = oracle.attention(**none, q=qs, scale=1.0, tail_k=keys[nt:], tail_v=vals[nt:])
+    only_comp = oracle.attention(**a, q=qs, scale=1.0)
+    assert not np.allclose(full, only_tail) and not np.allclose(full, only_comp)
+    lt = qs @ keys[nt:].T
+    lc = oracle.logits(a["k_idx"], a["k_sbit"], a["k_nhat"], a["k_ghat"], a["pi_k"], a["s_k"], a["c_k"], qs,
+                       qjl=True)
+    zt, zc = np.exp(lt).sum(1, keepdims=True), np.exp(lc).sum(1, keepdims=True)
+    assert np.allclose(full, (zt * only_tail + zc * only_comp) / (zt + zc), rtol=1e-12, atol=1e-12)
+
+
 def test_topk_matches_full_sort():
     c, t, pi, s, x, q = _setup(n=500)
     qs = np.random.default_rng(7).standard_normal((6, 64))
