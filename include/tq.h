@@ -161,7 +161,8 @@ int tq_pv(const tq_codec* codec, const void* packed_v, int64_t n_seq, int n_kv, 
  *   q        device [n_seq, n_kv * g, d], fp32 or bf16; query head j reads kv-head j / g.
  *   g        query heads per kv-head, 1, 2 or 4 (else TQ_ERR_UNSUPPORTED).
  *   tail_k, tail_v  device bf16 [n_seq, n_kv, n_tail, d] recent keys and values, the
- *            tokens that follow the compressed ones; NULL with n_tail = 0.
+ *            tokens that follow the compressed ones (tail_v 8-byte aligned); NULL with
+ *            n_tail = 0.
  *            n_tail <= TQ_ATTN_MAX_TAIL, else TQ_ERR_UNSUPPORTED.
  *   out      device fp32 [n_seq, n_kv * g, d].
  *   ws       tq_attention_workspace_bytes(kcodec, vcodec, n_seq, n_kv, n_tok, g, n_tail) bytes,

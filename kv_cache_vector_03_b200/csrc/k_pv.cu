@@ -4,15 +4,15 @@
 //   o_h = sum_t w_t |v_t| Pi^T c[idx_t] = Pi^T ( sum_t w_t |v_t| c[idx_t] )
 // so the weighted sum is accumulated in the rotated domain and rotated back once.
 //
-// Kernel 1 (split): one CTA of 4 warps per (stream, block range); warp w takes blocks
-// w, w + 4, ... of the range. Each warp keeps a ring of NS stages in shared memory: the packed
+// Kernel 1 (split): one CTA of 8 warps per (stream, block range); warp w takes blocks
+// w, w + 8, ... of the range. Each warp keeps a ring of NS stages in shared memory: the packed
 // 32-token block arrives by a bulk copy (TMA engine, mbarrier completion) and its P values by
 // 4-byte asynchronous copies. Per block and head the warp updates a running maximum (online
 // softmax: a new maximum rescales the accumulators), computes one exp per (head, token) and
 // stages the weights exp(P - m) |v| as fp16 hi + lo columns. The codes are dequantized
 // straight into fp16 MMA A fragments (rows = coordinates, K = tokens) through a per-lane
 // table that maps a 2B-bit field (two tokens' codes of one coordinate) to a half2 of
-// centroids, and multiplied on the tensor cores. The 4 warps meet at the CTA's maximum;
+// centroids, and multiplied on the tensor cores. The 8 warps meet at the CTA's maximum;
 // partial sums, maxima and denominators go to the workspace.
 // Kernel 2 (merge): one CTA per query head combines the partials (log-sum-exp rescale) and
 // rotates by Pi^T.
@@ -20,8 +20,8 @@
 
 namespace {
 
-constexpr int kPvWarps = 4;
-constexpr int kPvNS = 4;              // ring stages per warp
+constexpr int kPvWarps = 8;
+constexpr int kPvNS = 3;              // ring stages per warp
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kWCol = 20;             // words per staged weight column (16 used; 20 spreads the banks)
 
@@ -32,7 +32,7 @@ constexpr size_t pv_smem_bytes() {
 }
 
 template <int B, int KT, int NT>  // KT = D/16 coordinate tiles, NT = n-tiles of 4 heads
-__global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
+__global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvParams p) {
     constexpr int NS = kPvNS;
     constexpr int E = 1 << (2 * B);          // table entries
     constexpr int CH = KT * B / 8;           // 16-byte chunks per lane per block (D*B/128)
@@ -59,9 +59,10 @@ __global__ void __launch_bounds__(kPvWarps * 32) k_pv_split(PvParams p) {
     const float* Pst = p.P + (size_t)stream * G * p.n_tok;
     const uint8_t* sbase = p.packed + (size_t)stream * p.nb * BBYTES;
 
-    for (int e = threadIdx.x; e < E * 32; e += blockDim.x) {
-        const int ent = e >> 5;
-        lut[e] = p.cb.lut_half[ent & ((1 << B) - 1)] | (p.cb.lut_half[ent >> B] << 16);
+    for (int e = threadIdx.x; e < E * 8; e += blockDim.x) {   // 32 equal words per entry
+        const int ent = e >> 3;
+        const uint32_t v = p.cb.lut_half[ent & ((1 << B) - 1)] | (p.cb.lut_half[ent >> B] << 16);
+        reinterpret_cast<uint4*>(lut)[e] = make_uint4(v, v, v, v);
     }
     for (int e = threadIdx.x; e < HP * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
     if (threadIdx.x < HP) s_l[threadIdx.x] = 0.f;

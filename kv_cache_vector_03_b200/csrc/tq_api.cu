@@ -125,7 +125,7 @@ struct PvWs { int nsplit, bps; size_t part, ml, total; };
 PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
     PvWs w;
     const int64_t nb = (n_tok + 31) / 32;
-    int64_t bps = (nb * n_streams + 4 * kNumSms - 1) / (4 * kNumSms);
+    int64_t bps = (nb * n_streams + 2 * kNumSms - 1) / (2 * kNumSms);   // about two CTAs per SM
     if (bps < 8) bps = 8;
     if (bps > nb) bps = nb;
     if (bps < 1) bps = 1;
@@ -139,14 +139,15 @@ PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
 }
 
 // fused attention: the logits prologue's fragments, the exact tail logits, split partials.
-// One CTA per (stream, range) at about two resident CTAs per SM; ranges of at least 4 blocks.
+// One CTA per (stream, range) at about two resident CTAs per SM; ranges of at least 8 blocks
+// (one per warp).
 struct AttnWs { int nsplit, bps; LogitsWs lg; size_t tl, part, ml, total; };
 AttnWs attn_ws(const TqDims& tk, int64_t n_streams, int64_t n_tok, int g, int n_tail) {
     AttnWs w;
     w.lg = logits_ws(tk, n_streams, g);
     const int64_t nb = (n_tok + 31) / 32;
     int64_t bps = (nb * n_streams + 2 * kNumSms - 1) / (2 * kNumSms);
-    bps = std::max<int64_t>(4, bps);
+    bps = std::max<int64_t>(8, bps);
     bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
     w.bps = (int)bps;
     w.nsplit = (int)((nb + bps - 1) / bps);
@@ -400,7 +401,7 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
         return TQ_ERR_ARG;
     if ((n_tok > 0 && (!aligned(packed_k, 16) || !aligned(packed_v, 16))) || !aligned(out, 4) ||
         !aligned(ws, 256) || !aligned(q, q_dtype == TQ_F32 ? 4 : 2) ||
-        (n_tail > 0 && (!aligned(tail_k, 2) || !aligned(tail_v, 2))))
+        (n_tail > 0 && (!aligned(tail_k, 2) || !aligned(tail_v, 8))))
         return TQ_ERR_ARG;
     if (!std::isfinite(scale)) return TQ_ERR_ARG;
     const TqDims tk = dims_of(kcodec), tv = dims_of(vcodec);

@@ -346,7 +346,6 @@ def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
     c_v, _ = _cb(d, Bv)
     q = ti.bf16_to_f64(qb)
     kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
-    worst = 0.0
     for sq in range(n_seq):
         for h in range(n_kv):
             st = sq * n_kv + h
@@ -374,8 +373,8 @@ def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
             assert np.all(np.isfinite(got[sq, h * g:(h + 1) * g]))
             bound = TOL + np.expm1(2 * dl) + 1e-5
             assert np.all(err <= bound), f"stream {st}: normalised error {err} above {bound}"
-            worst = max(worst, float(err.max()))
-    return worst
+            print(f"attention stream {st}: normalised error {err.max():.2e}, bound {bound.min():.2e}, "
+                  f"logit error {dl_norm.max():.2e}")
 
 
 def test_attention_rejects_unsupported():
