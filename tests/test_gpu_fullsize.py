@@ -1,7 +1,8 @@
 """GPU parity at the workloads' full sizes, in the launch configurations the benchmark uses,
 checked against the oracle on sampled outputs (tolerances as in test_gpu_parity.py).
 
-  c2: Llama-3.1-8B-shaped decode, 8 kv-heads x 32768 tokens (last 128 kept in bf16), b = 4, 3
+  c2: Llama-3.1-8B-shaped decode, 8 kv-heads x 32768 tokens (last 128 kept in bf16), b = 4, 3;
+      also fused with the values (tq_attention, b-bit value cache)
   c3: values at 128K context, 8 x 131072, MSE-only 3 and 4 bits, P ~ N(0, 4), 32 q-heads
   c4: batched decode, 64 sequences x 8 kv-heads x 8192 tokens, b = 3, 32 q-heads per sequence
   c5: vector search, 1,000,000 x d=200 database, 10,000 queries, b = 2 and 4, top-10
@@ -15,7 +16,7 @@ import oracle
 import tq_inputs as ti
 from gpu_helpers import (TOL, compare_codes, gpu_quantize, make_codec, to_dev_bf16, to_dev_f32, torch_cuda, tq,
                          unpack)
-from test_gpu_parity import _check_logits, _check_pv, _logits_gpu, _pv_gpu, _topk_gpu, check_topk
+from test_gpu_parity import _attention_gpu, _check_logits, _check_pv, _logits_gpu, _pv_gpu, _topk_gpu, check_topk
 
 pytestmark = pytest.mark.gpu
 RNG = np.random.default_rng(2026)
@@ -57,6 +58,51 @@ def test_c2_llama_decode(b):
         _check_logits(got[h * g:(h + 1) * g, samp], want, qh, np.linalg.norm(kf[h, samp], axis=1), 1.0 / math.sqrt(d))
         wt = oracle.exact_dot(kf[h, n_tok:], qh, 1.0 / math.sqrt(d))
         _check_logits(got[h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[h, n_tok:], axis=1), 1.0 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("b", [4, 3])
+def test_c2_fused_attention(b):
+    """The c2 decode step fused: keys at b bits (b - 1 MSE + QJL), values at b bits (MSE), the last
+    128 tokens in bf16. Two kv-heads are checked against the oracle composition over all 32768
+    tokens, under the bound of test_gpu_parity.test_attention (P.V tolerance plus expm1(2 dl)
+    for the logit error dl tq_logits makes on the same codes)."""
+    d = m = 128
+    n_kv, n_all, n_tail, g = 8, 32768, 128, 4
+    n_tok = n_all - n_tail
+    pik, sk, piv = ti.C2.pi(), ti.C2.s(), ti.C3.pi()
+    keys = np.stack([ti.key_stream(2, 0, h, n_all) for h in range(n_kv)])
+    vals = np.stack([ti.value_stream(h, n_all) for h in range(n_kv)])
+    qb = ti.decode_queries(2, 1, n_kv * g)
+    kc = make_codec(d, m, b - 1, True, pik, sk)
+    vc = make_codec(d, 0, b, False, piv, None)
+    pk, st = gpu_quantize(kc, to_dev_bf16(keys), n_kv, n_tok, stride=n_all * d)
+    assert st == tq().TQ_OK
+    pvv, st = gpu_quantize(vc, to_dev_bf16(vals), n_kv, n_tok, stride=n_all * d)
+    assert st == tq().TQ_OK
+    tk = to_dev_bf16(np.ascontiguousarray(keys[:, n_tok:]))
+    tv = to_dev_bf16(np.ascontiguousarray(vals[:, n_tok:]))
+    scale = 1.0 / math.sqrt(d)
+    got = _attention_gpu(kc, vc, pk, pvv, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)[0]
+    lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
+    kidx, ksb, knh, kgh = unpack(kc, pk, n_kv, n_tok)
+    vidx, vnh = unpack(vc, pvv, n_kv, n_tok)
+    c_k, _ = _cb(d, b - 1)
+    c_v, _ = _cb(d, b)
+    q = ti.bf16_to_f64(qb)[0]
+    kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
+    for h in (0, 5):
+        qh = q[h * g:(h + 1) * g]
+        want = oracle.attention(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, vidx[h], vnh[h], piv, c_v, qh, scale,
+                                tail_k=kf[h, n_tok:], tail_v=vf[h, n_tok:])
+        lo = oracle.logits(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, qh, qjl=True, scale=scale)
+        L = np.concatenate([lo, oracle.exact_dot(kf[h, n_tok:], qh, scale)], axis=1)
+        w = np.exp(L - L.max(axis=1, keepdims=True))
+        w /= w.sum(axis=1, keepdims=True)
+        vnorm = np.concatenate([vnh[h], np.linalg.norm(vf[h, n_tok:], axis=1)])
+        dl = np.abs(lg[h * g:(h + 1) * g] - L).max(axis=1)
+        err = np.max(np.abs(got[h * g:(h + 1) * g] - want), axis=1) / (w @ vnorm)
+        assert np.all(np.isfinite(got[h * g:(h + 1) * g]))
+        assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), f"kv-head {h}: {err}"
 
 
 @pytest.mark.parametrize("B", [3, 4])
