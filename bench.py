@@ -418,6 +418,15 @@ def extra_workloads(torch, tq, ti, gen, peaks):
             "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA-graph replays of 12 calls"}
+        # sparse values: blocks whose weights are all below 1e-4 of the running maximum skip
+        # their values (the bytes still stream: the value block shares the key block's stage)
+        ms = time_graph(torch, lambda i: tq.tq_attention(codec, vcodec, packs[i % copies], vpacks[i % copies], 1, n_kv,
+                                                         n_tok, q, 4, tail, tail_v, n_tail, 1.0 / math.sqrt(d), ao,
+                                                         aws, v_skip=1e-4), copies)
+        out[f"c2_llama8b_decode_attention_k{b}v{b}_sparse_v1e-4"] = {
+            "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "timing": "CUDA-graph replays of 12 calls"}
         del keys, packs, vals, vpacks
     # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
     n_kv, n_tok, g = 8, 131072, 4

@@ -164,6 +164,13 @@ int tq_pv(const tq_codec* codec, const void* packed_v, int64_t n_seq, int n_kv, 
  *            tokens that follow the compressed ones (tail_v 8-byte aligned); NULL with
  *            n_tail = 0.
  *            n_tail <= TQ_ATTN_MAX_TAIL, else TQ_ERR_UNSUPPORTED.
+ *   v_skip   sparse values (ai-coding.wiselychen.com "Google TurboQuant KV-cache compression",
+ *            community extensions: "Sparse V" skips the dequantization of low-weight values),
+ *            in [0, 1]: a 32-token block of compressed values is skipped when every softmax
+ *            weight in it, relative to the largest weight seen so far, is below v_skip; the
+ *            softmax denominator still counts them. 0 = dense. A skipped token's final
+ *            relative weight is below v_skip too, so the result differs from the dense one by
+ *            at most the weight mass of the tokens whose relative weight is below v_skip.
  *   out      device fp32 [n_seq, n_kv * g, d].
  *   ws       tq_attention_workspace_bytes(kcodec, vcodec, n_seq, n_kv, n_tok, g, n_tail) bytes,
  *            256-byte aligned. n_tok + n_tail = 0 is TQ_ERR_ARG (a softmax over no tokens). */
@@ -172,8 +179,8 @@ size_t tq_attention_workspace_bytes(const tq_codec* kcodec, const tq_codec* vcod
                                     int64_t n_tok, int g, int n_tail);
 int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* packed_k, const void* packed_v,
                  int64_t n_seq, int n_kv, int64_t n_tok, const void* q, tq_dtype q_dtype, int g,
-                 const void* tail_k, const void* tail_v, int n_tail, float scale, float* out, void* ws,
-                 size_t ws_bytes, void* stream);
+                 const void* tail_k, const void* tail_v, int n_tail, float scale, float v_skip, float* out,
+                 void* ws, size_t ws_bytes, void* stream);
 
 /* Top-k inner-product search over a packed database (a2a-mcp.org, benchmark section:
  * GloVe d=200 recall; scores are the same estimator as tq_logits with scale 1).

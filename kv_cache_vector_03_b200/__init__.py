@@ -51,7 +51,7 @@ _sig = {
     "tq_logits_noalloc": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P]),
     "tq_pv": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _P, _P, _SZ, _P]),
     "tq_attention_workspace_bytes": (_SZ, [_CP, _CP, _I64, _I, _I64, _I, _I]),
-    "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _P, _P, _SZ, _P]),
+    "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _F, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "tq_dequantize": (_I, [_CP, _P, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_reset_status": (_I, [_P, _P]),
@@ -179,10 +179,10 @@ def tq_attention_workspace_bytes(kcodec: Codec, vcodec: Codec, n_seq, n_kv, n_to
 
 
 def tq_attention(kcodec: Codec, vcodec: Codec, packed_k, packed_v, n_seq, n_kv, n_tok, q, g, tail_k, tail_v, n_tail,
-                 scale, out, ws, stream=None):
+                 scale, out, ws, v_skip=0.0, stream=None):
     return _check("tq_attention", lib.tq_attention(kcodec.ref, vcodec.ref, _ptr(packed_k), _ptr(packed_v), n_seq, n_kv,
                                                    n_tok, _ptr(q), _dtype(q), g, _ptr(tail_k), _ptr(tail_v), n_tail,
-                                                   scale, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+                                                   scale, v_skip, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=None):

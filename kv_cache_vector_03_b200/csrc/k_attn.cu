@@ -189,12 +189,26 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
         }
         const float ml2 = m_run * kLog2e;
         const uint16_t* vn = reinterpret_cast<const uint16_t*>(vb + SEC_AV);
+        float ev[4];
+        bool low = true;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            ev[u] = m_run > -INFINITY ? tq_exp2(fmaf(l[u], kLog2e, -ml2)) : 0.f;
+            lsum += ev[u];
+            low = low && ev[u] < p.v_skip;
+        }
+        // sparse values: every weight of the block is below v_skip (relative to the running
+        // maximum, so also to the final one): the softmax sum keeps them, the values are skipped
+        if (__all_sync(0xffffffffu, low)) {
+            __syncwarp();
+            if (lane == 0) tq_fence_proxy_async();
+            issue(k + NS);
+            continue;
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int tok = 8 * u + g;
-            const float e = m_run > -INFINITY ? tq_exp2(fmaf(l[u], kLog2e, -ml2)) : 0.f;
-            lsum += e;
-            const float wt = e * tq_half_val(vn[tok]);
+            const float wt = ev[u] * tq_half_val(vn[tok]);
             const __half hi = __float2half_rn(wt);
             reinterpret_cast<__half*>(&wst[w][2 * t][0])[tok] = hi;
             reinterpret_cast<__half*>(&wst[w][2 * t + 1][0])[tok] = __float2half_rn(wt - __half2float(hi));

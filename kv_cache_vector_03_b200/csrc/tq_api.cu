@@ -388,7 +388,8 @@ size_t tq_attention_workspace_bytes(const tq_codec* kcodec, const tq_codec* vcod
 
 int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* packed_k, const void* packed_v,
                  int64_t n_seq, int n_kv, int64_t n_tok, const void* q, tq_dtype q_dtype, int g, const void* tail_k,
-                 const void* tail_v, int n_tail, float scale, float* out, void* ws, size_t ws_bytes, void* stream) {
+                 const void* tail_v, int n_tail, float scale, float v_skip, float* out, void* ws, size_t ws_bytes,
+                 void* stream) {
     int st = check_attention_codecs(kcodec, vcodec);
     if (st != TQ_OK) return st;
     if (g != 1 && g != 2 && g != 4) return TQ_ERR_UNSUPPORTED;
@@ -403,7 +404,7 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
         !aligned(ws, 256) || !aligned(q, q_dtype == TQ_F32 ? 4 : 2) ||
         (n_tail > 0 && (!aligned(tail_k, 2) || !aligned(tail_v, 8))))
         return TQ_ERR_ARG;
-    if (!std::isfinite(scale)) return TQ_ERR_ARG;
+    if (!std::isfinite(scale) || !(v_skip >= 0.f && v_skip <= 1.f)) return TQ_ERR_ARG;
     const TqDims tk = dims_of(kcodec), tv = dims_of(vcodec);
     const int64_t n_streams = n_seq * n_kv;
     if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
@@ -452,6 +453,7 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
     p.status = static_cast<uint32_t*>(ws);
     p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
     p.g = g; p.nsplit = p.nb > 0 ? W.nsplit : 0; p.blocks_per_split = W.bps; p.n_tail = n_tail;
+    p.v_skip = v_skip;
     p.tk = tk; p.tv = tv;
     if ((st = codebook_consts(vcodec, &p.cbv)) != TQ_OK) return st;
 

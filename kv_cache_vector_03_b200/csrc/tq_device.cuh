@@ -326,6 +326,7 @@ struct AttnParams {
     uint32_t* status;
     int64_t n_streams, n_tok, nb;
     int g, nsplit, blocks_per_split, n_tail;
+    float v_skip;                 // sparse values: a block whose weights are all below it skips its values
     TqDims tk, tv;
     TqCodebookConsts cbv;         // value codebook (binary16 decode table)
 };

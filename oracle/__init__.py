@@ -185,29 +185,62 @@ def pv(idx, nhat, pi, c, P) -> np.ndarray:
     return out
 
 
-def attention(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale: float,
-              tail_k=None, tail_v=None) -> np.ndarray:
-    """Decode attention of the query heads q [nh, d] of one kv stream, in fp64:
-    softmax over [estimated logits of the compressed keys, exact logits of the tail keys]
-    times [reconstructed compressed values, tail values] (a2a-mcp.org "What is TurboQuant":
-    scores from the codes, the weighted sum over the dequantized values; blog.hotdry.top
-    "TurboQuant vector-search compression", engineering configuration list: the recent
-    tokens kept at full precision). Either part may be empty (None or zero tokens)."""
+def _attention_parts(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale,
+                     tail_k, tail_v):
+    """Logits [nh, n], values [n, d] and the compressed-token count of one kv stream."""
     q = _f64(q)
     q = q.reshape(-1, q.shape[-1])
-    lgs, vals = [], []
+    lgs, vals, n_comp = [], [], 0
     if k_idx is not None and len(k_idx):
         lgs.append(logits(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, q, qjl=True, scale=scale))
         vals.append(reconstruct(v_idx, None, v_nhat, None, pi_v, None, c_v, qjl=False))
+        n_comp = len(k_idx)
     if tail_k is not None and len(tail_k):
         lgs.append(exact_dot(tail_k, q, scale))
         vals.append(_f64(tail_v))
     if not lgs:
         raise ValueError("attention over no tokens")
-    lg = np.concatenate(lgs, axis=1)
-    w = np.exp(lg - lg.max(axis=1, keepdims=True))
-    w /= w.sum(axis=1, keepdims=True)
-    return w @ np.concatenate(vals, axis=0)
+    return np.concatenate(lgs, axis=1), np.concatenate(vals, axis=0), n_comp
+
+
+def attention(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale: float,
+              tail_k=None, tail_v=None, v_skip: float = 0.0) -> np.ndarray:
+    """Decode attention of the query heads q [nh, d] of one kv stream, in fp64:
+    softmax over [estimated logits of the compressed keys, exact logits of the tail keys]
+    times [reconstructed compressed values, tail values] (a2a-mcp.org "What is TurboQuant":
+    scores from the codes, the weighted sum over the dequantized values; blog.hotdry.top
+    "TurboQuant vector-search compression", engineering configuration list: the recent
+    tokens kept at full precision). Either part may be empty (None or zero tokens).
+
+    v_skip > 0: sparse values (ai-coding.wiselychen.com "Google TurboQuant KV-cache
+    compression", community extensions, "Sparse V"): a compressed token whose weight relative
+    to the largest weight, exp(l_t - max l), is below v_skip drops out of the weighted sum of
+    values; the softmax denominator keeps it."""
+    lg, vals, n_comp = _attention_parts(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q,
+                                        scale, tail_k, tail_v)
+    rel = np.exp(lg - lg.max(axis=1, keepdims=True))
+    w = rel / rel.sum(axis=1, keepdims=True)
+    if v_skip > 0.0:
+        w = w.copy()
+        drop = rel < v_skip
+        drop[:, n_comp:] = False
+        w[drop] = 0.0
+    return w @ vals
+
+
+def attention_skip_mass(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale: float,
+                        tail_k=None, tail_v=None, v_skip: float = 0.0) -> np.ndarray:
+    """Per head, sum over the compressed tokens with relative weight below v_skip of w_t |v_t|,
+    divided by sum_t w_t |v_t|: a bound on the normalised change any subset of those tokens
+    can make when dropped from the value sum (the sparse-value error bound)."""
+    lg, vals, n_comp = _attention_parts(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q,
+                                        scale, tail_k, tail_v)
+    rel = np.exp(lg - lg.max(axis=1, keepdims=True))
+    w = rel / rel.sum(axis=1, keepdims=True)
+    wv = w * np.linalg.norm(vals, axis=1)[None, :]
+    drop = rel < v_skip
+    drop[:, n_comp:] = False
+    return (wv * drop).sum(axis=1) / wv.sum(axis=1)
 
 
 def topk(idx, sbit, nhat, ghat, pi, s, c, q, k: int, qjl: bool = True):

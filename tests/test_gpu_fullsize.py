@@ -60,12 +60,13 @@ def test_c2_llama_decode(b):
         _check_logits(got[h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[h, n_tok:], axis=1), 1.0 / math.sqrt(d))
 
 
-@pytest.mark.parametrize("b", [4, 3])
-def test_c2_fused_attention(b):
+@pytest.mark.parametrize("b,vs", [(4, 0.0), (3, 0.0), (3, 1e-4)])
+def test_c2_fused_attention(b, vs):
     """The c2 decode step fused: keys at b bits (b - 1 MSE + QJL), values at b bits (MSE), the last
     128 tokens in bf16. Two kv-heads are checked against the oracle composition over all 32768
     tokens, under the bound of test_gpu_parity.test_attention (P.V tolerance plus expm1(2 dl)
-    for the logit error dl tq_logits makes on the same codes)."""
+    for the logit error dl tq_logits makes on the same codes, plus the dropped weight mass
+    when sparse values are on)."""
     d = m = 128
     n_kv, n_all, n_tail, g = 8, 32768, 128, 4
     n_tok = n_all - n_tail
@@ -82,7 +83,7 @@ def test_c2_fused_attention(b):
     tk = to_dev_bf16(np.ascontiguousarray(keys[:, n_tok:]))
     tv = to_dev_bf16(np.ascontiguousarray(vals[:, n_tok:]))
     scale = 1.0 / math.sqrt(d)
-    got = _attention_gpu(kc, vc, pk, pvv, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)[0]
+    got = _attention_gpu(kc, vc, pk, pvv, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale, vs)[0]
     lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
     kidx, ksb, knh, kgh = unpack(kc, pk, n_kv, n_tok)
     vidx, vnh = unpack(vc, pvv, n_kv, n_tok)
@@ -102,7 +103,12 @@ def test_c2_fused_attention(b):
         dl = np.abs(lg[h * g:(h + 1) * g] - L).max(axis=1)
         err = np.max(np.abs(got[h * g:(h + 1) * g] - want), axis=1) / (w @ vnorm)
         assert np.all(np.isfinite(got[h * g:(h + 1) * g]))
-        assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), f"kv-head {h}: {err}"
+        bound = TOL + np.expm1(2 * dl) + 1e-5
+        if vs > 0.0:
+            bound = bound + oracle.attention_skip_mass(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, vidx[h], vnh[h],
+                                                       piv, c_v, qh, scale, tail_k=kf[h, n_tok:],
+                                                       tail_v=vf[h, n_tok:], v_skip=vs)
+        assert np.all(err <= bound), f"kv-head {h}: {err} above {bound}"
 
 
 @pytest.mark.parametrize("B", [3, 4])

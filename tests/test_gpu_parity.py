@@ -285,12 +285,12 @@ def test_pv_one_hot_and_uniform():
 
 
 # ----------------------------------------------------------------------------- fused attention
-def _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale):
+def _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale, v_skip=0.0):
     torch = torch_cuda()
     m = tq()
     out = torch.full((n_seq, n_kv * g, kc.c.d), float("nan"), dtype=torch.float32, device="cuda")
     ws = m.workspace(m.tq_attention_workspace_bytes(kc, vc, n_seq, n_kv, n_tok, g, n_tail))
-    m.tq_attention(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale, out, ws)
+    m.tq_attention(kc, vc, pk, pvv, n_seq, n_kv, n_tok, q_dev, g, tk_dev, tv_dev, n_tail, scale, out, ws, v_skip=v_skip)
     torch.cuda.synchronize()
     assert m.tq_get_status(ws) == m.TQ_OK
     return out.cpu().numpy().astype(np.float64)
@@ -301,23 +301,26 @@ def _normal_stream(seed, seq, head, n):
     return ti.value_stream(head, n, cfg_id=seed * 1000 + seq)
 
 
-@pytest.mark.parametrize("Bk,Bv,g,n_seq,n_kv,n_tok,n_tail,law,qs", [
-    (2, 3, 4, 2, 3, 301, 5, "normal", 1.0),      # several streams, ragged last block
-    (3, 4, 4, 1, 2, 5000, 128, "normal", 1.0),   # many ranges per stream, a 128-token tail
-    (1, 2, 1, 1, 2, 64, 0, "normal", 1.0),       # no tail
-    (2, 4, 2, 1, 2, 0, 33, "normal", 1.0),       # tail only
-    (3, 3, 4, 1, 1, 1000, 1, "normal", 8.0),     # peaked softmax: the running maximum moves
-    (2, 1, 4, 3, 1, 33, 7, "normal", 1.0),       # 1-bit values, a block of one valid token
-    (3, 4, 4, 1, 2, 3000, 128, "c2", 1.0),       # the decode key law (outlier channels, long keys)
+@pytest.mark.parametrize("Bk,Bv,g,n_seq,n_kv,n_tok,n_tail,law,qs,vs", [
+    (2, 3, 4, 2, 3, 301, 5, "normal", 1.0, 0.0),      # several streams, ragged last block
+    (3, 4, 4, 1, 2, 5000, 128, "normal", 1.0, 0.0),   # many ranges per stream, a 128-token tail
+    (1, 2, 1, 1, 2, 64, 0, "normal", 1.0, 0.0),       # no tail
+    (2, 4, 2, 1, 2, 0, 33, "normal", 1.0, 0.0),       # tail only
+    (3, 3, 4, 1, 1, 1000, 1, "normal", 8.0, 0.0),     # peaked softmax: the running maximum moves
+    (2, 1, 4, 3, 1, 33, 7, "normal", 1.0, 0.0),       # 1-bit values, a block of one valid token
+    (3, 4, 4, 1, 2, 3000, 128, "c2", 1.0, 0.0),       # the decode key law (outlier channels, long keys)
+    (3, 4, 4, 1, 2, 3000, 128, "c2", 1.0, 1e-4),      # sparse values on the same data
+    (2, 3, 4, 2, 2, 2000, 16, "normal", 4.0, 1e-2),   # sparse values, a milder softmax
 ])
-def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
+def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs, vs):
     """softmax(scale q . K) . V against the oracle composition on the same codes.
 
     Bound, from the step tolerances: a logit error of at most dl moves every softmax weight by
     a factor within exp(+-2 dl), so |do| <= (expm1(2 dl) + TOL) sum_t w_t |v_t| with the P.V
     tolerance TOL. dl is the logit error tq_logits makes on the same codes and queries (the
     fused kernel evaluates the same fragments with the same arithmetic); it is itself held to
-    the logits tolerance."""
+    the logits tolerance. With sparse values (vs > 0) the oracle's dropped weight mass (tokens
+    whose relative weight is below vs) is added: the kernel drops a subset of them."""
     d = m = 128
     pik, sk, piv = ti.haar_rotation(d, 95), ti.gaussian_sketch(m, d, 96), ti.haar_rotation(d, 97)
     n = n_tok + n_tail
@@ -337,7 +340,7 @@ def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
     tv = to_dev_bf16(np.ascontiguousarray(vals[:, :, n_tok:])) if n_tail else None
     qb = ti.decode_queries(12, n_seq, n_kv * g)
     scale = qs / math.sqrt(d)
-    got = _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)
+    got = _attention_gpu(kc, vc, pk, pvv, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale, vs)
     lg = _logits_gpu(kc, pk, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)
     if n_tok:
         kidx, ksb, knh, kgh = unpack(kc, pk, S, n_tok)
@@ -372,6 +375,8 @@ def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs):
             err = np.max(np.abs(got[sq, h * g:(h + 1) * g] - want), axis=1) / (w @ vnorm)
             assert np.all(np.isfinite(got[sq, h * g:(h + 1) * g]))
             bound = TOL + np.expm1(2 * dl) + 1e-5
+            if vs > 0.0:
+                bound = bound + oracle.attention_skip_mass(**a, q=qh, scale=scale, tail_k=tkh, tail_v=tvh, v_skip=vs)
             assert np.all(err <= bound), f"stream {st}: normalised error {err} above {bound}"
             print(f"attention stream {st}: normalised error {err.max():.2e}, bound {bound.min():.2e}, "
                   f"logit error {dl_norm.max():.2e}")

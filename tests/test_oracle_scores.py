@@ -147,6 +147,32 @@ def test_attention_uniform_and_one_hot_tail():
     assert np.allclose(full, (zt * only_tail + zc * only_comp) / (zt + zc), rtol=1e-12, atol=1e-12)
 
 
+def test_attention_sparse_values():
+    a, keys, vals = _attention_setup(n_tail=0)
+    qs = np.random.default_rng(23).standard_normal((3, 64)) * 0.3
+    dense = oracle.attention(**a, q=qs, scale=1.0)
+    # a threshold below every relative weight changes nothing
+    assert np.array_equal(oracle.attention(**a, q=qs, scale=1.0, v_skip=1e-300), dense)
+    # v_skip = 1 keeps only the largest-weight token in the value sum, the denominator keeps all
+    lg = oracle.logits(a["k_idx"], a["k_sbit"], a["k_nhat"], a["k_ghat"], a["pi_k"], a["s_k"], a["c_k"], qs,
+                       qjl=True)
+    vh = oracle.reconstruct(a["v_idx"], None, a["v_nhat"], None, a["pi_v"], None, a["c_v"], qjl=False)
+    top = lg.argmax(axis=1)
+    z = np.exp(lg - lg.max(axis=1, keepdims=True)).sum(axis=1)
+    assert np.allclose(oracle.attention(**a, q=qs, scale=1.0, v_skip=1.0), vh[top] / z[:, None], rtol=1e-12,
+                       atol=1e-14)
+    # the change is bounded by the dropped weight mass, which grows with the threshold
+    sumwv = (np.exp(lg - lg.max(axis=1, keepdims=True)) / z[:, None]) @ np.linalg.norm(vh, axis=1)
+    prev = np.zeros(3)
+    for tau in (1e-3, 1e-2, 1e-1, 0.5):
+        sp = oracle.attention(**a, q=qs, scale=1.0, v_skip=tau)
+        mass = oracle.attention_skip_mass(**a, q=qs, scale=1.0, v_skip=tau)
+        assert np.all(mass >= prev) and np.all(mass < 1.0)
+        assert np.all(np.max(np.abs(sp - dense), axis=1) <= mass * sumwv * (1 + 1e-12))
+        prev = mass
+    assert prev.min() > 0.0
+
+
 def test_topk_matches_full_sort():
     c, t, pi, s, x, q = _setup(n=500)
     qs = np.random.default_rng(7).standard_normal((6, 64))
