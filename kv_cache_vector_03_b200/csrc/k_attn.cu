@@ -291,9 +291,10 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
 
 // One CTA per query head: the ranges and the exact tail under one maximum M,
 //   out = (Pi^T sum_s e^{m_s - M} part_s + sum_t e^{l_t - M} v_t) / (sum_s e^{m_s - M} l_s + sum_t e^{l_t - M}).
-// The two sums run side by side: thread (group, coordinate quad) takes every 8th range of the
-// rotated-domain partials and every 8th tail token (8-byte loads of 4 bf16 coordinates, a
-// warp reads one 256-byte row), then the groups are added in shared memory.
+// Every global load is issued in one round: thread (group, coordinate quad) folds every 8th
+// range (rotated-domain partial quads) and every 8th tail token (exact logit, 8-byte load of
+// 4 bf16 coordinates; a warp reads one 256-byte row) under its own running maximum, into a
+// rotated-domain and an original-domain sum; the groups then meet in shared memory.
 constexpr int kMergeThreads = 256;
 constexpr int kMergeGroups = kMergeThreads / 32;   // 32 coordinate quads = 128 coordinates
 
@@ -301,95 +302,93 @@ __global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
     const int d = p.tv.d, ns = p.nsplit, nt = p.n_tail;   // D = 128
     const int64_t hq = blockIdx.x;   // stream * g + head
     const int64_t stream = hq / p.g;
-    extern __shared__ float msm[];
-    float* fs = msm;                       // [ns] split weights, padded to 4 floats
-    float* ft = fs + ((ns + 3) & ~3);      // [n_tail] tail weights, padded to 4 floats
-    float* red = ft + ((nt + 3) & ~3);     // [8][128] range partials, 16-byte aligned
-    float* redt = red + 1024;              // [8][128] tail partials
-    float* s_o = redt + 1024;              // [128] rotated-domain sum
-    float* s_t = s_o + 128;                // [128] tail sum
-    __shared__ float s_w[kMergeThreads / 32];
-    __shared__ float s_M, s_den;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    __shared__ __align__(16) float s_acc[kMergeGroups * 128], s_tac[kMergeGroups * 128];
+    __shared__ __align__(16) float s_o[128];
+    __shared__ float s_t[128], s_gm[kMergeGroups], s_gl[kMergeGroups];
+    const int tid = threadIdx.x, grp = tid >> 5, qd = tid & 31;
     const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
-    const float* tl = p.tail_logit + (size_t)hq * nt;
-
-    float mx = -INFINITY;
-    for (int s = tid; s < ns; s += kMergeThreads) {
-        const float2 v = ml[s];
-        if (v.y > 0.f) mx = fmaxf(mx, v.x);
-    }
-    for (int j = tid; j < nt; j += kMergeThreads) mx = fmaxf(mx, tl[j]);
-    mx = tq_warp_max(mx);
-    if (lane == 0) s_w[wid] = mx;
-    __syncthreads();
-    if (tid == 0) {
-        float M = s_w[0];
-        for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, s_w[i]);
-        s_M = M;
-    }
-    __syncthreads();
-    const float M = s_M;
-    float den = 0.f;
-    for (int s = tid; s < ns; s += kMergeThreads) {
-        const float2 v = ml[s];
-        const float f = v.y > 0.f ? __expf(v.x - M) : 0.f;
-        fs[s] = f;
-        den = fmaf(f, v.y, den);
-    }
-    for (int j = tid; j < nt; j += kMergeThreads) {
-        const float f = __expf(tl[j] - M);
-        ft[j] = f;
-        den += f;
-    }
-    den = tq_warp_sum(den);
-    __syncthreads();   // s_w reused; fs and ft complete
-    if (lane == 0) s_w[wid] = den;
-    const int grp = wid, qd = lane;
-    // ranges: every range wrote its partial (zeros where it saw no weight)
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * 128) + qd;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = grp; s < ns; s += kMergeGroups) {
-        const float f = fs[s];
-        const float4 v = src[(size_t)s * 32];
-        a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
-    }
-    reinterpret_cast<float4*>(red)[grp * 32 + qd] = a;
-    // tail tokens, original domain
-    float4 b = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (qd < d / 4) {
-        const uint2* tv = reinterpret_cast<const uint2*>(p.tail_v + (size_t)stream * nt * d) + qd;
-#pragma unroll 4
-        for (int tt = grp; tt < nt; tt += kMergeGroups) {
-            const uint2 v = __ldg(tv + (size_t)tt * (d / 4));
-            const float f = ft[tt];
-            b.x = fmaf(f, __uint_as_float(v.x << 16), b.x);
-            b.y = fmaf(f, __uint_as_float(v.x & 0xffff0000u), b.y);
-            b.z = fmaf(f, __uint_as_float(v.y << 16), b.z);
-            b.w = fmaf(f, __uint_as_float(v.y & 0xffff0000u), b.w);
+    float m = -INFINITY, l = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = make_float4(0.f, 0.f, 0.f, 0.f);
+    // batches whose loads are all issued before any is used; one rescale per batch
+    constexpr int RB = 8, TB = 16;
+    for (int s0 = grp; s0 < ns; s0 += RB * kMergeGroups) {
+        float2 v[RB];
+        float4 x[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int s = s0 + u * kMergeGroups;
+            v[u] = s < ns ? ml[s] : make_float2(-INFINITY, 0.f);
+            x[u] = s < ns ? src[(size_t)s * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mn = m;
+#pragma unroll
+        for (int u = 0; u < RB; ++u) mn = v[u].y > 0.f ? fmaxf(mn, v[u].x) : mn;
+        if (mn > -INFINITY) {   // a range with weight (every range wrote its partial)
+            const float so = __expf(m - mn);
+            a.x *= so; a.y *= so; a.z *= so; a.w *= so;
+            l *= so;
+#pragma unroll
+            for (int u = 0; u < RB; ++u) {
+                const float sn = v[u].y > 0.f ? __expf(v[u].x - mn) : 0.f;
+                a.x = fmaf(sn, x[u].x, a.x); a.y = fmaf(sn, x[u].y, a.y);
+                a.z = fmaf(sn, x[u].z, a.z); a.w = fmaf(sn, x[u].w, a.w);
+                l = fmaf(sn, v[u].y, l);
+            }
+            m = mn;
         }
     }
-    reinterpret_cast<float4*>(redt)[grp * 32 + qd] = b;
+    const float* tl = p.tail_logit + (size_t)hq * nt;
+    const uint2* tv = reinterpret_cast<const uint2*>(p.tail_v + (size_t)stream * nt * d) + qd;
+    const bool qv = qd < d / 4;
+    for (int t0 = grp; t0 < nt; t0 += TB * kMergeGroups) {
+        float lt[TB];
+        uint2 vv[TB];
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+            const int tt = t0 + u * kMergeGroups;
+            lt[u] = tt < nt ? tl[tt] : -INFINITY;
+            vv[u] = tt < nt && qv ? __ldg(tv + (size_t)tt * (d / 4)) : make_uint2(0u, 0u);
+        }
+        float mn = m;
+#pragma unroll
+        for (int u = 0; u < TB; ++u) mn = fmaxf(mn, lt[u]);
+        const float so = __expf(m - mn);   // m = -inf the first time: 0
+        a.x *= so; a.y *= so; a.z *= so; a.w *= so;
+        b.x *= so; b.y *= so; b.z *= so; b.w *= so;
+        l *= so;
+#pragma unroll
+        for (int u = 0; u < TB; ++u) {
+            const float sn = __expf(lt[u] - mn);   // 0 past the tail
+            b.x = fmaf(sn, __uint_as_float(vv[u].x << 16), b.x);
+            b.y = fmaf(sn, __uint_as_float(vv[u].x & 0xffff0000u), b.y);
+            b.z = fmaf(sn, __uint_as_float(vv[u].y << 16), b.z);
+            b.w = fmaf(sn, __uint_as_float(vv[u].y & 0xffff0000u), b.w);
+            l += sn;
+        }
+        m = mn;
+    }
+    reinterpret_cast<float4*>(s_acc)[grp * 32 + qd] = a;
+    reinterpret_cast<float4*>(s_tac)[grp * 32 + qd] = b;
+    if (qd == 0) { s_gm[grp] = m; s_gl[grp] = l; }
     __syncthreads();
-    if (tid < 128) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < kMergeGroups; ++q) M = fmaxf(M, s_gm[q]);
+    float den = 0.f;
+#pragma unroll
+    for (int q = 0; q < kMergeGroups; ++q) den += s_gm[q] > -INFINITY ? __expf(s_gm[q] - M) * s_gl[q] : 0.f;
+    {
+        const int i = tid & 127;
+        const float* accp = tid < 128 ? s_acc : s_tac;
         float v = 0.f;
 #pragma unroll
-        for (int q = 0; q < kMergeGroups; ++q) v += red[q * 128 + tid];
-        s_o[tid] = v;
-    } else {
-        float v = 0.f;
-#pragma unroll
-        for (int q = 0; q < kMergeGroups; ++q) v += redt[q * 128 + tid - 128];
-        s_t[tid - 128] = v;
-    }
-    if (tid == 0) {
-        float v = 0.f;
-        for (int i = 0; i < kMergeThreads / 32; ++i) v += s_w[i];
-        s_den = v;
+        for (int q = 0; q < kMergeGroups; ++q)
+            if (s_gm[q] > -INFINITY) v = fmaf(__expf(s_gm[q] - M), accp[q * 128 + i], v);
+        (tid < 128 ? s_o : s_t)[i] = v;
     }
     __syncthreads();
-    const float inv = 1.f / s_den;
+    const float inv = 1.f / den;
     // out[j] = (<row j of Pi^T, o> + t_j) / den: pair (j, half), the halves joined by a shuffle
     // of neighbouring lanes under a block-uniform trip count
     for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
@@ -434,10 +433,6 @@ cudaError_t launch_bv(const AttnParams& p, cudaStream_t st) {
 
 }  // namespace
 
-size_t tq_attn_merge_smem(int nsplit, int n_tail) {
-    return (((size_t)nsplit + 3) / 4 * 4 + ((size_t)n_tail + 3) / 4 * 4 + 2048 + 256) * 4;
-}
-
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
     if (p.tk.D != 128 || p.tk.Mp != 128 || p.tv.D != 128 || p.g < 1 || p.g > 4) return cudaErrorInvalidValue;
     if (p.nsplit > 0) {   // no compressed tokens: the merge sees only the tail
@@ -449,10 +444,8 @@ cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
         }
         if (e != cudaSuccess) return e;
     }
-    const size_t msmem = tq_attn_merge_smem(p.nsplit, p.n_tail);
-    if (msmem > 48 * 1024) return cudaErrorInvalidValue;
     // a plain launch: as a programmatic dependent of the split the merge measured 17 us slower
     // per call at 8 x 32768 tokens
-    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, msmem, st>>>(p);
+    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }

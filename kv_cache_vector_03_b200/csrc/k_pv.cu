@@ -271,73 +271,67 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
 }
 
 // One CTA per query head: o = sum_s e^{m_s - M} part_s / sum_s e^{m_s - M} l_s, then Pi^T o.
+// Every global load of the partials is issued in one round: thread (group, coordinate quad)
+// reads the maxima, sums and partial quads of every ngrp-th range and folds them under its
+// own running maximum; the groups then meet in shared memory under the common one.
 constexpr int kMergeThreads = 256;
 
 __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
     const int D = p.t.D, d = p.t.d, ns = p.nsplit;
     const int64_t hq = blockIdx.x;   // stream * g + head
-    extern __shared__ float msm[];
-    float* fs = msm;                     // [ns] split weights e^{m_s - M}, padded to 4 floats
-    float* red = fs + ((ns + 3) & ~3);   // [1024], 16-byte aligned: [groups][D] partial sums, later [2][256]
-    float* s_o = red + 1024;             // [256]
-    __shared__ float s_w[kMergeThreads / 32];
-    __shared__ float s_M, s_den;
-    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
-
-    float mx = -INFINITY;
-    for (int s = tid; s < ns; s += kMergeThreads) {
-        const float2 v = ml[s];
-        if (v.y > 0.f) mx = fmaxf(mx, v.x);
-    }
-    mx = tq_warp_max(mx);
-    if (lane == 0) s_w[wid] = mx;
-    __syncthreads();
-    if (tid == 0) {
-        float M = s_w[0];
-        for (int i = 1; i < kMergeThreads / 32; ++i) M = fmaxf(M, s_w[i]);
-        s_M = M;
-    }
-    __syncthreads();
-    const float M = s_M;
-    float den = 0.f;
-    for (int s = tid; s < ns; s += kMergeThreads) {
-        const float2 v = ml[s];
-        const float f = v.y > 0.f ? __expf(v.x - M) : 0.f;
-        fs[s] = f;
-        den = fmaf(f, v.y, den);
-    }
-    den = tq_warp_sum(den);
-    __syncthreads();   // s_w reused
-    if (lane == 0) s_w[wid] = den;
-    __syncthreads();
-    if (tid == 0) {
-        float v = 0.f;
-        for (int i = 0; i < kMergeThreads / 32; ++i) v += s_w[i];
-        s_den = v;
-    }
-    // weighted sum over splits: thread (group, column quad)
+    __shared__ __align__(16) float s_acc[kMergeThreads * 4];   // [group][D]
+    __shared__ __align__(16) float s_o[256];
+    __shared__ float s_gm[8], s_gl[8];
+    const int tid = threadIdx.x;
     const int nq = D / 4, ngrp = kMergeThreads / nq;
     const int grp = tid / nq, qd = tid % nq;
+    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
+    float m = -INFINITY, l = 0.f;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    // every split wrote its partial (zeros where it saw no weight), so the loads need no guard
-    // and can all be in flight at once
-#pragma unroll 8
-    for (int s = grp; s < ns; s += ngrp) {
-        const float f = fs[s];
-        const float4 v = src[(size_t)s * nq];
-        a.x = fmaf(f, v.x, a.x); a.y = fmaf(f, v.y, a.y); a.z = fmaf(f, v.z, a.z); a.w = fmaf(f, v.w, a.w);
+    // batches whose loads are all issued before any is used; one rescale per batch
+    constexpr int RB = 8;
+    for (int s0 = grp; s0 < ns; s0 += RB * ngrp) {
+        float2 v[RB];
+        float4 x[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int s = s0 + u * ngrp;
+            v[u] = s < ns ? ml[s] : make_float2(-INFINITY, 0.f);
+            x[u] = s < ns ? src[(size_t)s * nq] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mn = m;
+#pragma unroll
+        for (int u = 0; u < RB; ++u) mn = v[u].y > 0.f ? fmaxf(mn, v[u].x) : mn;
+        if (mn > -INFINITY) {   // a range with weight (every range wrote its partial)
+            const float so = __expf(m - mn);
+            a.x *= so; a.y *= so; a.z *= so; a.w *= so;
+            l *= so;
+#pragma unroll
+            for (int u = 0; u < RB; ++u) {
+                const float sn = v[u].y > 0.f ? __expf(v[u].x - mn) : 0.f;
+                a.x = fmaf(sn, x[u].x, a.x); a.y = fmaf(sn, x[u].y, a.y);
+                a.z = fmaf(sn, x[u].z, a.z); a.w = fmaf(sn, x[u].w, a.w);
+                l = fmaf(sn, v[u].y, l);
+            }
+            m = mn;
+        }
     }
-    reinterpret_cast<float4*>(red)[grp * nq + qd] = a;
+    reinterpret_cast<float4*>(s_acc)[grp * nq + qd] = a;
+    if (qd == 0) { s_gm[grp] = m; s_gl[grp] = l; }
     __syncthreads();
-    const float inv = 1.f / s_den;
+    float M = -INFINITY;
+    for (int q = 0; q < ngrp; ++q) M = fmaxf(M, s_gm[q]);
+    float den = 0.f;
+    for (int q = 0; q < ngrp; ++q) den += s_gm[q] > -INFINITY ? __expf(s_gm[q] - M) * s_gl[q] : 0.f;
     for (int i = tid; i < D; i += kMergeThreads) {
         float v = 0.f;
-        for (int q = 0; q < ngrp; ++q) v += red[q * D + i];
-        s_o[i] = v * inv;
+        for (int q = 0; q < ngrp; ++q)
+            if (s_gm[q] > -INFINITY) v = fmaf(__expf(s_gm[q] - M), s_acc[q * D + i], v);
+        s_o[i] = v;
     }
     __syncthreads();
+    const float inv = 1.f / den;
     // out[j] = sum_i Pi[i][j] o_i = <row j of Pi^T, o> (its columns i >= d are zero): pair
     // (j, half), 16-byte loads of the row; the block-uniform trip count keeps warps whole for
     // the shuffle that joins the halves (neighbouring lanes)
@@ -356,7 +350,7 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
             }
         }
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (valid && hf == 0) p.out[(size_t)hq * d + j] = acc;
+        if (valid && hf == 0) p.out[(size_t)hq * d + j] = acc * inv;
     }
 }
 
@@ -382,8 +376,6 @@ cudaError_t launch_b(const PvParams& p, cudaStream_t st) {
     return cudaErrorInvalidValue;
 }
 
-size_t pv_merge_smem(int nsplit) { return (((size_t)nsplit + 3) / 4 * 4 + 1024 + 256) * 4; }
-
 }  // namespace
 
 cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
@@ -393,8 +385,6 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
     else if (p.t.D == 256) e = nt == 1 ? launch_b<16, 1>(p, st) : launch_b<16, 2>(p, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
-    const size_t msmem = pv_merge_smem(p.nsplit);
-    if (msmem > 48 * 1024) return cudaErrorInvalidValue;
-    k_pv_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, msmem, st>>>(p);
+    k_pv_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
