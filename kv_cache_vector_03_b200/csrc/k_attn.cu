@@ -37,6 +37,13 @@ __device__ __forceinline__ size_t qf_word(int64_t stream, int nmg, int mg, int c
     return (((size_t)stream * nmg + mg) * 4 + c) * 64 + lane * 2;
 }
 
+// order-preserving map between floats and ints, for integer atomicMax on float maxima
+__device__ __forceinline__ int ord_of(float f) {
+    const int i = __float_as_int(f);
+    return i >= 0 ? i : i ^ 0x7fffffff;
+}
+__device__ __forceinline__ float float_of(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
+
 template <int BK, int BV>   // key MSE bits (1..3), value bits (1..4); d <= 128, m <= 128, g <= 4
 __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p) {
     constexpr int NS = kAttnNS;
@@ -54,6 +61,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
     __shared__ uint32_t wst[kAttnWarps][8][kWCol];             // column 2 head + part: token pairs
     __shared__ float s_acc[4][KT * 16];
     __shared__ float s_m[kAttnWarps][4], s_l[kAttnWarps][4];
+    __shared__ int s_cmax[4];   // CTA-wide running maximum per head (order-preserving int image)
     __shared__ uint64_t bars[kAttnWarps][NS];
 
     const int G = p.g;
@@ -70,6 +78,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
         reinterpret_cast<uint4*>(lut)[e] = make_uint4(v, v, v, v);
     }
     for (int e = threadIdx.x; e < 4 * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
+    if (threadIdx.x < 4) s_cmax[threadIdx.x] = ord_of(-INFINITY);
     if (lane == 0)
         for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[w][s], 2);
     tq_fence_mbar_init();
@@ -178,6 +187,13 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+        // sparse values compare against the largest logit any warp of the CTA has seen (never
+        // above the final maximum), so a warp skips from its first block on
+        float cmax = bm;
+        if (p.v_skip > 0.f) {
+            if (g == 0) atomicMax(&s_cmax[t], ord_of(bm));
+            cmax = fmaxf(bm, float_of(*reinterpret_cast<volatile int*>(&s_cmax[t])));
+        }
         if (bm > m_run) {
             const float fac = tq_exp2((m_run - bm) * kLog2e);   // 0 while the maximum was -inf
 #pragma unroll
@@ -191,14 +207,16 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
         const uint16_t* vn = reinterpret_cast<const uint16_t*>(vb + SEC_AV);
         float ev[4];
         bool low = true;
+        const float lthr = cmax + __logf(p.v_skip);   // -inf when v_skip = 0
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             ev[u] = m_run > -INFINITY ? tq_exp2(fmaf(l[u], kLog2e, -ml2)) : 0.f;
             lsum += ev[u];
-            low = low && ev[u] < p.v_skip;
+            low = low && (l[u] < lthr || l[u] == -INFINITY);
         }
-        // sparse values: every weight of the block is below v_skip (relative to the running
-        // maximum, so also to the final one): the softmax sum keeps them, the values are skipped
+        // sparse values: every weight of the block is below v_skip relative to the CTA's
+        // running maximum (so also to the final one): the softmax sum keeps them, the values
+        // are skipped
         if (__all_sync(0xffffffffu, low)) {
             __syncwarp();
             if (lane == 0) tq_fence_proxy_async();
