@@ -324,6 +324,16 @@ __global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
     __shared__ __align__(16) float s_o[128];
     __shared__ float s_t[128], s_gm[kMergeGroups], s_gl[kMergeGroups];
     const int tid = threadIdx.x, grp = tid >> 5, qd = tid & 31;
+    // the half row of Pi^T this thread rotates with (output j = tid / 2, half tid % 2), loaded
+    // first so that its latency overlaps the partials' (d <= 128: one pair per thread)
+    const int jr = tid >> 1, hr = tid & 1;
+    const bool rv = tid < 2 * d;
+    float4 wrow[16];
+    {
+        const float4* rowp = reinterpret_cast<const float4*>(p.piT_v + (size_t)(rv ? jr : 0) * 128 + hr * 64);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) wrow[k] = __ldg(rowp + k);
+    }
     const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * 128) + qd;
     float m = -INFINITY, l = 0.f;
@@ -407,24 +417,17 @@ __global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
     }
     __syncthreads();
     const float inv = 1.f / den;
-    // out[j] = (<row j of Pi^T, o> + t_j) / den: pair (j, half), the halves joined by a shuffle
-    // of neighbouring lanes under a block-uniform trip count
-    for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
-        const int e = e0 + tid, j = e >> 1, hf = e & 1;
-        const bool valid = e < 2 * d;
-        float acc = 0.f;
-        if (valid) {
-            const float4* rowp = reinterpret_cast<const float4*>(p.piT_v + (size_t)j * 128 + hf * 64);
-            const float4* op = reinterpret_cast<const float4*>(s_o + hf * 64);
+    // out[j] = (<row j of Pi^T, o> + t_j) / den; the two halves meet by a shuffle of
+    // neighbouring lanes (all 256 threads take part)
+    float acc = 0.f;
+    const float4* op = reinterpret_cast<const float4*>(s_o + hr * 64);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const float4 w = __ldg(rowp + k), o = op[k];
-                acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
-            }
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (valid && hf == 0) p.out[(size_t)hq * d + j] = (acc + s_t[j]) * inv;
+    for (int k = 0; k < 16; ++k) {
+        const float4 w = wrow[k], o = op[k];
+        acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
     }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (rv && hr == 0) p.out[(size_t)hq * d + jr] = (acc + s_t[jr]) * inv;
 }
 
 template <int BK, int BV>

@@ -276,15 +276,26 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
 // own running maximum; the groups then meet in shared memory under the common one.
 constexpr int kMergeThreads = 256;
 
+template <int D>   // 128 or 256
 __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
-    const int D = p.t.D, d = p.t.d, ns = p.nsplit;
+    const int d = p.t.d, ns = p.nsplit;
     const int64_t hq = blockIdx.x;   // stream * g + head
     __shared__ __align__(16) float s_acc[kMergeThreads * 4];   // [group][D]
     __shared__ __align__(16) float s_o[256];
     __shared__ float s_gm[8], s_gl[8];
     const int tid = threadIdx.x;
-    const int nq = D / 4, ngrp = kMergeThreads / nq;
+    constexpr int nq = D / 4, ngrp = kMergeThreads / nq;
     const int grp = tid / nq, qd = tid % nq;
+    // D = 128: the half row of Pi^T this thread rotates with (output tid / 2, half tid % 2) is
+    // loaded first so that its latency overlaps the partials'
+    const int jr = tid >> 1, hr = tid & 1;
+    const bool rv = tid < 2 * d;
+    float4 wrow[D == 128 ? 16 : 1];
+    if constexpr (D == 128) {
+        const float4* rowp = reinterpret_cast<const float4*>(p.piT + (size_t)(rv ? jr : 0) * 128 + hr * 64);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) wrow[k] = __ldg(rowp + k);
+    }
     const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
     float m = -INFINITY, l = 0.f;
@@ -333,8 +344,20 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
     __syncthreads();
     const float inv = 1.f / den;
     // out[j] = sum_i Pi[i][j] o_i = <row j of Pi^T, o> (its columns i >= d are zero): pair
-    // (j, half), 16-byte loads of the row; the block-uniform trip count keeps warps whole for
-    // the shuffle that joins the halves (neighbouring lanes)
+    // (j, half), the halves joined by a shuffle of neighbouring lanes
+    if constexpr (D == 128) {
+        float acc = 0.f;
+        const float4* op = reinterpret_cast<const float4*>(s_o + hr * 64);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float4 w = wrow[k], o = op[k];
+            acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        if (rv && hr == 0) p.out[(size_t)hq * d + jr] = acc * inv;
+        return;
+    }
+    // D = 256: 16-byte loads of the row; the block-uniform trip count keeps warps whole
     const int hl = D / 2;
     for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
         const int e = e0 + tid, j = e >> 1, hf = e & 1;
@@ -385,6 +408,7 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
     else if (p.t.D == 256) e = nt == 1 ? launch_b<16, 1>(p, st) : launch_b<16, 2>(p, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
-    k_pv_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    if (p.t.D == 128) k_pv_merge<128><<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    else k_pv_merge<256><<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }

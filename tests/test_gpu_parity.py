@@ -382,6 +382,41 @@ def test_attention(Bk, Bv, g, n_seq, n_kv, n_tok, n_tail, law, qs, vs):
                   f"logit error {dl_norm.max():.2e}")
 
 
+def test_attention_narrow_codec():
+    """d = 96, m = 64: the zero-padded coordinates and sketch rows of the 128-wide blocks."""
+    d, m, g, n_tok, n_tail = 96, 64, 2, 200, 9
+    pik, sk, piv = ti.haar_rotation(d, 98), ti.gaussian_sketch(m, d, 99), ti.haar_rotation(d, 100)
+    rng = np.random.default_rng(101)
+    keys = ti.f32_to_bf16_bits(rng.standard_normal((n_tok + n_tail, d)).astype(np.float32))
+    vals = ti.f32_to_bf16_bits(rng.standard_normal((n_tok + n_tail, d)).astype(np.float32))
+    qb = ti.f32_to_bf16_bits(rng.standard_normal((1, g, d)).astype(np.float32))
+    kc = make_codec(d, m, 2, True, pik, sk)
+    vc = make_codec(d, 0, 3, False, piv, None)
+    pk, _ = gpu_quantize(kc, to_dev_bf16(keys[:n_tok]), 1, n_tok)
+    pvv, _ = gpu_quantize(vc, to_dev_bf16(vals[:n_tok]), 1, n_tok)
+    tk, tv = to_dev_bf16(keys[n_tok:]), to_dev_bf16(vals[n_tok:])
+    scale = 1.0 / math.sqrt(d)
+    got = _attention_gpu(kc, vc, pk, pvv, 1, 1, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)[0]
+    lg = _logits_gpu(kc, pk, 1, 1, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
+    kidx, ksb, knh, kgh = unpack(kc, pk, 1, n_tok)
+    vidx, vnh = unpack(vc, pvv, 1, n_tok)
+    c_k, _ = _cb(d, 2)
+    c_v, _ = _cb(d, 3)
+    q = ti.bf16_to_f64(qb)[0]
+    kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
+    want = oracle.attention(kidx[0], ksb[0], knh[0], kgh[0], pik, sk, c_k, vidx[0], vnh[0], piv, c_v, q, scale,
+                            tail_k=kf[n_tok:], tail_v=vf[n_tok:])
+    lo = oracle.logits(kidx[0], ksb[0], knh[0], kgh[0], pik, sk, c_k, q, qjl=True, scale=scale)
+    L = np.concatenate([lo, oracle.exact_dot(kf[n_tok:], q, scale)], axis=1)
+    w = np.exp(L - L.max(axis=1, keepdims=True))
+    w /= w.sum(axis=1, keepdims=True)
+    vnorm = np.concatenate([vnh[0], np.linalg.norm(vf[n_tok:], axis=1)])
+    dl = np.abs(lg - L).max(axis=1)
+    err = np.max(np.abs(got - want), axis=1) / (w @ vnorm)
+    assert np.all(np.isfinite(got))
+    assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), err
+
+
 def test_attention_rejects_unsupported():
     torch = torch_cuda()
     m = tq()
