@@ -133,23 +133,32 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         uint8_t* bt = at + 2 * 16 * 256;                            // Pi hi, Pi lo, M hi, M lo [128][256 B]
         __shared__ float s_qsc[16];
         const uint32_t sat = tq_smem_addr(at), sbt = tq_smem_addr(bt);
+        // every global load of this phase is issued before any is used: the query row of
+        // this warp's head, then the 16 B-tile chunks of this thread
+        float xq[4];
+        {
+            const int h = wid;   // 16 warps, 16 rows
+            const bool ok = h < H && (int64_t)(h_base + h) < p.n_heads_valid;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * lane + k;
+                xq[k] = ok && j < d ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
+            }
+        }
         {   // B tiles, swizzled rows
             const uint16_t* srcs[4] = {p.pih, p.pil, p.mh, p.ml};
+            uint4 v[16];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint4 v[8];
+            for (int k = 0; k < 16; ++k) {
+                const int e = tid + kPrologueThreads * k;
+                const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
+                v[k] = __ldg(reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8));
+            }
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int e = tid + kPrologueThreads * (8 * half + k);
-                    const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
-                    v[k] = __ldg(reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8));
-                }
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int e = tid + kPrologueThreads * (8 * half + k);
-                    const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
-                    *reinterpret_cast<uint4*>(bt + m * 32768 + tq_swz256(row, ch)) = v[k];
-                }
+            for (int k = 0; k < 16; ++k) {
+                const int e = tid + kPrologueThreads * k;
+                const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
+                *reinterpret_cast<uint4*>(bt + m * 32768 + tq_swz256(row, ch)) = v[k];
             }
         }
         // A rows: warp w = head w; lane l holds coordinates 4l .. 4l + 3, scaled per row by a power
@@ -171,17 +180,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                                                                    *reinterpret_cast<const uint32_t*>(&l1));
             if (lane == 0) s_qsc[row] = scale_of_max / sc;
         };
-        {
-            const int h = wid;   // 16 warps, 16 rows
-            const bool ok = h < H && (int64_t)(h_base + h) < p.n_heads_valid;
-            float x[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = 4 * lane + k;
-                x[k] = ok && j < d ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
-            }
-            put_row(h, x, 1.f / 256.f);
-        }
+        put_row(wid, xq, 1.f / 256.f);
         __syncthreads();
         // one 16 x 8 output tile per warp over K = 128: A hi/lo x B hi/lo (three passes)
         const int mi = lane >> 3, r8 = lane & 7;
