@@ -287,7 +287,7 @@ def run_gpu(args, world, rank, local):
 
     # DRAM bytes (read + write) per launch of these kernels on this workload, from one ncu
     # capture each (profiles/k_quantize_tc_c4_append.md, profiles/k_logits_stream_c4.md)
-    ncu_traffic = {"tq_quantize": 67.31e6 + 2.05e6, "tq_logits": 0.69e6 + 220.86e6 + 48.48e6}
+    ncu_traffic = {"tq_quantize": 67.31e6 + 1.41e6, "tq_logits": 0.69e6 + 220.82e6 + 48.26e6}
     # kernels launched per step: quantize 1, logits 2 (prologue + stream)
     launches_per_step = 3
     dominant = "tq_logits" if t_logit >= t_quant else "tq_quantize"
