@@ -103,3 +103,39 @@ def test_argument_checks_fail_before_device_work(tq):
     assert tq.lib.tq_make_codebook(2, 2, np.zeros(4).ctypes.data, np.zeros(3).ctypes.data, None) == \
         tq.TQ_ERR_UNSUPPORTED
     assert tq.lib.tq_status_string(tq.TQ_ERR_RANGE).decode().startswith("norm")
+
+
+def test_attention_host_checks(tq):
+    """tq_attention: workspace sizing and argument checks, all before any device work."""
+    k, keep_k = _codec(tq, B=3)
+    v, keep_v = _codec(tq, qjl=0, m=0, B=4)
+    for c in (k, v):
+        c.prep, c.prep_bytes = 0x100000, 1 << 30
+    K, V = ctypes.byref(k), ctypes.byref(v)
+    ws = tq.lib.tq_attention_workspace_bytes
+    w0 = ws(K, V, 1, 8, 32640, 4, 0)
+    w1 = ws(K, V, 1, 8, 32640, 4, 128)
+    assert w0 > 0 and w0 % 256 == 0
+    assert w1 - w0 >= 8 * 4 * 128 * 4          # one fp32 tail logit per (query head, tail token)
+    assert ws(K, V, 1, 8, 320, 4, 128) < w1    # two ranges per stream instead of about one per SM
+    assert ws(K, V, 1, 8, 32640, 8, 0) == 0    # g = 8: outside the fused head tile
+    assert ws(V, K, 1, 8, 32640, 4, 0) == 0    # key and value codecs swapped
+    wide, keep_w = _codec(tq, d=200, m=200, B=2)
+    wide.prep, wide.prep_bytes = 0x100000, 1 << 30
+    assert ws(ctypes.byref(wide), V, 1, 8, 320, 4, 0) == 0   # d > 128
+
+    def call(n_seq=1, n_tok=320, g=4, tail_k=0x5000, tail_v=0x6000, n_tail=8, scale=0.125, v_skip=0.0,
+             wsb=1 << 24, packed_k=0x1000, q_dtype=tq.TQ_BF16):
+        return tq.lib.tq_attention(K, V, packed_k, 0x2000, n_seq, 8, n_tok, 0x3000, q_dtype, g, tail_k, tail_v,
+                                   n_tail, scale, v_skip, 0x4000, 0x100000, wsb, None)
+    assert call(n_seq=0) == tq.TQ_OK                                   # nothing to do
+    assert call(g=8) == tq.TQ_ERR_UNSUPPORTED
+    assert call(n_tok=0, n_tail=0) == tq.TQ_ERR_ARG                    # a softmax over no tokens
+    assert call(n_tail=9000) == tq.TQ_ERR_UNSUPPORTED                  # above TQ_ATTN_MAX_TAIL
+    assert call(tail_v=0x6004) == tq.TQ_ERR_ARG                        # tail values need 8-byte rows
+    assert call(packed_k=0x1008) == tq.TQ_ERR_ARG                      # packed caches are 16-byte aligned
+    assert call(v_skip=1.5) == tq.TQ_ERR_ARG
+    assert call(v_skip=float("nan")) == tq.TQ_ERR_ARG
+    assert call(scale=float("inf")) == tq.TQ_ERR_ARG
+    assert call(q_dtype=5) == tq.TQ_ERR_ARG
+    assert call(wsb=ws(K, V, 1, 8, 320, 4, 8) - 1) == tq.TQ_ERR_WORKSPACE
