@@ -185,6 +185,27 @@ def pv(idx, nhat, pi, c, P) -> np.ndarray:
     return out
 
 
+def fwht_rotate(x, signs) -> np.ndarray:
+    """y = H (D x) / sqrt(d) for every row of x, by the O(d log d) butterflies of the fast
+    Walsh-Hadamard transform (ai-coding.wiselychen.com "Google TurboQuant KV-cache
+    compression", community ports: the rotation as a Walsh-Hadamard transform); d a power of
+    two, signs the +-1 diagonal D. The structured counterpart of a dense Pi = H D / sqrt(d)."""
+    y = _f64(x) * _f64(signs)[None, :]
+    y = y.reshape(-1, y.shape[-1]).copy()
+    d = y.shape[1]
+    if d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = 1
+    while h < d:
+        for i in range(0, d, 2 * h):
+            a = y[:, i:i + h].copy()
+            b = y[:, i + h:i + 2 * h].copy()
+            y[:, i:i + h] = a + b
+            y[:, i + h:i + 2 * h] = a - b
+        h *= 2
+    return y / np.sqrt(d)
+
+
 def _attention_parts(k_idx, k_sbit, k_nhat, k_ghat, pi_k, s_k, c_k, v_idx, v_nhat, pi_v, c_v, q, scale,
                      tail_k, tail_v):
     """Logits [nh, n], values [n, d] and the compressed-token count of one kv stream."""

@@ -417,6 +417,51 @@ def test_attention_narrow_codec():
     assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), err
 
 
+def test_hadamard_rotation_path():
+    """A randomized Walsh-Hadamard rotation H D / sqrt(d) as Pi (dense operand) for keys and
+    values: codes against the oracle's quantization, logits and fused attention against the
+    oracle on the same codes."""
+    d = m = 128
+    pik, piv = ti.hadamard_rotation(d, 31), ti.hadamard_rotation(d, 32)
+    sk = ti.gaussian_sketch(m, d, 33)
+    n_kv, n_tok, n_tail, g, B = 2, 700, 6, 4, 2
+    keys = np.stack([ti.key_stream(4, 0, h, n_tok + n_tail) for h in range(n_kv)])
+    vals = np.stack([_normal_stream(71, 0, h, n_tok + n_tail) for h in range(n_kv)])
+    kc = make_codec(d, m, B, True, pik, sk)
+    vc = make_codec(d, 0, 3, False, piv, None)
+    pk, st = gpu_quantize(kc, to_dev_bf16(np.ascontiguousarray(keys[:, :n_tok]).reshape(-1, d)), n_kv, n_tok)
+    assert st == tq().TQ_OK
+    pvv, _ = gpu_quantize(vc, to_dev_bf16(np.ascontiguousarray(vals[:, :n_tok]).reshape(-1, d)), n_kv, n_tok)
+    kidx, ksb, knh, kgh = unpack(kc, pk, n_kv, n_tok)
+    vidx, vnh = unpack(vc, pvv, n_kv, n_tok)
+    c_k, t_k = _cb(d, B)
+    c_v, _ = _cb(d, 3)
+    kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
+    for h in range(n_kv):
+        ref = oracle.quantize(kf[h, :n_tok], pik, sk, c_k, t_k, B, qjl=True)
+        compare_codes(kidx[h], ksb[h], knh[h], kgh[h], ref, t_k, x=kf[h, :n_tok], pi=pik, s=sk, c=c_k, t=t_k, B=B)
+    qb = ti.decode_queries(13, 1, n_kv * g)
+    scale = 1.0 / math.sqrt(d)
+    tk = to_dev_bf16(np.ascontiguousarray(keys[:, n_tok:]))
+    tv = to_dev_bf16(np.ascontiguousarray(vals[:, n_tok:]))
+    lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
+    got = _attention_gpu(kc, vc, pk, pvv, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale)[0]
+    q = ti.bf16_to_f64(qb)[0]
+    for h in range(n_kv):
+        qh = q[h * g:(h + 1) * g]
+        lo = oracle.logits(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, qh, qjl=True, scale=scale)
+        _check_logits(lg[h * g:(h + 1) * g, :n_tok], lo, qh, np.linalg.norm(kf[h, :n_tok], axis=1), scale)
+        want = oracle.attention(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, vidx[h], vnh[h], piv, c_v, qh, scale,
+                                tail_k=kf[h, n_tok:], tail_v=vf[h, n_tok:])
+        L = np.concatenate([lo, oracle.exact_dot(kf[h, n_tok:], qh, scale)], axis=1)
+        w = np.exp(L - L.max(axis=1, keepdims=True))
+        w /= w.sum(axis=1, keepdims=True)
+        vnorm = np.concatenate([vnh[h], np.linalg.norm(vf[h, n_tok:], axis=1)])
+        dl = np.abs(lg[h * g:(h + 1) * g] - L).max(axis=1)
+        err = np.max(np.abs(got[h * g:(h + 1) * g] - want), axis=1) / (w @ vnorm)
+        assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), err
+
+
 def test_attention_rejects_unsupported():
     torch = torch_cuda()
     m = tq()

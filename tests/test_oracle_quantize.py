@@ -39,6 +39,39 @@ def test_rotation_gaussianises_outlier_data():
     assert abs(k_after - g["kurt_after"]) < 0.1 and k_after < g["kurt_gauss"]
 
 
+def test_hadamard_rotation_and_fast_transform():
+    # randomized Walsh-Hadamard rotation H D / sqrt(d) (ai-coding.wiselychen.com, community
+    # ports: rotation by a Walsh-Hadamard transform): orthogonal, entries +-1/sqrt(d), and the
+    # oracle's butterflies give the dense product
+    s2 = ti.hadamard_signs(2, 5)
+    assert np.allclose(ti.hadamard_rotation(2, 5), np.array([[s2[0], s2[1]], [s2[0], -s2[1]]]) / math.sqrt(2))
+    rng = np.random.default_rng(12)
+    for d in (2, 8, 128):
+        p = ti.hadamard_rotation(d, 40 + d)
+        assert np.max(np.abs(p.T @ p - np.eye(d))) < 1e-12
+        assert np.allclose(np.abs(p), 1.0 / math.sqrt(d), rtol=0, atol=1e-15)
+        x = rng.standard_normal((7, d))
+        y = oracle.fwht_rotate(x, ti.hadamard_signs(d, 40 + d))
+        assert np.max(np.abs(y - x @ p.T)) < 1e-12
+        # without the signs the normalised transform is an involution
+        assert np.max(np.abs(oracle.fwht_rotate(oracle.fwht_rotate(x, np.ones(d)), np.ones(d)) - x)) < 1e-12
+    with pytest.raises(ValueError):
+        ti.hadamard_rotation(200, 1)
+
+
+def test_hadamard_rotation_kurtosis_closed_form():
+    # Each rotated coordinate of a fixed unit vector u is a Rademacher sum sum_j +-u_j, whose
+    # fourth moment is 3 - 2 sum_j u_j^4: an outlier key keeps lighter tails than under a
+    # Haar rotation (3d/(d+2)).
+    d = 128
+    keys = ti.bf16_to_f64(ti.key_stream(2, 0, 0, 1, d))
+    u = keys[0] / np.linalg.norm(keys[0])
+    y = np.concatenate([oracle.fwht_rotate(u[None, :], ti.hadamard_signs(d, 9000 + k))[0] for k in range(400)])
+    y *= math.sqrt(d)
+    assert abs(stats.kurtosis(y, fisher=False) - (3.0 - 2.0 * np.sum(u ** 4))) < 0.05
+    assert abs(np.mean(y ** 2) - 1.0) < 0.02
+
+
 def _codebook(d, bits):
     c, t, _, _ = oracle.codebook(d, bits)
     return c, t

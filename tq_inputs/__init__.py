@@ -53,6 +53,23 @@ def haar_rotation(d: int, seed: int) -> np.ndarray:
     return q * np.sign(np.diag(r))[None, :]
 
 
+def hadamard_signs(d: int, seed: int) -> np.ndarray:
+    """The random +-1 diagonal D of a randomized Hadamard rotation (fp64 [d])."""
+    return np.where(np.random.default_rng(seed).integers(0, 2, d) == 1, 1.0, -1.0)
+
+
+def hadamard_rotation(d: int, seed: int) -> np.ndarray:
+    """Structured random rotation H D / sqrt(d) (fp64 [d, d]) for d a power of two: H the
+    Sylvester Walsh-Hadamard matrix (H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]]), D the
+    seeded +-1 diagonal of hadamard_signs. It enters the library as a dense Pi."""
+    if d < 1 or d & (d - 1):
+        raise ValueError("d must be a power of two")
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h * hadamard_signs(d, seed)[None, :] / np.sqrt(d)
+
+
 def gaussian_sketch(m: int, d: int, seed: int) -> np.ndarray:
     """QJL projection S (fp64), i.i.d. N(0,1), row-major [m, d]."""
     return np.random.default_rng(seed).standard_normal((m, d))
