@@ -77,6 +77,14 @@ typedef struct {
     size_t prep_bytes;
 } tq_codec;
 
+/* Score estimators for packed keys (tq_logits_est, tq_topk_est):
+ *   TQ_EST_QJL  |x| (<Pi q, c[idx]> + gamma sqrt(pi/2)/m <S q, s>), unbiased (the default);
+ *   TQ_EST_MSE  |x| <Pi q, c[idx]>, the MSE stage alone: the stored signs and gamma are not
+ *               used (blog.hotdry.top, monitoring notes: in some settings the QJL correction
+ *               lowers ranking quality and an MSE-only mode is preferred). The key records
+ *               are the same; only the estimate changes.                                    */
+enum { TQ_EST_QJL = 0, TQ_EST_MSE = 1 };
+
 /* Operations, for tq_workspace_bytes */
 enum { TQ_OP_QUANTIZE = 0, TQ_OP_LOGITS = 1, TQ_OP_PV = 2, TQ_OP_TOPK = 3, TQ_OP_DEQUANTIZE = 4 };
 
@@ -138,6 +146,11 @@ int tq_quantize(const tq_codec* codec, const void* x, tq_dtype dtype, int64_t n_
 int tq_logits(const tq_codec* codec, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok,
               const void* q, tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale,
               float* out, void* ws, size_t ws_bytes, void* stream);
+/* tq_logits with the estimator chosen (TQ_EST_QJL or TQ_EST_MSE; else TQ_ERR_ARG); the same
+ * workspace and layouts. tq_logits is tq_logits_est with TQ_EST_QJL.                      */
+int tq_logits_est(const tq_codec* codec, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok,
+                  const void* q, tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale,
+                  float* out, void* ws, size_t ws_bytes, int estimator, void* stream);
 
 /* softmax(P) . V over MSE-only packed values (friday-blog-bgf.pages.dev, section 1, step 1;
  * accumulated in the rotated domain and rotated back once by Pi^T).
@@ -191,6 +204,11 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
  *   ws       tq_workspace_bytes(codec, TQ_OP_TOPK, n_q, n_db, k) bytes.                   */
 int tq_topk(const tq_codec* codec, const void* packed_db, int64_t n_db, const float* q,
             int64_t n_q, int k, int64_t* idx, float* score, void* ws, size_t ws_bytes, void* stream);
+/* tq_topk with the estimator chosen (TQ_EST_QJL or TQ_EST_MSE; else TQ_ERR_ARG); tq_topk is
+ * tq_topk_est with TQ_EST_QJL.                                                               */
+int tq_topk_est(const tq_codec* codec, const void* packed_db, int64_t n_db, const float* q,
+                int64_t n_q, int k, int64_t* idx, float* score, void* ws, size_t ws_bytes,
+                int estimator, void* stream);
 
 /* tq_logits without a caller workspace, for callers that cannot allocate device memory:
  * code inside a host framework whose pool owns all device memory, plugins that may only use

@@ -24,10 +24,11 @@ TQ_OK, TQ_ERR_ARG, TQ_ERR_UNSUPPORTED, TQ_ERR_CUDA = 0, -1, -2, -3
 TQ_ERR_RANGE, TQ_ERR_TIMEOUT, TQ_ERR_NOCONV, TQ_ERR_WORKSPACE = -4, -5, -6, -7
 TQ_F32, TQ_BF16 = 0, 1
 TQ_OP_QUANTIZE, TQ_OP_LOGITS, TQ_OP_PV, TQ_OP_TOPK, TQ_OP_DEQUANTIZE = 0, 1, 2, 3, 4
+TQ_EST_QJL, TQ_EST_MSE = 0, 1
 EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_bytes", "tq_prep_bytes",
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
             "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",
-            "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes"]
+            "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes", "tq_logits_est", "tq_topk_est"]
 
 
 class tq_codec(ctypes.Structure):
@@ -53,6 +54,8 @@ _sig = {
     "tq_attention_workspace_bytes": (_SZ, [_CP, _CP, _I64, _I, _I64, _I, _I]),
     "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _F, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
+    "tq_logits_est": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _I, _P]),
+    "tq_topk_est": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _I, _P]),
     "tq_dequantize": (_I, [_CP, _P, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_reset_status": (_I, [_P, _P]),
     "tq_get_status": (_I, [_P, _P]),
@@ -156,10 +159,15 @@ def tq_quantize(codec: Codec, x, n_streams, n_tok, x_stream_stride, packed, ws, 
                                                  _ptr(packed), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def tq_logits(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_tail, scale, out, ws, stream=None):
-    return _check("tq_logits", lib.tq_logits(codec.ref, _ptr(packed), n_seq, n_kv, n_tok, _ptr(q), _dtype(q), g,
-                                             _ptr(tail), n_tail, scale, _ptr(out), _ptr(ws), ws.numel(),
-                                             _stream(stream)))
+def tq_logits(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_tail, scale, out, ws, stream=None,
+              estimator=None):
+    if estimator is None:
+        return _check("tq_logits", lib.tq_logits(codec.ref, _ptr(packed), n_seq, n_kv, n_tok, _ptr(q), _dtype(q), g,
+                                                 _ptr(tail), n_tail, scale, _ptr(out), _ptr(ws), ws.numel(),
+                                                 _stream(stream)))
+    return _check("tq_logits_est", lib.tq_logits_est(codec.ref, _ptr(packed), n_seq, n_kv, n_tok, _ptr(q), _dtype(q),
+                                                     g, _ptr(tail), n_tail, scale, _ptr(out), _ptr(ws), ws.numel(),
+                                                     estimator, _stream(stream)))
 
 
 def tq_logits_noalloc(codec: Codec, packed, n_seq, n_kv, n_tok, q, g, tail, n_tail, scale, out, stream=None):
@@ -185,9 +193,12 @@ def tq_attention(kcodec: Codec, vcodec: Codec, packed_k, packed_v, n_seq, n_kv, 
                                                    scale, v_skip, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=None):
-    return _check("tq_topk", lib.tq_topk(codec.ref, _ptr(packed_db), n_db, _ptr(q), n_q, k, _ptr(idx), _ptr(score),
-                                         _ptr(ws), ws.numel(), _stream(stream)))
+def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=None, estimator=None):
+    if estimator is None:
+        return _check("tq_topk", lib.tq_topk(codec.ref, _ptr(packed_db), n_db, _ptr(q), n_q, k, _ptr(idx),
+                                             _ptr(score), _ptr(ws), ws.numel(), _stream(stream)))
+    return _check("tq_topk_est", lib.tq_topk_est(codec.ref, _ptr(packed_db), n_db, _ptr(q), n_q, k, _ptr(idx),
+                                                 _ptr(score), _ptr(ws), ws.numel(), estimator, _stream(stream)))
 
 
 def tq_dequantize(codec: Codec, packed, n_streams, n_tok, out, ws=None, stream=None):

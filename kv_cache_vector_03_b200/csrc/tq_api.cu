@@ -303,11 +303,12 @@ int tq_quantize(const tq_codec* c, const void* x, tq_dtype dtype, int64_t n_stre
     return cuda_status(tq_launch_quantize(p, static_cast<cudaStream_t>(stream)));
 }
 
-int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
-              tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
-              size_t ws_bytes, void* stream) {
+int tq_logits_est(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+                  tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
+                  size_t ws_bytes, int estimator, void* stream) {
     int st = check_codec(c, true);
     if (st != TQ_OK) return st;
+    if (estimator != TQ_EST_QJL && estimator != TQ_EST_MSE) return TQ_ERR_ARG;
     if (!c->qjl) return TQ_ERR_ARG;
     if (g != 1 && g != 2 && g != 4 && g != 8) return TQ_ERR_UNSUPPORTED;
     if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0) return TQ_ERR_ARG;
@@ -339,7 +340,8 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.n_seq = n_seq; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
     p.n_kv = n_kv; p.g = g; p.ntiles = g > 4 ? 2 : 1; p.n_tail = n_tail;
     p.scale = scale;
-    p.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
+    // the MSE-only estimator drops the QJL term (its constants become zero)
+    p.kappa = estimator == TQ_EST_MSE ? 0.f : (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.status = static_cast<uint32_t*>(ws);
     p.n_heads_valid = n_streams * g;
     // the tail runs on a second grid dimension of 16-token CTAs (at most 65535)
@@ -348,6 +350,13 @@ int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, in
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_logits(p, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+              tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
+              size_t ws_bytes, void* stream) {
+    return tq_logits_est(c, packed, n_seq, n_kv, n_tok, q, q_dtype, g, tail, n_tail, scale, out, ws, ws_bytes,
+                         TQ_EST_QJL, stream);
 }
 
 int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int64_t n_tok, const float* P, int g,
@@ -463,10 +472,11 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
     return cuda_status(tq_launch_attention(p, cs));
 }
 
-int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,
-            float* score, void* ws, size_t ws_bytes, void* stream) {
+int tq_topk_est(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k,
+                int64_t* idx, float* score, void* ws, size_t ws_bytes, int estimator, void* stream) {
     int st = check_codec(c, true);
     if (st != TQ_OK) return st;
+    if (estimator != TQ_EST_QJL && estimator != TQ_EST_MSE) return TQ_ERR_ARG;
     if (!c->qjl) return TQ_ERR_ARG;
     if (n_q < 0 || n_db < 1 || n_db > 0x7fffffffLL || k < 1 || k > 32 || k > n_db) return TQ_ERR_ARG;
     if (n_q == 0) return TQ_OK;
@@ -494,7 +504,7 @@ int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float*
     lp.status = static_cast<uint32_t*>(ws);
     lp.n_seq = 1; lp.n_kv = W.n_groups; lp.g = 4; lp.ntiles = 1; lp.n_tok = 0; lp.nb = 0; lp.n_tail = 0;
     lp.scale = 1.f;
-    lp.kappa = (float)(std::sqrt(M_PI / 2.0) / c->m);
+    lp.kappa = estimator == TQ_EST_MSE ? 0.f : (float)(std::sqrt(M_PI / 2.0) / c->m);
     lp.n_heads_valid = n_q;
     lp.t = t;
     if ((st = codebook_consts(c, &lp.cb)) != TQ_OK) return st;
@@ -513,6 +523,11 @@ int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float*
     p.k = k; p.nsplit = W.nsplit; p.blocks_per_split = W.bps; p.n_groups = W.n_groups;
     p.t = t;
     return cuda_status(tq_launch_topk(p, cs));
+}
+
+int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,
+            float* score, void* ws, size_t ws_bytes, void* stream) {
+    return tq_topk_est(c, packed_db, n_db, q, n_q, k, idx, score, ws, ws_bytes, TQ_EST_QJL, stream);
 }
 
 int tq_dequantize(const tq_codec* c, const void* packed, int64_t n_streams, int64_t n_tok, float* out, void* ws,

@@ -509,13 +509,13 @@ def test_dequantize_reconstruction(qjl, B):
 
 
 # ----------------------------------------------------------------------------- top-k
-def _topk_gpu(codec, packed, n_db, q_dev, n_q, k):
+def _topk_gpu(codec, packed, n_db, q_dev, n_q, k, estimator=None):
     torch = torch_cuda()
     m = tq()
     idx = torch.full((n_q, k), -7, dtype=torch.int64, device="cuda")
     score = torch.full((n_q, k), float("nan"), dtype=torch.float32, device="cuda")
     ws = m.workspace(codec.workspace_bytes(m.TQ_OP_TOPK, n_q, n_db, k))
-    m.tq_topk(codec, packed, n_db, q_dev, n_q, k, idx, score, ws)
+    m.tq_topk(codec, packed, n_db, q_dev, n_q, k, idx, score, ws, estimator=estimator)
     torch.cuda.synchronize()
     return idx.cpu().numpy(), score.cpu().numpy().astype(np.float64)
 
@@ -560,6 +560,48 @@ def test_topk_against_oracle(B, n_db, n_q, k):
                         k=min(k, 500))
     assert oi.shape == (3, min(k, 500))
     print(f"top-{k}: {swaps} near-tie swaps over {n_q} queries")
+
+
+def test_mse_only_estimator():
+    """TQ_EST_MSE on QJL key records: logits and top-k equal the oracle's MSE-stage estimate
+    |x| <Pi q, c[idx]> on the same codes (signs and gamma unused)."""
+    torch = torch_cuda()
+    m = tq()
+    d = mm = 128
+    pi, s = ti.haar_rotation(d, 111), ti.gaussian_sketch(mm, d, 112)
+    n_kv, n_tok, g, B = 2, 333, 4, 3
+    keys = np.stack([ti.key_stream(4, 1, h, n_tok) for h in range(n_kv)])
+    codec = make_codec(d, mm, B, True, pi, s)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(keys.reshape(-1, d)), n_kv, n_tok)
+    qb = ti.decode_queries(14, 1, n_kv * g)
+    out = torch.full((1, n_kv * g, n_tok), float("nan"), dtype=torch.float32, device="cuda")
+    ws = m.workspace(codec.workspace_bytes(m.TQ_OP_LOGITS, 1, n_kv, g))
+    m.tq_logits(codec, packed, 1, n_kv, n_tok, to_dev_bf16(qb), g, None, 0, 0.5, out, ws, estimator=m.TQ_EST_MSE)
+    got = out.cpu().numpy().astype(np.float64)[0]
+    idx, sbit, nhat, ghat = unpack(codec, packed, n_kv, n_tok)
+    c, _ = _cb(d, B)
+    q = ti.bf16_to_f64(qb)[0]
+    kf = ti.bf16_to_f64(keys)
+    for h in range(n_kv):
+        qh = q[h * g:(h + 1) * g]
+        want = oracle.logits(idx[h], sbit[h], nhat[h], ghat[h], pi, s, c, qh, qjl=False, scale=0.5)
+        _check_logits(got[h * g:(h + 1) * g], want, qh, np.linalg.norm(kf[h], axis=1), 0.5)
+        full = oracle.logits(idx[h], sbit[h], nhat[h], ghat[h], pi, s, c, qh, qjl=True, scale=0.5)
+        assert np.max(np.abs(want - full)) > 1e-2   # the QJL term is really gone
+    with pytest.raises(m.TQError):
+        m.tq_logits(codec, packed, 1, n_kv, n_tok, to_dev_bf16(qb), g, None, 0, 0.5, out, ws, estimator=7)
+    # top-k with the MSE-only score
+    dd = 200
+    pi5, s5 = ti.C5.pi(), ti.C5.s()
+    x = ti.c5_rows("db", 0, 3000)
+    qs = ti.c5_rows("q", 0, 21)
+    c5 = make_codec(dd, dd, 2, True, pi5, s5)
+    pk5, _ = gpu_quantize(c5, to_dev_f32(x), 1, 3000)
+    gidx, gsc = _topk_gpu(c5, pk5, 3000, to_dev_f32(qs), 21, 10, estimator=m.TQ_EST_MSE)
+    i5, sb5, nh5, gh5 = unpack(c5, pk5, 1, 3000)
+    cc5, _ = _cb(dd, 2)
+    all_scores = oracle.logits(i5[0], sb5[0], nh5[0], gh5[0], pi5, s5, cc5, qs.astype(np.float64), qjl=False)
+    check_topk(gidx, gsc, all_scores, qs.astype(np.float64), np.linalg.norm(x.astype(np.float64), axis=1), 10)
 
 
 def test_topk_d128_codec():
