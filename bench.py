@@ -428,6 +428,25 @@ def extra_workloads(torch, tq, ti, gen, peaks):
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
             "timing": "CUDA-graph replays of 12 calls"}
         del keys, packs, vals, vpacks
+    # the key side of the asymmetric configuration at c2: 8-bit keys (q8_0-style), same queries and tail
+    keys = make_keys_device(torch, gen, n_kv, n_all, n_kv)
+    copies = 12
+    q8s = []
+    for _ in range(copies):
+        pk = torch.empty(tq.tq_q8_packed_bytes(d, n_kv, n_tok), dtype=torch.uint8, device="cuda")
+        tq.tq_q8_quantize(keys, d, n_kv, n_tok, n_all * d, pk, tq.workspace(256))
+        q8s.append(pk)
+    tail = keys[:, n_tok:].contiguous()
+    q = torch.randn((1, n_kv * 4, d), generator=gen, device="cuda").to(torch.bfloat16)
+    lo = torch.empty((1, n_kv * 4, n_all), dtype=torch.float32, device="cuda")
+    ms = time_graph(torch, lambda i: tq.tq_q8_logits(q8s[i % copies], d, 1, n_kv, n_tok, q, 4, tail, n_tail,
+                                                     1.0 / math.sqrt(d), lo), copies)
+    byts = n_kv * n_tok * 136 + n_kv * n_tail * d * 2 + lo.numel() * 4
+    out["c2_llama8b_decode_logits_q8_keys"] = {
+        "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
+        "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA-graph replays of 12 calls"}
+    del keys, q8s
     # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
     n_kv, n_tok, g = 8, 131072, 4
     vals = torch.randn((n_kv, n_tok, d), generator=gen, device="cuda").to(torch.bfloat16)

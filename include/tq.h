@@ -230,6 +230,33 @@ int tq_logits_noalloc(const tq_codec* codec, const void* packed, int64_t n_seq, 
                       const void* q, tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale,
                       float* out, void* stream);
 
+/* 8-bit keys, the key side of the asymmetric K/V configuration (blog.hotdry.top "TurboQuant
+ * vector-search compression", engineering configuration list: q8_0 keys with TurboQuant
+ * values). No rotation or codebook: per 32-coordinate chunk of a key, scale
+ * s = max|x| / 127 (fp32), codes rint(x / s) (fp32 division, round half to even, clamped to
+ * +-127), stored scale = s rounded to binary16; the key reads back as code * scale.
+ * Record: d <= 128 (multiple of 8) padded to 128 coordinates, 136 bytes per key, in blocks
+ * of 32 tokens: codes [column j = 0..7][token][16 B] (coordinates 16j .. 16j+15), then
+ * scales [chunk c = 0..3][token] binary16. Stream s occupies blocks
+ * [s * ceil(n_tok/32), (s+1) * ceil(n_tok/32)); padding tokens are zero.
+ *   tq_q8_packed_bytes: bytes of n_streams x n_tok keys, 0 if d is unsupported.
+ *   tq_q8_quantize: x device fp32 or bf16, vector t of stream s at s * x_stream_stride + t * d;
+ *            packed 16-byte aligned; ws: TQ_STATUS_BYTES (status word: TQ_ERR_RANGE when a
+ *            value is not finite or a scale overflows binary16).
+ *   tq_q8_logits: out fp32 [n_seq, n_kv * g, n_tok + n_tail] = scale <q, k~> for the packed
+ *            keys followed by the exact scale <q, k> of the bf16 tail ([n_seq, n_kv, n_tail,
+ *            d], n_tail <= TQ_Q8_MAX_TAIL); q device [n_seq, n_kv * g, d] fp32 or bf16;
+ *            g in {1, 2, 4}. The query is rounded to int16 fixed point per head (step
+ *            max|q| / 16383): the error is at most sqrt(d) / 32766 of scale |q| |k~|. No
+ *            workspace.                                                                        */
+#define TQ_Q8_MAX_TAIL 65536
+size_t tq_q8_packed_bytes(int d, int64_t n_streams, int64_t n_tok);
+int tq_q8_quantize(const void* x, tq_dtype dtype, int d, int64_t n_streams, int64_t n_tok,
+                   int64_t x_stream_stride, void* packed, void* ws, size_t ws_bytes, void* stream);
+int tq_q8_logits(const void* packed, int d, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+                 tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out,
+                 void* stream);
+
 /* Diagnostic reconstruction (not on the hot path): x~ = |x|(Pi^T c[idx] + gamma
  * sqrt(pi/2)/m S^T s) for keys, |x| Pi^T c[idx] for values (blog.hotdry.top, "QJL residual
  * correction"). out: device fp32 [n_streams, n_tok, d].                                  */

@@ -28,7 +28,8 @@ TQ_EST_QJL, TQ_EST_MSE = 0, 1
 EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_bytes", "tq_prep_bytes",
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
             "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",
-            "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes", "tq_logits_est", "tq_topk_est"]
+            "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes", "tq_logits_est", "tq_topk_est",
+            "tq_q8_packed_bytes", "tq_q8_quantize", "tq_q8_logits"]
 
 
 class tq_codec(ctypes.Structure):
@@ -55,6 +56,9 @@ _sig = {
     "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _F, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "tq_logits_est": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _I, _P]),
+    "tq_q8_packed_bytes": (_SZ, [_I, _I64, _I64]),
+    "tq_q8_quantize": (_I, [_P, _I, _I, _I64, _I64, _I64, _P, _P, _SZ, _P]),
+    "tq_q8_logits": (_I, [_P, _I, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P]),
     "tq_topk_est": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _I, _P]),
     "tq_dequantize": (_I, [_CP, _P, _I64, _I64, _P, _P, _SZ, _P]),
     "tq_reset_status": (_I, [_P, _P]),
@@ -199,6 +203,20 @@ def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=Non
                                              _ptr(score), _ptr(ws), ws.numel(), _stream(stream)))
     return _check("tq_topk_est", lib.tq_topk_est(codec.ref, _ptr(packed_db), n_db, _ptr(q), n_q, k, _ptr(idx),
                                                  _ptr(score), _ptr(ws), ws.numel(), estimator, _stream(stream)))
+
+
+def tq_q8_packed_bytes(d, n_streams, n_tok):
+    return lib.tq_q8_packed_bytes(d, n_streams, n_tok)
+
+
+def tq_q8_quantize(x, d, n_streams, n_tok, x_stream_stride, packed, ws, stream=None):
+    return _check("tq_q8_quantize", lib.tq_q8_quantize(_ptr(x), _dtype(x), d, n_streams, n_tok, x_stream_stride,
+                                                       _ptr(packed), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def tq_q8_logits(packed, d, n_seq, n_kv, n_tok, q, g, tail, n_tail, scale, out, stream=None):
+    return _check("tq_q8_logits", lib.tq_q8_logits(_ptr(packed), d, n_seq, n_kv, n_tok, _ptr(q), _dtype(q), g,
+                                                   _ptr(tail), n_tail, scale, _ptr(out), _stream(stream)))
 
 
 def tq_dequantize(codec: Codec, packed, n_streams, n_tok, out, ws=None, stream=None):

@@ -530,6 +530,56 @@ int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float*
     return tq_topk_est(c, packed_db, n_db, q, n_q, k, idx, score, ws, ws_bytes, TQ_EST_QJL, stream);
 }
 
+size_t tq_q8_packed_bytes(int d, int64_t n_streams, int64_t n_tok) {
+    if (d < 8 || d > 128 || d % 8 || n_streams < 0 || n_tok < 0) return 0;
+    return (size_t)n_streams * (size_t)((n_tok + 31) / 32) * kQ8Block;
+}
+
+int tq_q8_quantize(const void* x, tq_dtype dtype, int d, int64_t n_streams, int64_t n_tok, int64_t x_stream_stride,
+                   void* packed, void* ws, size_t ws_bytes, void* stream) {
+    if (d < 8 || d > 128 || d % 8) return TQ_ERR_UNSUPPORTED;
+    if (dtype != TQ_F32 && dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_streams < 0 || n_tok < 0) return TQ_ERR_ARG;
+    if (n_streams == 0 || n_tok == 0) return TQ_OK;
+    if (!x || !packed || !ws || !aligned(packed, 16) || !aligned(x, dtype == TQ_F32 ? 4 : 2) || !aligned(ws, 4))
+        return TQ_ERR_ARG;
+    if (n_streams > 1 && x_stream_stride < n_tok * d) return TQ_ERR_ARG;
+    if (ws_bytes < TQ_STATUS_BYTES) return TQ_ERR_WORKSPACE;
+    Q8QuantParams p;
+    p.x = x; p.dtype = dtype; p.packed = static_cast<uint8_t*>(packed); p.status = static_cast<uint32_t*>(ws);
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32; p.x_stride = x_stream_stride; p.d = d;
+    return cuda_status(tq_launch_q8_quantize(p, static_cast<cudaStream_t>(stream)));
+}
+
+int tq_q8_logits(const void* packed, int d, int64_t n_seq, int n_kv, int64_t n_tok, const void* q, tq_dtype q_dtype,
+                 int g, const void* tail, int n_tail, float scale, float* out, void* stream) {
+    if (d < 8 || d > 128 || d % 8) return TQ_ERR_UNSUPPORTED;
+    if (g != 1 && g != 2 && g != 4) return TQ_ERR_UNSUPPORTED;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_seq == 0 || n_tok + n_tail == 0) return TQ_OK;
+    if (n_tail > TQ_Q8_MAX_TAIL) return TQ_ERR_UNSUPPORTED;
+    if (!q || !out || (n_tok > 0 && !packed) || (n_tail > 0 && !tail)) return TQ_ERR_ARG;
+    if ((n_tok > 0 && !aligned(packed, 16)) || !aligned(out, 4) || !aligned(q, q_dtype == TQ_F32 ? 4 : 2) ||
+        (n_tail > 0 && !aligned(tail, 2)))
+        return TQ_ERR_ARG;
+    if (!std::isfinite(scale)) return TQ_ERR_ARG;
+    const int64_t n_streams = n_seq * n_kv;
+    const int64_t nb = (n_tok + 31) / 32;
+    // one CTA per (stream, range), about four CTAs per SM; ranges of at least 8 blocks
+    int64_t bps = (nb * n_streams + 4 * kNumSms - 1) / (4 * kNumSms);
+    bps = std::max<int64_t>(8, bps);
+    bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
+    const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;
+    if (n_streams * nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    Q8LogitsParams p;
+    p.packed = static_cast<const uint8_t*>(packed);
+    p.q = q; p.q_dtype = q_dtype; p.tail = static_cast<const uint16_t*>(tail); p.out = out;
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = nb;
+    p.g = g; p.n_tail = n_tail; p.d = d; p.nsplit = (int)nsplit; p.bps = (int)bps; p.scale = scale;
+    return cuda_status(tq_launch_q8_logits(p, static_cast<cudaStream_t>(stream)));
+}
+
 int tq_dequantize(const tq_codec* c, const void* packed, int64_t n_streams, int64_t n_tok, float* out, void* ws,
                   size_t ws_bytes, void* stream) {
     int st = check_codec(c, false);

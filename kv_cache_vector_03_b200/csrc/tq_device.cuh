@@ -331,6 +331,27 @@ struct AttnParams {
     TqCodebookConsts cbv;         // value codebook (binary16 decode table)
 };
 
+// 8-bit keys (per 32-coordinate chunk: int8 codes and one binary16 scale), d <= 128
+constexpr uint32_t kQ8Block = 4096u + 256u;   // 32 tokens: codes [column 0..7][token][16 B], scales [chunk][token]
+struct Q8QuantParams {
+    const void* x;
+    int dtype;
+    uint8_t* packed;
+    uint32_t* status;
+    int64_t n_streams, n_tok, nb, x_stride;
+    int d;
+};
+struct Q8LogitsParams {
+    const uint8_t* packed;
+    const void* q;
+    int q_dtype;
+    const uint16_t* tail;   // bf16 [stream][n_tail][d] or null
+    float* out;
+    int64_t n_streams, n_tok, nb;
+    int g, n_tail, d, nsplit, bps;
+    float scale;
+};
+
 struct DequantParams {
     const uint8_t* packed;
     float* out;
@@ -352,3 +373,5 @@ cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
+cudaError_t tq_launch_q8_quantize(const Q8QuantParams& p, cudaStream_t st);
+cudaError_t tq_launch_q8_logits(const Q8LogitsParams& p, cudaStream_t st);

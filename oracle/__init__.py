@@ -185,6 +185,34 @@ def pv(idx, nhat, pi, c, P) -> np.ndarray:
     return out
 
 
+def q8_quantize(x):
+    """8-bit keys of the asymmetric K/V configuration (blog.hotdry.top "TurboQuant vector-search
+    compression", engineering configuration list: q8_0 keys). Per 32-coordinate chunk:
+    s = max|x| / 127 in fp32, codes rint(x / s) in fp32 (round half to even, clamped to
+    +-127; the integer decision is taken in the kernel's precision), stored scale = s rounded
+    to binary16. x [n, d] with d <= 128 -> (codes int8 [n, d], scales fp64 of binary16
+    [n, ceil(d / 32)])."""
+    x32 = np.ascontiguousarray(x, dtype=np.float32)
+    n, d = x32.shape
+    nc = (d + 31) // 32
+    xp = np.zeros((n, nc * 32), np.float32)
+    xp[:, :d] = x32
+    ch = xp.reshape(n, nc, 32)
+    am = np.abs(ch).max(axis=2)
+    s = (am / np.float32(127.0)).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(am[:, :, None] > 0, np.clip(np.rint(ch / s[:, :, None]), -127, 127), 0)
+    return q.reshape(n, nc * 32)[:, :d].astype(np.int8), s.astype(np.float16).astype(np.float64)
+
+
+def q8_logits(codes, scales, q, scale: float = 1.0) -> np.ndarray:
+    """scale <q, k~> with k~ = code * scale of its chunk, in fp64, for every (query, key)."""
+    codes = np.asarray(codes, dtype=np.float64)
+    n, d = codes.shape
+    k = codes * np.repeat(np.asarray(scales, dtype=np.float64), 32, axis=1)[:, :d]
+    return scale * (_f64(q).reshape(-1, d) @ k.T)
+
+
 def fwht_rotate(x, signs) -> np.ndarray:
     """y = H (D x) / sqrt(d) for every row of x, by the O(d log d) butterflies of the fast
     Walsh-Hadamard transform (ai-coding.wiselychen.com "Google TurboQuant KV-cache

@@ -139,3 +139,21 @@ def test_attention_host_checks(tq):
     assert call(scale=float("inf")) == tq.TQ_ERR_ARG
     assert call(q_dtype=5) == tq.TQ_ERR_ARG
     assert call(wsb=ws(K, V, 1, 8, 320, 4, 8) - 1) == tq.TQ_ERR_WORKSPACE
+
+
+def test_q8_host_checks(tq):
+    assert tq.lib.tq_q8_packed_bytes(128, 3, 33) == 3 * 2 * 4352
+    assert tq.lib.tq_q8_packed_bytes(200, 1, 32) == 0
+    assert tq.lib.tq_q8_quantize(0x1000, tq.TQ_BF16, 136, 1, 32, 4352, 0x2000, 0x3000, 256, None) == \
+        tq.TQ_ERR_UNSUPPORTED
+    assert tq.lib.tq_q8_quantize(0x1000, tq.TQ_BF16, 128, 1, 32, 4096, 0x2008, 0x3000, 256, None) == tq.TQ_ERR_ARG
+    assert tq.lib.tq_q8_quantize(0x1000, tq.TQ_BF16, 128, 1, 32, 4096, 0x2000, 0x3000, 8, None) == \
+        tq.TQ_ERR_WORKSPACE
+    assert tq.lib.tq_q8_quantize(0x1000, tq.TQ_BF16, 128, 0, 32, 4096, 0x2000, 0x3000, 256, None) == tq.TQ_OK
+    assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 64, 0x3000, tq.TQ_BF16, 8, None, 0, 1.0, 0x4000, None) == \
+        tq.TQ_ERR_UNSUPPORTED
+    assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 64, 0x3000, tq.TQ_BF16, 4, None, 70000, 1.0, 0x4000, None) == \
+        tq.TQ_ERR_UNSUPPORTED
+    assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 64, 0x3000, tq.TQ_BF16, 4, None, 3, 1.0, 0x4000, None) == \
+        tq.TQ_ERR_ARG
+    assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 0, 0x3000, tq.TQ_BF16, 4, None, 0, 1.0, 0x4000, None) == tq.TQ_OK

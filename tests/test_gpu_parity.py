@@ -462,6 +462,67 @@ def test_hadamard_rotation_path():
         assert np.all(err <= TOL + np.expm1(2 * dl) + 1e-5), err
 
 
+def _unpack_q8(packed_dev, d, n_streams, n_tok):
+    """Decode the 8-bit key blocks as the header describes them: codes [column][token][16 B],
+    then binary16 scales [chunk][token]."""
+    nb = (n_tok + 31) // 32
+    raw = packed_dev.cpu().numpy().reshape(n_streams * nb, 4352)
+    codes = raw[:, :4096].reshape(-1, 8, 32, 16).transpose(0, 2, 1, 3).reshape(n_streams, nb * 32, 128)
+    scales = np.ascontiguousarray(raw[:, 4096:]).view(np.float16).reshape(-1, 4, 32).transpose(0, 2, 1)
+    scales = scales.reshape(n_streams, nb * 32, 4).astype(np.float64)
+    return codes.view(np.int8)[:, :n_tok, :d], scales[:, :n_tok, :(d + 31) // 32], codes.view(np.int8)[:, :, d:]
+
+
+@pytest.mark.parametrize("d,g,n_seq,n_kv,n_tok,n_tail", [(128, 4, 1, 3, 301, 5), (96, 2, 2, 2, 64, 0),
+                                                        (128, 1, 1, 2, 0, 9), (128, 4, 1, 2, 4100, 128)])
+def test_q8_keys(d, g, n_seq, n_kv, n_tok, n_tail):
+    """8-bit keys: codes and scales bit-exact against the oracle (the integer decisions are
+    taken in fp32 on both sides), logits within sqrt(d)/32766 of scale |q| |k~| (the query's
+    int16 rounding) under the 1e-3 tolerance."""
+    torch = torch_cuda()
+    m = tq()
+    n = n_tok + n_tail
+    keys = np.stack([np.stack([ti.key_stream(4, sq, h, n, d) for h in range(n_kv)]) for sq in range(n_seq)])
+    S = n_seq * n_kv
+    kd = to_dev_bf16(np.ascontiguousarray(keys[:, :, :n_tok]).reshape(-1, d)) if n_tok else None
+    packed = torch.zeros(max(m.tq_q8_packed_bytes(d, S, n_tok), 16), dtype=torch.uint8, device="cuda")
+    ws = m.workspace(256)
+    if n_tok:
+        m.tq_q8_quantize(kd, d, S, n_tok, n_tok * d, packed, ws)
+        assert m.tq_get_status(ws) == m.TQ_OK
+    kf = ti.bf16_to_f64(keys)
+    if n_tok:
+        codes, scales, pad = _unpack_q8(packed, d, S, n_tok)
+        assert not pad.any()
+        for st in range(S):
+            want_c, want_s = oracle.q8_quantize(kf.reshape(S, n, d)[st, :n_tok])
+            assert np.array_equal(codes[st], want_c)
+            assert np.array_equal(scales[st], want_s)
+    qb = ti.decode_queries(15, n_seq, n_kv * g, d)
+    out = torch.full((n_seq, n_kv * g, n), float("nan"), dtype=torch.float32, device="cuda")
+    tail = to_dev_bf16(np.ascontiguousarray(keys[:, :, n_tok:])) if n_tail else None
+    scale = 1.0 / math.sqrt(d)
+    m.tq_q8_logits(packed, d, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tail, n_tail, scale, out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy().astype(np.float64)
+    q = ti.bf16_to_f64(qb)
+    for sq in range(n_seq):
+        for h in range(n_kv):
+            st = sq * n_kv + h
+            qh = q[sq, h * g:(h + 1) * g]
+            if n_tok:
+                c_, s_ = oracle.q8_quantize(kf[sq, h, :n_tok])
+                want = oracle.q8_logits(c_, s_, qh, scale)
+                rec = c_.astype(np.float64) * np.repeat(s_, 32, axis=1)[:, :d]
+                err = np.abs(got[sq, h * g:(h + 1) * g, :n_tok] - want) / (
+                    scale * np.linalg.norm(qh, axis=1)[:, None] * np.linalg.norm(rec, axis=1)[None, :])
+                assert err.max() <= min(TOL, math.sqrt(d) / 32766 * 1.01), err.max()
+            if n_tail:
+                wt = oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)
+                _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1),
+                              scale)
+
+
 def test_attention_rejects_unsupported():
     torch = torch_cuda()
     m = tq()
