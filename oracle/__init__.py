@@ -1,9 +1,11 @@
 """fp64 CPU oracle of the TurboQuant KV-vector hot path -- TEST INFRASTRUCTURE ONLY.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
-import this package. It shares no code with the CUDA library: the arithmetic lives in
-``tq_oracle.c`` (plain C, fp64, one vector at a time), built into ``liboracle.so`` by
-``build()``; this module only marshals numpy arrays.
+import this package. It shares no code with the CUDA library. The codebook, quantizer,
+estimator, reconstruction, P.V and top-k arithmetic lives in ``tq_oracle.c`` (plain C, fp64,
+one vector at a time), built into ``liboracle.so`` by ``build()``; the compositions and
+variants written here in numpy (decode attention over those functions, sparse values, the
+Walsh-Hadamard butterflies, 8-bit keys) use library primitives only (matmul, exp, rint).
 
 Parity status of each function (what pins it) is listed in the repository's design notes;
 every function here is pinned by a test in ``tests/test_oracle_*.py``.
