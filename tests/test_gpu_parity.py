@@ -268,6 +268,25 @@ def test_pv(B, g, n_tok):
         _check_pv(got[h * g:(h + 1) * g], want, Ph.astype(np.float64), nhat[h])
 
 
+@pytest.mark.parametrize("B,g", [(3, 4), (4, 8)])
+def test_pv_d200_values(B, g):
+    """d = 200 values pad to 256 coordinates: the 16-tile split kernel and the 256-wide merge."""
+    d, n_kv, n_tok = 200, 2, 1000
+    pi = ti.haar_rotation(d, 121)
+    rng = np.random.default_rng(122)
+    bits = ti.f32_to_bf16_bits(rng.standard_normal((n_kv * n_tok, d)).astype(np.float32))
+    codec = make_codec(d, 0, B, False, pi, None)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(bits), n_kv, n_tok)
+    P = ti.logits_p(n_kv * g, n_tok)
+    got = _pv_gpu(codec, packed, 1, n_kv, n_tok, to_dev_f32(P), g)[0]
+    idx, nhat = unpack(codec, packed, n_kv, n_tok)
+    c, _ = _cb(d, B)
+    for h in range(n_kv):
+        Ph = P[h * g:(h + 1) * g]
+        want = oracle.pv(idx[h], nhat[h], pi, c, Ph)
+        _check_pv(got[h * g:(h + 1) * g], want, Ph.astype(np.float64), nhat[h])
+
+
 def test_pv_one_hot_and_uniform():
     d, B, n_tok = 128, 3, 300
     pi = ti.C3.pi()
