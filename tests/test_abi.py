@@ -157,3 +157,11 @@ def test_q8_host_checks(tq):
     assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 64, 0x3000, tq.TQ_BF16, 4, None, 3, 1.0, 0x4000, None) == \
         tq.TQ_ERR_ARG
     assert tq.lib.tq_q8_logits(0x2000, 128, 1, 8, 0, 0x3000, tq.TQ_BF16, 4, None, 0, 1.0, 0x4000, None) == tq.TQ_OK
+
+
+def test_header_is_plain_c():
+    """include/tq.h is a C header: it compiles as C99 and as C++ with no CUDA headers."""
+    import subprocess
+    hdr = os.path.join(ROOT, "include", "tq.h")
+    subprocess.check_call(["gcc", "-fsyntax-only", "-std=c99", "-Wall", "-Werror", "-x", "c", hdr])
+    subprocess.check_call(["g++", "-fsyntax-only", "-Wall", "-Werror", "-x", "c++", hdr])
