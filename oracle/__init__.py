@@ -215,6 +215,24 @@ def q8_logits(codes, scales, q, scale: float = 1.0) -> np.ndarray:
     return scale * (_f64(q).reshape(-1, d) @ k.T)
 
 
+def attention_q8(k_codes, k_scales, v_idx, v_nhat, pi_v, c_v, q, scale: float, tail_k=None,
+                 tail_v=None) -> np.ndarray:
+    """Decode attention of the asymmetric configuration (blog.hotdry.top, engineering
+    configuration list: 8-bit keys, TurboQuant values): softmax over [logits of the 8-bit
+    keys, exact logits of the tail keys] times [reconstructed values, tail values], fp64."""
+    q = _f64(q)
+    q = q.reshape(-1, q.shape[-1])
+    lg = [q8_logits(k_codes, k_scales, q, scale)]
+    vals = [reconstruct(v_idx, None, v_nhat, None, pi_v, None, c_v, qjl=False)]
+    if tail_k is not None and len(tail_k):
+        lg.append(exact_dot(tail_k, q, scale))
+        vals.append(_f64(tail_v))
+    lg = np.concatenate(lg, axis=1)
+    w = np.exp(lg - lg.max(axis=1, keepdims=True))
+    w /= w.sum(axis=1, keepdims=True)
+    return w @ np.concatenate(vals, axis=0)
+
+
 def fwht_rotate(x, signs) -> np.ndarray:
     """y = H (D x) / sqrt(d) for every row of x, by the O(d log d) butterflies of the fast
     Walsh-Hadamard transform (ai-coding.wiselychen.com "Google TurboQuant KV-cache

@@ -56,3 +56,24 @@ def test_logits_brute_force():
             for i in range(40):
                 want += q[a, i] * float(codes[b, i]) * scales[b, i // 32]
             assert abs(got[a, b] - 0.25 * want) <= 1e-12 * max(1.0, abs(want))
+
+
+def test_attention_over_8bit_keys():
+    # no tail: P.V of the 8-bit-key logits (separately pinned functions); q = 0: the mean of
+    # the compressed and tail values together
+    rng = np.random.default_rng(4)
+    d, nt = 64, 150
+    keys = rng.standard_normal((nt + 5, d)) * 3.0
+    vals = rng.standard_normal((nt + 5, d))
+    c_v, t_v, _, _ = oracle.codebook(d, 3)
+    pi_v = np.linalg.qr(rng.standard_normal((d, d)))[0]
+    vq = oracle.quantize(vals[:nt], pi_v, None, c_v, t_v, 3, qjl=False)
+    kc, ks = oracle.q8_quantize(keys[:nt])
+    qs = rng.standard_normal((3, d)) * 0.2
+    o = oracle.attention_q8(kc, ks, vq.idx, vq.nhat, pi_v, c_v, qs, 0.5)
+    want = oracle.pv(vq.idx, vq.nhat, pi_v, c_v, oracle.q8_logits(kc, ks, qs, 0.5))
+    assert np.allclose(o, want, rtol=1e-5, atol=1e-6 * np.abs(want).max())
+    vh = oracle.reconstruct(vq.idx, None, vq.nhat, None, pi_v, None, c_v, qjl=False)
+    o0 = oracle.attention_q8(kc, ks, vq.idx, vq.nhat, pi_v, c_v, np.zeros((1, d)), 1.0, tail_k=keys[nt:],
+                             tail_v=vals[nt:])
+    assert np.allclose(o0[0], np.concatenate([vh, vals[nt:]]).mean(0), rtol=1e-12, atol=1e-12)
