@@ -20,6 +20,7 @@ import argparse
 import json
 import math
 import os
+import socket
 import subprocess
 import sys
 import time
@@ -560,6 +561,32 @@ def run_reference(args, world, rank):
             "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def relaunch(argv, n_ranks):
+    """`--gpus N` run without a torchrun environment: start N ranks on this node, one process
+    per GPU, through torch.distributed.run (loopback rendezvous), and return its exit code."""
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n_ranks}",
+           "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_plumbing(args, world, rank):
+    """The N-rank plumbing alone (process group, barrier, max over ranks), no GPU work: each
+    rank times a fixed host wait; rank 0 reports the slowest rank's time and the world size."""
+    barrier(world)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time.sleep(0.001 * (rank + 1))
+    ms = max_over_ranks(world, (time.perf_counter() - t0) * 1e3 / args.steps)
+    barrier(world)
+    if rank != 0:
+        return None
+    return {"plumbing_only": True, "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "scaling": "weak"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -568,9 +595,25 @@ def main():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the c2/c3/c5 side measurements")
+    ap.add_argument("--plumbing-only", action="store_true",
+                    help="run only the multi-rank plumbing over gloo (no GPU work); for tests")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        sys.exit(relaunch(sys.argv[1:], args.gpus))
+    if env_world is not None and int(env_world) != args.gpus:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={env_world}: launch one rank per GPU")
+    if args.plumbing_only:
+        world, rank, _ = dist_init(backend="gloo")
+        line = run_plumbing(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     world, rank, local = dist_init() if args.impl == "tq" else (int(os.environ.get("WORLD_SIZE", "1")),
                                                                  int(os.environ.get("RANK", "0")), 0)
     if args.impl == "reference":

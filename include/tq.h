@@ -45,7 +45,7 @@ typedef enum {
     TQ_ERR_UNSUPPORTED = -2,  /* valid request outside the supported shapes */
     TQ_ERR_CUDA = -3,         /* a CUDA runtime call failed */
     TQ_ERR_RANGE = -4,        /* (status word) a norm overflowed binary16 or an input was not finite */
-    TQ_ERR_TIMEOUT = -5,      /* (status word) a bounded wait for a bulk copy ran out */
+    TQ_ERR_TIMEOUT = -5,      /* (status word) a bounded wait of a kernel ran out */
     TQ_ERR_NOCONV = -6,       /* codebook iteration did not converge */
     TQ_ERR_WORKSPACE = -7     /* workspace or prepared buffer too small / not prepared */
 } tq_status;
@@ -84,6 +84,13 @@ typedef struct {
  *               lowers ranking quality and an MSE-only mode is preferred). The key records
  *               are the same; only the estimate changes.                                    */
 enum { TQ_EST_QJL = 0, TQ_EST_MSE = 1 };
+
+/* Test hook, OR-ed into the estimator of tq_logits_est: every warp of the logits stream
+ * kernel first waits on a barrier that nothing arrives at, with a limit of a few thousand
+ * polls. The wait runs out as a lost copy would: the kernel records TQ_ERR_TIMEOUT in the
+ * status word, waits (bounded) for the copies it has in flight and returns without writing
+ * logits, leaving the context usable. It exists to test that path; it is not for use.     */
+#define TQ_TEST_STALL 0x100
 
 /* Operations, for tq_workspace_bytes */
 enum { TQ_OP_QUANTIZE = 0, TQ_OP_LOGITS = 1, TQ_OP_PV = 2, TQ_OP_TOPK = 3, TQ_OP_DEQUANTIZE = 4 };
@@ -219,11 +226,16 @@ int tq_topk_est(const tq_codec* codec, const void* packed_db, int64_t n_db, cons
  *   GPU that loads the library until the process exits. A request whose
  *   tq_workspace_bytes(codec, TQ_OP_LOGITS, n_seq, n_kv, g) exceeds it returns
  *   TQ_ERR_WORKSPACE and enqueues nothing.
- *   The first call on a device resolves the array's device address (cudaGetSymbolAddress,
- *   with that device current): make that first call before any stream capture.
+ *   The array's device address belongs to the CUDA context that loaded the library's
+ *   module. The first call in a context resolves it (cudaGetSymbolAddress, with that context
+ *   current): the first call on a device, and the first after cudaDeviceReset or any other
+ *   change of the device's current context. Make such a first call before any stream
+ *   capture.
  *   Every call on a device shares the array: calls whose GPU work may overlap (other
- *   streams, other threads) race and must be serialised by the caller. Each call clears
- *   the status word first; data-dependent faults are not reported by this variant.
+ *   streams, other threads) race and must be serialised by the caller. Arguments are
+ *   checked first; a rejected call enqueues nothing and leaves the array untouched. An
+ *   accepted call clears the status word on the stream before its kernels; data-dependent
+ *   faults are not reported by this variant.
  *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine.        */
 #define TQ_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
 int tq_logits_noalloc(const tq_codec* codec, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok,
@@ -266,7 +278,8 @@ int tq_dequantize(const tq_codec* codec, const void* packed, int64_t n_streams, 
 /* Status word. Data-dependent faults of every call that used `ws` accumulate in its first
  * word until read. tq_reset_status enqueues a clear (do it once on a new workspace);
  * tq_get_status synchronises `stream`, reads the word and clears it, returning TQ_OK,
- * TQ_ERR_RANGE, or TQ_ERR_CUDA if the read itself failed.                                */
+ * TQ_ERR_TIMEOUT if a bounded wait of a kernel ran out (it takes precedence), TQ_ERR_RANGE,
+ * or TQ_ERR_CUDA if the read itself failed.                                              */
 int tq_reset_status(void* ws, void* stream);
 int tq_get_status(void* ws, void* stream);
 

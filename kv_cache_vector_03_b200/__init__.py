@@ -25,6 +25,7 @@ TQ_ERR_RANGE, TQ_ERR_TIMEOUT, TQ_ERR_NOCONV, TQ_ERR_WORKSPACE = -4, -5, -6, -7
 TQ_F32, TQ_BF16 = 0, 1
 TQ_OP_QUANTIZE, TQ_OP_LOGITS, TQ_OP_PV, TQ_OP_TOPK, TQ_OP_DEQUANTIZE = 0, 1, 2, 3, 4
 TQ_EST_QJL, TQ_EST_MSE = 0, 1
+TQ_TEST_STALL = 0x100   # test hook: see include/tq.h
 EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_bytes", "tq_prep_bytes",
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
             "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",

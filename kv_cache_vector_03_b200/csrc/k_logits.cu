@@ -418,12 +418,13 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     // exact int32 combination of the hi/lo columns while 128 * 8 kTqQueryMax * K < 2^31
     constexpr bool kIntComb = NP * GD <= 4 && GM <= 4;
     extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ uint64_t bars[kStreamWarps][NS];
+    // one barrier per ring stage, plus one that nothing arrives at (the test stall)
+    __shared__ uint64_t bars[kStreamWarps][NS + 1];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     uint8_t* my_ring = ring + (size_t)warp * NS * BB;
     if (lane == 0)
-        for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[warp][s], 1);
+        for (int s = 0; s <= NS; ++s) tq_mbar_init(&bars[warp][s], 1);
     tq_fence_mbar_init();
     __syncwarp();
 
@@ -432,10 +433,12 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     FlatWalk prod, cons;
     prod.init(p, gw * n_blocks / n_warps, (gw + 1) * n_blocks / n_warps);
     cons = prod;
+    uint32_t issued = 0;   // copies issued so far (lane 0): copy k fills stage k % NS
     if (lane == 0) {
         for (int s = 0; s < NS && prod.valid(); ++s) {
             tq_bulk_load(my_ring + s * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB, &bars[warp][s]);
             prod.advance(p);
+            ++issued;
         }
     }
 
@@ -448,8 +451,10 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     bool hv[NT];
     int cur_stream = -1;
     uint32_t seq = 0;
-    bool ok = true;
-    while (cons.valid()) {
+    // test stall: a bounded wait on the barrier nothing arrives at runs out, exactly as a
+    // copy that never lands would
+    bool ok = p.test_stall == 0u || __all_sync(0xffffffffu, tq_mbar_wait(&bars[warp][NS], 0u, p.test_stall));
+    while (ok && cons.valid()) {
         if (cons.stream != cur_stream) {
             cur_stream = cons.stream;
 #pragma unroll
@@ -548,15 +553,17 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
             tq_bulk_load(my_ring + stage * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB,
                          &bars[warp][stage]);
             prod.advance(p);
+            ++issued;
         }
         ++seq;
         cons.advance(p);
     }
     if (!ok) {
-        // a wait ran out: record it, then give the outstanding copies a bounded time to land
+        // a wait ran out: record it, then give each copy still in flight (copies seq .. issued-1)
+        // a bounded time to land before the CTA's shared memory is released
         if (lane == 0) {
             tq_raise(p.status, TQ_FLAG_TIMEOUT);
-            for (int s = 0; s < NS; ++s) tq_mbar_wait(&bars[warp][(seq + s) % NS], ((seq + s) / NS) & 1u, kWaitLimit);
+            for (uint32_t k = seq; k < issued; ++k) tq_mbar_wait(&bars[warp][k % NS], (k / NS) & 1u, kWaitLimit);
         }
         __syncwarp();
     }
@@ -589,7 +596,10 @@ cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
 }  // namespace
 
 // heads per prologue CTA: about one CTA per SM
-static int prologue_hpc(int64_t n_heads) { return n_heads <= 148 * 4 ? 4 : n_heads <= 148 * 8 ? 8 : 16; }
+static int prologue_hpc(int64_t n_heads) {
+    const int64_t sms = tq_device_sms();
+    return n_heads <= sms * 4 ? 4 : n_heads <= sms * 8 ? 8 : 16;
+}
 
 // MMA path (D + Mp = 256): qo [16][256] fp32 + A hi/lo [16][256 B] + four [128][256 B] B tiles
 constexpr size_t kPrologueSmemMma = (size_t)16 * 256 * 4 + 2 * 16 * 256 + 4 * 128 * 256;

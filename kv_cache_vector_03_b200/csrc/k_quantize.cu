@@ -193,16 +193,7 @@ __global__ void __launch_bounds__(128) k_quantize_f32(QuantParams p) {
     }
 }
 
-// ---------------------------------------------------------------------------------------
-// Tensor-core quantizer for d <= 128 (D = Mp = 128 or values): persistent CTAs of 8 warps,
-// 128-vector tiles (four 32-vector blocks); warp w owns tile rows 16w..16w+15.
-//   Y = (2^e x) (256 Pi)^T on mma.sync m16n8k16 fp16 -> fp32: x scaled by a power of two so
-//       that max |2^e x| is in [2^14, 2^15), split hi/lo (bf16 inputs are exact in the hi
-//       part: 2 passes; fp32 inputs: 3 passes); Pi as the prepared hi/lo pair.
-//   y = Y / (|x| 2^(e+8)); codes, residual r = y - c[idx] and gamma per row.
-//   Z = (2^12 r)(256 M)^T, 3 passes (hi.hi + hi.lo + lo.hi): only its sign is kept.
-// Operands live in shared memory with 16-byte chunks XOR-swizzled by (row & 7), read with
-// ldmatrix. Pi and M stay resident for the whole kernel.
+// one CTA of 4 warps per 32-vector block
 template <int KD, int KM, int B>
 cudaError_t launch(const QuantParams& p, cudaStream_t st) {
     const size_t smem_bytes = (size_t)32 * KD * 32 * 4 + (size_t)32 * KD * 32;

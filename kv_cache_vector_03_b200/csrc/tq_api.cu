@@ -13,7 +13,8 @@
 
 namespace {
 
-constexpr int kNumSms = 148;
+// polls of the wait that TQ_TEST_STALL makes run out (a few milliseconds at most)
+constexpr uint32_t kTestStallPolls = 2000;
 
 size_t align_up(size_t v) { return (v + TQ_ALIGN - 1) / TQ_ALIGN * TQ_ALIGN; }
 
@@ -108,7 +109,7 @@ TopkWs topk_ws(const TqDims& t, int64_t n_q, int64_t n_db, int k) {
     const int64_t nb = (n_db + 31) / 32;
     w.n_groups = (int)((n_q + 3) / 4);
     const int64_t qgroups = (w.n_groups + 7) / 8;
-    int64_t ns = (4 * kNumSms + qgroups - 1) / qgroups;
+    int64_t ns = (4 * tq_device_sms() + qgroups - 1) / qgroups;
     ns = std::max<int64_t>(1, std::min<int64_t>(ns, nb));
     w.bps = (int)((nb + ns - 1) / ns);
     w.nsplit = (int)((nb + w.bps - 1) / w.bps);
@@ -125,7 +126,7 @@ struct PvWs { int nsplit, bps; size_t part, ml, total; };
 PvWs pv_ws(const TqDims& t, int64_t n_streams, int64_t n_tok, int g) {
     PvWs w;
     const int64_t nb = (n_tok + 31) / 32;
-    int64_t bps = (nb * n_streams + 2 * kNumSms - 1) / (2 * kNumSms);   // about two CTAs per SM
+    int64_t bps = (nb * n_streams + 2 * tq_device_sms() - 1) / (2 * tq_device_sms());   // about two CTAs per SM
     if (bps < 8) bps = 8;
     if (bps > nb) bps = nb;
     if (bps < 1) bps = 1;
@@ -146,7 +147,7 @@ AttnWs attn_ws(const TqDims& tk, int64_t n_streams, int64_t n_tok, int g, int n_
     AttnWs w;
     w.lg = logits_ws(tk, n_streams, g);
     const int64_t nb = (n_tok + 31) / 32;
-    int64_t bps = (nb * n_streams + 2 * kNumSms - 1) / (2 * kNumSms);
+    int64_t bps = (nb * n_streams + 2 * tq_device_sms() - 1) / (2 * tq_device_sms());
     bps = std::max<int64_t>(8, bps);
     bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
     w.bps = (int)bps;
@@ -303,11 +304,17 @@ int tq_quantize(const tq_codec* c, const void* x, tq_dtype dtype, int64_t n_stre
     return cuda_status(tq_launch_quantize(p, static_cast<cudaStream_t>(stream)));
 }
 
-int tq_logits_est(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+}  // extern "C"
+
+// tq_logits_est behind its argument checks; with clear_status the status word is cleared on
+// the stream once every check has passed (the no-workspace variant shares one scratch array).
+int tq_logits_run(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
                   tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
-                  size_t ws_bytes, int estimator, void* stream) {
+                  size_t ws_bytes, int estimator, int clear_status, void* stream) {
     int st = check_codec(c, true);
     if (st != TQ_OK) return st;
+    const bool test_stall = (estimator & TQ_TEST_STALL) != 0;
+    estimator &= ~TQ_TEST_STALL;
     if (estimator != TQ_EST_QJL && estimator != TQ_EST_MSE) return TQ_ERR_ARG;
     if (!c->qjl) return TQ_ERR_ARG;
     if (g != 1 && g != 2 && g != 4 && g != 8) return TQ_ERR_UNSUPPORTED;
@@ -344,12 +351,24 @@ int tq_logits_est(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv
     p.kappa = estimator == TQ_EST_MSE ? 0.f : (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.status = static_cast<uint32_t*>(ws);
     p.n_heads_valid = n_streams * g;
+    p.test_stall = test_stall ? kTestStallPolls : 0u;
     // the tail runs on a second grid dimension of 16-token CTAs (at most 65535)
     if (n_streams * g > 0x7fffffffLL || n_streams * p.nb > (1LL << 40) || n_tail > 16 * 65534)
         return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    if (clear_status && cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return TQ_ERR_CUDA;
     return cuda_status(tq_launch_logits(p, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" {
+
+int tq_logits_est(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+                  tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
+                  size_t ws_bytes, int estimator, void* stream) {
+    return tq_logits_run(c, packed, n_seq, n_kv, n_tok, q, q_dtype, g, tail, n_tail, scale, out, ws, ws_bytes,
+                         estimator, 0, stream);
 }
 
 int tq_logits(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
@@ -426,6 +445,7 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
 
     // 1. query fragments and exact tail logits: the logits prologue with no compressed tokens
     LogitsParams lp;
+    std::memset(&lp, 0, sizeof(lp));
     lp.packed = nullptr;
     lp.q = q; lp.q_dtype = q_dtype;
     lp.tail = static_cast<const uint16_t*>(tail_k);
@@ -567,7 +587,7 @@ int tq_q8_logits(const void* packed, int d, int64_t n_seq, int n_kv, int64_t n_t
     const int64_t n_streams = n_seq * n_kv;
     const int64_t nb = (n_tok + 31) / 32;
     // one CTA per (stream, range), about four CTAs per SM; ranges of at least 8 blocks
-    int64_t bps = (nb * n_streams + 4 * kNumSms - 1) / (4 * kNumSms);
+    int64_t bps = (nb * n_streams + 4 * tq_device_sms() - 1) / (4 * tq_device_sms());
     bps = std::max<int64_t>(8, bps);
     bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
     const int64_t nsplit = nb > 0 ? (nb + bps - 1) / bps : 1;

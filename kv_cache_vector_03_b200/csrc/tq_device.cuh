@@ -49,6 +49,27 @@ inline cudaError_t tq_kernel_setup(Kernel kern, int threads, size_t max_smem, Tq
     return cudaSuccess;
 }
 
+// SM count of the current device (cached per device). Split counts, and so workspace sizes,
+// follow it; with no usable device (a size query on a machine without a GPU) the B200's 148
+// is assumed.
+inline int tq_device_sms() {
+    constexpr int kDevices = 64;
+    static std::atomic<int> cache[kDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) {
+        cudaGetLastError();
+        return 148;
+    }
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
 TQ_DEVICE uint32_t tq_half_bits(float v) { return (uint32_t)__half_as_ushort(__float2half_rn(v)); }
 TQ_DEVICE float tq_half_val(uint32_t bits) { return __half2float(__ushort_as_half((unsigned short)bits)); }
 
@@ -280,6 +301,7 @@ struct LogitsParams {
     int n_kv, g, ntiles, n_tail;
     float scale, kappa;
     int64_t n_heads_valid;                   // query rows that exist (later heads read as zero)
+    uint32_t test_stall;                     // 0, or the poll limit of a wait that is made to run out
     TqDims t;
     TqCodebookConsts cb;
 };

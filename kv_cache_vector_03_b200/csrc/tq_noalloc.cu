@@ -6,11 +6,18 @@
 // no-allocation policy. This entry point takes the same inputs and outputs as tq_logits
 // but no workspace: its scratch (status word, query fragments, per-head constants) lives
 // in a fixed array in device memory that every GPU loading the library keeps until exit.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
 #include "tq.h"
+
+// tq_logits_est behind its argument checks (tq_api.cu); clear_status clears the status word
+// on the stream once every check has passed
+int tq_logits_run(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv, int64_t n_tok, const void* q,
+                  tq_dtype q_dtype, int g, const void* tail, int n_tail, float scale, float* out, void* ws,
+                  size_t ws_bytes, int estimator, int clear_status, void* stream);
 
 namespace {
 
@@ -18,21 +25,69 @@ constexpr size_t kScratchBytes = TQ_NOALLOC_SCRATCH_BYTES;
 __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
 // Host code must not pass g_scratch to a kernel: on the host it names a shadow, not a
-// device address. The address is resolved once per device, with that device current.
+// device address. The address belongs to the module as loaded in one CUDA context, so it is
+// resolved (cudaGetSymbolAddress, with that context current) on the first call in a context
+// and again whenever the current context of a device changes, e.g. after cudaDeviceReset
+// reloaded the module. Contexts are told apart by the driver's unique context ID.
 constexpr int kMaxDevices = 64;
-void* g_ptr[kMaxDevices];
+struct Slot {
+    unsigned long long ctx_id;   // 0: not resolved
+    void* ptr;
+};
+Slot g_slot[kMaxDevices];
 std::mutex g_lock;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_get_current = nullptr;
+CtxGetIdFn g_get_id = nullptr;
+
+// driver entry points through the runtime (the library does not link libcuda itself)
+bool resolve_driver_calls() {
+    if (g_get_current && g_get_id) return true;
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || !a)
+        return false;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess || !b)
+        return false;
+    g_get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    g_get_id = reinterpret_cast<CtxGetIdFn>(b);
+    return true;
+}
+
+// ID of the context the runtime uses for `dev` on this thread (made current if need be)
+bool current_context_id(int dev, unsigned long long* id) {
+    CUcontext ctx = nullptr;
+    if (g_get_current(&ctx) != CUDA_SUCCESS) return false;
+    if (!ctx) {
+        // the runtime makes its context current lazily; cudaSetDevice initialises it
+        if (cudaSetDevice(dev) != cudaSuccess || g_get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+    }
+    return g_get_id(ctx, id) == CUDA_SUCCESS && *id != 0;
+}
 
 int scratch_of_current_device(void** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TQ_ERR_CUDA;
     std::lock_guard<std::mutex> guard(g_lock);
-    if (!g_ptr[dev]) {
+    unsigned long long id = 0;
+    if (!resolve_driver_calls() || !current_context_id(dev, &id)) return TQ_ERR_CUDA;
+    Slot& s = g_slot[dev];
+    if (s.ctx_id != id || !s.ptr) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) return TQ_ERR_CUDA;
-        g_ptr[dev] = p;
+        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || !p) {
+            s.ctx_id = 0;
+            s.ptr = nullptr;
+            return TQ_ERR_CUDA;
+        }
+        s.ctx_id = id;
+        s.ptr = p;
     }
-    *out = g_ptr[dev];
+    *out = s.ptr;
     return TQ_OK;
 }
 
@@ -47,8 +102,8 @@ extern "C" int tq_logits_noalloc(const tq_codec* codec, const void* packed, int6
     void* ws = nullptr;
     const int st = scratch_of_current_device(&ws);
     if (st != TQ_OK) return st;
-    // the status word starts at zero for every call; the rest is written before it is read
-    if (cudaMemsetAsync(ws, 0, 4, static_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
-    return tq_logits(codec, packed, n_seq, n_kv, n_tok, q, q_dtype, g, tail, n_tail, scale, out, ws, kScratchBytes,
-                     stream);
+    // every argument is checked before the status word is cleared and the kernels are
+    // enqueued: a rejected call leaves the stream and the shared array untouched
+    return tq_logits_run(codec, packed, n_seq, n_kv, n_tok, q, q_dtype, g, tail, n_tail, scale, out, ws,
+                         kScratchBytes, TQ_EST_QJL, 1, stream);
 }

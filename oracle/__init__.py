@@ -7,8 +7,9 @@ one vector at a time), built into ``liboracle.so`` by ``build()``; the compositi
 variants written here in numpy (decode attention over those functions, sparse values, the
 Walsh-Hadamard butterflies, 8-bit keys) use library primitives only (matmul, exp, rint).
 
-Parity status of each function (what pins it) is listed in the repository's design notes;
-every function here is pinned by a test in ``tests/test_oracle_*.py``.
+Every function here is pinned by a test in ``tests/test_oracle_*.py`` against something
+other than itself: closed forms, the printed distortions, brute force on tiny inputs,
+exhaustive search, invariants (unbiasedness, orthogonality, rotate-once) and special cases.
 """
 from __future__ import annotations
 

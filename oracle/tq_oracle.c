@@ -26,7 +26,7 @@
  *   [V]  friday-blog-bgf.pages.dev "TurboQuant deep dive II", section 1, step 1:
  *        values use the rotation + MSE scalar quantizer only.
  *
- * Readings where the pages are loose (each is listed in the design notes):
+ * Readings where the pages are loose or silent:
  *   - the QJL factor is sqrt(pi/2)/m (the pages print /d; m = d in every workload);
  *   - vectors are normalised first: n = |x|, u = x/n, and gamma is |r| of the unit vector;
  *     scores are n * (<Pi q, c[idx]> + gamma sqrt(pi/2)/m <S q, s>);

@@ -95,3 +95,51 @@ def unpack(codec, packed_dev, n_streams, n_tok):
     if c.qjl:
         return unpack_keys(buf, c.d, c.m, c.mse_bits, n_streams, n_tok)
     return unpack_values(buf, c.d, c.mse_bits, n_streams, n_tok)
+
+
+ATTN_CEIL = 5e-3     # ceiling of the fused-attention error against the full oracle
+
+
+def _softmax_rows(L):
+    w = np.exp(L - L.max(axis=1, keepdims=True))
+    return w / w.sum(axis=1, keepdims=True)
+
+
+def check_attention(got, want, L, lg, n_tok, V, vnorm, v_skip=0.0, skip_mass=None):
+    """Fused decode attention of the g heads of one kv stream, two checks.
+
+    got [g, d] GPU output; want [g, d] the oracle's attention; L [g, n] the oracle's logits
+    (estimator on the compressed keys, exact on the tail); lg [g, n] the GPU's tq_logits on the
+    same codes and queries; V [n, d] the oracle's reconstructed compressed values followed by
+    the exact tail values; vnorm [n] the stored value norms, then the tail norms.
+
+    1. Composed (the step tolerance of P.V): the oracle's softmax(P) . V with P = the GPU's
+       compressed-key logits followed by the exact tail logits. The fused kernel evaluates the
+       same logit fragments, so this isolates its softmax, value decode and merge: the error
+       is held to TOL of sum_t w_t |v_t| on every workload, whatever the logit scale.
+    2. Full oracle: a logit error dl moves every softmax weight by a factor within
+       exp(+-2 dl), so the error is at most (expm1(2 dl) + TOL) sum_t w_t |v_t|; the bound is
+       capped by the fixed ATTN_CEIL, so a large logit scale cannot widen it.
+    With sparse values the dropped weight mass (tokens whose relative weight is below v_skip)
+    is added to both bounds. Returns (full error, composed error), per head."""
+    assert np.all(np.isfinite(got))
+    Lc = np.concatenate([lg[:, :n_tok], L[:, n_tok:]], axis=1)
+    wc = _softmax_rows(Lc)
+    comp = wc @ V
+    skip_c = np.zeros(len(got))
+    if v_skip > 0.0:
+        rel = np.exp(Lc - Lc.max(axis=1, keepdims=True))
+        drop = rel < v_skip
+        drop[:, n_tok:] = False
+        wv = wc * vnorm[None, :]
+        skip_c = (wv * drop).sum(axis=1) / wv.sum(axis=1)
+    err_c = np.max(np.abs(got - comp), axis=1) / (wc @ vnorm)
+    assert np.all(err_c <= TOL + skip_c), f"composed check: normalised error {err_c} above {TOL + skip_c}"
+    w = _softmax_rows(L)
+    dl = np.abs(lg - L).max(axis=1)
+    err = np.max(np.abs(got - want), axis=1) / (w @ vnorm)
+    bound = np.minimum(TOL + np.expm1(2 * dl) + 1e-5, ATTN_CEIL)
+    if skip_mass is not None:
+        bound = bound + skip_mass
+    assert np.all(err <= bound), f"full oracle: normalised error {err} above {bound}"
+    return err, err_c

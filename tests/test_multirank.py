@@ -59,3 +59,27 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(1, 3.5) == 3.5
     bench.barrier(1)
+
+
+def test_bench_launches_its_own_ranks():
+    """`python bench.py --gpus 2` with no torchrun environment starts two ranks itself (one
+    process per GPU) and rank 0 reports n_gpus = 2; here over gloo, with no GPU work."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR",
+                                                            "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--plumbing-only",
+                        "--steps", "3", "--warmup", "3"], capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [json.loads(ln) for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["plumbing_only"]
+    assert lines[0]["ms_per_step"] >= 2.0      # the slower rank (2 ms per step) sets the time
+
+
+def test_bench_refuses_a_mismatched_world_size():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--plumbing-only"],
+                       capture_output=True, text=True, timeout=120, env=env)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr

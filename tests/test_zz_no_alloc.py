@@ -54,3 +54,35 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     st = m.lib.tq_logits_noalloc(codec.ref, ctypes.c_void_p(16), 4096, 1, 32, ctypes.c_void_p(16), 0, 4, None, 0,
                                  1.0, ctypes.c_void_p(16), None)
     assert st == m.TQ_ERR_WORKSPACE
+
+
+def test_noalloc_rejected_arguments_enqueue_nothing():
+    """Argument errors come back synchronously, before the shared array is touched: a null
+    output, a misaligned packed cache and a non-finite scale are refused, and a following
+    valid call still matches tq_logits."""
+    torch = torch_cuda()
+    m = tq()
+    d = 128
+    pi, s = ti.haar_rotation(d, 105), ti.gaussian_sketch(d, d, 106)
+    n_kv, n_tok, g = 2, 300, 4
+    codec = make_codec(d, d, 2, True, pi, s)
+    keys = np.concatenate([ti.key_stream(4, 0, h, n_tok) for h in range(n_kv)])
+    packed, _ = gpu_quantize(codec, to_dev_bf16(keys), n_kv, n_tok)
+    q = to_dev_bf16(ti.decode_queries(30, 1, n_kv * g))
+    got = torch.full((1, n_kv * g, n_tok), float("nan"), dtype=torch.float32, device="cuda")
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())
+    lib = m.lib
+    assert lib.tq_logits_noalloc(codec.ref, vp(packed), 1, n_kv, n_tok, vp(q), 1, g, None, 0, 1.0, None,
+                                 None) == m.TQ_ERR_ARG
+    assert lib.tq_logits_noalloc(codec.ref, ctypes.c_void_p(packed.data_ptr() + 4), 1, n_kv, n_tok, vp(q), 1, g,
+                                 None, 0, 1.0, vp(got), None) == m.TQ_ERR_ARG
+    assert lib.tq_logits_noalloc(codec.ref, vp(packed), 1, n_kv, n_tok, vp(q), 1, g, None, 0, float("inf"),
+                                 vp(got), None) == m.TQ_ERR_ARG
+    torch.cuda.synchronize()
+    assert torch.isnan(got).all()
+    ref = torch.zeros_like(got)
+    ws = m.workspace(codec.workspace_bytes(m.TQ_OP_LOGITS, 1, n_kv, g))
+    m.tq_logits(codec, packed, 1, n_kv, n_tok, q, g, None, 0, 1.0, ref, ws)
+    m.tq_logits_noalloc(codec, packed, 1, n_kv, n_tok, q, g, None, 0, 1.0, got)
+    torch.cuda.synchronize()
+    assert torch.equal(ref, got)
