@@ -286,26 +286,33 @@ def run_gpu(args, world, rank, local):
     h2d = h_append.numel() * 2 + h_q.numel() * 2
     d2h = h_out.numel() * 4
 
-    # DRAM bytes (read + write) per launch of these kernels on this workload, from one ncu
-    # capture each (profiles/k_quantize_tc_c4_append.md, profiles/k_logits_stream_c4.md)
-    ncu_traffic = {"tq_quantize": 67.31e6 + 1.41e6, "tq_logits": 0.69e6 + 220.82e6 + 48.26e6}
     # kernels launched per step: quantize 1, logits 2 (prologue + stream)
     launches_per_step = 3
     dominant = "tq_logits" if t_logit >= t_quant else "tq_quantize"
     logits_roof = {"kernel": "tq_logits (prologue + int8-MMA stream)", "bound": "hbm", "achieved": round(logit_gbs, 1),
                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(logit_gbs / peaks["hbm_gbs"], 4),
-                   "traffic": ncu_traffic["tq_logits"], "peak_kind": peak_kind,
+                   "traffic": ncu_traffic("tq_logits"), "peak_kind": peak_kind,
                    "algorithmic_bytes_per_launch": logit_bytes}
-    # the d = 128 quantize runs its two contractions on fp16 tensor cores, split into hi/lo
-    # passes for fp32-equivalent precision (2 passes for Pi x with bf16 input, 3 for M r):
-    # measured against the bf16 (= fp16) dense peak, with and without the split passes
+    # quantize: the roofline time is the larger of its algorithmic bytes at the HBM peak and its
+    # algorithmic flops (two d x d contractions per vector, one pass each) at the dense bf16
+    # peak; the kernel runs the contractions as split passes for fp32-equivalent precision
+    # (three bf16 passes for Pi x, three fp16 passes for M r), reported beside it
     tpeak = peaks["bf16_tflops"]
-    passes = 2.5
-    quant_roof = {"kernel": "tq_quantize (fp16 tensor-core split, tcgen05.mma)", "bound": "tensor",
-                  "achieved": round(quant_tf, 2), "peak": tpeak, "unit": "TFLOP/s",
-                  "frac": round(quant_tf / tpeak, 4), "frac_with_split_passes": round(passes * quant_tf / tpeak, 4),
-                  "traffic": ncu_traffic["tq_quantize"], "algorithmic_flops_per_launch": quant_flops,
-                  "peak_kind": peak_kind + " (bf16 burst)"}
+    t_hbm = quant_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = quant_flops / (tpeak * 1e12)
+    passes = 3.0
+    q_bound = "hbm" if t_hbm >= t_tc else "tensor"
+    quant_roof = {"kernel": "tq_quantize (warp-specialized tcgen05: TMA rows, split-precision MMAs, TMEM epilogue)",
+                  "bound": q_bound,
+                  "achieved": round(quant_bytes / (t_quant * 1e-3) / 1e9, 1) if q_bound == "hbm" else round(quant_tf, 2),
+                  "peak": peaks["hbm_gbs"] if q_bound == "hbm" else tpeak,
+                  "unit": "GB/s" if q_bound == "hbm" else "TFLOP/s",
+                  "frac": round(max(t_hbm, t_tc) / (t_quant * 1e-3), 4),
+                  "traffic": ncu_traffic("tq_quantize"), "algorithmic_bytes_per_launch": quant_bytes,
+                  "algorithmic_flops_per_launch": quant_flops, "tensor_TFLOP_per_s": round(quant_tf, 2),
+                  "tensor_frac": round(quant_tf / tpeak, 4), "split_passes": passes,
+                  "tensor_frac_with_split_passes": round(passes * quant_tf / tpeak, 4),
+                  "peak_kind": peak_kind + (" (HBM copy)" if q_bound == "hbm" else " (bf16 burst)")}
     also = {} if args.no_extras else extra_workloads(torch, tq, ti, gen, peaks)
     line = {
         "metric": METRIC, "value": keys_per_step * world / (ms_step * 1e-3), "unit": "keys/s",
@@ -331,6 +338,33 @@ def run_gpu(args, world, rank, local):
         "also": also,
     }
     return line
+
+
+# DRAM bytes (read + write) per launch of the step's kernels on the c4 workload, each from one
+# ncu capture (profiles/), valid only while the kernel sources it was taken on are unchanged:
+# name -> (bytes, {source file: sha256 prefix at capture time})
+NCU_TRAFFIC = {
+    "tq_logits": (0.69e6 + 220.82e6 + 48.26e6, {"k_logits.cu": None}),
+    "tq_quantize": (None, {"k_quantize_ws.cu": None}),
+}
+
+
+def _src_sha(name):
+    import hashlib
+    path = os.path.join(ROOT, "kv_cache_vector_03_b200", "csrc", name)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def ncu_traffic(kernel):
+    """The captured DRAM traffic of a kernel, or None once its source has changed since."""
+    byts, srcs = NCU_TRAFFIC[kernel]
+    if byts is None:
+        return None
+    for name, sha in srcs.items():
+        if sha is None or _src_sha(name) != sha:
+            return None
+    return byts
 
 
 def time_calls(torch, fn, n_iter, n_warm=3):

@@ -55,10 +55,36 @@ __global__ void k_prepare(PrepParams p) {
     }
 }
 
+// Operand images of the warp-specialized quantize (D = Mp = 128): Pi as three bf16 pieces
+// (Pi_1 = bf16(Pi), Pi_2 = bf16(Pi - Pi_1), Pi_3 = bf16(Pi - Pi_1 - Pi_2): each difference
+// is exact in fp32 and the three pieces sum to the fp32 matrix), and the fp16 hi/lo pair of
+// 256 M, all in the swizzled shared-memory layout. Runs after k_prepare_split (reads M).
+__global__ void k_prepare_images(PrepParams p) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < 128 * 128; e += gridDim.x * blockDim.x) {
+        const int i = e >> 7, j = e & 127;
+        const uint32_t off = tq_sw128_offset(i, j);
+        const float v = (i < p.d && j < p.d) ? p.pi[(int64_t)i * p.d + j] : 0.f;
+        const __nv_bfloat16 b1 = __float2bfloat16_rn(v);
+        const float r1 = v - __bfloat162float(b1);
+        const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 b3 = __float2bfloat16_rn(r1 - __bfloat162float(b2));
+        *reinterpret_cast<__nv_bfloat16*>(p.img + 0 * kTqImageBytes + off) = b1;
+        *reinterpret_cast<__nv_bfloat16*>(p.img + 1 * kTqImageBytes + off) = b2;
+        *reinterpret_cast<__nv_bfloat16*>(p.img + 2 * kTqImageBytes + off) = b3;
+        *reinterpret_cast<uint16_t*>(p.img + 3 * kTqImageBytes + off) = p.mh[e];
+        *reinterpret_cast<uint16_t*>(p.img + 4 * kTqImageBytes + off) = p.ml[e];
+    }
+}
+
 cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
     k_prepare<<<296, 256, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     k_prepare_split<<<296, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (p.img) {
+        k_prepare_images<<<64, 256, 0, st>>>(p);
+        e = cudaGetLastError();
+    }
+    return e;
 }

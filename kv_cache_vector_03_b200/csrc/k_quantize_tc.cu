@@ -824,6 +824,7 @@ cudaError_t launch_b(const QuantParams& p, cudaStream_t st) {
 // d <= 128 with m <= 128 (or no sketch)
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st) {
     const bool f32 = p.dtype == 0;
+    if (tq_quantize_ws_eligible(p)) return tq_launch_quantize_ws(p, st);
     if (p.t.qjl && !f32) {
         switch (p.t.B) {
             case 1: return launch_tc_pipe<1>(p, st);

@@ -1,0 +1,508 @@
+// tq_quantize for bf16 keys with d, m <= 128: a warp-specialized tcgen05 pipeline (rotate,
+// nearest Lloyd-Max centroid, residual, QJL sign sketch, pack; blog.hotdry.top "TurboQuant
+// vector-search compression", sections "Random rotation and scalar quantization" and "QJL
+// residual correction"; a2a-mcp.org "What is TurboQuant", stage 1).
+//
+// One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with ten warps:
+//   warp 8 (one thread)  TMA: the tile's raw bf16 rows, as four 32-row boxes per 64-column
+//                        K-block, straight into the 128-byte-swizzled K-major operand layout
+//                        (two stages);
+//   warp 9 (one thread)  tensor cores: Y = X (Pi_1 + Pi_2 + Pi_3)^T, three bf16 passes
+//                        whose sum is the fp32 rotation applied to the exact bf16 input, into
+//                        TMEM; later Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo +
+//                        lo.hi) with the residual operand R read from TMEM;
+//   warps 0-3, 4-7       epilogue, two warpgroups taking alternate tiles, one thread per
+//                        vector (TMEM lane) over all of its coordinates:
+//                          |x| = |Y row| (Pi is orthogonal), per-row thresholds t_k |x| and
+//                          centroids, the code planes from sign bits, the scaled residual
+//                          r |x| 2^k split into an integer-valued fp16 hi part and an fp16
+//                          lo part written to TMEM, gamma^2; then the sign plane from Z.
+// Resident in shared memory: Pi_1..3 (bf16) and 256 M hi/lo (fp16), 160 KB, loaded once by
+// bulk copies from the prepared images; two 32 KB stages of X. TMEM (512 columns): per
+// warpgroup 128 columns for Y then Z of its tile, and 128 for the residual operand.
+#include <cuda.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "tq_device.cuh"
+
+namespace {
+
+constexpr int kWsThreads = 320;
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr uint32_t kMat = 32768;          // one 128 x 128 16-bit operand
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+// shared memory map (from a 1024-aligned base)
+constexpr uint32_t oPi = 0;               // Pi_1, Pi_2, Pi_3 (bf16)
+constexpr uint32_t oM = 3 * kMat;         // M_hi, M_lo (fp16)
+constexpr uint32_t oX = 5 * kMat;         // X stage 0, 1 (bf16)
+constexpr uint32_t oBar = 7 * kMat;       // barriers, TMEM base, abort flag
+constexpr size_t kWsSmem = (size_t)7 * kMat + 256 + 1024;
+
+// barrier indices
+enum { bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bTEmpty = 10, bOps = 12, bDrain = 13, kNumBars = 14 };
+
+// instruction descriptors, kind::f16, fp32 D, K-major A and B, M = N = 128
+constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdescBF16 = kIdescF16 | (1u << 7) | (1u << 10);
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// K-step k (16 elements) of a 128 x 128 operand: K-block k / 4, 32 bytes per step inside it
+__device__ __forceinline__ uint32_t kstep(int k) { return (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u; }
+
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n}\n" ::"r"(d),
+        "l"(a), "l"(b), "r"(acc), "r"(idesc));
+}
+// A from TMEM (row = lane, two 16-bit elements per column), B from shared memory
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n}\n" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(acc), "r"(idesc));
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     tq_smem_addr(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// Bounded wait that also gives up when another role has aborted; a wait that runs out sets
+// the abort flag itself.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
+    const uint32_t a = tq_smem_addr(bar);
+    for (uint32_t it = 0; it < kWaitLimit; ++it) {
+        if (mbar_try(a, parity)) return true;
+        if ((it & 31u) == 31u && *abort_flag) return false;
+    }
+    *abort_flag = 1u;
+    return false;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tq_smem_addr(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tq_smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(tq_smem_addr(bar))
+                 : "memory");
+}
+// one box of the 3-D tensor map [stream][token][coordinate] (no multicast)
+__device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                          uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(tq_smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? ~0u : n <= 0 ? 0u : (1u << n) - 1u; }
+__device__ __forceinline__ uint32_t shl_in(uint32_t w, uint32_t v) { return __funnelshift_l(v, w, 1); }
+__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+struct WsParams {
+    uint8_t* packed;
+    const uint8_t* img;        // prepared operand images (Pi_1..3, M_hi, M_lo)
+    uint32_t* status;
+    int64_t n_streams, n_tok, nb;
+    int d, m;
+    TqDims t;
+    TqCodebookConsts cb;
+};
+
+template <int B, bool FULL>
+__global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_constant__ CUtensorMap xmap, WsParams p) {
+    constexpr int L = 1 << B, H = L / 2;
+    extern __shared__ uint8_t raw_smem[];
+    const uint32_t raw = tq_smem_addr(raw_smem);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
+    uint8_t* sm = raw_smem + pad;
+    const uint32_t sb = raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + oBar);
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + oBar + 8 * kNumBars);
+    volatile uint32_t* s_abort = s_tmem + 1;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t total_blocks = p.n_streams * p.nb;
+    const int64_t n_tiles = (total_blocks + 3) / 4;
+    const int n_local = (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);   // tiles of this CTA
+
+    if (tid == 0) {
+        for (int i = 0; i < kNumBars; ++i) {
+            const bool four = (i >= bRFull && i < bRFull + 2) || (i >= bTEmpty && i < bTEmpty + 2);
+            tq_mbar_init(&bars[i], four ? 4 : 1);
+        }
+        *s_abort = 0u;
+        tq_fence_mbar_init();
+    }
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tq_smem_addr(s_tmem)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+            // resident operands: five 32 KB images
+            mbar_expect_tx(&bars[bOps], 5 * kMat);
+            for (int i = 0; i < 5; ++i) bulk_copy(sb + oPi + i * kMat, p.img + (size_t)i * kMat, kMat, &bars[bOps]);
+            int issued = 0;
+            for (int i = 0; i < n_local; ++i) {
+                const int xs = i & 1;
+                if (i >= 2 && !wait_bar(&bars[bXEmpty + xs], ((i >> 1) - 1) & 1, s_abort)) break;
+                const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+                const int64_t left = total_blocks - tile * 4;
+                const int nvb = left < 4 ? (int)left : 4;
+                mbar_expect_tx(&bars[bXFull + xs], (uint32_t)nvb * 8192u);
+                for (int jb = 0; jb < nvb; ++jb) {
+                    const int64_t gb = tile * 4 + jb;
+                    const int s = (int)(gb / p.nb), tok0 = (int)(gb % p.nb) * 32;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tma_load3(sb + oX + xs * kMat + h * 16384 + jb * 4096, &xmap, 64 * h, tok0, s, &bars[bXFull + xs]);
+                }
+                issued = i + 1;
+            }
+            // nothing may be in flight when the CTA exits: wait (bounded) for the last load of
+            // each stage (a completed phase returns at once)
+            for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i)
+                tq_mbar_wait(&bars[bXFull + (i & 1)], (i >> 1) & 1, kWaitLimit);
+            tq_mbar_wait(&bars[bOps], 0, kWaitLimit);
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            bool ok = wait_bar(&bars[bOps], 0, s_abort);
+            auto issue_z = [&](int i) -> bool {
+                const int b = i & 1;
+                if (!wait_bar(&bars[bRFull + b], (i >> 1) & 1, s_abort)) return false;
+                fence_after();
+                const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
+#pragma unroll
+                for (int ps = 0; ps < 3; ++ps) {
+                    const uint32_t ra = r + (ps == 2 ? 64u : 0u);
+                    const uint32_t mb = sb + oM + (ps == 1 ? kMat : 0u);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
+                }
+                mma_commit(&bars[bZFull + b]);
+                return true;
+            };
+            for (int i = 0; ok && i < n_local; ++i) {
+                const int b = i & 1;
+                if (!wait_bar(&bars[bXFull + b], (i >> 1) & 1, s_abort)) { ok = false; break; }
+                if (i >= 2 && !wait_bar(&bars[bTEmpty + b], ((i >> 1) - 1) & 1, s_abort)) { ok = false; break; }
+                fence_after();
+                const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat;
+#pragma unroll
+                for (int ps = 0; ps < 3; ++ps)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ss(d, sdesc(xa + kstep(k)), sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16, (ps | k) != 0);
+                mma_commit(&bars[bYFull + b]);
+                mma_commit(&bars[bXEmpty + b]);
+                if (i >= 1 && !issue_z(i - 1)) { ok = false; break; }
+            }
+            if (ok && n_local >= 1) issue_z(n_local - 1);
+            // every MMA this thread issued completes before TMEM is released (a commit tracks
+            // all earlier MMAs of the thread)
+            mma_commit(&bars[bDrain]);
+            tq_mbar_wait(&bars[bDrain], 0, kWaitLimit);
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue
+        const int wg = warp >> 2, wq = warp & 3;
+        const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+        const uint32_t tY = tmem + lane_base + 128u * wg;               // Y, then Z, of this warpgroup's tiles
+        const uint32_t tR = tmem + lane_base + 256u + 128u * wg;        // residual operand hi | lo
+        const int u = lane >> 3, gq = lane & 7;
+        float tb[H > 1 ? H - 1 : 1], cmg[H];
+#pragma unroll
+        for (int k = 0; k < H - 1; ++k) tb[k] = p.cb.bounds[H + k];
+#pragma unroll
+        for (int k = 0; k < H; ++k) cmg[k] = p.cb.cent[H + k];
+        int j = 0;
+        for (int i = wg; i < n_local; i += 2, ++j) {
+            const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+            const int64_t gb = tile * 4 + wq;
+            const bool blk_ok = gb < total_blocks;
+            const int64_t tok = blk_ok ? (gb % p.nb) * 32 + lane : 0;
+            const bool rvalid = blk_ok && tok < p.n_tok;
+            bool w_ok = true;
+            if (lane == 0) w_ok = wait_bar(&bars[bYFull + wg], j & 1, s_abort);
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+            fence_after();
+            // |x| from the rotated row (orthogonal Pi)
+            float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float y[32];
+                tmem_ld32(tY + 32u * c, y);
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    ss0 = fmaf(y[e], y[e], ss0);
+                    ss1 = fmaf(y[e + 1], y[e + 1], ss1);
+                }
+            }
+            float ss = ss0 + ss1;
+            const bool tiny = ss < 1e-30f && ss > 0.f;
+            if (__any_sync(0xffffffffu, tiny)) {
+                // a tiny vector in the warp: its sum of squares is taken again on the row scaled by
+                // 2^60 (the TMEM loads are warp-wide, so every lane takes part)
+                float acc = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float y[32];
+                    tmem_ld32(tY + 32u * c, y);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float v = y[e] * 0x1p60f;
+                        acc = fmaf(v, v, acc);
+                    }
+                }
+                if (tiny) ss = fmaxf(acc * 0x1p-120f, 0x1p-149f);
+            }
+            const float n = sqrtf(ss);
+            const bool finite = isfinite(n);
+            const float ne = (n > 0.f && finite) ? n : 1.f;
+            // kap = 2^(10 - floor(log2 ne)): |residual| * ne * kap < 2^11 (integer hi part exact in fp16)
+            const int ex = ((__float_as_int(ne) >> 23) & 0xff) - 127;
+            const float kap = __int_as_float((127 + min(max(10 - ex, -126), 127)) << 23);
+            float th[H > 1 ? H - 1 : 1], cs[H];
+#pragma unroll
+            for (int k = 0; k < H - 1; ++k) th[k] = tb[k] * ne;
+#pragma unroll
+            for (int k = 0; k < H; ++k) cs[k] = cmg[k] * ne * kap;
+            float g2a = 0.f, g2b = 0.f;
+            uint8_t* blk = p.packed + (size_t)(blk_ok ? gb : 0) * p.t.block_bytes;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float y[32], rr[32];
+                tmem_ld32(tY + 32u * c, y);
+                uint32_t pw[B];
+#pragma unroll
+                for (int pl = 0; pl < B; ++pl) pw[pl] = 0u;
+#pragma unroll
+                for (int e = 31; e >= 0; --e) {
+                    const float yv = y[e];
+                    const uint32_t w = __float_as_uint(0.f - yv);      // sign bit: y > 0
+                    const float ay = fabsf(yv);
+                    float cm = cs[0];
+                    uint32_t dbits[H > 1 ? H - 1 : 1];
+#pragma unroll
+                    for (int k = 0; k < H - 1; ++k) {
+                        const float dk = th[k] - ay;                     // sign bit: |y| above boundary k
+                        dbits[k] = __float_as_uint(dk);
+                        cm = dk < 0.f ? cs[k + 1] : cm;
+                    }
+                    // the centroid takes the sign of y (negative for y <= 0: the lower cell)
+                    const float csg = __uint_as_float(__float_as_uint(cm) ^ (~w & 0x80000000u));
+                    float r = fmaf(yv, kap, -csg);
+                    if (!FULL && 32 * c + e >= p.d) r = 0.f;
+                    rr[e] = r;
+                    if (e & 1) g2a = fmaf(r, r, g2a);
+                    else g2b = fmaf(r, r, g2b);
+                    // index bits: top bit = [y > 0]; lower bits = level bits XNOR [y > 0]
+                    pw[B - 1] = shl_in(pw[B - 1], w);
+                    if constexpr (B == 2) {
+                        pw[0] = shl_in(pw[0], ~(dbits[0] ^ w));
+                    } else if constexpr (B == 3) {
+                        pw[1] = shl_in(pw[1], ~(dbits[1] ^ w));
+                        pw[0] = shl_in(pw[0], ~(dbits[0] ^ dbits[1] ^ dbits[2] ^ w));
+                    }
+                }
+                // residual operand: an integer-valued hi part (|hi| <= 2048, exact in fp16) and
+                // the remainder in [-1/2, 1/2] as lo
+                uint32_t hw[16], lw[16];
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                    const float h0 = (rr[2 * q] + 12582912.f) - 12582912.f;
+                    const float h1 = (rr[2 * q + 1] + 12582912.f) - 12582912.f;
+                    hw[q] = pack_half2(h0, h1);
+                    lw[q] = pack_half2(rr[2 * q] - h0, rr[2 * q + 1] - h1);
+                }
+                tmem_st16(tR + 16u * c, hw);
+                tmem_st16(tR + 64u + 16u * c, lw);
+                // code planes of this vector (zero for padding tokens and coordinates beyond d)
+                if (blk_ok) {
+                    const uint32_t keep = rvalid ? low_bits(p.d - 32 * c) : 0u;
+#pragma unroll
+                    for (int pl = 0; pl < B; ++pl)
+                        reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + c) * 4 + u] = pw[pl] & keep;
+                }
+            }
+            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[bRFull + wg]);
+            // signs of Z = R M^T
+            if (lane == 0) w_ok = wait_bar(&bars[bZFull + wg], j & 1, s_abort);
+            if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+            fence_after();
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                float z[32];
+                tmem_ld32(tY + 32u * c, z);
+                uint32_t sw = 0u;
+#pragma unroll
+                for (int e = 31; e >= 0; --e) sw = shl_in(sw, __float_as_uint(z[e]));
+                // bit = [z >= 0]: the sign bit inverted (an exact zero has sign bit 0)
+                if (blk_ok)
+                    reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + c) * 4 + u] =
+                        rvalid ? ~sw & low_bits(p.m - 32 * c) : 0u;
+            }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[bTEmpty + wg]);
+            if (blk_ok) {
+                const float gam = sqrtf(g2a + g2b) / (ne * kap);
+                const uint32_t nh = rvalid ? tq_half_bits(n) : 0u;
+                const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
+                if (rvalid && (!finite || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
+                reinterpret_cast<uint32_t*>(blk + p.t.sec_a)[gq * 4 + u] = nh | (gh << 16);
+            }
+        }
+    }
+    __syncthreads();
+    if (*s_abort) {
+        if (tid == 0) tq_raise(p.status, TQ_FLAG_TIMEOUT);
+    }
+    if (warp == kMmaWarp) {
+        fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+    }
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (libtq does not link libcuda)
+EncodeTiledFn encode_tiled() {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (f) return f;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !ptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    f = reinterpret_cast<EncodeTiledFn>(ptr);
+    fn.store(f, std::memory_order_release);
+    return f;
+}
+
+template <int B, bool FULL>
+cudaError_t launch_ws(const CUtensorMap& map, const WsParams& wp, cudaStream_t st) {
+    auto kern = k_quantize_ws<B, FULL>;
+    static TqLaunchCache cache;
+    int sms = 0;
+    cudaError_t e = tq_kernel_setup(kern, kWsThreads, kWsSmem, cache, &sms, nullptr);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = (wp.n_streams * wp.nb + 3) / 4;
+    const int64_t grid = std::min<int64_t>(tiles, sms);
+    if (grid > 0) kern<<<(unsigned)grid, kWsThreads, kWsSmem, st>>>(map, wp);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+// Whether the warp-specialized kernel takes this request: bf16 keys with D = Mp = 128, B <= 3,
+// the prepared images present, and rows a tensor map can describe (16-byte aligned base, stream
+// stride a multiple of 8 elements).
+bool tq_quantize_ws_eligible(const QuantParams& p) {
+    if (!p.t.qjl || p.dtype != 1 || p.t.D != 128 || p.t.Mp != 128 || !p.img) return false;
+    if (p.t.B < 1 || p.t.B > 3) return false;
+    if ((reinterpret_cast<uintptr_t>(p.x) & 15) != 0) return false;
+    if (p.n_streams > 1 && p.x_stride % 8 != 0) return false;
+    if (p.n_tok > 0x7fffffffLL || p.n_streams > 0x7fffffffLL) return false;
+    return encode_tiled() != nullptr;
+}
+
+cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t dims[3] = {(cuuint64_t)p.t.d, (cuuint64_t)p.n_tok, (cuuint64_t)p.n_streams};
+    const int64_t stride = p.n_streams > 1 ? p.x_stride : p.n_tok * p.t.d;
+    const cuuint64_t strides[2] = {(cuuint64_t)p.t.d * 2, (cuuint64_t)stride * 2};
+    const cuuint32_t box[3] = {64, 32, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.x), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+    WsParams wp;
+    wp.packed = p.packed;
+    wp.img = p.img;
+    wp.status = p.status;
+    wp.n_streams = p.n_streams;
+    wp.n_tok = p.n_tok;
+    wp.nb = p.nb;
+    wp.d = p.t.d;
+    wp.m = p.t.m;
+    wp.t = p.t;
+    wp.cb = p.cb;
+    const bool full = p.t.d == 128;
+    switch (p.t.B) {
+        case 1: return full ? launch_ws<1, true>(map, wp, st) : launch_ws<1, false>(map, wp, st);
+        case 2: return full ? launch_ws<2, true>(map, wp, st) : launch_ws<2, false>(map, wp, st);
+        case 3: return full ? launch_ws<3, true>(map, wp, st) : launch_ws<3, false>(map, wp, st);
+    }
+    return cudaErrorInvalidValue;
+}

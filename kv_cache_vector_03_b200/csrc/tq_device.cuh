@@ -268,8 +268,17 @@ struct PrepParams {
     float* sT;
     float* mT;
     uint16_t *pih, *pil, *mh, *ml;
+    uint8_t* img;          // operand images of the warp-specialized quantize, or null
     int d, m, D, Mp, qjl;
 };
+
+// Byte offset of element (row r, column c) in a 128 x 128 16-bit tensor-core operand laid
+// out as two K-blocks of 64 columns, [128 rows][128 B] each, in 8-row atoms of 1024 B with
+// the 16-byte chunk index XOR (row mod 8) (the canonical K-major 128-byte swizzle).
+TQ_DEVICE uint32_t tq_sw128_offset(int r, int c) {
+    const int kc = c >> 3;
+    return (uint32_t)((kc >> 3) * 16384 + (r >> 3) * 1024 + (r & 7) * 128 + (((kc & 7) ^ (r & 7)) << 4) + (c & 7) * 2);
+}
 
 struct QuantParams {
     const void* x;
@@ -279,6 +288,7 @@ struct QuantParams {
     const float* piT;
     const float* mT;
     const uint16_t *pih, *pil, *mh, *ml;
+    const uint8_t* img;    // operand images of the warp-specialized kernel, or null
     uint32_t* status;
     int vec_ok;            // rows can be read 4 elements at a time (alignment of x, stride, d)
     TqDims t;
@@ -393,6 +403,8 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st);
 cudaError_t tq_launch_dequant(const DequantParams& p, cudaStream_t st);
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st);
+bool tq_quantize_ws_eligible(const QuantParams& p);
+cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
 cudaError_t tq_launch_q8_quantize(const Q8QuantParams& p, cudaStream_t st);
