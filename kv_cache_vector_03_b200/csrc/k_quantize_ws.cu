@@ -3,23 +3,26 @@
 // vector-search compression", sections "Random rotation and scalar quantization" and "QJL
 // residual correction"; a2a-mcp.org "What is TurboQuant", stage 1).
 //
-// One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with ten warps:
-//   warp 8 (one thread)  TMA: the tile's raw bf16 rows, as four 32-row boxes per 64-column
-//                        K-block, straight into the 128-byte-swizzled K-major operand layout
-//                        (two stages);
-//   warp 9 (one thread)  tensor cores: Y = X (Pi_1 + Pi_2 + Pi_3)^T, three bf16 passes
-//                        whose sum is the fp32 rotation applied to the exact bf16 input, into
-//                        TMEM; later Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo +
-//                        lo.hi) with the residual operand R read from TMEM;
-//   warps 0-3, 4-7       epilogue, two warpgroups taking alternate tiles, one thread per
-//                        vector (TMEM lane) over all of its coordinates:
-//                          |x| = |Y row| (Pi is orthogonal), per-row thresholds t_k |x| and
-//                          centroids, the code planes from sign bits, the scaled residual
-//                          r |x| 2^k split into an integer-valued fp16 hi part and an fp16
-//                          lo part written to TMEM, gamma^2; then the sign plane from Z.
+// One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with 18 warps:
+//   warp 16 (one thread)  TMA: the tile's raw bf16 rows, as four 32-row boxes per 64-column
+//                         K-block, straight into the 128-byte-swizzled K-major operand layout
+//                         (two stages);
+//   warp 17 (one thread)  tensor cores: Y = X (Pi_1 + Pi_2 + Pi_3)^T, three bf16 passes
+//                         whose sum is the fp32 rotation applied to the exact bf16 input, into
+//                         TMEM; Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo + lo.hi) with
+//                         the residual operand R read from TMEM. Whichever of the next Y and
+//                         the next Z is ready is issued first;
+//   warps 0-15            epilogue: warps 0-7 take even tiles, 8-15 odd ones; in each group
+//                         warp w reads TMEM lanes 32 (w mod 4) .. +31 (one vector per thread)
+//                         and columns 64 ((w / 4) mod 2) .. +63:
+//                           |x| = |Y row| over all 128 columns (Pi is orthogonal), per-row
+//                           thresholds t_k |x| and centroids, the code planes from sign bits,
+//                           the scaled residual r |x| 2^k split into an integer-valued fp16 hi
+//                           part and an fp16 lo part written to TMEM, gamma^2 (the two column
+//                           halves meet through shared memory); then the sign plane from Z.
 // Resident in shared memory: Pi_1..3 (bf16) and 256 M hi/lo (fp16), 160 KB, loaded once by
-// bulk copies from the prepared images; two 32 KB stages of X. TMEM (512 columns): per
-// warpgroup 128 columns for Y then Z of its tile, and 128 for the residual operand.
+// bulk copies from the prepared images; two 32 KB stages of X. TMEM (512 columns): per tile
+// parity 128 columns for Y then Z, and 128 for the residual operand (hi 64 | lo 64).
 #include <cuda.h>
 
 #include <algorithm>
@@ -29,20 +32,27 @@
 
 namespace {
 
-constexpr int kWsThreads = 320;
-constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kWsThreads = 576;
+constexpr int kEpiWarps = 16, kTmaWarp = 16, kMmaWarp = 17;
 constexpr uint32_t kMat = 32768;          // one 128 x 128 16-bit operand
 constexpr uint32_t kWaitLimit = 1u << 22;
+constexpr uint32_t kIdleLimit = 1u << 24; // polls of the MMA issuer with nothing to issue
 
 // shared memory map (from a 1024-aligned base)
 constexpr uint32_t oPi = 0;               // Pi_1, Pi_2, Pi_3 (bf16)
 constexpr uint32_t oM = 3 * kMat;         // M_hi, M_lo (fp16)
 constexpr uint32_t oX = 5 * kMat;         // X stage 0, 1 (bf16)
-constexpr uint32_t oBar = 7 * kMat;       // barriers, TMEM base, abort flag
-constexpr size_t kWsSmem = (size_t)7 * kMat + 256 + 1024;
+constexpr uint32_t oG2 = 7 * kMat;        // gamma^2 of the upper column half [tile parity][row]
+constexpr uint32_t oBar = oG2 + 2 * 128 * 4;   // barriers, then the TMEM base and the abort flag
 
-// barrier indices
-enum { bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bTEmpty = 10, bOps = 12, bDrain = 13, kNumBars = 14 };
+// barrier indices: per X stage, per tile parity, per (tile parity, lane quarter)
+enum {
+    bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bTEmpty = 10, bOps = 12, bDrain = 13,
+    bG2Full = 14, bG2Empty = 22, kNumBars = 30
+};
+constexpr size_t kWsSmemUsed = (size_t)oBar + 8 * kNumBars + 8;
+constexpr size_t kWsSmem = 232448;        // the per-CTA maximum: the used bytes plus the alignment pad
+static_assert(kWsSmemUsed + 1023 <= kWsSmem, "shared memory map too large");
 
 // instruction descriptors, kind::f16, fp32 D, K-major A and B, M = N = 128
 constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
@@ -98,6 +108,40 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
         "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
+}
+
+// 16 columns of this thread's TMEM lane, without waiting (tmem_wait_ld before use)
+__device__ __forceinline__ void tld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+// wait for this thread's TMEM loads; the registers of the last one are operands, so no use of
+// them can be scheduled before the wait
+__device__ __forceinline__ void twait(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tst8(uint32_t taddr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(v[0]),
+                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(tq_smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
 }
 
 __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
@@ -159,6 +203,58 @@ struct WsParams {
     TqCodebookConsts cb;
 };
 
+// One row's worth of the code and residual work on 16 TMEM columns: codes into the low
+// 16 bits of pw[] (coordinate e at bit e), the residual operand into hw / lw (two fp16 per
+// word), gamma^2 into g2. Column index col0 + e; coordinates beyond d (when !FULL) count zero.
+template <int B, bool FULL>
+__device__ __forceinline__ void residual16(const uint32_t (&yb)[16], const float (&th)[(1 << B) / 2 > 1 ? (1 << B) / 2 - 1 : 1],
+                                           const float (&cs)[(1 << B) / 2], float kap, int col0, int d,
+                                           uint32_t (&pw)[B], uint32_t (&hw)[8], uint32_t (&lw)[8], float& g2a,
+                                           float& g2b) {
+    constexpr int H = (1 << B) / 2;
+    float rr[16];
+#pragma unroll
+    for (int pl = 0; pl < B; ++pl) pw[pl] = 0u;
+#pragma unroll
+    for (int e = 15; e >= 0; --e) {
+        const float yv = __uint_as_float(yb[e]);
+        const uint32_t w = __float_as_uint(0.f - yv);      // sign bit: y > 0
+        const float ay = fabsf(yv);
+        float cm = cs[0];
+        uint32_t dbits[H > 1 ? H - 1 : 1];
+#pragma unroll
+        for (int k = 0; k < H - 1; ++k) {
+            const float dk = th[k] - ay;                     // sign bit: |y| above boundary k
+            dbits[k] = __float_as_uint(dk);
+            cm = dk < 0.f ? cs[k + 1] : cm;
+        }
+        // the centroid takes the sign of y (negative for y <= 0: the lower cell)
+        const float csg = __uint_as_float(__float_as_uint(cm) ^ (~w & 0x80000000u));
+        float r = fmaf(yv, kap, -csg);
+        if (!FULL && col0 + e >= d) r = 0.f;
+        rr[e] = r;
+        if (e & 1) g2a = fmaf(r, r, g2a);
+        else g2b = fmaf(r, r, g2b);
+        // index bits: top bit = [y > 0]; lower bits = level bits XNOR [y > 0]
+        pw[B - 1] = shl_in(pw[B - 1], w);
+        if constexpr (B == 2) {
+            pw[0] = shl_in(pw[0], ~(dbits[0] ^ w));
+        } else if constexpr (B == 3) {
+            pw[1] = shl_in(pw[1], ~(dbits[1] ^ w));
+            pw[0] = shl_in(pw[0], ~(dbits[0] ^ dbits[1] ^ dbits[2] ^ w));
+        }
+    }
+    // residual operand: an integer-valued hi part (|hi| <= 2048, exact in fp16) and the
+    // remainder in [-1/2, 1/2] as lo
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+        const float h0 = (rr[2 * q] + 12582912.f) - 12582912.f;
+        const float h1 = (rr[2 * q + 1] + 12582912.f) - 12582912.f;
+        hw[q] = pack_half2(h0, h1);
+        lw[q] = pack_half2(rr[2 * q] - h0, rr[2 * q + 1] - h1);
+    }
+}
+
 template <int B, bool FULL>
 __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_constant__ CUtensorMap xmap, WsParams p) {
     constexpr int L = 1 << B, H = L / 2;
@@ -167,6 +263,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
     uint8_t* sm = raw_smem + pad;
     const uint32_t sb = raw + pad;
+    float* s_g2 = reinterpret_cast<float*>(sm + oG2);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + oBar);
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + oBar + 8 * kNumBars);
     volatile uint32_t* s_abort = s_tmem + 1;
@@ -178,8 +275,11 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
 
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
-            const bool four = (i >= bRFull && i < bRFull + 2) || (i >= bTEmpty && i < bTEmpty + 2);
-            tq_mbar_init(&bars[i], four ? 4 : 1);
+            int count = 1;
+            if (i >= bRFull && i < bRFull + 2) count = 8;         // the 8 warps of a tile
+            if (i >= bTEmpty && i < bTEmpty + 2) count = 8;
+            if (i >= bG2Full && i < bG2Full + 8) count = 32;      // every lane of the upper-half warp
+            tq_mbar_init(&bars[i], count);
         }
         *s_abort = 0u;
         tq_fence_mbar_init();
@@ -224,39 +324,57 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             tq_mbar_wait(&bars[bOps], 0, kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0) {
-            bool ok = wait_bar(&bars[bOps], 0, s_abort);
-            auto issue_z = [&](int i) -> bool {
-                const int b = i & 1;
-                if (!wait_bar(&bars[bRFull + b], (i >> 1) & 1, s_abort)) return false;
-                fence_after();
-                const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
+        if (lane == 0 && wait_bar(&bars[bOps], 0, s_abort)) {
+            int ny = 0, nz = 0;
+            uint32_t idle = 0;
+            while (nz < n_local) {
+                bool progress = false;
+                if (ny < n_local) {
+                    const int b = ny & 1;
+                    if (mbar_test(&bars[bXFull + b], (ny >> 1) & 1) &&
+                        (ny < 2 || mbar_test(&bars[bTEmpty + b], ((ny >> 1) - 1) & 1))) {
+                        fence_after();
+                        const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat;
 #pragma unroll
-                for (int ps = 0; ps < 3; ++ps) {
-                    const uint32_t ra = r + (ps == 2 ? 64u : 0u);
-                    const uint32_t mb = sb + oM + (ps == 1 ? kMat : 0u);
+                        for (int ps = 0; ps < 3; ++ps)
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
+                            for (int k = 0; k < 8; ++k)
+                                mma_ss(d, sdesc(xa + kstep(k)), sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16,
+                                       (ps | k) != 0);
+                        mma_commit(&bars[bYFull + b]);
+                        mma_commit(&bars[bXEmpty + b]);
+                        ++ny;
+                        progress = true;
+                    }
                 }
-                mma_commit(&bars[bZFull + b]);
-                return true;
-            };
-            for (int i = 0; ok && i < n_local; ++i) {
-                const int b = i & 1;
-                if (!wait_bar(&bars[bXFull + b], (i >> 1) & 1, s_abort)) { ok = false; break; }
-                if (i >= 2 && !wait_bar(&bars[bTEmpty + b], ((i >> 1) - 1) & 1, s_abort)) { ok = false; break; }
-                fence_after();
-                const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat;
+                if (nz < ny) {
+                    const int b = nz & 1;
+                    if (mbar_test(&bars[bRFull + b], (nz >> 1) & 1)) {
+                        fence_after();
+                        const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
 #pragma unroll
-                for (int ps = 0; ps < 3; ++ps)
+                        for (int ps = 0; ps < 3; ++ps) {
+                            const uint32_t ra = r + (ps == 2 ? 64u : 0u);
+                            const uint32_t mb = sb + oM + (ps == 1 ? kMat : 0u);
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ss(d, sdesc(xa + kstep(k)), sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16, (ps | k) != 0);
-                mma_commit(&bars[bYFull + b]);
-                mma_commit(&bars[bXEmpty + b]);
-                if (i >= 1 && !issue_z(i - 1)) { ok = false; break; }
+                            for (int k = 0; k < 8; ++k)
+                                mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
+                        }
+                        mma_commit(&bars[bZFull + b]);
+                        ++nz;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    idle = 0;
+                } else {
+                    if (++idle >= kIdleLimit) { *s_abort = 1u; break; }
+                    if ((idle & 31u) == 0u && *s_abort) break;
+                    __nanosleep(20);
+                }
             }
-            if (ok && n_local >= 1) issue_z(n_local - 1);
+        }
+        if (lane == 0) {
             // every MMA this thread issued completes before TMEM is released (a commit tracks
             // all earlier MMAs of the thread)
             mma_commit(&bars[bDrain]);
@@ -264,52 +382,71 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
         }
     } else {
         // ------------------------------------------------------------------ epilogue
-        const int wg = warp >> 2, wq = warp & 3;
+        const int par = warp >> 3, half = (warp >> 2) & 1, wq = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        const uint32_t tY = tmem + lane_base + 128u * wg;               // Y, then Z, of this warpgroup's tiles
-        const uint32_t tR = tmem + lane_base + 256u + 128u * wg;        // residual operand hi | lo
-        const int u = lane >> 3, gq = lane & 7;
+        const uint32_t tY = tmem + lane_base + 128u * par;          // Y, then Z, of this tile parity
+        const uint32_t tR = tmem + lane_base + 256u + 128u * par;   // residual operand hi | lo
+        const int row = 32 * wq + lane, u = lane >> 3, gq = lane & 7;
+        float* g2x = s_g2 + par * 128 + row;
+        uint64_t* g2full = &bars[bG2Full + 4 * par + wq];
+        uint64_t* g2empty = &bars[bG2Empty + 4 * par + wq];
         float tb[H > 1 ? H - 1 : 1], cmg[H];
 #pragma unroll
         for (int k = 0; k < H - 1; ++k) tb[k] = p.cb.bounds[H + k];
 #pragma unroll
         for (int k = 0; k < H; ++k) cmg[k] = p.cb.cent[H + k];
+        // every lane waits (and acquires); the warp continues only if all of them succeeded
+        auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, wait_bar(bar, parity, s_abort)) != 0;
+        };
         int j = 0;
-        for (int i = wg; i < n_local; i += 2, ++j) {
+        for (int i = par; i < n_local; i += 2, ++j) {
             const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
             const int64_t gb = tile * 4 + wq;
             const bool blk_ok = gb < total_blocks;
             const int64_t tok = blk_ok ? (gb % p.nb) * 32 + lane : 0;
             const bool rvalid = blk_ok && tok < p.n_tok;
-            bool w_ok = true;
-            if (lane == 0) w_ok = wait_bar(&bars[bYFull + wg], j & 1, s_abort);
-            if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+            uint8_t* blk = p.packed + (size_t)(blk_ok ? gb : 0) * p.t.block_bytes;
+            if (!warp_wait(&bars[bYFull + par], j & 1)) break;
             fence_after();
-            // |x| from the rotated row (orthogonal Pi)
-            float ss0 = 0.f, ss1 = 0.f;
+            // |x| from the whole rotated row (orthogonal Pi), TMEM loads one step ahead
+            float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
+            {
+                uint32_t ya[16], yb[16];
+                tld16(tY, ya);
+                twait(ya);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float y[32];
-                tmem_ld32(tY + 32u * c, y);
+                for (int c = 0; c < 8; c += 2) {
+                    tld16(tY + 16u * (c + 1), yb);
 #pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    ss0 = fmaf(y[e], y[e], ss0);
-                    ss1 = fmaf(y[e + 1], y[e + 1], ss1);
+                    for (int e = 0; e < 16; e += 2) {
+                        ss0 = fmaf(__uint_as_float(ya[e]), __uint_as_float(ya[e]), ss0);
+                        ss1 = fmaf(__uint_as_float(ya[e + 1]), __uint_as_float(ya[e + 1]), ss1);
+                    }
+                    twait(yb);
+                    if (c + 2 < 8) tld16(tY + 16u * (c + 2), ya);
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        ss2 = fmaf(__uint_as_float(yb[e]), __uint_as_float(yb[e]), ss2);
+                        ss3 = fmaf(__uint_as_float(yb[e + 1]), __uint_as_float(yb[e + 1]), ss3);
+                    }
+                    if (c + 2 < 8) twait(ya);
                 }
             }
-            float ss = ss0 + ss1;
+            float ss = (ss0 + ss1) + (ss2 + ss3);
             const bool tiny = ss < 1e-30f && ss > 0.f;
             if (__any_sync(0xffffffffu, tiny)) {
                 // a tiny vector in the warp: its sum of squares is taken again on the row scaled by
                 // 2^60 (the TMEM loads are warp-wide, so every lane takes part)
                 float acc = 0.f;
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    float y[32];
-                    tmem_ld32(tY + 32u * c, y);
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t yv[16];
+                    tld16(tY + 16u * c, yv);
+                    twait(yv);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float v = y[e] * 0x1p60f;
+                    for (int e = 0; e < 16; ++e) {
+                        const float v = __uint_as_float(yv[e]) * 0x1p60f;
                         acc = fmaf(v, v, acc);
                     }
                 }
@@ -326,93 +463,88 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             for (int k = 0; k < H - 1; ++k) th[k] = tb[k] * ne;
 #pragma unroll
             for (int k = 0; k < H; ++k) cs[k] = cmg[k] * ne * kap;
+            // codes and residual of this warp's 64 columns: two plane words (chunks 2 half, +1)
             float g2a = 0.f, g2b = 0.f;
-            uint8_t* blk = p.packed + (size_t)(blk_ok ? gb : 0) * p.t.block_bytes;
+            {
+                uint32_t ya[16], yb[16];
+                const uint32_t y0 = tY + 64u * half, r0 = tR + 32u * half;
+                tld16(y0, ya);
+                twait(ya);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float y[32], rr[32];
-                tmem_ld32(tY + 32u * c, y);
-                uint32_t pw[B];
+                for (int q = 0; q < 2; ++q) {
+                    const int c = 2 * half + q;      // 32-coordinate chunk = plane word index
+                    uint32_t pa[B], pb[B], hw[8], lw[8];
+                    tld16(y0 + 32u * q + 16u, yb);
+                    residual16<B, FULL>(ya, th, cs, kap, 32 * c, p.d, pa, hw, lw, g2a, g2b);
+                    tst8(r0 + 16u * q, hw);
+                    tst8(r0 + 64u + 16u * q, lw);
+                    twait(yb);
+                    if (q == 0) tld16(y0 + 32u, ya);
+                    residual16<B, FULL>(yb, th, cs, kap, 32 * c + 16, p.d, pb, hw, lw, g2a, g2b);
+                    tst8(r0 + 16u * q + 8u, hw);
+                    tst8(r0 + 64u + 16u * q + 8u, lw);
+                    if (blk_ok) {
+                        const uint32_t keep = rvalid ? low_bits(p.d - 32 * c) : 0u;
 #pragma unroll
-                for (int pl = 0; pl < B; ++pl) pw[pl] = 0u;
-#pragma unroll
-                for (int e = 31; e >= 0; --e) {
-                    const float yv = y[e];
-                    const uint32_t w = __float_as_uint(0.f - yv);      // sign bit: y > 0
-                    const float ay = fabsf(yv);
-                    float cm = cs[0];
-                    uint32_t dbits[H > 1 ? H - 1 : 1];
-#pragma unroll
-                    for (int k = 0; k < H - 1; ++k) {
-                        const float dk = th[k] - ay;                     // sign bit: |y| above boundary k
-                        dbits[k] = __float_as_uint(dk);
-                        cm = dk < 0.f ? cs[k + 1] : cm;
+                        for (int pl = 0; pl < B; ++pl)
+                            reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + c) * 4 + u] =
+                                ((pb[pl] << 16) | pa[pl]) & keep;
                     }
-                    // the centroid takes the sign of y (negative for y <= 0: the lower cell)
-                    const float csg = __uint_as_float(__float_as_uint(cm) ^ (~w & 0x80000000u));
-                    float r = fmaf(yv, kap, -csg);
-                    if (!FULL && 32 * c + e >= p.d) r = 0.f;
-                    rr[e] = r;
-                    if (e & 1) g2a = fmaf(r, r, g2a);
-                    else g2b = fmaf(r, r, g2b);
-                    // index bits: top bit = [y > 0]; lower bits = level bits XNOR [y > 0]
-                    pw[B - 1] = shl_in(pw[B - 1], w);
-                    if constexpr (B == 2) {
-                        pw[0] = shl_in(pw[0], ~(dbits[0] ^ w));
-                    } else if constexpr (B == 3) {
-                        pw[1] = shl_in(pw[1], ~(dbits[1] ^ w));
-                        pw[0] = shl_in(pw[0], ~(dbits[0] ^ dbits[1] ^ dbits[2] ^ w));
-                    }
-                }
-                // residual operand: an integer-valued hi part (|hi| <= 2048, exact in fp16) and
-                // the remainder in [-1/2, 1/2] as lo
-                uint32_t hw[16], lw[16];
-#pragma unroll
-                for (int q = 0; q < 16; ++q) {
-                    const float h0 = (rr[2 * q] + 12582912.f) - 12582912.f;
-                    const float h1 = (rr[2 * q + 1] + 12582912.f) - 12582912.f;
-                    hw[q] = pack_half2(h0, h1);
-                    lw[q] = pack_half2(rr[2 * q] - h0, rr[2 * q + 1] - h1);
-                }
-                tmem_st16(tR + 16u * c, hw);
-                tmem_st16(tR + 64u + 16u * c, lw);
-                // code planes of this vector (zero for padding tokens and coordinates beyond d)
-                if (blk_ok) {
-                    const uint32_t keep = rvalid ? low_bits(p.d - 32 * c) : 0u;
-#pragma unroll
-                    for (int pl = 0; pl < B; ++pl)
-                        reinterpret_cast<uint32_t*>(blk)[(pl * 32 + 4 * gq + c) * 4 + u] = pw[pl] & keep;
+                    if (q == 0) twait(ya);
                 }
             }
             asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[bRFull + wg]);
-            // signs of Z = R M^T
-            if (lane == 0) w_ok = wait_bar(&bars[bZFull + wg], j & 1, s_abort);
-            if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+            if (lane == 0) mbar_arrive(&bars[bRFull + par]);
+            // gamma^2: the upper column half hands its partial sum to the lower one
+            float g2 = g2a + g2b;
+            if (half == 1) {
+                if (j > 0 && !warp_wait(g2empty, (j - 1) & 1)) break;
+                *g2x = g2;
+                mbar_arrive(g2full);
+            }
+            // signs of Z = R M^T over this warp's columns
+            if (!warp_wait(&bars[bZFull + par], j & 1)) break;
             fence_after();
+            {
+                uint32_t za[16], zb[16];
+                const uint32_t z0 = tY + 64u * half;
+                tld16(z0, za);
+                twait(za);
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                float z[32];
-                tmem_ld32(tY + 32u * c, z);
-                uint32_t sw = 0u;
+                for (int q = 0; q < 2; ++q) {
+                    const int c = 2 * half + q;
+                    tld16(z0 + 32u * q + 16u, zb);
+                    uint32_t sa = 0u, sbw = 0u;
 #pragma unroll
-                for (int e = 31; e >= 0; --e) sw = shl_in(sw, __float_as_uint(z[e]));
-                // bit = [z >= 0]: the sign bit inverted (an exact zero has sign bit 0)
-                if (blk_ok)
-                    reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + c) * 4 + u] =
-                        rvalid ? ~sw & low_bits(p.m - 32 * c) : 0u;
+                    for (int e = 15; e >= 0; --e) sa = shl_in(sa, za[e]);
+                    twait(zb);
+                    if (q == 0) tld16(z0 + 32u, za);
+#pragma unroll
+                    for (int e = 15; e >= 0; --e) sbw = shl_in(sbw, zb[e]);
+                    // bit = [z >= 0]: the sign bit inverted (an exact zero has sign bit 0)
+                    if (blk_ok)
+                        reinterpret_cast<uint32_t*>(blk)[(B * 32 + 4 * gq + c) * 4 + u] =
+                            rvalid ? ~((sbw << 16) | sa) & low_bits(p.m - 32 * c) : 0u;
+                    if (q == 0) twait(za);
+                }
             }
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[bTEmpty + wg]);
-            if (blk_ok) {
-                const float gam = sqrtf(g2a + g2b) / (ne * kap);
-                const uint32_t nh = rvalid ? tq_half_bits(n) : 0u;
-                const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
-                if (rvalid && (!finite || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
-                reinterpret_cast<uint32_t*>(blk + p.t.sec_a)[gq * 4 + u] = nh | (gh << 16);
+            if (lane == 0) mbar_arrive(&bars[bTEmpty + par]);
+            if (half == 0) {
+                if (!warp_wait(g2full, j & 1)) break;
+                g2 += *g2x;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(g2empty);
+                if (blk_ok) {
+                    const float gam = sqrtf(g2) / (ne * kap);
+                    const uint32_t nh = rvalid ? tq_half_bits(n) : 0u;
+                    const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
+                    if (rvalid && (!finite || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
+                    reinterpret_cast<uint32_t*>(blk + p.t.sec_a)[gq * 4 + u] = nh | (gh << 16);
+                }
             }
         }
     }
