@@ -314,6 +314,15 @@ def run_gpu(args, world, rank, local):
                   "tensor_frac_with_split_passes": round(passes * quant_tf / tpeak, 4),
                   "peak_kind": peak_kind + (" (HBM copy)" if q_bound == "hbm" else " (bf16 burst)")}
     also = {} if args.no_extras else extra_workloads(torch, tq, ti, gen, peaks)
+    if not args.no_extras:
+        # the same append with a randomized Walsh-Hadamard rotation H D / sqrt(d): the rotation
+        # is an exact +-1 operand, one tensor-core pass instead of three
+        hcodec = tq.Codec(D, D, MSE_BITS, True, torch.from_numpy(ti.hadamard_rotation(D, 1004).astype(np.float32)), s)
+        hms = time_calls(torch, lambda i: tq.tq_quantize(hcodec, append, n_streams, N_APPEND, N_APPEND * D,
+                                                          append_packed, wsq, stream), 20, 3)
+        also["c4_append_quantize_hadamard_rotation"] = {
+            "ms": hms, "vectors_per_s": vec_per_step / (hms * 1e-3), "dense_rotation_ms": t_quant,
+            "GB_per_s": quant_bytes / (hms * 1e-3) / 1e9}
     line = {
         "metric": METRIC, "value": keys_per_step * world / (ms_step * 1e-3), "unit": "keys/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -59,11 +59,27 @@ __global__ void k_prepare(PrepParams p) {
 // (Pi_1 = bf16(Pi), Pi_2 = bf16(Pi - Pi_1), Pi_3 = bf16(Pi - Pi_1 - Pi_2): each difference
 // is exact in fp32 and the three pieces sum to the fp32 matrix), and the fp16 hi/lo pair of
 // 256 M, all in the swizzled shared-memory layout. Runs after k_prepare_split (reads M).
+// Header: whether every entry of the d x d Pi is +-1/sqrt(d) (within fp32 rounding), i.e. Pi
+// is a scaled Hadamard rotation such as H D / sqrt(d); the flag word starts with the bit set.
+__global__ void k_check_pm1(PrepParams p) {
+    const double r = sqrt((double)p.d);
+    bool ok = true;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < (int64_t)p.d * p.d;
+         e += (int64_t)gridDim.x * blockDim.x)
+        ok = ok && fabs(fabs((double)p.pi[e]) * r - 1.0) < 1e-6;
+    if (!__syncthreads_and(ok) && threadIdx.x == 0) atomicAnd(&p.hdr[0], 0u);
+}
+
 __global__ void k_prepare_images(PrepParams p) {
+    const bool pm1 = (p.hdr[0] & TQ_PREP_PM1) != 0;
+    const float up = pm1 ? sqrtf((float)p.d) : 1.f;
+    if (blockIdx.x == 0 && threadIdx.x == 0) reinterpret_cast<float*>(p.hdr)[1] = pm1 ? up : 1.f;
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < 128 * 128; e += gridDim.x * blockDim.x) {
         const int i = e >> 7, j = e & 127;
         const uint32_t off = tq_sw128_offset(i, j);
-        const float v = (i < p.d && j < p.d) ? p.pi[(int64_t)i * p.d + j] : 0.f;
+        const float v0 = (i < p.d && j < p.d) ? p.pi[(int64_t)i * p.d + j] : 0.f;
+        // a +-1/sqrt(d) rotation: the first piece is exactly +-1 and the others vanish
+        const float v = pm1 ? (v0 > 0.f ? 1.f : v0 < 0.f ? -1.f : 0.f) : v0;
         const __nv_bfloat16 b1 = __float2bfloat16_rn(v);
         const float r1 = v - __bfloat162float(b1);
         const __nv_bfloat16 b2 = __float2bfloat16_rn(r1);
@@ -76,6 +92,22 @@ __global__ void k_prepare_images(PrepParams p) {
     }
 }
 
+// Chunked images of 256 Pi and 256 M for the 256-wide quantize (D = Mp = 256): chunk
+// 4 nh + kb holds rows 128 nh .. +127 and columns 64 kb .. +63 as fp16 hi then lo, each in
+// the swizzled [128 rows][128 B] layout. Runs after k_prepare_split (reads its hi/lo pairs).
+__global__ void k_prepare_wide_images(PrepParams p) {
+    for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < 2 * 256 * 256; e += gridDim.x * blockDim.x) {
+        const int mat = e >> 16, r = (e >> 8) & 255, c = e & 255;
+        const size_t src = (size_t)r * 256 + c;
+        const uint16_t hi = mat == 0 ? p.pih[src] : p.mh[src];
+        const uint16_t lo = mat == 0 ? p.pil[src] : p.ml[src];
+        uint8_t* chunk = p.wimg + ((size_t)mat * 8 + (r >> 7) * 4 + (c >> 6)) * kTqWideChunk;
+        const uint32_t off = tq_sw128_offset(r & 127, c & 63);
+        *reinterpret_cast<uint16_t*>(chunk + off) = hi;
+        *reinterpret_cast<uint16_t*>(chunk + 16384 + off) = lo;
+    }
+}
+
 cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
     k_prepare<<<296, 256, 0, st>>>(p);
     cudaError_t e = cudaGetLastError();
@@ -83,7 +115,15 @@ cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
     k_prepare_split<<<296, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.img) {
+        // flag word: TQ_PREP_PM1 set (bytes 0x01) until an entry disproves it
+        if ((e = cudaMemsetAsync(p.hdr, 1, 4, st)) != cudaSuccess) return e;
+        k_check_pm1<<<64, 256, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         k_prepare_images<<<64, 256, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (p.wimg) {
+        k_prepare_wide_images<<<256, 256, 0, st>>>(p);
         e = cudaGetLastError();
     }
     return e;

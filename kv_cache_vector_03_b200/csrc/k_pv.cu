@@ -23,12 +23,12 @@ namespace {
 constexpr int kPvWarps = 8;
 constexpr int kPvNS = 3;              // ring stages per warp
 constexpr uint32_t kWaitLimit = 1u << 22;
-constexpr int kWCol = 20;             // words per staged weight column (16 used; 20 spreads the banks)
+constexpr int kPRow = 40;             // floats per staged P row (32 used; 40 spreads the banks)
 
 template <int B, int KT, int NT>
 constexpr size_t pv_smem_bytes() {
     return (size_t)(1 << (2 * B)) * 128 + (size_t)kPvWarps * kPvNS * (512 * (KT * B / 8) + 64) +
-           (size_t)kPvWarps * kPvNS * 4 * NT * 32 * 4;
+           (size_t)kPvWarps * kPvNS * 4 * NT * kPRow * 4;
 }
 
 template <int B, int KT, int NT>  // KT = D/16 coordinate tiles, NT = n-tiles of 4 heads
@@ -43,8 +43,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
     extern __shared__ __align__(128) uint8_t smem[];
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem);                              // [E][32]
     uint8_t* ring = smem + (size_t)E * 128;                                          // [warp][NS][BBYTES]
-    float* pring = reinterpret_cast<float*>(ring + (size_t)kPvWarps * NS * BBYTES);  // [warp][NS][HP][32]
-    __shared__ uint32_t wst[kPvWarps][2 * HP][kWCol];   // column 2h (hi) / 2h + 1 (lo): token pairs
+    float* pring = reinterpret_cast<float*>(ring + (size_t)kPvWarps * NS * BBYTES);  // [warp][NS][HP][kPRow]
     __shared__ float s_acc[HP][KT * 16];
     __shared__ float s_m[kPvWarps][HP], s_l[HP];
     __shared__ uint64_t bars[kPvWarps][NS];
@@ -72,7 +71,7 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
     __syncthreads();
 
     uint8_t* my_ring = ring + (size_t)w * NS * BBYTES;
-    float* my_p = pring + (size_t)w * NS * HP * 32;
+    float* my_p = pring + (size_t)w * NS * HP * kPRow;
     const int64_t first = b0 + w;
     const int nmine = first < b1 ? (int)((b1 - first + kPvWarps - 1) / kPvWarps) : 0;
     // block k of this warp (first + 4k) into stage k % NS; every lane commits one copy group.
@@ -84,10 +83,10 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
             const int s = k % NS;
             if (lane == 0) tq_bulk_load(my_ring + s * BBYTES, vk, BBYTES, &bars[w][s]);
             const bool in = (first + (int64_t)kPvWarps * k) * 32 + lane < p.n_tok;
-            float* dst = my_p + s * HP * 32 + lane;
+            float* dst = my_p + s * HP * kPRow + lane;
 #pragma unroll
             for (int h = 0; h < HP; ++h)
-                if (h < G) tq_cp_async4(dst + h * 32, in ? pk + (size_t)h * p.n_tok : p.P, in ? 4u : 0u);
+                if (h < G) tq_cp_async4(dst + h * kPRow, in ? pk + (size_t)h * p.n_tok : p.P, in ? 4u : 0u);
             pk += 32 * kPvWarps;
             vk += (size_t)kPvWarps * BBYTES;
         }
@@ -102,12 +101,17 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int r = 0; r < 4; ++r) acc[k][n][r] = 0.f;
-    // m_run (the same in every lane) and ml2 = m_run log2(e); lsum holds the lane's tokens
-    float m_run[HP], ml2[HP], lsum[HP];
+    // Thread (g, t) feeds column g of each n-tile n of the B operand: head hb = 4n + g/2, the
+    // fp16 hi (g even) or lo (g odd) part of its weights exp(P - m) |v| for the tokens
+    // 2t, 2t+1, 2t+8, 2t+9, 16+2t, 17+2t, 24+2t, 25+2t of the block (the K rows of its B
+    // fragments). m_run / ml2 / lsum belong to head hb; the accumulator columns 2t, 2t+1 of
+    // n-tile n belong to head 4n + t, whose rescale factor comes from lane 8t.
+    float m_run[NT], ml2[NT], lsum[NT];
 #pragma unroll
-    for (int h = 0; h < HP; ++h) { m_run[h] = -INFINITY; ml2[h] = -INFINITY; lsum[h] = 0.f; }
+    for (int n = 0; n < NT; ++n) { m_run[n] = -INFINITY; ml2[n] = -INFINITY; lsum[n] = 0.f; }
     constexpr float kLog2e = 1.4426950408889634f;
     const uint32_t lane4 = (uint32_t)lane * 4u;
+    const bool lo_col = (g & 1) != 0;
 
     bool ok = true;
     int k = 0;
@@ -118,67 +122,76 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
         if (!ok) break;
         __syncwarp();                 // and those of the other lanes are visible
         const uint8_t* bp = my_ring + s * BBYTES;
-        const int64_t tok = (first + (int64_t)kPvWarps * k) * 32 + lane;
-        const bool in = tok < p.n_tok;
-        const float nrm = tq_half_val(reinterpret_cast<const uint16_t*>(bp + SEC_A)[lane]);
-        // online maximum and weights of this lane's token, one head at a time
-        float myf[NT];   // rescale factor of this thread's accumulator head 4n + t
+        const int64_t tok0 = (first + (int64_t)kPvWarps * k) * 32;
+        const int64_t rem = p.n_tok - tok0;
+        const int nval = rem < 32 ? (int)rem : 32;   // valid tokens of the block
+        // norms of the thread's 8 tokens (pairs 2t + 8j, +1)
+        float nrm[8];
 #pragma unroll
-        for (int n = 0; n < NT; ++n) myf[n] = 1.f;
+        for (int jj = 0; jj < 4; ++jj) {
+            const uint32_t nw = reinterpret_cast<const uint32_t*>(bp + SEC_A)[4 * jj + t];
+            nrm[2 * jj] = tq_half_val(nw & 0xffffu);
+            nrm[2 * jj + 1] = tq_half_val(nw >> 16);
+        }
+        uint32_t bw[NT][2][2];
+        float fac_b[NT];
         bool grew = false;
-        float wt[HP];
 #pragma unroll
-        for (int h = 0; h < HP; ++h) {
-            wt[h] = 0.f;
-            if (h < G) {
-                const float pv = in ? my_p[(s * HP + h) * 32 + lane] : -INFINITY;
-                if (__any_sync(0xffffffffu, pv > m_run[h])) {
-                    const float bm = tq_warp_max(pv);
-                    const float fac = tq_exp2((m_run[h] - bm) * kLog2e);   // 0 while the maximum was -inf
-                    if ((h & 3) == t) myf[h >> 2] = fac;
-                    lsum[h] *= fac;
-                    m_run[h] = bm;
-                    ml2[h] = bm * kLog2e;
-                    grew = true;
+        for (int n = 0; n < NT; ++n) {
+            const int hb = 4 * n + (g >> 1);
+            fac_b[n] = 1.f;
+            float pv[8];
+            const float* prow = my_p + (s * HP + (hb < G ? hb : 0)) * kPRow + 2 * t;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const float2 v2 = *reinterpret_cast<const float2*>(prow + 8 * jj);
+                const int tt = 8 * jj + 2 * t;
+                pv[2 * jj] = (hb < G && tt < nval) ? v2.x : -INFINITY;
+                pv[2 * jj + 1] = (hb < G && tt + 1 < nval) ? v2.y : -INFINITY;
+            }
+            float bm = fmaxf(fmaxf(fmaxf(pv[0], pv[1]), fmaxf(pv[2], pv[3])), fmaxf(fmaxf(pv[4], pv[5]), fmaxf(pv[6], pv[7])));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+            if (bm > m_run[n]) {
+                fac_b[n] = tq_exp2((m_run[n] - bm) * kLog2e);   // 0 while the maximum was -inf
+                lsum[n] *= fac_b[n];
+                m_run[n] = bm;
+                ml2[n] = bm * kLog2e;
+                grew = true;
+            }
+            float wv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float ex = m_run[n] > -INFINITY ? tq_exp2(fmaf(pv[e], kLog2e, -ml2[n])) : 0.f;
+                lsum[n] += ex;
+                wv[e] = ex * nrm[e];
+            }
+            // fp16 hi, or the lo remainder, of the weights as the B fragments of both K halves
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __half2 hi = __floats2half2_rn(wv[2 * q], wv[2 * q + 1]);
+                uint32_t v;
+                if (lo_col) {
+                    const float2 hf = __half22float2(hi);
+                    const __half2 lo = __floats2half2_rn(wv[2 * q] - hf.x, wv[2 * q + 1] - hf.y);
+                    v = *reinterpret_cast<const uint32_t*>(&lo);
+                } else {
+                    v = *reinterpret_cast<const uint32_t*>(&hi);
                 }
-                const float ex = m_run[h] > -INFINITY ? tq_exp2(fmaf(pv, kLog2e, -ml2[h])) : 0.f;
-                lsum[h] += ex;
-                wt[h] = ex * nrm;
+                bw[n][q >> 1][q & 1] = v;
             }
         }
-        // fp16 hi / lo of the weights, two heads per packed conversion
+        if (__any_sync(0xffffffffu, grew)) {
+            // accumulator columns 2t, 2t + 1 of n-tile n belong to head 4n + t (factor at lane 8t)
 #pragma unroll
-        for (int h = 0; h < HP; h += 2) {
-            if (h < G) {
-                const __half2 hi = __floats2half2_rn(wt[h], wt[h + 1]);
-                const float2 hf = __half22float2(hi);
-                const __half2 lo = __floats2half2_rn(wt[h] - hf.x, wt[h + 1] - hf.y);
-                reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = __low2half(hi);
-                reinterpret_cast<__half*>(&wst[w][2 * h + 1][0])[lane] = __low2half(lo);
-                if (h + 1 < G) {
-                    reinterpret_cast<__half*>(&wst[w][2 * h + 2][0])[lane] = __high2half(hi);
-                    reinterpret_cast<__half*>(&wst[w][2 * h + 3][0])[lane] = __high2half(lo);
-                }
-            }
-        }
-        if (grew) {
-            // accumulator columns 2t, 2t + 1 of n-tile n belong to head 4n + t
-#pragma unroll
-            for (int n = 0; n < NT; ++n)
+            for (int n = 0; n < NT; ++n) {
+                const float f = __shfl_sync(0xffffffffu, fac_b[n], 8 * t);
 #pragma unroll
                 for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) acc[kk][n][r] *= myf[n];
+                    for (int r = 0; r < 4; ++r) acc[kk][n][r] *= f;
+            }
         }
-        __syncwarp();
-        // B fragments: column g of n-tile n (head 4n + g/2, hi or lo), tokens 16c + 8hv + 2t, +1
-        uint32_t bw[NT][2][2];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int c = 0; c < 2; ++c)
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) bw[n][c][hv] = wst[w][8 * n + g][8 * c + 4 * hv + t];
         uint32_t W[NW + 1];
 #pragma unroll
         for (int c = 0; c < CH; ++c) {
@@ -222,24 +235,25 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
         }
         __syncwarp();
     }
-    // the CTA's maximum per head; each warp's sums are rescaled to it
-    if (lane == 0)
+    // the CTA's maximum per head; each warp's sums are rescaled to it. Head h's running
+    // maximum is held by the lanes whose B column belongs to it (lane 8 (h mod 4) of n-tile h / 4).
+    if (t == 0 && (g & 1) == 0)
 #pragma unroll
-        for (int h = 0; h < HP; ++h) s_m[w][h] = m_run[h];
+        for (int n = 0; n < NT; ++n) s_m[w][4 * n + (g >> 1)] = m_run[n];
     __syncthreads();
-    float scl[HP], mys[NT];
+    float scl_b[NT];
 #pragma unroll
-    for (int h = 0; h < HP; ++h) {
-        float M = s_m[0][h];
+    for (int n = 0; n < NT; ++n) {
+        const int hb = 4 * n + (g >> 1);
+        float M = s_m[0][hb];
 #pragma unroll
-        for (int v = 1; v < kPvWarps; ++v) M = fmaxf(M, s_m[v][h]);
-        scl[h] = m_run[h] > -INFINITY ? __expf(m_run[h] - M) : 0.f;
-        if ((h & 3) == t) mys[h >> 2] = scl[h];
+        for (int v = 1; v < kPvWarps; ++v) M = fmaxf(M, s_m[v][hb]);
+        scl_b[n] = m_run[n] > -INFINITY ? __expf(m_run[n] - M) : 0.f;
     }
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int head = n * 4 + t;
-        const float f = mys[n];
+        const float f = __shfl_sync(0xffffffffu, scl_b[n], 8 * t);
         if (head < G) {
 #pragma unroll
             for (int kk = 0; kk < KT; ++kk) {
@@ -248,12 +262,14 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
             }
         }
     }
+    // denominators: the hi lanes of a head (t = 0..3) hold its 32 tokens between them
 #pragma unroll
-    for (int h = 0; h < HP; ++h) {
-        if (h < G) {
-            const float ls = tq_warp_sum(lsum[h]) * scl[h];
-            if (lane == 0) atomicAdd(&s_l[h], ls);
-        }
+    for (int n = 0; n < NT; ++n) {
+        float ls = (g & 1) == 0 ? lsum[n] * scl_b[n] : 0.f;
+        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+        const int hb = 4 * n + (g >> 1);
+        if (t == 0 && (g & 1) == 0 && hb < G) atomicAdd(&s_l[hb], ls);
     }
     __syncthreads();
     const int D = KT * 16;

@@ -230,8 +230,10 @@ cudaError_t launch_kd(const QuantParams& p, cudaStream_t st, int kd, int km) {
 }
 
 cudaError_t tq_launch_quantize(const QuantParams& p, cudaStream_t st) {
-    // d <= 128 with m <= 128 (or no sketch): tensor cores (k_quantize_tc.cu); otherwise fp32
+    // d <= 128 with m <= 128 (or no sketch): tensor cores (k_quantize_tc.cu, k_quantize_ws.cu);
+    // keys with d, m in 129..256: tensor cores (k_quantize_wide.cu); otherwise fp32
     if (p.t.D == 128 && (p.t.Mp == 128 || !p.t.qjl)) return tq_launch_quantize_tc(p, st);
+    if (p.t.qjl && p.t.D == 256 && p.t.Mp == 256 && p.wimg && p.t.B <= 3) return tq_launch_quantize_wide(p, st);
     const int kd = p.t.D / 32, km = p.t.Mp / 32;
     return launch_kd(p, st, kd, km);
 }

@@ -6,12 +6,13 @@
 // One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with 18 warps:
 //   warp 16 (one thread)  TMA: the tile's raw bf16 rows, as four 32-row boxes per 64-column
 //                         K-block, straight into the 128-byte-swizzled K-major operand layout
-//                         (two stages);
-//   warp 17 (one thread)  tensor cores: Y = X (Pi_1 + Pi_2 + Pi_3)^T, three bf16 passes
-//                         whose sum is the fp32 rotation applied to the exact bf16 input, into
-//                         TMEM; Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo + lo.hi) with
-//                         the residual operand R read from TMEM. Whichever of the next Y and
-//                         the next Z is ready is issued first;
+//                         (two stages); and the rotation Y = X (Pi_1 + Pi_2 + Pi_3)^T on the
+//                         tensor cores, three bf16 passes whose sum is the fp32 rotation applied
+//                         to the exact bf16 input, into TMEM, with X first copied from shared
+//                         memory into TMEM (tcgen05.cp) so that the passes read only Pi there;
+//   warp 17 (one thread)  the sketch Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo + lo.hi)
+//                         with the residual operand R read from TMEM, as soon as the epilogue
+//                         has written it (the two issuers wait on their own events);
 //   warps 0-15            epilogue: warps 0-7 take even tiles, 8-15 odd ones; in each group
 //                         warp w reads TMEM lanes 32 (w mod 4) .. +31 (one vector per thread)
 //                         and columns 64 ((w / 4) mod 2) .. +63:
@@ -33,10 +34,9 @@
 namespace {
 
 constexpr int kWsThreads = 576;
-constexpr int kEpiWarps = 16, kTmaWarp = 16, kMmaWarp = 17;
+constexpr int kTmaWarp = 16, kMmaWarp = 17;   // warps 0-15: epilogue
 constexpr uint32_t kMat = 32768;          // one 128 x 128 16-bit operand
 constexpr uint32_t kWaitLimit = 1u << 22;
-constexpr uint32_t kIdleLimit = 1u << 24; // polls of the MMA issuer with nothing to issue
 
 // shared memory map (from a 1024-aligned base)
 constexpr uint32_t oPi = 0;               // Pi_1, Pi_2, Pi_3 (bf16)
@@ -48,7 +48,7 @@ constexpr uint32_t oBar = oG2 + 2 * 128 * 4;   // barriers, then the TMEM base a
 // barrier indices: per X stage, per tile parity, per (tile parity, lane quarter)
 enum {
     bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bTEmpty = 10, bOps = 12, bDrain = 13,
-    bG2Full = 14, bG2Empty = 22, kNumBars = 30
+    bG2Full = 14, bG2Empty = 22, bDrainY = 30, kNumBars = 31
 };
 constexpr size_t kWsSmemUsed = (size_t)oBar + 8 * kNumBars + 8;
 constexpr size_t kWsSmem = 232448;        // the per-CTA maximum: the used bytes plus the alignment pad
@@ -66,18 +66,17 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
 // K-step k (16 elements) of a 128 x 128 operand: K-block k / 4, 32 bytes per step inside it
 __device__ __forceinline__ uint32_t kstep(int k) { return (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u; }
 
-__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %4, p;\n}\n" ::"r"(d),
-        "l"(a), "l"(b), "r"(acc), "r"(idesc));
-}
 // A from TMEM (row = lane, two 16-bit elements per column), B from shared memory
 __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n}\n" ::"r"(d),
         "r"(a_tmem), "l"(b), "r"(acc), "r"(idesc));
+}
+// 128 rows x 32 bytes (one K-step of 16 16-bit elements per row) from a shared-memory
+// operand to 8 TMEM columns, row r to lane r (the layout of an A operand in TMEM)
+__device__ __forceinline__ void tmem_cp(uint32_t taddr, uint64_t sd) {
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sd) : "memory");
 }
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -87,28 +86,6 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};\n" ::"r"(
-            taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
-        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
-        : "memory");
-}
 
 // 16 columns of this thread's TMEM lane, without waiting (tmem_wait_ld before use)
 __device__ __forceinline__ void tld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -133,15 +110,6 @@ __device__ __forceinline__ void tst8(uint32_t taddr, const uint32_t (&v)[8]) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(v[0]),
                  "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
                  : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(tq_smem_addr(bar)), "r"(parity)
-        : "memory");
-    return done != 0;
 }
 
 __device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
@@ -196,6 +164,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 struct WsParams {
     uint8_t* packed;
     const uint8_t* img;        // prepared operand images (Pi_1..3, M_hi, M_lo)
+    const uint32_t* hdr;       // prep header: +-1 rotation flag, image scale
     uint32_t* status;
     int64_t n_streams, n_tok, nb;
     int d, m;
@@ -300,11 +269,10 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             // resident operands: five 32 KB images
             mbar_expect_tx(&bars[bOps], 5 * kMat);
             for (int i = 0; i < 5; ++i) bulk_copy(sb + oPi + i * kMat, p.img + (size_t)i * kMat, kMat, &bars[bOps]);
-            int issued = 0;
-            for (int i = 0; i < n_local; ++i) {
-                const int xs = i & 1;
-                if (i >= 2 && !wait_bar(&bars[bXEmpty + xs], ((i >> 1) - 1) & 1, s_abort)) break;
-                const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+            // tile t of this CTA into X stage t & 1
+            auto load_tile = [&](int t) {
+                const int xs = t & 1;
+                const int64_t tile = blockIdx.x + (int64_t)t * gridDim.x;
                 const int64_t left = total_blocks - tile * 4;
                 const int nvb = left < 4 ? (int)left : 4;
                 mbar_expect_tx(&bars[bXFull + xs], (uint32_t)nvb * 8192u);
@@ -315,68 +283,60 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                     for (int h = 0; h < 2; ++h)
                         tma_load3(sb + oX + xs * kMat + h * 16384 + jb * 4096, &xmap, 64 * h, tok0, s, &bars[bXFull + xs]);
                 }
-                issued = i + 1;
+            };
+            int issued = 0;
+            for (; issued < 2 && issued < n_local; ++issued) load_tile(issued);
+            const int y_passes = (p.hdr[0] & TQ_PREP_PM1) ? 1 : 3;
+            bool ok = wait_bar(&bars[bOps], 0, s_abort);
+            for (int i = 0; ok && i < n_local; ++i) {
+                const int b = i & 1;
+                if (!wait_bar(&bars[bXFull + b], (i >> 1) & 1, s_abort)) break;
+                if (i >= 2 && !wait_bar(&bars[bTEmpty + b], ((i >> 1) - 1) & 1, s_abort)) break;
+                fence_after();
+                // X into TMEM (the residual columns of this buffer, free until the epilogue writes
+                // R after Y): the tensor cores then read only Pi from shared memory. A +-1/sqrt(d)
+                // rotation needs the first (exact +-1) piece only.
+                const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat, xt = tmem + 256u + 128u * b;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) tmem_cp(xt + 8u * k, sdesc(xa + kstep(k)));
+                mma_commit(&bars[bXEmpty + b]);
+                for (int ps = 0; ps < y_passes; ++ps)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ts(d, xt + 8u * k, sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16, (ps | k) != 0);
+                mma_commit(&bars[bYFull + b]);
+                // the stage of tile i - 1 is refilled with tile i + 1 once Y(i - 1) has read it
+                if (i >= 1 && issued < n_local) {
+                    if (!wait_bar(&bars[bXEmpty + (b ^ 1)], ((i - 1) >> 1) & 1, s_abort)) break;
+                    load_tile(issued++);
+                }
             }
-            // nothing may be in flight when the CTA exits: wait (bounded) for the last load of
-            // each stage (a completed phase returns at once)
+            // nothing may be in flight when the CTA exits: every Y has completed (a commit tracks
+            // all earlier MMAs of this thread), and the last load of each stage has landed (a
+            // completed phase returns at once)
+            mma_commit(&bars[bDrainY]);
+            tq_mbar_wait(&bars[bDrainY], 0, kWaitLimit);
             for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i)
                 tq_mbar_wait(&bars[bXFull + (i & 1)], (i >> 1) & 1, kWaitLimit);
             tq_mbar_wait(&bars[bOps], 0, kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
-        if (lane == 0 && wait_bar(&bars[bOps], 0, s_abort)) {
-            int ny = 0, nz = 0;
-            uint32_t idle = 0;
-            while (nz < n_local) {
-                bool progress = false;
-                if (ny < n_local) {
-                    const int b = ny & 1;
-                    if (mbar_test(&bars[bXFull + b], (ny >> 1) & 1) &&
-                        (ny < 2 || mbar_test(&bars[bTEmpty + b], ((ny >> 1) - 1) & 1))) {
-                        fence_after();
-                        const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat;
-#pragma unroll
-                        for (int ps = 0; ps < 3; ++ps)
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                mma_ss(d, sdesc(xa + kstep(k)), sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16,
-                                       (ps | k) != 0);
-                        mma_commit(&bars[bYFull + b]);
-                        mma_commit(&bars[bXEmpty + b]);
-                        ++ny;
-                        progress = true;
-                    }
-                }
-                if (nz < ny) {
-                    const int b = nz & 1;
-                    if (mbar_test(&bars[bRFull + b], (nz >> 1) & 1)) {
-                        fence_after();
-                        const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
-#pragma unroll
-                        for (int ps = 0; ps < 3; ++ps) {
-                            const uint32_t ra = r + (ps == 2 ? 64u : 0u);
-                            const uint32_t mb = sb + oM + (ps == 1 ? kMat : 0u);
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
-                        }
-                        mma_commit(&bars[bZFull + b]);
-                        ++nz;
-                        progress = true;
-                    }
-                }
-                if (progress) {
-                    idle = 0;
-                } else {
-                    if (++idle >= kIdleLimit) { *s_abort = 1u; break; }
-                    if ((idle & 31u) == 0u && *s_abort) break;
-                    __nanosleep(20);
-                }
-            }
-        }
         if (lane == 0) {
-            // every MMA this thread issued completes before TMEM is released (a commit tracks
-            // all earlier MMAs of the thread)
+            for (int i = 0; i < n_local; ++i) {
+                const int b = i & 1;
+                if (!wait_bar(&bars[bRFull + b], (i >> 1) & 1, s_abort)) break;
+                fence_after();
+                const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
+#pragma unroll
+                for (int ps = 0; ps < 3; ++ps) {
+                    const uint32_t ra = r + (ps == 2 ? 64u : 0u);
+                    const uint32_t mb = sb + oM + (ps == 1 ? kMat : 0u);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
+                }
+                mma_commit(&bars[bZFull + b]);
+            }
+            // every Z has completed before TMEM is released
             mma_commit(&bars[bDrain]);
             tq_mbar_wait(&bars[bDrain], 0, kWaitLimit);
         }
@@ -390,6 +350,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
         float* g2x = s_g2 + par * 128 + row;
         uint64_t* g2full = &bars[bG2Full + 4 * par + wq];
         uint64_t* g2empty = &bars[bG2Empty + 4 * par + wq];
+        // Y rows are the rotation scaled by the Pi_1 image factor (sqrt(d) for a +-1 rotation)
+        const float n_unscale = 1.f / reinterpret_cast<const float*>(p.hdr)[1];
         float tb[H > 1 ? H - 1 : 1], cmg[H];
 #pragma unroll
         for (int k = 0; k < H - 1; ++k) tb[k] = p.cb.bounds[H + k];
@@ -540,7 +502,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                 if (lane == 0) mbar_arrive(g2empty);
                 if (blk_ok) {
                     const float gam = sqrtf(g2) / (ne * kap);
-                    const uint32_t nh = rvalid ? tq_half_bits(n) : 0u;
+                    const uint32_t nh = rvalid ? tq_half_bits(n * n_unscale) : 0u;
                     const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
                     if (rvalid && (!finite || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
                     reinterpret_cast<uint32_t*>(blk + p.t.sec_a)[gq * 4 + u] = nh | (gh << 16);
@@ -622,6 +584,7 @@ cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st) {
     WsParams wp;
     wp.packed = p.packed;
     wp.img = p.img;
+    wp.hdr = p.hdr;
     wp.status = p.status;
     wp.n_streams = p.n_streams;
     wp.n_tok = p.n_tok;

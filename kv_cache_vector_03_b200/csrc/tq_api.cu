@@ -229,7 +229,9 @@ int tq_prepare(const tq_codec* c, void* stream) {
     p.pil = reinterpret_cast<uint16_t*>(base + L.pil);
     p.mh = reinterpret_cast<uint16_t*>(base + L.mh);
     p.ml = reinterpret_cast<uint16_t*>(base + L.ml);
-    p.img = L.total > L.img ? base + L.img : nullptr;
+    p.img = L.wimg > L.img ? base + L.img : nullptr;
+    p.wimg = L.total > L.wimg ? base + L.wimg : nullptr;
+    p.hdr = reinterpret_cast<uint32_t*>(base + L.hdr);
     p.d = t.d; p.m = t.m; p.D = t.D; p.Mp = t.Mp; p.qjl = t.qjl;
     return cuda_status(tq_launch_prepare(p, static_cast<cudaStream_t>(stream)));
 }
@@ -298,7 +300,9 @@ int tq_quantize(const tq_codec* c, const void* x, tq_dtype dtype, int64_t n_stre
     p.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
     p.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
     p.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
-    p.img = L.total > L.img ? static_cast<const uint8_t*>(c->prep) + L.img : nullptr;
+    p.img = L.wimg > L.img ? static_cast<const uint8_t*>(c->prep) + L.img : nullptr;
+    p.wimg = L.total > L.wimg ? static_cast<const uint8_t*>(c->prep) + L.wimg : nullptr;
+    p.hdr = reinterpret_cast<const uint32_t*>(static_cast<const uint8_t*>(c->prep) + L.hdr);
     p.status = static_cast<uint32_t*>(ws);
     p.vec_ok = aligned(x, dtype == TQ_F32 ? 16 : 8) && x_stream_stride % 4 == 0 && c->d % 4 == 0;
     p.t = t;

@@ -269,6 +269,8 @@ struct PrepParams {
     float* mT;
     uint16_t *pih, *pil, *mh, *ml;
     uint8_t* img;          // operand images of the warp-specialized quantize, or null
+    uint8_t* wimg;         // chunked operand images of the 256-wide quantize, or null
+    uint32_t* hdr;         // prep header (flags)
     int d, m, D, Mp, qjl;
 };
 
@@ -289,6 +291,8 @@ struct QuantParams {
     const float* mT;
     const uint16_t *pih, *pil, *mh, *ml;
     const uint8_t* img;    // operand images of the warp-specialized kernel, or null
+    const uint8_t* wimg;   // chunked operand images of the 256-wide kernel, or null
+    const uint32_t* hdr;   // prep header (flags)
     uint32_t* status;
     int vec_ok;            // rows can be read 4 elements at a time (alignment of x, stride, d)
     TqDims t;
@@ -404,6 +408,7 @@ cudaError_t tq_launch_dequant(const DequantParams& p, cudaStream_t st);
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_tc(const QuantParams& p, cudaStream_t st);
 bool tq_quantize_ws_eligible(const QuantParams& p);
+cudaError_t tq_launch_quantize_wide(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);

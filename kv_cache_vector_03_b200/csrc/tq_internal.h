@@ -62,20 +62,29 @@ static inline TqDims tq_dims(int d, int m, int B, int qjl) {
 }
 
 // Prepared (derived) operands, laid out in the caller's prep buffer:
-//   header (256 B) | PiT fp32 [D][D] | ST fp32 [D][Mp] | MT fp32 [D][Mp]
+//   header (256 B: word 0 = TQ_PREP_PM1 when every entry of the d x d Pi is +-1/sqrt(d), a
+//   scaled Hadamard rotation; float word 1 = the factor by which the Pi_1 image exceeds Pi)
+//   | PiT fp32 [D][D] | ST fp32 [D][Mp] | MT fp32 [D][Mp]
 //   | Pi_hi, Pi_lo fp16 [D][D] | M_hi, M_lo fp16 [Mp][D]     (tensor-core quantize)
 //   | images (keys with D = Mp = 128 only): Pi_1, Pi_2, Pi_3 bf16, M_hi, M_lo fp16
+//   | wide images (keys with D = Mp = 256 only): 256 Pi then 256 M, each as 8 chunks of
+//     32 KB, chunk 4 nh + kb = rows 128 nh .. +127, columns 64 kb .. +63: fp16 hi (16 KB)
+//     then lo (16 KB), each [128 rows][128 B] with the same 128-byte swizzle
 // PiT[j][i] = Pi[i][j], ST[j][k] = S[k][j], MT[i][k] = M[k][i] with M = S Pi^T, all zero
 // outside the d x d / m x d corners. The fp16 pairs hold 256 Pi and 256 M split as
 // hi = half(v), lo = half(v - hi), row-major (row = output coordinate).
+// For a +-1/sqrt(d) rotation the Pi_1 image holds sqrt(d) Pi (exactly +-1) and Pi_2 = Pi_3 = 0,
+// so one bf16 pass rotates exactly (up to the fp32 rounding of the stored Pi).
 // The images are 128 x 128 16-bit operands (row = output coordinate, column = K) stored
 // byte for byte as the tensor cores read them from shared memory: two K-blocks of 64
 // columns, each [128 rows][128 B] in 8-row atoms of 1024 B, 16-byte chunk index XOR
 // (row mod 8) (the 128-byte swizzle). Pi = Pi_1 + Pi_2 + Pi_3 exactly (bf16 pieces of the
 // fp32 matrix: 8 + 8 + 8 significant bits); M_hi, M_lo as above.
+#define TQ_PREP_PM1 1u
 constexpr size_t kTqImageBytes = 128 * 128 * 2;
+constexpr size_t kTqWideChunk = 32768;
 struct TqPrepLayout {
-    size_t hdr, piT, sT, mT, pih, pil, mh, ml, img, total;
+    size_t hdr, piT, sT, mT, pih, pil, mh, ml, img, wimg, total;
 };
 
 static inline TqPrepLayout tq_prep_layout(const TqDims& t) {
@@ -90,6 +99,7 @@ static inline TqPrepLayout tq_prep_layout(const TqDims& t) {
     L.mh = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
     L.ml = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
     L.img = off; off += (t.qjl && t.D == 128 && t.Mp == 128) ? 5 * kTqImageBytes : 0;
+    L.wimg = off; off += (t.qjl && t.D == 256 && t.Mp == 256) ? 16 * kTqWideChunk : 0;
     L.total = off;
     return L;
 }

@@ -94,6 +94,26 @@ def test_quantize_d200_vector_search(B):
     compare_codes(idx[0], sbit[0], nhat[0], ghat[0], ref, t, x=x.astype(np.float64), pi=pi, s=s, c=c, t=t, B=B)
 
 
+@pytest.mark.parametrize("d,m,B", [(256, 256, 2), (136, 200, 3), (200, 136, 1)])
+def test_quantize_wide_bf16_ragged(d, m, B):
+    """Keys with 129..256 coordinates and sketch rows (the 256-wide tensor-core path) from
+    bf16 rows: several streams with a ragged last block, padded coordinates and sketch rows."""
+    pi, s = ti.haar_rotation(d, 121 + d), ti.gaussian_sketch(m, d, 122 + m)
+    n_streams, n_tok = 3, 777
+    rng = np.random.default_rng(123 + d)
+    x = ti.f32_to_bf16_bits((rng.standard_normal((n_streams * n_tok, d)) * rng.uniform(0.5, 50, (n_streams * n_tok, 1)))
+                            .astype(np.float32))
+    codec = make_codec(d, m, B, True, pi, s)
+    packed, st = gpu_quantize(codec, to_dev_bf16(x), n_streams, n_tok)
+    assert st == tq().TQ_OK
+    idx, sbit, nhat, ghat = unpack(codec, packed, n_streams, n_tok)
+    c, t = _cb(d, B)
+    xf = ti.bf16_to_f64(x).reshape(n_streams, n_tok, d)
+    for st_i in range(n_streams):
+        ref = oracle.quantize(xf[st_i], pi, s, c, t, B, qjl=True)
+        compare_codes(idx[st_i], sbit[st_i], nhat[st_i], ghat[st_i], ref, t, x=xf[st_i], pi=pi, s=s, c=c, t=t, B=B)
+
+
 def test_quantize_range_status_and_zero_vector():
     d = m = 128
     pi, s = ti.haar_rotation(d, 81), ti.gaussian_sketch(m, d, 82)
