@@ -202,6 +202,24 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
                  const void* tail_k, const void* tail_v, int n_tail, float scale, float v_skip, float* out,
                  void* ws, size_t ws_bytes, void* stream);
 
+/* Decode attention of the asymmetric K/V configuration (blog.hotdry.top "TurboQuant
+ * vector-search compression", engineering configuration list: 8-bit keys with TurboQuant
+ * values) in one pass over the 8-bit key cache and the compressed values:
+ *   out_h = sum_t softmax_t(l_h) v_t,  l_h,t = scale <q_h, k~_t> (k~ = code * scale of its chunk)
+ * with the logits of tq_q8_logits (int16 fixed-point query) on the 8-bit tokens and exact on the
+ * bf16 tail, and the values of tq_pv; the logits never leave the SM.
+ *   vcodec   value codec, qjl = 0, d <= 128 (the keys have the same d), prepared.
+ *   packed_k8 device 8-bit key cache of n_seq * n_kv streams of n_tok tokens (tq_q8_quantize).
+ *   packed_v device value cache, the same streams and tokens.
+ *   q, g, tail_k, tail_v, n_tail, scale, v_skip, out: as tq_attention (g in 1, 2, 4).
+ *   ws       tq_attention_q8_workspace_bytes(vcodec, n_seq, n_kv, n_tok, g, n_tail) bytes,
+ *            256-byte aligned. n_tok + n_tail = 0 is TQ_ERR_ARG.                          */
+size_t tq_attention_q8_workspace_bytes(const tq_codec* vcodec, int64_t n_seq, int n_kv, int64_t n_tok, int g,
+                                       int n_tail);
+int tq_attention_q8(const tq_codec* vcodec, const void* packed_k8, const void* packed_v, int64_t n_seq, int n_kv,
+                    int64_t n_tok, const void* q, tq_dtype q_dtype, int g, const void* tail_k, const void* tail_v,
+                    int n_tail, float scale, float v_skip, float* out, void* ws, size_t ws_bytes, void* stream);
+
 /* Top-k inner-product search over a packed database (a2a-mcp.org, benchmark section:
  * GloVe d=200 recall; scores are the same estimator as tq_logits with scale 1).
  *   packed_db device, one stream of n_db key records (qjl = 1).

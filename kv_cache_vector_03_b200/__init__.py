@@ -30,7 +30,8 @@ EXPORTED = ["tq_make_codebook", "tq_block_bytes", "tq_record_bytes", "tq_packed_
             "tq_prepare", "tq_workspace_bytes", "tq_quantize", "tq_logits", "tq_pv", "tq_topk",
             "tq_dequantize", "tq_reset_status", "tq_get_status", "tq_status_string", "tq_abi_version",
             "tq_logits_noalloc", "tq_attention", "tq_attention_workspace_bytes", "tq_logits_est", "tq_topk_est",
-            "tq_q8_packed_bytes", "tq_q8_quantize", "tq_q8_logits"]
+            "tq_q8_packed_bytes", "tq_q8_quantize", "tq_q8_logits", "tq_attention_q8",
+            "tq_attention_q8_workspace_bytes"]
 
 
 class tq_codec(ctypes.Structure):
@@ -55,6 +56,8 @@ _sig = {
     "tq_pv": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _P, _P, _SZ, _P]),
     "tq_attention_workspace_bytes": (_SZ, [_CP, _CP, _I64, _I, _I64, _I, _I]),
     "tq_attention": (_I, [_CP, _CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _F, _P, _P, _SZ, _P]),
+    "tq_attention_q8_workspace_bytes": (_SZ, [_CP, _I64, _I, _I64, _I, _I]),
+    "tq_attention_q8": (_I, [_CP, _P, _P, _I64, _I, _I64, _P, _I, _I, _P, _P, _I, _F, _F, _P, _P, _SZ, _P]),
     "tq_topk": (_I, [_CP, _P, _I64, _P, _I64, _I, _P, _P, _P, _SZ, _P]),
     "tq_logits_est": (_I, [_CP, _P, _I64, _I, _I64, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _I, _P]),
     "tq_q8_packed_bytes": (_SZ, [_I, _I64, _I64]),
@@ -196,6 +199,18 @@ def tq_attention(kcodec: Codec, vcodec: Codec, packed_k, packed_v, n_seq, n_kv, 
     return _check("tq_attention", lib.tq_attention(kcodec.ref, vcodec.ref, _ptr(packed_k), _ptr(packed_v), n_seq, n_kv,
                                                    n_tok, _ptr(q), _dtype(q), g, _ptr(tail_k), _ptr(tail_v), n_tail,
                                                    scale, v_skip, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def tq_attention_q8_workspace_bytes(vcodec: Codec, n_seq, n_kv, n_tok, g, n_tail):
+    return lib.tq_attention_q8_workspace_bytes(vcodec.ref, n_seq, n_kv, n_tok, g, n_tail)
+
+
+def tq_attention_q8(vcodec: Codec, packed_k8, packed_v, n_seq, n_kv, n_tok, q, g, tail_k, tail_v, n_tail, scale, out,
+                    ws, v_skip=0.0, stream=None):
+    return _check("tq_attention_q8", lib.tq_attention_q8(vcodec.ref, _ptr(packed_k8), _ptr(packed_v), n_seq, n_kv,
+                                                         n_tok, _ptr(q), _dtype(q), g, _ptr(tail_k), _ptr(tail_v),
+                                                         n_tail, scale, v_skip, _ptr(out), _ptr(ws), ws.numel(),
+                                                         _stream(stream)))
 
 
 def tq_topk(codec: Codec, packed_db, n_db, q, n_q, k, idx, score, ws, stream=None, estimator=None):

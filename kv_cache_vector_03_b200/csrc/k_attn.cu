@@ -14,10 +14,16 @@
 // fp16 tensor cores (as tq_pv). Kernel 3 (merge): one CTA per query head combines the ranges
 // (log-sum-exp), rotates the value sum by Pi^T once and adds the exact tail.
 #include <algorithm>
+#include <cfloat>
 
 #include "tq_device.cuh"
 
 namespace {
+
+__device__ __forceinline__ uint32_t q8_pack4(int a, int b, int c, int d) {
+    return (uint32_t)(a & 0xff) | ((uint32_t)(b & 0xff) << 8) | ((uint32_t)(c & 0xff) << 16) |
+           ((uint32_t)(d & 0xff) << 24);
+}
 
 constexpr int kAttnWarps = 8;
 constexpr int kAttnNS = 2;             // ring stages per warp (key + value block each)
@@ -44,6 +50,48 @@ __device__ __forceinline__ int ord_of(float f) {
 }
 __device__ __forceinline__ float float_of(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7fffffff); }
 
+// The value side of one 32-token block: B fragments from the staged weights (column g = head
+// g/2, hi or lo part; token pairs), A fragments decoded through the per-lane half2 tables from
+// the value block's two-token fields, accumulated on the fp16 tensor cores (rows = 128
+// rotated coordinates in 8 tiles of 16, K = the 32 tokens).
+template <int BV>
+__device__ __forceinline__ void attn_values(float (&acc)[8][4], const uint32_t (&wst)[8][kWCol], const uint8_t* vb,
+                                            const uint32_t* lut, int lane) {
+    constexpr int KT = 8, CH = KT * BV / 8, NW = 4 * CH, E = 1 << (2 * BV);
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t lane4 = (uint32_t)lane * 4u;
+    uint32_t bw[2][2];
+#pragma unroll
+    for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int hv2 = 0; hv2 < 2; ++hv2) bw[c][hv2] = wst[g][8 * c + 4 * hv2 + t];
+    uint32_t W[NW + 1];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(vb + (c * 32 + lane) * 16);
+        W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
+    }
+    W[NW] = 0u;
+#pragma unroll
+    for (int kt = 0; kt < KT; ++kt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t a[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                // field (a, pp) at bit (4a + pp) * 2BV of the lane string; the field lands at
+                // bits 7.., i.e. already times the 128-byte entry stride
+                const int f = 4 * (2 * kt + (r & 1)) + 2 * c + (r >> 1);
+                const int bit = f * 2 * BV;
+                const int wi = bit >> 5, sh = bit & 31;
+                const uint32_t x = sh >= 7 ? __funnelshift_r(W[wi], W[wi + 1], sh - 7) : W[wi] << (7 - sh);
+                const uint32_t off = (x & ((uint32_t)(E - 1) << 7)) | lane4;
+                a[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(lut) + off);
+            }
+            tq_hmma(acc[kt], a[0], a[1], a[2], a[3], bw[c][0], bw[c][1]);
+        }
+}
+
 template <int BK, int BV>   // key MSE bits (1..3), value bits (1..4); d <= 128, m <= 128, g <= 4
 __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p) {
     constexpr int NS = kAttnNS;
@@ -51,7 +99,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
     constexpr int NPG = BK + 1;            // stored key plane groups (one 128-coordinate group each)
     constexpr int NMG = NP + 1;            // MMA plane groups
     constexpr uint32_t BBK = 512u * NPG + 128u;
-    constexpr int KT = 8, CH = KT * BV / 8, NW = 4 * CH;
+    constexpr int KT = 8, CH = KT * BV / 8;
     constexpr uint32_t SEC_AV = 512u * CH;
     constexpr uint32_t STG = attn_stage_bytes<BK, BV>();
     constexpr int E = 1 << (2 * BV);
@@ -116,7 +164,6 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
     const float4 sc = reinterpret_cast<const float4*>(p.qscale)[(size_t)stream * 4 + t];
     const bool hv = t < G;
     constexpr float kLog2e = 1.4426950408889634f;
-    const uint32_t lane4 = (uint32_t)lane * 4u;
 
     float acc[KT][4];
 #pragma unroll
@@ -232,35 +279,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
             reinterpret_cast<__half*>(&wst[w][2 * t + 1][0])[tok] = __float2half_rn(wt - __half2float(hi));
         }
         __syncwarp();
-        // ---- values: B fragments (column g = head g/2, hi / lo) and table-decoded A fragments
-        uint32_t bw[2][2];
-#pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-            for (int hv2 = 0; hv2 < 2; ++hv2) bw[c][hv2] = wst[w][g][8 * c + 4 * hv2 + t];
-        uint32_t W[NW + 1];
-#pragma unroll
-        for (int c = 0; c < CH; ++c) {
-            const uint4 v = *reinterpret_cast<const uint4*>(vb + (c * 32 + lane) * 16);
-            W[4 * c] = v.x; W[4 * c + 1] = v.y; W[4 * c + 2] = v.z; W[4 * c + 3] = v.w;
-        }
-        W[NW] = 0u;
-#pragma unroll
-        for (int kt = 0; kt < KT; ++kt)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint32_t a[4];
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int f = 4 * (2 * kt + (r & 1)) + 2 * c + (r >> 1);
-                    const int bit = f * 2 * BV;
-                    const int wi = bit >> 5, sh = bit & 31;
-                    const uint32_t x = sh >= 7 ? __funnelshift_r(W[wi], W[wi + 1], sh - 7) : W[wi] << (7 - sh);
-                    const uint32_t off = (x & ((uint32_t)(E - 1) << 7)) | lane4;
-                    a[r] = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint8_t*>(lut) + off);
-                }
-                tq_hmma(acc[kt], a[0], a[1], a[2], a[3], bw[c][0], bw[c][1]);
-            }
+        attn_values<BV>(acc, wst[w], vb, lut, lane);
         // the stage is consumed: refill it
         __syncwarp();
         if (lane == 0) tq_fence_proxy_async();
@@ -452,6 +471,306 @@ cudaError_t launch_bv(const AttnParams& p, cudaStream_t st) {
     return cudaErrorInvalidValue;
 }
 
+
+// ---------------------------------------------------------------------------------------
+// Decode attention over 8-bit keys and TurboQuant values (the asymmetric K/V configuration of
+// blog.hotdry.top "TurboQuant vector-search compression", engineering configuration list):
+// the split kernel scores each 32-token block with dp4a on the int8 key codes (lane = token,
+// the query heads as int16 fixed point in hi / lo bytes, exact int32 per 32-coordinate chunk,
+// scaled per chunk, as tq_q8_logits), runs the online softmax of every head across the warp,
+// stages exp(l - m) |v| as fp16 hi + lo and accumulates the values as the TurboQuant split
+// kernel does; the first range of a stream also writes the exact logits of its bf16 tail.
+// The merge is the same kernel.
+template <int BV>
+constexpr uint32_t q8_stage_bytes() {
+    return kQ8Block + (512u * BV + 64u);
+}
+template <int BV>
+constexpr size_t q8_attn_smem() {
+    return (size_t)(1 << (2 * BV)) * 128 + (size_t)kAttnWarps * kAttnNS * q8_stage_bytes<BV>();
+}
+
+template <int BV>
+__global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_q8_split(AttnParams p) {
+    constexpr int NS = kAttnNS;
+    constexpr int KT = 8, CH = KT * BV / 8;
+    constexpr uint32_t SEC_AV = 512u * CH;
+    constexpr uint32_t STG = q8_stage_bytes<BV>();
+    constexpr int E = 1 << (2 * BV);
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem);        // [E][32]
+    uint8_t* ring = smem + (size_t)E * 128;                    // [warp][NS][STG]
+    __shared__ uint32_t wst[kAttnWarps][8][kWCol];
+    __shared__ float s_acc[4][KT * 16];
+    __shared__ float s_m[kAttnWarps][4], s_l[kAttnWarps][4];
+    __shared__ int s_cmax[4];
+    __shared__ uint64_t bars[kAttnWarps][NS];
+    __shared__ uint4 s_q[4][2][8];   // per head: hi / lo bytes of the int16 query, per 16-coordinate column
+    __shared__ float s_qs[4];        // scale * fixed-point step
+
+    const int G = p.g, d = p.d;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t stream = blockIdx.x / p.nsplit;
+    const int split = blockIdx.x % p.nsplit;
+    const int64_t b0 = (int64_t)split * p.blocks_per_split;
+    const int64_t b1 = min(b0 + p.blocks_per_split, p.nb);
+
+    for (int e = threadIdx.x; e < E * 8; e += blockDim.x) {
+        const int ent = e >> 3;
+        const uint32_t v = p.cbv.lut_half[ent & ((1 << BV) - 1)] | (p.cbv.lut_half[ent >> BV] << 16);
+        reinterpret_cast<uint4*>(lut)[e] = make_uint4(v, v, v, v);
+    }
+    for (int e = threadIdx.x; e < 4 * KT * 16; e += blockDim.x) (&s_acc[0][0])[e] = 0.f;
+    if (threadIdx.x < 4) s_cmax[threadIdx.x] = ord_of(-INFINITY);
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) tq_mbar_init(&bars[w][s], 2);
+    tq_fence_mbar_init();
+    // query heads as int16 fixed point (step max|q| / 16383), hi / lo int8 bytes
+    if (w < 4) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (w < G) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * lane + k;
+                if (j < d) v[k] = tq_load_elem(p.q, p.q_dtype, (stream * G + w) * d + j);
+            }
+        }
+        const float am = tq_warp_max(fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+        const float step = am > 0.f && am <= FLT_MAX ? am / 16383.f : 1.f;
+        int hi[4], lo[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int qi = (int)fminf(fmaxf(rintf(v[k] / step), -16383.f), 16383.f);
+            hi[k] = (qi + 128) >> 8;
+            lo[k] = qi - 256 * hi[k];
+        }
+        reinterpret_cast<uint32_t*>(&s_q[w][0][lane >> 2])[lane & 3] = q8_pack4(hi[0], hi[1], hi[2], hi[3]);
+        reinterpret_cast<uint32_t*>(&s_q[w][1][lane >> 2])[lane & 3] = q8_pack4(lo[0], lo[1], lo[2], lo[3]);
+        if (lane == 0) s_qs[w] = p.scale * step;
+    }
+    __syncthreads();
+
+    uint8_t* my_ring = ring + (size_t)w * NS * STG;
+    const int64_t first = b0 + w;
+    const int nmine = first < b1 ? (int)((b1 - first + kAttnWarps - 1) / kAttnWarps) : 0;
+    const uint8_t* kk = p.packed_k8 + ((size_t)stream * p.nb + first) * kQ8Block;
+    const uint8_t* vk = p.packed_v + ((size_t)stream * p.nb + first) * p.tv.block_bytes;
+    auto issue = [&](int k) {
+        if (k < nmine && lane == 0) {
+            const int s = k % NS;
+            tq_bulk_load(my_ring + s * STG, kk, kQ8Block, &bars[w][s]);
+            tq_bulk_load(my_ring + s * STG + kQ8Block, vk, (uint32_t)p.tv.block_bytes, &bars[w][s]);
+        }
+        if (k < nmine) {
+            kk += (size_t)kAttnWarps * kQ8Block;
+            vk += (size_t)kAttnWarps * p.tv.block_bytes;
+        }
+    };
+    for (int k = 0; k < NS; ++k) issue(k);
+
+    // the first range of each stream writes the exact logits of its tail (read by the merge)
+    if (split == 0) {
+        for (int tt = w; tt < p.n_tail; tt += kAttnWarps) {
+            const uint16_t* kp = p.tail_k + ((size_t)stream * p.n_tail + tt) * d;
+            float kv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * lane + k;
+                kv[k] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
+            }
+            for (int h = 0; h < G; ++h) {
+                float a = 0.f;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int j = 4 * lane + k;
+                    if (j < d) a = fmaf(kv[k], tq_load_elem(p.q, p.q_dtype, (stream * G + h) * d + j), a);
+                }
+                a = tq_warp_sum(a);
+                if (lane == 0) p.tail_logit[(stream * G + h) * p.n_tail + tt] = p.scale * a;
+            }
+        }
+    }
+
+    constexpr float kLog2e = 1.4426950408889634f;
+    float acc[KT][4];
+#pragma unroll
+    for (int i = 0; i < KT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    float m_run[4], lsum[4];   // every lane: the running maxima (warp-uniform) and its tokens' sums
+#pragma unroll
+    for (int h = 0; h < 4; ++h) { m_run[h] = -INFINITY; lsum[h] = 0.f; }
+
+    bool ok = true;
+    int k = 0;
+    for (; k < nmine; ++k) {
+        const int s = k % NS;
+        ok = __all_sync(0xffffffffu, tq_mbar_wait(&bars[w][s], (uint32_t)(k / NS) & 1u, kWaitLimit));
+        if (!ok) break;
+        const uint8_t* kb = my_ring + s * STG;
+        const uint8_t* vb = kb + kQ8Block;
+        const int64_t blk = first + (int64_t)kAttnWarps * k;
+        // ---- logits of token `lane` for the 4 heads: dp4a per 32-coordinate chunk
+        uint4 kc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kc[j] = *reinterpret_cast<const uint4*>(kb + j * 512 + lane * 16);
+        float res[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const float csc = tq_half_val(reinterpret_cast<const uint16_t*>(kb + 4096)[c * 32 + lane]);
+            int ah[4] = {0, 0, 0, 0}, al[4] = {0, 0, 0, 0};
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int j = 2 * c + jj;
+                const int kw[4] = {(int)kc[j].x, (int)kc[j].y, (int)kc[j].z, (int)kc[j].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const uint4 qh = s_q[h][0][j], ql = s_q[h][1][j];
+                    ah[h] = __dp4a(kw[0], (int)qh.x, ah[h]);
+                    ah[h] = __dp4a(kw[1], (int)qh.y, ah[h]);
+                    ah[h] = __dp4a(kw[2], (int)qh.z, ah[h]);
+                    ah[h] = __dp4a(kw[3], (int)qh.w, ah[h]);
+                    al[h] = __dp4a(kw[0], (int)ql.x, al[h]);
+                    al[h] = __dp4a(kw[1], (int)ql.y, al[h]);
+                    al[h] = __dp4a(kw[2], (int)ql.z, al[h]);
+                    al[h] = __dp4a(kw[3], (int)ql.w, al[h]);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < 4; ++h) res[h] = fmaf(csc, (float)(256 * ah[h] + al[h]), res[h]);
+        }
+        const bool tok_in = blk * 32 + lane < p.n_tok;
+        float l[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) l[h] = (h < G && tok_in) ? s_qs[h] * res[h] : -INFINITY;
+        // ---- online softmax, every head across the warp
+        float fac[4];
+        bool low = true;
+        const float vn = tq_half_val(reinterpret_cast<const uint16_t*>(vb + SEC_AV)[lane]);
+        float wt[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const float bm = tq_warp_max(l[h]);
+            float cmax = bm;
+            if (p.v_skip > 0.f) {
+                if (lane == 0) atomicMax(&s_cmax[h], ord_of(bm));
+                cmax = fmaxf(bm, float_of(*reinterpret_cast<volatile int*>(&s_cmax[h])));
+            }
+            fac[h] = 1.f;
+            if (bm > m_run[h]) {
+                fac[h] = tq_exp2((m_run[h] - bm) * kLog2e);   // 0 while the maximum was -inf
+                lsum[h] *= fac[h];
+                m_run[h] = bm;
+            }
+            const float ev = m_run[h] > -INFINITY ? tq_exp2(fmaf(l[h], kLog2e, -m_run[h] * kLog2e)) : 0.f;
+            lsum[h] += ev;
+            wt[h] = ev * vn;
+            low = low && (l[h] < cmax + __logf(p.v_skip) || l[h] == -INFINITY);
+        }
+        // accumulator columns 2t, 2t + 1 belong to head t
+        const float ft = t == 0 ? fac[0] : t == 1 ? fac[1] : t == 2 ? fac[2] : fac[3];
+        if (ft != 1.f) {
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+                acc[i][0] *= ft; acc[i][1] *= ft; acc[i][2] *= ft; acc[i][3] *= ft;
+            }
+        }
+        if (__all_sync(0xffffffffu, low)) {
+            __syncwarp();
+            if (lane == 0) tq_fence_proxy_async();
+            issue(k + NS);
+            continue;
+        }
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const __half hi = __float2half_rn(wt[h]);
+            reinterpret_cast<__half*>(&wst[w][2 * h][0])[lane] = hi;
+            reinterpret_cast<__half*>(&wst[w][2 * h + 1][0])[lane] = __float2half_rn(wt[h] - __half2float(hi));
+        }
+        __syncwarp();
+        attn_values<BV>(acc, wst[w], vb, lut, lane);
+        __syncwarp();
+        if (lane == 0) tq_fence_proxy_async();
+        issue(k + NS);
+    }
+    if (!ok) {
+        if (lane == 0) {
+            tq_raise(p.status, TQ_FLAG_TIMEOUT);
+            for (int j = k; j < min(k + NS, nmine); ++j)
+                tq_mbar_wait(&bars[w][j % NS], (uint32_t)(j / NS) & 1u, kWaitLimit);
+        }
+        __syncwarp();
+    }
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        const float ls = tq_warp_sum(lsum[h]);
+        if (lane == 0) { s_m[w][h] = m_run[h]; s_l[w][h] = ls; }
+    }
+    __syncthreads();
+    float M = s_m[0][t];
+#pragma unroll
+    for (int v = 1; v < kAttnWarps; ++v) M = fmaxf(M, s_m[v][t]);
+    const float mt = s_m[w][t];
+    const float f = mt > -INFINITY ? tq_exp2((mt - M) * kLog2e) : 0.f;
+    if (t < G) {
+#pragma unroll
+        for (int kt = 0; kt < KT; ++kt) {
+            atomicAdd(&s_acc[t][16 * kt + g], f * (acc[kt][0] + acc[kt][1]));
+            atomicAdd(&s_acc[t][16 * kt + 8 + g], f * (acc[kt][2] + acc[kt][3]));
+        }
+    }
+    __syncthreads();
+    const int D = KT * 16;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, i = e % D;
+        p.part[(((size_t)stream * G + h) * p.nsplit + split) * D + i] = s_acc[h][i];
+    }
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float Mh = s_m[0][h], L = 0.f;
+        for (int v = 1; v < kAttnWarps; ++v) Mh = fmaxf(Mh, s_m[v][h]);
+        for (int v = 0; v < kAttnWarps; ++v)
+            if (s_m[v][h] > -INFINITY) L += s_l[v][h] * tq_exp2((s_m[v][h] - Mh) * kLog2e);
+        reinterpret_cast<float2*>(p.part_ml)[((size_t)stream * G + h) * p.nsplit + split] = make_float2(Mh, L);
+    }
+}
+
+template <int BV>
+cudaError_t launch_q8_split(const AttnParams& p, cudaStream_t st) {
+    constexpr size_t smem = q8_attn_smem<BV>();
+    if (p.tv.block_bytes != 512u * BV + 64u) return cudaErrorInvalidValue;
+    auto kern = k_attn_q8_split<BV>;
+    static TqLaunchCache cache;
+    cudaError_t e = tq_kernel_setup(kern, kAttnWarps * 32, smem, cache, nullptr, nullptr);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)(p.n_streams * p.nsplit), kAttnWarps * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+// tail-only calls: the tail logits of every stream (one CTA per stream)
+__global__ void __launch_bounds__(kAttnWarps * 32) k_attn_q8_tail(AttnParams p) {
+    const int G = p.g, d = p.d;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t stream = blockIdx.x;
+    for (int tt = w; tt < p.n_tail; tt += kAttnWarps) {
+        const uint16_t* kp = p.tail_k + ((size_t)stream * p.n_tail + tt) * d;
+        float kv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int j = 4 * lane + k;
+            kv[k] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
+        }
+        for (int h = 0; h < G; ++h) {
+            float a = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int j = 4 * lane + k;
+                if (j < d) a = fmaf(kv[k], tq_load_elem(p.q, p.q_dtype, (stream * G + h) * d + j), a);
+            }
+            a = tq_warp_sum(a);
+            if (lane == 0) p.tail_logit[(stream * G + h) * p.n_tail + tt] = p.scale * a;
+        }
+    }
+}
 }  // namespace
 
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
@@ -467,6 +786,26 @@ cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
     }
     // a plain launch: as a programmatic dependent of the split the merge measured 17 us slower
     // per call at 8 x 32768 tokens
+    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st) {
+    if (p.tv.D != 128 || p.d > 128 || p.g < 1 || p.g > 4) return cudaErrorInvalidValue;
+    cudaError_t e = cudaSuccess;
+    if (p.nsplit > 0) {
+        switch (p.tv.B) {
+            case 1: e = launch_q8_split<1>(p, st); break;
+            case 2: e = launch_q8_split<2>(p, st); break;
+            case 3: e = launch_q8_split<3>(p, st); break;
+            case 4: e = launch_q8_split<4>(p, st); break;
+            default: e = cudaErrorInvalidValue;
+        }
+    } else if (p.n_tail > 0) {
+        k_attn_q8_tail<<<(unsigned)p.n_streams, kAttnWarps * 32, 0, st>>>(p);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) return e;
     k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }

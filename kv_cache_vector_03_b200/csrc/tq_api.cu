@@ -160,6 +160,24 @@ AttnWs attn_ws(const TqDims& tk, int64_t n_streams, int64_t n_tok, int g, int n_
     return w;
 }
 
+// attention over 8-bit keys: the tail logits, split partials (no query fragments)
+struct AttnQ8Ws { int nsplit, bps; size_t tl, part, ml, total; };
+AttnQ8Ws attn_q8_ws(int64_t n_streams, int64_t n_tok, int g, int n_tail) {
+    AttnQ8Ws w;
+    const int64_t nb = (n_tok + 31) / 32;
+    int64_t bps = (nb * n_streams + 2 * tq_device_sms() - 1) / (2 * tq_device_sms());
+    bps = std::max<int64_t>(8, bps);
+    bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
+    w.bps = (int)bps;
+    w.nsplit = (int)((nb + bps - 1) / bps);
+    size_t off = TQ_STATUS_BYTES;
+    w.tl = off; off = align_up(off + (size_t)n_streams * g * n_tail * 4);
+    w.part = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * 128 * 4);
+    w.ml = off; off = align_up(off + (size_t)n_streams * g * w.nsplit * 8);
+    w.total = off;
+    return w;
+}
+
 // key codec (qjl = 1, d and m <= 128) and value codec (qjl = 0, the same d) of tq_attention
 int check_attention_codecs(const tq_codec* kc, const tq_codec* vc) {
     int st = check_codec(kc, true);
@@ -496,6 +514,63 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
     cudaError_t e = tq_launch_logits_prologue(lp, cs);
     if (e != cudaSuccess) return TQ_ERR_CUDA;
     return cuda_status(tq_launch_attention(p, cs));
+}
+
+size_t tq_attention_q8_workspace_bytes(const tq_codec* vcodec, int64_t n_seq, int n_kv, int64_t n_tok, int g,
+                                       int n_tail) {
+    if (check_codec(vcodec, true) != TQ_OK || vcodec->qjl || vcodec->d > 128) return 0;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0 || g < 1 || g > 4) return 0;
+    return attn_q8_ws(n_seq * n_kv, n_tok, g, n_tail).total;
+}
+
+int tq_attention_q8(const tq_codec* vcodec, const void* packed_k8, const void* packed_v, int64_t n_seq, int n_kv,
+                    int64_t n_tok, const void* q, tq_dtype q_dtype, int g, const void* tail_k, const void* tail_v,
+                    int n_tail, float scale, float v_skip, float* out, void* ws, size_t ws_bytes, void* stream) {
+    int st = check_codec(vcodec, true);
+    if (st != TQ_OK) return st;
+    if (vcodec->qjl) return TQ_ERR_ARG;
+    if (vcodec->d > 128) return TQ_ERR_UNSUPPORTED;
+    if (g != 1 && g != 2 && g != 4) return TQ_ERR_UNSUPPORTED;
+    if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0) return TQ_ERR_ARG;
+    if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return TQ_ERR_ARG;
+    if (n_seq == 0) return TQ_OK;
+    if (n_tok + n_tail == 0) return TQ_ERR_ARG;   // softmax over no tokens
+    if (n_tail > TQ_ATTN_MAX_TAIL) return TQ_ERR_UNSUPPORTED;
+    if (!q || !out || !ws || (n_tok > 0 && (!packed_k8 || !packed_v)) || (n_tail > 0 && (!tail_k || !tail_v)))
+        return TQ_ERR_ARG;
+    if ((n_tok > 0 && (!aligned(packed_k8, 16) || !aligned(packed_v, 16))) || !aligned(out, 4) ||
+        !aligned(ws, 256) || !aligned(q, q_dtype == TQ_F32 ? 4 : 2) ||
+        (n_tail > 0 && (!aligned(tail_k, 2) || !aligned(tail_v, 8))))
+        return TQ_ERR_ARG;
+    if (!std::isfinite(scale) || !(v_skip >= 0.f && v_skip <= 1.f)) return TQ_ERR_ARG;
+    const TqDims tv = dims_of(vcodec);
+    const int64_t n_streams = n_seq * n_kv;
+    if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
+    const AttnQ8Ws W = attn_q8_ws(n_streams, n_tok, g, n_tail);
+    if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
+    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.packed_k8 = static_cast<const uint8_t*>(packed_k8);
+    p.packed_v = static_cast<const uint8_t*>(packed_v);
+    p.q = q; p.q_dtype = q_dtype;
+    p.tail_k = static_cast<const uint16_t*>(tail_k);
+    p.tail_logit = reinterpret_cast<float*>(wsb + W.tl);
+    p.tail_v = static_cast<const uint16_t*>(tail_v);
+    p.piT_v = reinterpret_cast<const float*>(static_cast<const uint8_t*>(vcodec->prep) + tq_prep_layout(tv).piT);
+    p.out = out;
+    p.part = reinterpret_cast<float*>(wsb + W.part);
+    p.part_ml = reinterpret_cast<float*>(wsb + W.ml);
+    p.status = static_cast<uint32_t*>(ws);
+    p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
+    p.g = g; p.nsplit = p.nb > 0 ? W.nsplit : 0; p.blocks_per_split = W.bps; p.n_tail = n_tail;
+    p.v_skip = v_skip;
+    p.tv = tv;
+    p.scale = scale;
+    p.d = vcodec->d;
+    if ((st = codebook_consts(vcodec, &p.cbv)) != TQ_OK) return st;
+    return cuda_status(tq_launch_attention_q8(p, static_cast<cudaStream_t>(stream)));
 }
 
 int tq_topk_est(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k,

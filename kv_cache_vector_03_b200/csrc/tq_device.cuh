@@ -353,7 +353,7 @@ struct AttnParams {
     const uint8_t* packed_v;      // value blocks (qjl = 0), same d
     const uint32_t* qfrag;        // query fragments of the key codec (logits prologue)
     const float* qscale;          // per-head constants (attention scale folded in)
-    const float* tail_logit;      // [stream * g + head][n_tail] exact tail logits (prologue)
+    float* tail_logit;            // [stream * g + head][n_tail] exact tail logits (prologue, or the q8 split)
     const uint16_t* tail_v;       // bf16 [stream][n_tail][d] full-precision recent values
     const float* piT_v;           // prepared Pi^T of the value codec, fp32 [D][D]
     float* out;                   // fp32 [stream * g + head][d]
@@ -365,6 +365,14 @@ struct AttnParams {
     float v_skip;                 // sparse values: a block whose weights are all below it skips its values
     TqDims tk, tv;
     TqCodebookConsts cbv;         // value codebook (binary16 decode table)
+    // 8-bit keys (tq_attention_q8): the key cache, the raw queries and the bf16 tail keys,
+    // whose exact logits the split kernel writes to tail_logit
+    const uint8_t* packed_k8;
+    const void* q;
+    int q_dtype;
+    const uint16_t* tail_k;
+    float scale;
+    int d;
 };
 
 // 8-bit keys (per 32-coordinate chunk: int8 codes and one binary16 scale), d <= 128
@@ -411,6 +419,7 @@ bool tq_quantize_ws_eligible(const QuantParams& p);
 cudaError_t tq_launch_quantize_wide(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
+cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
 cudaError_t tq_launch_q8_quantize(const Q8QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_q8_logits(const Q8LogitsParams& p, cudaStream_t st);

@@ -552,6 +552,78 @@ def test_q8_keys(d, g, n_seq, n_kv, n_tok, n_tail):
                               scale)
 
 
+@pytest.mark.parametrize("Bv,g,n_seq,n_kv,n_tok,n_tail,law,vs", [
+    (3, 4, 1, 2, 3000, 128, "c2", 0.0),     # the decode key law, a 128-token tail
+    (4, 2, 2, 2, 301, 5, "normal", 0.0),    # several streams, ragged last block
+    (2, 1, 1, 1, 64, 0, "normal", 0.0),     # no tail
+    (3, 4, 1, 2, 2000, 16, "c2", 1e-4),     # sparse values
+])
+def test_attention_q8_keys(Bv, g, n_seq, n_kv, n_tok, n_tail, law, vs):
+    """Decode attention over 8-bit keys and TurboQuant values (the asymmetric configuration)
+    against the oracle's attention_q8 on the GPU's own codes, by the two checks of
+    gpu_helpers.check_attention: the oracle's P.V over the logits of tq_q8_logits (softmax,
+    value decode, merge) and the full oracle composition."""
+    torch = torch_cuda()
+    m = tq()
+    d = 128
+    n = n_tok + n_tail
+    piv = ti.haar_rotation(d, 131)
+    if law == "c2":
+        keys = np.stack([np.stack([ti.key_stream(4, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    else:
+        keys = np.stack([np.stack([_normal_stream(81, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    vals = np.stack([np.stack([_normal_stream(82, sq, h, n) for h in range(n_kv)]) for sq in range(n_seq)])
+    S = n_seq * n_kv
+    vc = make_codec(d, 0, Bv, False, piv, None)
+    pk8 = torch.zeros(m.tq_q8_packed_bytes(d, S, n_tok), dtype=torch.uint8, device="cuda")
+    ws0 = m.workspace(256)
+    m.tq_q8_quantize(to_dev_bf16(np.ascontiguousarray(keys[:, :, :n_tok]).reshape(-1, d)), d, S, n_tok, n_tok * d,
+                     pk8, ws0)
+    assert m.tq_get_status(ws0) == m.TQ_OK
+    pvv, _ = gpu_quantize(vc, to_dev_bf16(np.ascontiguousarray(vals[:, :, :n_tok]).reshape(-1, d)), S, n_tok)
+    tk = to_dev_bf16(np.ascontiguousarray(keys[:, :, n_tok:])) if n_tail else None
+    tv = to_dev_bf16(np.ascontiguousarray(vals[:, :, n_tok:])) if n_tail else None
+    qb = ti.decode_queries(16, n_seq, n_kv * g)
+    scale = 1.0 / math.sqrt(d)
+    out = torch.full((n_seq, n_kv * g, d), float("nan"), dtype=torch.float32, device="cuda")
+    ws = m.workspace(m.tq_attention_q8_workspace_bytes(vc, n_seq, n_kv, n_tok, g, n_tail))
+    m.tq_attention_q8(vc, pk8, pvv, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, tv, n_tail, scale, out, ws, v_skip=vs)
+    torch.cuda.synchronize()
+    assert m.tq_get_status(ws) == m.TQ_OK
+    got = out.cpu().numpy().astype(np.float64)
+    lgt = torch.full((n_seq, n_kv * g, n), float("nan"), dtype=torch.float32, device="cuda")
+    m.tq_q8_logits(pk8, d, n_seq, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale, lgt)
+    torch.cuda.synchronize()
+    lg = lgt.cpu().numpy().astype(np.float64)
+    codes, scales, _ = _unpack_q8(pk8, d, S, n_tok)
+    vidx, vnh = unpack(vc, pvv, S, n_tok)
+    c_v, _ = _cb(d, Bv)
+    q = ti.bf16_to_f64(qb)
+    kf, vf = ti.bf16_to_f64(keys), ti.bf16_to_f64(vals)
+    for sq in range(n_seq):
+        for h in range(n_kv):
+            st = sq * n_kv + h
+            qh = q[sq, h * g:(h + 1) * g]
+            tkh, tvh = (kf[sq, h, n_tok:], vf[sq, h, n_tok:]) if n_tail else (None, None)
+            want = oracle.attention_q8(codes[st], scales[st], vidx[st], vnh[st], piv, c_v, qh, scale, tail_k=tkh,
+                                       tail_v=tvh)
+            L = np.concatenate([oracle.q8_logits(codes[st], scales[st], qh, scale),
+                                oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)], axis=1)
+            vhat = oracle.reconstruct(vidx[st], None, vnh[st], None, piv, None, c_v, qjl=False)
+            V = np.concatenate([vhat, vf[sq, h, n_tok:]])
+            vnorm = np.concatenate([vnh[st], np.linalg.norm(vf[sq, h, n_tok:], axis=1)])
+            skip = None
+            if vs > 0.0:
+                rel = np.exp(L - L.max(axis=1, keepdims=True))
+                wv = rel / rel.sum(axis=1, keepdims=True) * vnorm[None, :]
+                drop = rel < vs
+                drop[:, n_tok:] = False
+                skip = (wv * drop).sum(axis=1) / wv.sum(axis=1)
+            err, err_c = check_attention(got[sq, h * g:(h + 1) * g], want, L, lg[sq, h * g:(h + 1) * g], n_tok, V,
+                                         vnorm, v_skip=vs, skip_mass=skip)
+            print(f"q8 attention stream {st}: {err.max():.2e} (full), {err_c.max():.2e} (composed)")
+
+
 def test_attention_rejects_unsupported():
     torch = torch_cuda()
     m = tq()
