@@ -588,302 +588,6 @@ cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
     return tq_launch_pdl(kern, dim3((unsigned)grid), dim3(kStreamWarps * 32), smem, st, p);
 }
 
-// ---------------------------------------------------------------------------------------
-// Fused single-launch variant for d, m <= 128 and g <= 4 (one n-tile of heads): every CTA first
-// rotates the queries of the (at most kMaxCS) streams its warps visit, q' = Pi q and q'' = S q
-// on the CUDA cores from the prepared transposes, and builds their fixed-point fragments and
-// per-head constants in shared memory exactly as the prologue kernel would; the bulk copies
-// of its first key blocks are already in flight meanwhile. After the key blocks, the warps
-// share the exact logits of the bf16 tail tokens.
-constexpr int kMaxCS = 4;
-
-template <int B, int NS>
-__global__ void __launch_bounds__(kStreamWarps * 32) k_logits_fused(LogitsParams p) {
-    constexpr int NP = B == 3 ? 4 : B;
-    constexpr int NPG = B + 1, NMG = NP + 1;
-    constexpr uint32_t BB = 512u * NPG + 128u;
-    constexpr int W = 256;                 // q' (128) then q'' (128)
-    extern __shared__ __align__(128) uint8_t ring[];
-    __shared__ uint64_t bars[kStreamWarps][NS + 1];
-    __shared__ __align__(16) uint32_t s_frag[kMaxCS][NMG * 256];
-    __shared__ __align__(16) float4 s_sc[kMaxCS][4];
-    __shared__ float s_step[2][4], s_inv[2][4];
-    __shared__ int s_sum[2][4];
-    float* s_q = reinterpret_cast<float*>(ring + (size_t)kStreamWarps * NS * BB);   // [4][128] raw queries
-    float* s_qo = s_q + 4 * 128;                                                     // [4][W]
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int G = p.g, d = p.t.d;
-    uint8_t* my_ring = ring + (size_t)warp * NS * BB;
-    if (lane == 0)
-        for (int s = 0; s <= NS; ++s) tq_mbar_init(&bars[warp][s], 1);
-    tq_fence_mbar_init();
-    __syncwarp();
-
-    const int64_t n_blocks = p.n_seq * p.n_kv * p.nb, n_warps = (int64_t)gridDim.x * kStreamWarps;
-    const int64_t gw = (int64_t)blockIdx.x * kStreamWarps + warp;
-    FlatWalk prod, cons;
-    prod.init(p, gw * n_blocks / n_warps, (gw + 1) * n_blocks / n_warps);
-    cons = prod;
-    uint32_t issued = 0;
-    if (lane == 0) {
-        for (int s = 0; s < NS && prod.valid(); ++s) {
-            tq_bulk_load(my_ring + s * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB, &bars[warp][s]);
-            prod.advance(p);
-            ++issued;
-        }
-    }
-    // streams of this CTA: from the first block of warp 0 to the last block of warp 7
-    const int64_t cb0 = (int64_t)blockIdx.x * kStreamWarps * n_blocks / n_warps;
-    const int64_t cb1 = ((int64_t)blockIdx.x + 1) * kStreamWarps * n_blocks / n_warps;
-    const int s_lo = (int)(cb0 / p.nb);
-    const int ncs = cb1 > cb0 ? (int)((cb1 - 1) / p.nb) - s_lo + 1 : 0;   // <= kMaxCS (checked at launch)
-
-    // 1-4, one stream of the CTA at a time (4 head slots: query row (s_lo + cs) g + h, h < g)
-    for (int e = tid; e < kMaxCS * NMG * 256; e += blockDim.x) (&s_frag[0][0])[e] = 0u;
-    float amax = 0.f;
-    for (int pl = 0; pl < NP; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
-    for (int cs = 0; cs < ncs; ++cs) {
-        // 1. raw queries
-        for (int e = tid; e < 4 * 128; e += blockDim.x) {
-            const int h = e >> 7, j = e & 127;
-            const int64_t qrow = (int64_t)(s_lo + cs) * G + h;
-            const bool qok = h < G && j < d && qrow < p.n_heads_valid;
-            s_q[e] = qok ? tq_load_elem(p.q, p.q_dtype, qrow * d + j) : 0.f;
-        }
-        if (tid < 8) s_sum[tid >> 2][tid & 3] = 0;
-        __syncthreads();
-        // 2. q' = Pi q (columns of PiT) and q'' = S q (columns of S^T), one output column per thread
-        {
-            const int c = tid;   // 256 threads, 256 output columns (D = Mp = 128)
-            const float* mat = c < 128 ? p.piT + c : p.sT + (c - 128);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-            for (int j = 0; j < d; ++j) {
-                const float m = __ldg(mat + (size_t)j * 128);
-#pragma unroll
-                for (int h = 0; h < 4; ++h) acc[h] = fmaf(s_q[h * 128 + j], m, acc[h]);
-            }
-#pragma unroll
-            for (int h = 0; h < 4; ++h) s_qo[h * W + c] = acc[h];
-        }
-        __syncthreads();
-        // 3. fixed-point steps, one head per warp
-        if (warp < 4) {
-            const int h = warp;
-            float ma = 0.f, ms = 0.f;
-            for (int i = lane; i < 128; i += 32) {
-                ma = fmaxf(ma, fabsf(s_qo[h * W + i]));
-                ms = fmaxf(ms, fabsf(s_qo[h * W + 128 + i]));
-            }
-            ma = tq_warp_max(ma) * amax;
-            ms = tq_warp_max(ms);
-            if (lane == 0) {
-                s_step[0][h] = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
-                s_step[1][h] = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
-                s_inv[0][h] = 1.f / s_step[0][h];
-                s_inv[1][h] = 1.f / s_step[1][h];
-            }
-        }
-        __syncthreads();
-        // 4. fragment words (the prologue kernel's layout, per stream in shared memory); a warp's
-        //    32 items share the head and the plane group
-        for (int e = tid; e < 4 * 32 * NMG; e += blockDim.x) {
-            const int head = e / (32 * NMG), w = e - head * (32 * NMG);
-            const int mg = w >> 5, c = (w >> 3) & 3, tt = (w >> 1) & 3, hh = w & 1;
-            const bool is_code = mg < NP;
-            int sum = 0;
-            if (head < G) {
-                const float coef = is_code ? 2.f * p.cb.plane_coef[mg] : 1.f;
-                const float inv = coef * s_inv[is_code ? 0 : 1][head];
-                const float* src = s_qo + head * W + (is_code ? 0 : 128) + 32 * tt + 2 * c + hh;
-                uint32_t whi = 0, wlo = 0;
-                // bit s = 2c + hh of the key bytes meets this register: factor 2^(3 - s mod 4)
-                const int f = 8 >> ((2 * c + hh) & 3);
-#pragma unroll
-                for (int bb = 0; bb < 4; ++bb) {
-                    const int v = __float2int_rn(src[8 * bb] * inv);
-                    sum += v;
-                    const int vf = v * f, hi = (vf + 128) >> 8, lo = vf - 256 * hi;
-                    whi |= (uint32_t)(hi & 0xff) << (8 * bb);
-                    wlo |= (uint32_t)(lo & 0xff) << (8 * bb);
-                }
-                const int wi = mg * 256 + c * 64 + 16 * head + 2 * tt + hh;
-                s_frag[cs][wi] = whi;
-                s_frag[cs][wi + 8] = wlo;
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-            if (lane == 0) atomicAdd(&s_sum[is_code ? 0 : 1][head], sum);
-        }
-        __syncthreads();
-        // per-head constants (scale and QJL factor folded in), as the prologue kernel's
-        if (tid < 4) {
-            const int head = tid;
-            const float dA = s_step[0][head], dS = s_step[1][head], sa = p.scale;
-            s_sc[cs][head] = head < G ? make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)s_sum[0][head],
-                                                    sa * p.kappa * 2.f * dS / 128.f,
-                                                    sa * p.kappa * dS * (float)s_sum[1][head])
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        __syncthreads();
-    }
-
-    // 5. the key blocks (as k_logits_stream, with the fragments in shared memory)
-    const int64_t row = p.n_tok + p.n_tail;
-    uint32_t qf[NMG][4][2];
-    float4 sc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float* orow = p.out;
-    bool hv = false;
-    int cur_stream = -1;
-    uint32_t seq = 0;
-    // test stall: a bounded wait on the barrier nothing arrives at runs out, as a lost copy would
-    bool ok = p.test_stall == 0u || __all_sync(0xffffffffu, tq_mbar_wait(&bars[warp][NS], 0u, p.test_stall));
-    while (ok && cons.valid()) {
-        if (cons.stream != cur_stream) {
-            cur_stream = cons.stream;
-            const uint32_t* fr = s_frag[cur_stream - s_lo];
-#pragma unroll
-            for (int mg = 0; mg < NMG; ++mg)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(fr + mg * 256 + c * 64 + lane * 2);
-                    qf[mg][c][0] = v.x;
-                    qf[mg][c][1] = v.y;
-                }
-            sc = s_sc[cur_stream - s_lo][t];
-            hv = t < G;
-            orow = p.out + ((int64_t)cur_stream * G + (hv ? t : 0)) * row;
-        }
-        const int stage = seq % NS;
-        ok = __all_sync(0xffffffffu, tq_mbar_wait(&bars[warp][stage], (seq / NS) & 1u, kWaitLimit));
-        if (!ok) break;
-        const uint8_t* bp = my_ring + stage * BB;
-        uint4 cur[NPG + 1];
-#pragma unroll
-        for (int pg = 0; pg < NPG; ++pg) cur[pg] = *reinterpret_cast<const uint4*>(bp + (pg * 32 + lane) * 16);
-        cur[NPG] = *reinterpret_cast<const uint4*>(bp + NPG * 512 + g * 16);
-        const bool full = (int64_t)(cons.blk + 1) * 32 <= p.n_tok;
-        const int n_valid = full ? 32 : (int)(p.n_tok - (int64_t)cons.blk * 32);
-        const int tok0 = cons.blk * 32 + g;
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            // code planes accumulate in two chains (chunks c odd / even), the sign plane in one
-            int accA[4], accA2[4], accS[4];
-#pragma unroll
-            for (int mg = 0; mg < NMG; ++mg) {
-                uint32_t w0, w1;   // words of rows g (u = 2mt) and g + 8 (u = 2mt + 1)
-                if (mg == 3 && mg < NP) {   // b0 ^ b1 ^ b2
-                    const uint32_t* c0 = reinterpret_cast<const uint32_t*>(&cur[0]);
-                    const uint32_t* c1 = reinterpret_cast<const uint32_t*>(&cur[1]);
-                    const uint32_t* c2 = reinterpret_cast<const uint32_t*>(&cur[2]);
-                    w0 = c0[2 * mt] ^ c1[2 * mt] ^ c2[2 * mt];
-                    w1 = c0[2 * mt + 1] ^ c1[2 * mt + 1] ^ c2[2 * mt + 1];
-                } else {
-                    const uint32_t* cw = reinterpret_cast<const uint32_t*>(&cur[mg < NP ? mg : B]);
-                    w0 = cw[2 * mt];
-                    w1 = cw[2 * mt + 1];
-                }
-                tq_expand_planes(w0, w1, [&](int c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-                    const uint32_t b0 = qf[mg][c][0], b1 = qf[mg][c][1];
-                    if (mg < NP) {
-                        int(&acc)[4] = (c & 1) ? accA : accA2;
-                        if (mg == 0 && c >= 2) tq_imma_u8_z(acc, a0, a1, a2, a3, b0, b1);
-                        else tq_imma_u8(acc, a0, a1, a2, a3, b0, b1);
-                    } else {
-                        if (c == 3) tq_imma_u8_z(accS, a0, a1, a2, a3, b0, b1);
-                        else tq_imma_u8(accS, a0, a1, a2, a3, b0, b1);
-                    }
-                });
-            }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) accA[r] += accA2[r];
-            const uint32_t* nrm = reinterpret_cast<const uint32_t*>(&cur[NPG]);
-#pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int u = 2 * mt + r;
-                const uint32_t nw = nrm[u];
-                const float nhv = tq_half_val(nw & 0xffffu), gh = tq_half_val(nw >> 16);
-                const float va = (float)(256 * accA[2 * r] + accA[2 * r + 1]);
-                const float vs = (float)(256 * accS[2 * r] + accS[2 * r + 1]);
-                const float est = fmaf(sc.x, va, -sc.y) + gh * fmaf(sc.z, vs, -sc.w);
-                if (hv && (full || 8 * u + g < n_valid)) orow[tok0 + 8 * u] = nhv * est;
-            }
-        }
-        // the stage's data are consumed (all reads above fed the MMAs): refill it
-        __syncwarp();
-        if (lane == 0 && prod.valid()) {
-            tq_fence_proxy_async();
-            tq_bulk_load(my_ring + stage * BB, p.packed + ((size_t)prod.stream * p.nb + prod.blk) * BB, BB,
-                         &bars[warp][stage]);
-            prod.advance(p);
-            ++issued;
-        }
-        ++seq;
-        cons.advance(p);
-    }
-    if (!ok) {
-        // a wait ran out: record it, then give each copy still in flight a bounded time to land
-        if (lane == 0) {
-            tq_raise(p.status, TQ_FLAG_TIMEOUT);
-            for (uint32_t k = seq; k < issued; ++k) tq_mbar_wait(&bars[warp][k % NS], (k / NS) & 1u, kWaitLimit);
-        }
-        __syncwarp();
-        return;
-    }
-    // 6. exact logits of the bf16 tail: items (stream, token), one per warp, strided over all warps
-    const int64_t n_items = p.n_seq * p.n_kv * (int64_t)p.n_tail;
-    for (int64_t it = gw; it < n_items; it += n_warps) {
-        const int64_t st = it / p.n_tail;
-        const int tt = (int)(it - st * p.n_tail);
-        const uint16_t* kp = p.tail + ((size_t)st * p.n_tail + tt) * d;
-        float kv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = lane + 32 * i;
-            kv[i] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
-        }
-        for (int h = 0; h < G; ++h) {
-            const int64_t qrow = st * G + h;
-            float a = 0.f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = lane + 32 * i;
-                if (j < d) a = fmaf(kv[i], tq_load_elem(p.q, p.q_dtype, qrow * d + j), a);
-            }
-            a = tq_warp_sum(a);
-            if (lane == 0 && qrow < p.n_heads_valid) p.out[qrow * row + p.n_tok + tt] = p.scale * a;
-        }
-    }
-}
-
-template <int B>
-constexpr size_t fused_smem() {
-    return (size_t)kStreamWarps * 4 * (512u * (B + 1) + 128u) + (size_t)4 * (128 + 256) * 4;
-}
-
-// the fused kernel's grid (persistent, as the stream kernel's); 0 if it does not apply
-template <int B>
-int fused_grid(const LogitsParams& p, TqLaunchCache& cache, cudaError_t* err) {
-    auto kern = k_logits_fused<B, 4>;
-    int sms = 0, per_sm = 0;
-    *err = tq_kernel_setup(kern, kStreamWarps * 32, fused_smem<B>(), cache, &sms, &per_sm);
-    if (*err != cudaSuccess) return 0;
-    const int64_t n_blocks = p.n_seq * p.n_kv * p.nb;
-    const int64_t grid = std::min<int64_t>((n_blocks + kStreamWarps - 1) / kStreamWarps, (int64_t)per_sm * sms);
-    if (grid <= 0) return 0;
-    // every CTA must visit at most kMaxCS streams: its range is about n_blocks / grid blocks
-    const int64_t per_cta = (n_blocks + grid - 1) / grid + 1;
-    if ((per_cta + p.nb - 1) / p.nb + 1 > kMaxCS) return 0;
-    return (int)grid;
-}
-
-template <int B>
-cudaError_t launch_fused(const LogitsParams& p, int grid, cudaStream_t st) {
-    k_logits_fused<B, 4><<<(unsigned)grid, kStreamWarps * 32, fused_smem<B>(), st>>>(p);
-    return cudaGetLastError();
-}
-
 template <int B, int GD, int GM>
 cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
     return p.ntiles == 1 ? launch_stream<B, GD, GM, 1>(p, st) : launch_stream<B, GD, GM, 2>(p, st);
@@ -933,26 +637,6 @@ cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
 }
 
 cudaError_t tq_launch_logits(const LogitsParams& p, cudaStream_t st) {
-    // one launch when every CTA's queries fit its shared memory (d, m <= 128, g <= 4 and CTAs
-    // that span at most kMaxCS streams)
-    if (p.nb > 0 && p.t.D == 128 && p.t.Mp == 128 && p.ntiles == 1) {
-        static TqLaunchCache c1, c2, c3;
-        cudaError_t e = cudaSuccess;
-        int grid = 0;
-        switch (p.t.B) {
-            case 1: grid = fused_grid<1>(p, c1, &e); break;
-            case 2: grid = fused_grid<2>(p, c2, &e); break;
-            case 3: grid = fused_grid<3>(p, c3, &e); break;
-        }
-        if (e != cudaSuccess) return e;
-        if (grid > 0) {
-            switch (p.t.B) {
-                case 1: return launch_fused<1>(p, grid, st);
-                case 2: return launch_fused<2>(p, grid, st);
-                case 3: return launch_fused<3>(p, grid, st);
-            }
-        }
-    }
     cudaError_t e = tq_launch_logits_prologue(p, st);
     if (e != cudaSuccess) return e;
     if (p.nb == 0) return cudaSuccess;

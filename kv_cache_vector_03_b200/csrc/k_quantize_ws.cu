@@ -3,37 +3,41 @@
 // vector-search compression", sections "Random rotation and scalar quantization" and "QJL
 // residual correction"; a2a-mcp.org "What is TurboQuant", stage 1).
 //
-// One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with 18 warps:
+// One persistent CTA per SM walks tiles of 128 vectors (four blocks of 32) with 19 warps:
 //   warp 16 (one thread)  TMA: the tile's raw bf16 rows, as four 32-row boxes per 64-column
 //                         K-block, straight into the 128-byte-swizzled K-major operand layout
-//                         (two stages); and the rotation Y = X (Pi_1 + Pi_2 + Pi_3)^T on the
+//                         (two stages);
+//   warp 17 (one thread)  the rotation Y = X (Pi_1 + Pi_2 + Pi_3)^T on the
 //                         tensor cores, three bf16 passes whose sum is the fp32 rotation applied
-//                         to the exact bf16 input, into TMEM, with X first copied from shared
-//                         memory into TMEM (tcgen05.cp) so that the passes read only Pi there;
-//   warp 17 (one thread)  the sketch Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo + lo.hi)
+//                         to the exact bf16 input (one pass when Pi is a +-1/sqrt(d) Hadamard
+//                         rotation, whose scaled image is exactly +-1), into TMEM;
+//   warp 18 (one thread)  the sketch Z = (R_hi + R_lo)(256 M)^T on fp16 (hi.hi + hi.lo + lo.hi)
 //                         with the residual operand R read from TMEM, as soon as the epilogue
-//                         has written it (the two issuers wait on their own events);
+//                         has written it;
 //   warps 0-15            epilogue: warps 0-7 take even tiles, 8-15 odd ones; in each group
-//                         warp w reads TMEM lanes 32 (w mod 4) .. +31 (one vector per thread)
-//                         and columns 64 ((w / 4) mod 2) .. +63:
-//                           |x| = |Y row| over all 128 columns (Pi is orthogonal), per-row
-//                           thresholds t_k |x| and centroids, the code planes from sign bits,
-//                           the scaled residual r |x| 2^k split into an integer-valued fp16 hi
-//                           part and an fp16 lo part written to TMEM, gamma^2 (the two column
-//                           halves meet through shared memory); then the sign plane from Z.
+//                         warp w owns rows 32 (w mod 4) .. +31 (one vector per thread) and the
+//                         column half (w / 4) mod 2:
+//                           |x| from the raw bf16 row in shared memory while Y is computed; per-row
+//                           thresholds t_k |x| and centroids; from Y the code planes (sign bits),
+//                           the scaled residual r |x| 2^k split into an integer-valued fp16 hi part
+//                           and an fp16 lo part written to TMEM, gamma^2; then the sign plane from Z.
 // Resident in shared memory: Pi_1..3 (bf16) and 256 M hi/lo (fp16), 160 KB, loaded once by
 // bulk copies from the prepared images; two 32 KB stages of X. TMEM (512 columns): per tile
-// parity 128 columns for Y then Z, and 128 for the residual operand (hi 64 | lo 64).
+// parity two 128-column regions that trade roles on each use: one takes Y and then Z, the
+// other the residual operand (hi 64 | lo 64). So the next Y of a parity starts as soon as Z
+// has consumed the residual, while the epilogue still reads the signs from the other region.
 #include <cuda.h>
 
 #include <algorithm>
 #include <atomic>
 
 #include "tq_device.cuh"
+#include "tq_tc.cuh"
 
 namespace {
+using namespace tqtc;
 
-constexpr int kWsThreads = 576;
+constexpr int kWsThreads = 608;
 constexpr int kTmaWarp = 16, kMmaWarp = 17;   // warps 0-15: epilogue
 constexpr uint32_t kMat = 32768;          // one 128 x 128 16-bit operand
 constexpr uint32_t kWaitLimit = 1u << 22;
@@ -45,105 +49,21 @@ constexpr uint32_t oX = 5 * kMat;         // X stage 0, 1 (bf16)
 constexpr uint32_t oG2 = 7 * kMat;        // gamma^2 of the upper column half [tile parity][row]
 constexpr uint32_t oBar = oG2 + 2 * 128 * 4;   // barriers, then the TMEM base and the abort flag
 
-// barrier indices: per X stage, per tile parity, per (tile parity, lane quarter)
+// barrier indices: per X stage / tile parity, then per (tile parity, lane quarter)
 enum {
-    bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bTEmpty = 10, bOps = 12, bDrain = 13,
-    bG2Full = 14, bG2Empty = 22, bDrainY = 30, kNumBars = 31
+    bXFull = 0, bXEmpty = 2, bYFull = 4, bRFull = 6, bZFull = 8, bOps = 10, bDrain = 11, bDrainY = 12,
+    bG2Full = 13, bG2Empty = 21, kNumBars = 29
 };
 constexpr size_t kWsSmemUsed = (size_t)oBar + 8 * kNumBars + 8;
 constexpr size_t kWsSmem = 232448;        // the per-CTA maximum: the used bytes plus the alignment pad
 static_assert(kWsSmemUsed + 1023 <= kWsSmem, "shared memory map too large");
 
-// instruction descriptors, kind::f16, fp32 D, K-major A and B, M = N = 128
-constexpr uint32_t kIdescF16 = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
-constexpr uint32_t kIdescBF16 = kIdescF16 | (1u << 7) | (1u << 10);
+constexpr uint32_t kIdescF16 = idesc_f16(128, 128);
+constexpr uint32_t kIdescBF16 = idesc_bf16(128, 128);
 
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 // K-step k (16 elements) of a 128 x 128 operand: K-block k / 4, 32 bytes per step inside it
 __device__ __forceinline__ uint32_t kstep(int k) { return (uint32_t)(k >> 2) * 16384u + (uint32_t)(k & 3) * 32u; }
 
-// A from TMEM (row = lane, two 16-bit elements per column), B from shared memory
-__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %3, 0;\n"
-        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %4, p;\n}\n" ::"r"(d),
-        "r"(a_tmem), "l"(b), "r"(acc), "r"(idesc));
-}
-// 128 rows x 32 bytes (one K-step of 16 16-bit elements per row) from a shared-memory
-// operand to 8 TMEM columns, row r to lane r (the layout of an A operand in TMEM)
-__device__ __forceinline__ void tmem_cp(uint32_t taddr, uint64_t sd) {
-    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sd) : "memory");
-}
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     tq_smem_addr(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-
-// 16 columns of this thread's TMEM lane, without waiting (tmem_wait_ld before use)
-__device__ __forceinline__ void tld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-// wait for this thread's TMEM loads; the registers of the last one are operands, so no use of
-// them can be scheduled before the wait
-__device__ __forceinline__ void twait(uint32_t (&r)[16]) {
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15])
-                 :
-                 : "memory");
-}
-__device__ __forceinline__ void tst8(uint32_t taddr, const uint32_t (&v)[8]) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n" ::"r"(taddr), "r"(v[0]),
-                 "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
-                 : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(a), "r"(parity)
-        : "memory");
-    return done != 0;
-}
-// Bounded wait that also gives up when another role has aborted; a wait that runs out sets
-// the abort flag itself.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile uint32_t* abort_flag) {
-    const uint32_t a = tq_smem_addr(bar);
-    for (uint32_t it = 0; it < kWaitLimit; ++it) {
-        if (mbar_try(a, parity)) return true;
-        if ((it & 31u) == 31u && *abort_flag) return false;
-    }
-    *abort_flag = 1u;
-    return false;
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(tq_smem_addr(bar)) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(tq_smem_addr(bar)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void bulk_copy(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(tq_smem_addr(bar))
-                 : "memory");
-}
 // one box of the 3-D tensor map [stream][token][coordinate] (no multicast)
 __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2,
                                           uint64_t* bar) {
@@ -156,10 +76,6 @@ __device__ __forceinline__ void tma_load3(uint32_t dst, const CUtensorMap* map, 
 
 __device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? ~0u : n <= 0 ? 0u : (1u << n) - 1u; }
 __device__ __forceinline__ uint32_t shl_in(uint32_t w, uint32_t v) { return __funnelshift_l(v, w, 1); }
-__device__ __forceinline__ uint32_t pack_half2(float a, float b) {
-    const __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
 
 struct WsParams {
     uint8_t* packed;
@@ -171,6 +87,24 @@ struct WsParams {
     TqDims t;
     TqCodebookConsts cb;
 };
+
+// sum of squares of the 128 bf16 coordinates of one row of a swizzled X stage (two K-blocks),
+// each scaled by sc; four 16-byte chunks in flight at a time
+__device__ __forceinline__ float row_ss(const uint8_t* stage, int row, float sc) {
+    float s0 = 0.f, s1 = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < 16; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + (c >> 3) * 16384 + sw128(row, c & 7));
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float lo = __uint_as_float(w[e] << 16) * sc, hi = __uint_as_float(w[e] & 0xffff0000u) * sc;
+            s0 = fmaf(lo, lo, s0);
+            s1 = fmaf(hi, hi, s1);
+        }
+    }
+    return s0 + s1;
+}
 
 // One row's worth of the code and residual work on 16 TMEM columns: codes into the low
 // 16 bits of pw[] (coordinate e at bit e), the residual operand into hw / lw (two fp16 per
@@ -245,23 +179,23 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
     if (tid == 0) {
         for (int i = 0; i < kNumBars; ++i) {
             int count = 1;
+            if (i >= bXEmpty && i < bXEmpty + 2) count = 9;       // the Y commit and the 8 warps of a tile
             if (i >= bRFull && i < bRFull + 2) count = 8;         // the 8 warps of a tile
-            if (i >= bTEmpty && i < bTEmpty + 2) count = 8;
             if (i >= bG2Full && i < bG2Full + 8) count = 32;      // every lane of the upper-half warp
             tq_mbar_init(&bars[i], count);
         }
         *s_abort = 0u;
         tq_fence_mbar_init();
     }
-    if (warp == kMmaWarp) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(tq_smem_addr(s_tmem)),
-                     "r"(512));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
+    if (warp == kMmaWarp) tmem_alloc(s_tmem, 512);
     fence_before();
     __syncthreads();
     fence_after();
     const uint32_t tmem = *s_tmem;
+    // TMEM regions of tile i (parity b = i & 1, use j = i >> 1 of that parity): Y then Z in
+    // acc(i), the residual operand in res(i); the two regions of a parity trade roles each use
+    auto acc_col = [](int i) { return 256u * (uint32_t)(i & 1) + 128u * (uint32_t)((i >> 1) & 1); };
+    auto res_col = [](int i) { return 256u * (uint32_t)(i & 1) + 128u * (uint32_t)(((i >> 1) + 1) & 1); };
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
@@ -269,10 +203,12 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             // resident operands: five 32 KB images
             mbar_expect_tx(&bars[bOps], 5 * kMat);
             for (int i = 0; i < 5; ++i) bulk_copy(sb + oPi + i * kMat, p.img + (size_t)i * kMat, kMat, &bars[bOps]);
-            // tile t of this CTA into X stage t & 1
-            auto load_tile = [&](int t) {
-                const int xs = t & 1;
-                const int64_t tile = blockIdx.x + (int64_t)t * gridDim.x;
+            int issued = 0;
+            for (int i = 0; i < n_local; ++i) {
+                const int xs = i & 1;
+                // the stage is free once Y(i - 2) and the epilogue's norm pass have read it
+                if (i >= 2 && !wait_bar(&bars[bXEmpty + xs], ((i >> 1) - 1) & 1, s_abort, kWaitLimit)) break;
+                const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
                 const int64_t left = total_blocks - tile * 4;
                 const int nvb = left < 4 ? (int)left : 4;
                 mbar_expect_tx(&bars[bXFull + xs], (uint32_t)nvb * 8192u);
@@ -283,50 +219,45 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                     for (int h = 0; h < 2; ++h)
                         tma_load3(sb + oX + xs * kMat + h * 16384 + jb * 4096, &xmap, 64 * h, tok0, s, &bars[bXFull + xs]);
                 }
-            };
-            int issued = 0;
-            for (; issued < 2 && issued < n_local; ++issued) load_tile(issued);
-            const int y_passes = (p.hdr[0] & TQ_PREP_PM1) ? 1 : 3;
-            bool ok = wait_bar(&bars[bOps], 0, s_abort);
-            for (int i = 0; ok && i < n_local; ++i) {
-                const int b = i & 1;
-                if (!wait_bar(&bars[bXFull + b], (i >> 1) & 1, s_abort)) break;
-                if (i >= 2 && !wait_bar(&bars[bTEmpty + b], ((i >> 1) - 1) & 1, s_abort)) break;
-                fence_after();
-                // X into TMEM (the residual columns of this buffer, free until the epilogue writes
-                // R after Y): the tensor cores then read only Pi from shared memory. A +-1/sqrt(d)
-                // rotation needs the first (exact +-1) piece only.
-                const uint32_t d = tmem + 128u * b, xa = sb + oX + b * kMat, xt = tmem + 256u + 128u * b;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) tmem_cp(xt + 8u * k, sdesc(xa + kstep(k)));
-                mma_commit(&bars[bXEmpty + b]);
-                for (int ps = 0; ps < y_passes; ++ps)
-#pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        mma_ts(d, xt + 8u * k, sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16, (ps | k) != 0);
-                mma_commit(&bars[bYFull + b]);
-                // the stage of tile i - 1 is refilled with tile i + 1 once Y(i - 1) has read it
-                if (i >= 1 && issued < n_local) {
-                    if (!wait_bar(&bars[bXEmpty + (b ^ 1)], ((i - 1) >> 1) & 1, s_abort)) break;
-                    load_tile(issued++);
-                }
+                issued = i + 1;
             }
-            // nothing may be in flight when the CTA exits: every Y has completed (a commit tracks
-            // all earlier MMAs of this thread), and the last load of each stage has landed (a
-            // completed phase returns at once)
-            mma_commit(&bars[bDrainY]);
-            tq_mbar_wait(&bars[bDrainY], 0, kWaitLimit);
+            // nothing may be in flight when the CTA exits (a completed phase returns at once)
             for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i)
                 tq_mbar_wait(&bars[bXFull + (i & 1)], (i >> 1) & 1, kWaitLimit);
             tq_mbar_wait(&bars[bOps], 0, kWaitLimit);
         }
     } else if (warp == kMmaWarp) {
+        // rotation issue: a +-1/sqrt(d) rotation needs the first (exact +-1) piece only
+        if (lane == 0) {
+            const int y_passes = (p.hdr[0] & TQ_PREP_PM1) ? 1 : 3;
+            bool ok = wait_bar(&bars[bOps], 0, s_abort, kWaitLimit);
+            for (int i = 0; ok && i < n_local; ++i) {
+                const int b = i & 1;
+                if (!wait_bar(&bars[bXFull + b], (i >> 1) & 1, s_abort, kWaitLimit)) break;
+                // the region takes Y(i) once Z(i - 2) has consumed the residual held there
+                if (i >= 2 && !wait_bar(&bars[bZFull + b], ((i >> 1) - 1) & 1, s_abort, kWaitLimit)) break;
+                fence_after();
+                const uint32_t d = tmem + acc_col(i), xa = sb + oX + b * kMat;
+                for (int ps = 0; ps < y_passes; ++ps)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_ss(d, sdesc(xa + kstep(k)), sdesc(sb + oPi + ps * kMat + kstep(k)), kIdescBF16,
+                               (ps | k) != 0);
+                commit(&bars[bYFull + b]);
+                commit(&bars[bXEmpty + b]);
+            }
+            // every Y has completed before TMEM is released
+            commit(&bars[bDrainY]);
+            tq_mbar_wait(&bars[bDrainY], 0, kWaitLimit);
+        }
+    } else if (warp == kMmaWarp + 1) {
+        // sketch issue
         if (lane == 0) {
             for (int i = 0; i < n_local; ++i) {
                 const int b = i & 1;
-                if (!wait_bar(&bars[bRFull + b], (i >> 1) & 1, s_abort)) break;
+                if (!wait_bar(&bars[bRFull + b], (i >> 1) & 1, s_abort, kWaitLimit)) break;
                 fence_after();
-                const uint32_t d = tmem + 128u * b, r = tmem + 256u + 128u * b;
+                const uint32_t d = tmem + acc_col(i), r = tmem + res_col(i);
 #pragma unroll
                 for (int ps = 0; ps < 3; ++ps) {
                     const uint32_t ra = r + (ps == 2 ? 64u : 0u);
@@ -334,24 +265,23 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
 #pragma unroll
                     for (int k = 0; k < 8; ++k) mma_ts(d, ra + 8u * k, sdesc(mb + kstep(k)), kIdescF16, (ps | k) != 0);
                 }
-                mma_commit(&bars[bZFull + b]);
+                commit(&bars[bZFull + b]);
             }
             // every Z has completed before TMEM is released
-            mma_commit(&bars[bDrain]);
+            commit(&bars[bDrain]);
             tq_mbar_wait(&bars[bDrain], 0, kWaitLimit);
         }
     } else {
         // ------------------------------------------------------------------ epilogue
         const int par = warp >> 3, half = (warp >> 2) & 1, wq = warp & 3;
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        const uint32_t tY = tmem + lane_base + 128u * par;          // Y, then Z, of this tile parity
-        const uint32_t tR = tmem + lane_base + 256u + 128u * par;   // residual operand hi | lo
         const int row = 32 * wq + lane, u = lane >> 3, gq = lane & 7;
         float* g2x = s_g2 + par * 128 + row;
         uint64_t* g2full = &bars[bG2Full + 4 * par + wq];
         uint64_t* g2empty = &bars[bG2Empty + 4 * par + wq];
+        const uint8_t* xst = sm + oX + par * kMat;   // this group's X stage
         // Y rows are the rotation scaled by the Pi_1 image factor (sqrt(d) for a +-1 rotation)
-        const float n_unscale = 1.f / reinterpret_cast<const float*>(p.hdr)[1];
+        const float y_scale = reinterpret_cast<const float*>(p.hdr)[1];
         float tb[H > 1 ? H - 1 : 1], cmg[H];
 #pragma unroll
         for (int k = 0; k < H - 1; ++k) tb[k] = p.cb.bounds[H + k];
@@ -359,7 +289,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
         for (int k = 0; k < H; ++k) cmg[k] = p.cb.cent[H + k];
         // every lane waits (and acquires); the warp continues only if all of them succeeded
         auto warp_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
-            return __all_sync(0xffffffffu, wait_bar(bar, parity, s_abort)) != 0;
+            return __all_sync(0xffffffffu, wait_bar(bar, parity, s_abort, kWaitLimit)) != 0;
         };
         int j = 0;
         for (int i = par; i < n_local; i += 2, ++j) {
@@ -369,54 +299,24 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             const int64_t tok = blk_ok ? (gb % p.nb) * 32 + lane : 0;
             const bool rvalid = blk_ok && tok < p.n_tok;
             uint8_t* blk = p.packed + (size_t)(blk_ok ? gb : 0) * p.t.block_bytes;
-            if (!warp_wait(&bars[bYFull + par], j & 1)) break;
-            fence_after();
-            // |x| from the whole rotated row (orthogonal Pi), TMEM loads one step ahead
-            float ss0 = 0.f, ss1 = 0.f, ss2 = 0.f, ss3 = 0.f;
-            {
-                uint32_t ya[16], yb[16];
-                tld16(tY, ya);
-                twait(ya);
-#pragma unroll 1
-                for (int c = 0; c < 8; c += 2) {
-                    tld16(tY + 16u * (c + 1), yb);
-#pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        ss0 = fmaf(__uint_as_float(ya[e]), __uint_as_float(ya[e]), ss0);
-                        ss1 = fmaf(__uint_as_float(ya[e + 1]), __uint_as_float(ya[e + 1]), ss1);
-                    }
-                    twait(yb);
-                    if (c + 2 < 8) tld16(tY + 16u * (c + 2), ya);
-#pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
-                        ss2 = fmaf(__uint_as_float(yb[e]), __uint_as_float(yb[e]), ss2);
-                        ss3 = fmaf(__uint_as_float(yb[e + 1]), __uint_as_float(yb[e + 1]), ss3);
-                    }
-                    if (c + 2 < 8) twait(ya);
-                }
-            }
-            float ss = (ss0 + ss1) + (ss2 + ss3);
+            const uint32_t tY = tmem + lane_base + acc_col(i);   // Y, then Z
+            const uint32_t tR = tmem + lane_base + res_col(i);   // residual operand hi | lo
+            // |x| from the raw row (exact bf16 inputs) while the tensor cores rotate it; both
+            // column halves take the whole row, in the same order
+            if (!warp_wait(&bars[bXFull + par], j & 1)) break;
+            float ss = row_ss(xst, row, 1.f);
             const bool tiny = ss < 1e-30f && ss > 0.f;
             if (__any_sync(0xffffffffu, tiny)) {
-                // a tiny vector in the warp: its sum of squares is taken again on the row scaled by
-                // 2^60 (the TMEM loads are warp-wide, so every lane takes part)
-                float acc = 0.f;
-#pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t yv[16];
-                    tld16(tY + 16u * c, yv);
-                    twait(yv);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float v = __uint_as_float(yv[e]) * 0x1p60f;
-                        acc = fmaf(v, v, acc);
-                    }
-                }
+                // a tiny vector in the warp: its sum of squares again on the whole row scaled by 2^60
+                const float acc = row_ss(xst, row, 0x1p60f);
                 if (tiny) ss = fmaxf(acc * 0x1p-120f, 0x1p-149f);
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[bXEmpty + par]);
             const float n = sqrtf(ss);
             const bool finite = isfinite(n);
-            const float ne = (n > 0.f && finite) ? n : 1.f;
+            const float ny = n * y_scale;
+            const float ne = (ny > 0.f && finite) ? ny : 1.f;
             // kap = 2^(10 - floor(log2 ne)): |residual| * ne * kap < 2^11 (integer hi part exact in fp16)
             const int ex = ((__float_as_int(ne) >> 23) & 0xff) - 127;
             const float kap = __int_as_float((127 + min(max(10 - ex, -126), 127)) << 23);
@@ -425,6 +325,8 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
             for (int k = 0; k < H - 1; ++k) th[k] = tb[k] * ne;
 #pragma unroll
             for (int k = 0; k < H; ++k) cs[k] = cmg[k] * ne * kap;
+            if (!warp_wait(&bars[bYFull + par], j & 1)) break;
+            fence_after();
             // codes and residual of this warp's 64 columns: two plane words (chunks 2 half, +1)
             float g2a = 0.f, g2b = 0.f;
             {
@@ -455,7 +357,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                     if (q == 0) twait(ya);
                 }
             }
-            asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+            twait_st();
             fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[bRFull + par]);
@@ -492,9 +394,6 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                     if (q == 0) twait(za);
                 }
             }
-            fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars[bTEmpty + par]);
             if (half == 0) {
                 if (!warp_wait(g2full, j & 1)) break;
                 g2 += *g2x;
@@ -502,7 +401,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
                 if (lane == 0) mbar_arrive(g2empty);
                 if (blk_ok) {
                     const float gam = sqrtf(g2) / (ne * kap);
-                    const uint32_t nh = rvalid ? tq_half_bits(n * n_unscale) : 0u;
+                    const uint32_t nh = rvalid ? tq_half_bits(n) : 0u;
                     const uint32_t gh = rvalid ? tq_half_bits(gam) : 0u;
                     if (rvalid && (!finite || (nh & 0x7fffu) >= 0x7c00u)) tq_raise(p.status, TQ_FLAG_RANGE);
                     reinterpret_cast<uint32_t*>(blk + p.t.sec_a)[gq * 4 + u] = nh | (gh << 16);
@@ -516,7 +415,7 @@ __global__ void __launch_bounds__(kWsThreads, 1) k_quantize_ws(const __grid_cons
     }
     if (warp == kMmaWarp) {
         fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+        tmem_dealloc(tmem, 512);
     }
 }
 

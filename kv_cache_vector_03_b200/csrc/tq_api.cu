@@ -103,19 +103,21 @@ LogitsWs logits_ws(const TqDims& t, int64_t n_streams, int g) {
     return w;
 }
 
-struct TopkWs { int nsplit, bps, n_groups; size_t qfrag, qscale, psc, pix, total; };
-TopkWs topk_ws(const TqDims& t, int64_t n_q, int64_t n_db, int k) {
+// tq_topk workspace: fp16 query operand rows of the padded query tiles, 1 / sigma per row,
+// then the per-range candidate lists
+struct TopkWs { int nsplit, n_qt, kb_mse, kb_sign, kq; int64_t n_tiles, tps; size_t qimg, qinv, psc, pix, total; };
+TopkWs topk_ws(const TqDims& t, int64_t n_q, int64_t n_db, int k, bool qjl_terms) {
     TopkWs w;
-    const int64_t nb = (n_db + 31) / 32;
-    w.n_groups = (int)((n_q + 3) / 4);
-    const int64_t qgroups = (w.n_groups + 7) / 8;
-    int64_t ns = (4 * tq_device_sms() + qgroups - 1) / qgroups;
-    ns = std::max<int64_t>(1, std::min<int64_t>(ns, nb));
-    w.bps = (int)((nb + ns - 1) / ns);
-    w.nsplit = (int)((nb + w.bps - 1) / w.bps);
+    w.n_tiles = (n_db + 127) / 128;
+    w.n_qt = (int)((n_q + 127) / 128);
+    w.kb_mse = (t.d + 63) / 64;
+    w.kb_sign = qjl_terms ? (t.m + 63) / 64 : 0;
+    w.kq = 64 * (w.kb_mse + w.kb_sign);
+    w.nsplit = tq_topk_nsplit(w.n_qt, std::max<int64_t>(1, w.n_tiles));
+    w.tps = (w.n_tiles + w.nsplit - 1) / w.nsplit;
     size_t off = TQ_STATUS_BYTES;
-    w.qfrag = off; off = align_up(off + (size_t)w.n_groups * t.nmg * 4 * 64 * 4);
-    w.qscale = off; off = align_up(off + (size_t)w.n_groups * 4 * 16);
+    w.qimg = off; off = align_up(off + (size_t)w.n_qt * 128 * (64 * (size_t)((t.d + 63) / 64 + (t.m + 63) / 64)) * 2);
+    w.qinv = off; off = align_up(off + (size_t)w.n_qt * 128 * 4);
     w.psc = off; off = align_up(off + (size_t)n_q * w.nsplit * k * 4);
     w.pix = off; off = align_up(off + (size_t)n_q * w.nsplit * k * 4);
     w.total = off;
@@ -269,7 +271,7 @@ size_t tq_workspace_bytes(const tq_codec* c, int op, int64_t a, int64_t b, int64
             return pv_ws(t, a, b, (int)cc).total;
         case TQ_OP_TOPK:
             if (!c->qjl || a < 1 || b < 1 || cc < 1 || cc > 32 || cc > b) return 0;
-            return topk_ws(t, a, b, (int)cc).total;
+            return topk_ws(t, a, b, (int)cc, true).total;
     }
     return 0;
 }
@@ -585,45 +587,32 @@ int tq_topk_est(const tq_codec* c, const void* packed_db, int64_t n_db, const fl
     if (!aligned(packed_db, 16) || !aligned(q, 4) || !aligned(idx, 8) || !aligned(score, 4) || !aligned(ws, 256))
         return TQ_ERR_ARG;
     const TqDims t = dims_of(c);
-    const TopkWs W = topk_ws(t, n_q, n_db, k);
+    const TopkWs W = topk_ws(t, n_q, n_db, k, estimator == TQ_EST_QJL);
     if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
-    if ((int64_t)((W.n_groups + 7) / 8) * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    if ((int64_t)W.n_qt * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
     const TqPrepLayout L = tq_prep_layout(t);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
-    // queries rotated once: groups of 4 queries are the heads of one prologue stream
-    LogitsParams lp;
-    std::memset(&lp, 0, sizeof(lp));
-    lp.q = q; lp.q_dtype = TQ_F32;
-    lp.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
-    lp.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
-    lp.pih = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pih);
-    lp.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
-    lp.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
-    lp.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
-    lp.qfrag = reinterpret_cast<uint32_t*>(wsb + W.qfrag);
-    lp.qscale = reinterpret_cast<float*>(wsb + W.qscale);
-    lp.status = static_cast<uint32_t*>(ws);
-    lp.n_seq = 1; lp.n_kv = W.n_groups; lp.g = 4; lp.ntiles = 1; lp.n_tok = 0; lp.nb = 0; lp.n_tail = 0;
-    lp.scale = 1.f;
-    lp.kappa = estimator == TQ_EST_MSE ? 0.f : (float)(std::sqrt(M_PI / 2.0) / c->m);
-    lp.n_heads_valid = n_q;
-    lp.t = t;
-    if ((st = codebook_consts(c, &lp.cb)) != TQ_OK) return st;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (tq_launch_logits_prologue(lp, cs) != cudaSuccess) return TQ_ERR_CUDA;
     TopkParams p;
+    std::memset(&p, 0, sizeof(p));
     p.packed = static_cast<const uint8_t*>(packed_db);
-    p.qfrag = lp.qfrag;
-    p.qscale = lp.qscale;
+    p.q = q;
+    p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
+    p.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
+    p.qimg = reinterpret_cast<uint16_t*>(wsb + W.qimg);
+    p.qinv = reinterpret_cast<float*>(wsb + W.qinv);
     p.part_score = reinterpret_cast<float*>(wsb + W.psc);
     p.part_idx = reinterpret_cast<int*>(wsb + W.pix);
     p.out_idx = idx;
     p.out_score = score;
     p.status = static_cast<uint32_t*>(ws);
-    p.n_db = n_db; p.nb = (n_db + 31) / 32; p.n_q = n_q;
-    p.k = k; p.nsplit = W.nsplit; p.blocks_per_split = W.bps; p.n_groups = W.n_groups;
+    p.n_db = n_db; p.nb = (n_db + 31) / 32; p.n_q = n_q; p.n_tiles = W.n_tiles;
+    p.k = k; p.nsplit = W.nsplit; p.tiles_per_split = (int)W.tps; p.n_qt = W.n_qt;
+    p.kb_mse = W.kb_mse; p.kb_sign = W.kb_sign; p.kq = W.kq;
+    p.d = c->d; p.m = c->m;
+    p.kappa = estimator == TQ_EST_MSE ? 0.f : (float)(std::sqrt(M_PI / 2.0) / c->m);
     p.t = t;
-    return cuda_status(tq_launch_topk(p, cs));
+    if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
+    return cuda_status(tq_launch_topk(p, static_cast<cudaStream_t>(stream)));
 }
 
 int tq_topk(const tq_codec* c, const void* packed_db, int64_t n_db, const float* q, int64_t n_q, int k, int64_t* idx,

@@ -336,16 +336,23 @@ struct PvParams {
 
 struct TopkParams {
     const uint8_t* packed;      // one stream of n_db key records
-    const uint32_t* qfrag;      // [group of 4 queries][1][nmg][4][32][2] (prologue output)
-    const float* qscale;        // [group][4][4]
+    const float* q;             // fp32 [n_q][d] queries
+    const float* piT;           // prepared PiT [D][D] and ST [D][Mp] (fp32)
+    const float* sT;
+    uint16_t* qimg;             // [n_qt * 128][kq] fp16 query operand rows (scaled by sigma)
+    float* qinv;                // [n_qt * 128] 1 / sigma
     float* part_score;          // [n_q][nsplit][k]
     int* part_idx;              // [n_q][nsplit][k]
     int64_t* out_idx;
     float* out_score;
     uint32_t* status;
-    int64_t n_db, nb, n_q;
-    int k, nsplit, blocks_per_split, n_groups;
+    int64_t n_db, nb, n_q, n_tiles;   // n_tiles: key tiles of 128
+    int k, nsplit, tiles_per_split, n_qt;
+    int kb_mse, kb_sign, kq;    // K-blocks of 64 of the two parts (kb_sign = 0: MSE-only), kq = 64 (kb_mse + kb_sign)
+    int d, m;
+    float kappa;                // sqrt(pi/2)/m, or 0 (MSE-only)
     TqDims t;
+    TqCodebookConsts cb;
 };
 
 struct AttnParams {
@@ -421,5 +428,6 @@ cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
+int tq_topk_nsplit(int64_t n_qt, int64_t n_tiles);   // key ranges per query tile
 cudaError_t tq_launch_q8_quantize(const Q8QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_q8_logits(const Q8LogitsParams& p, cudaStream_t st);

@@ -766,6 +766,32 @@ def test_mse_only_estimator():
     check_topk(gidx, gsc, all_scores, qs.astype(np.float64), np.linalg.norm(x.astype(np.float64), axis=1), 10)
 
 
+def test_topk_ties_and_query_tiles():
+    """Three tiles of 128 queries, several key ranges each, and every database record stored
+    twice: equal scores keep the lower index first, so a duplicate enters the top-k only with
+    its original, right after it."""
+    torch = torch_cuda()
+    d = m = 200
+    n, n_q, k = 1600, 300, 8
+    pi, s = ti.C5.pi(), ti.C5.s()
+    x = ti.c5_rows("db", 4096, n)
+    q = ti.c5_rows("q", 4096, n_q)
+    codec = make_codec(d, m, 2, True, pi, s)
+    packed, _ = gpu_quantize(codec, to_dev_f32(x), 1, n)
+    twice = torch.cat([packed, packed])
+    gidx, gsc = _topk_gpu(codec, twice, 2 * n, to_dev_f32(q), n_q, k)
+    idx, sbit, nhat, ghat = unpack(codec, packed, 1, n)
+    c, _ = _cb(d, 2)
+    sc = oracle.logits(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, q.astype(np.float64), qjl=True)
+    xn = np.linalg.norm(x.astype(np.float64), axis=1)
+    check_topk(gidx, gsc, np.concatenate([sc, sc], axis=1), q.astype(np.float64), np.concatenate([xn, xn]), k)
+    for r in range(n_q):
+        row = gidx[r].tolist()
+        for pos, i in enumerate(row):
+            if i >= n:
+                assert pos > 0 and row[pos - 1] == i - n and gsc[r][pos] == gsc[r][pos - 1], (r, row)
+
+
 def test_topk_d128_codec():
     d = m = 128
     pi, s = ti.haar_rotation(d, 111), ti.gaussian_sketch(m, d, 112)
