@@ -490,7 +490,25 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
         "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA-graph replays of 12 calls"}
-    del keys, q8s
+    # the asymmetric decode step fused: 8-bit keys, 4-bit TurboQuant values, 128 bf16 tail tokens
+    vcodec = tq.Codec(d, 0, 4, False, torch.from_numpy(ti.C3.pi().astype(np.float32)), None)
+    vals = torch.randn((n_kv, n_all, d), generator=gen, device="cuda").to(torch.bfloat16)
+    vpacks = []
+    for _ in range(copies):
+        pv_ = torch.empty(vcodec.packed_bytes(n_kv, n_tok), dtype=torch.uint8, device="cuda")
+        tq.tq_quantize(vcodec, vals, n_kv, n_tok, n_all * d, pv_, tq.workspace(256))
+        vpacks.append(pv_)
+    tail_v = vals[:, n_tok:].contiguous()
+    ao = torch.empty((1, n_kv * 4, d), dtype=torch.float32, device="cuda")
+    aws = tq.workspace(tq.tq_attention_q8_workspace_bytes(vcodec, 1, n_kv, n_tok, 4, n_tail))
+    ms = time_graph(torch, lambda i: tq.tq_attention_q8(vcodec, q8s[i % copies], vpacks[i % copies], 1, n_kv, n_tok, q,
+                                                        4, tail, tail_v, n_tail, 1.0 / math.sqrt(d), ao, aws), copies)
+    byts = n_kv * n_tok * (136 + vcodec.record_bytes()) + 2 * n_kv * n_tail * d * 2 + ao.numel() * 4
+    out["c2_llama8b_decode_attention_q8_keys_v4"] = {
+        "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
+        "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA-graph replays of 12 calls"}
+    del keys, q8s, vals, vpacks
     # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
     n_kv, n_tok, g = 8, 131072, 4
     vals = torch.randn((n_kv, n_tok, d), generator=gen, device="cuda").to(torch.bfloat16)

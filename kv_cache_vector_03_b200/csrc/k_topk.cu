@@ -15,7 +15,7 @@
 //                   warp 0      bulk copies of raw key tiles (4 blocks of 32 records) into a
 //                               3-stage ring;
 //                   warp 1      one thread issues the MMAs: A = the 128 query rows, resident in
-//                               TMEM; B = K-blocks of 64 coordinates x 128 keys from a 6-slot
+//                               TMEM; B = K-blocks of 64 coordinates x 128 keys from an 8-slot
 //                               shared ring; D = 128 x 128 fp32 scores in TMEM, double buffered;
 //                               K-steps of 16 coordinates past d (resp. m) are skipped;
 //                   warps 2-9   expand each raw tile into the fp16 B operand (128-byte swizzled,
@@ -23,9 +23,10 @@
 //                               two coordinates, sign pairs as gamma with the sign bits set from
 //                               a nibble table, |x| as fp32 for the epilogue;
 //                   warps 10-13 one thread per query row: scores of 128 keys per tile read from
-//                               TMEM, times |x|, against the row's threshold (its current k-th
-//                               best); candidates go to the row's list in shared memory, merged
-//                               into the k best when the list fills;
+//                               TMEM, times |x|, against the row's threshold (the worst of its
+//                               k best, kept unordered in registers); candidates wait in a
+//                               per-row buffer and replace the worst entry, the warp's lanes in
+//                               step, once the tile's accumulator is released;
 //   k_topk_merge  one warp per query folds the ranges' lists.
 // Order: score descending, ties to the lower index. Rounding: the query row and the centroids
 // are rounded to fp16 (relative 2^-11 each; gamma and the signs are exact), so a score differs
@@ -43,10 +44,10 @@ using namespace tqtc;
 constexpr int kList = 128;          // slots of a merge list (k_topk_merge)
 constexpr int kThreads = 448;       // 14 warps
 constexpr int kMmaWarp = 1, kExpWarp0 = 2, kEpiWarp0 = 10;
-constexpr int kSlots = 6;           // B ring: one K-block (128 keys x 64 fp16) per slot
+constexpr int kSlots = 8;           // B ring: one K-block (128 keys x 64 fp16) per slot
 constexpr int kRaw = 3;             // raw tile stages
-constexpr int kCand = 32;           // candidate slots of a query row's list (after its k best)
 constexpr int kMaxK = 32;
+constexpr int kCandSlots = 32;      // candidate buffer slots per query row
 constexpr uint32_t kSlotBytes = 16384;
 constexpr uint32_t kWaitLimit = 1u << 22;
 
@@ -63,9 +64,8 @@ struct TopkLayout {
     static constexpr uint32_t oRing = 0;
     static constexpr uint32_t oRaw = kSlots * kSlotBytes;
     static constexpr uint32_t oNrm = oRaw + kRaw * RAWB;   // |x| fp32 [stage][128]
-    static constexpr uint32_t oLsc = oNrm + kRaw * 512;    // list scores [slot][128]
-    static constexpr uint32_t oLix = oLsc + (kMaxK + kCand) * 512;
-    static constexpr uint32_t oLut = oLix + (kMaxK + kCand) * 512;   // pair table (64 words), nibble table (16 x 8 B)
+    static constexpr uint32_t oCand = oNrm + kRaw * 512;   // candidate buffers: scores, keys [slot][128]
+    static constexpr uint32_t oLut = oCand + kCandSlots * 128 * 8;   // pair table (64 words), nibble table (16 x 8 B)
     static constexpr uint32_t oBar = oLut + 64 * 4 + 16 * 8;
     static constexpr uint32_t used = oBar + 8 * kNumBars + 16;
     static constexpr size_t smem = used + 1024;            // + alignment pad
@@ -186,7 +186,7 @@ __device__ __forceinline__ void sign_word(uint32_t nws, uint32_t gbase, const ui
 }
 
 // ------------------------------------------------------------------ the scan
-template <int B, int GD, int GM>
+template <int B, int GD, int GM, int KM>
 __global__ void __launch_bounds__(kThreads, 1) k_topk_tc(TopkParams p) {
     using Lay = TopkLayout<B, GD, GM>;
     constexpr int NPG = Lay::NPG;
@@ -198,8 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_tc(TopkParams p) {
     uint8_t* sm = raw_smem + pad;
     const uint32_t sb = raw + pad;
     float* s_nrm = reinterpret_cast<float*>(sm + Lay::oNrm);
-    float* lsc = reinterpret_cast<float*>(sm + Lay::oLsc);
-    int* lix = reinterpret_cast<int*>(sm + Lay::oLix);
+    float* s_cand = reinterpret_cast<float*>(sm + Lay::oCand);
     uint32_t* s_lut = reinterpret_cast<uint32_t*>(sm + Lay::oLut);
     uint2* s_sgn = reinterpret_cast<uint2*>(sm + Lay::oLut + 256);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Lay::oBar);
@@ -376,56 +375,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_tc(TopkParams p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(&bars[bAReady]);
         }
+        // this row's k best in registers, unordered: slots 0 .. k-1 start at (-inf, INT_MAX);
+        // slots k .. KM-1 hold (+inf, -1), which is never the worst. The worst slot (the last in
+        // "before" order) is the threshold and is the one a better score replaces.
         const int k = p.k;
-        int nk = 0, nc = 0, wpos = 0, wix = INT_MAX;
-        float wsc = -INFINITY, tau = qvalid ? -INFINITY : INFINITY;
-        // the worst of the k best: the last in "before" order
-        auto find_worst = [&]() {
-            wpos = 0; wsc = lsc[r]; wix = lix[r];
-            for (int e = 1; e < nk; ++e) {
-                const float s = lsc[e * 128 + r];
-                const int ix = lix[e * 128 + r];
-                if (before(wsc, wix, s, ix)) { wsc = s; wix = ix; wpos = e; }
+        float bsc[KM];
+        int bix[KM];
+#pragma unroll
+        for (int e = 0; e < KM; ++e) {
+            bsc[e] = e < k ? -INFINITY : INFINITY;
+            bix[e] = e < k ? INT_MAX : -1;
+        }
+        float wsc = -INFINITY;
+        int wix = INT_MAX, wpos = 0;
+        if (!qvalid) wsc = INFINITY;    // a padding row keeps nothing
+        auto insert = [&](float sv, int iv) {
+#pragma unroll
+            for (int e = 0; e < KM; ++e)
+                if (e == wpos) { bsc[e] = sv; bix[e] = iv; }
+            float w = bsc[0];
+            int wi = bix[0], wp = 0;
+#pragma unroll
+            for (int e = 1; e < KM; ++e) {
+                const bool later = before(w, wi, bsc[e], bix[e]);
+                w = later ? bsc[e] : w;
+                wi = later ? bix[e] : wi;
+                wp = later ? e : wp;
             }
+            wsc = w; wix = wi; wpos = wp;
         };
-        auto merge = [&]() {
-            for (int c = 0; c < nc; ++c) {
-                const float s = lsc[(k + c) * 128 + r];
-                const int ix = lix[(k + c) * 128 + r];
-                if (nk < k) {
-                    lsc[nk * 128 + r] = s; lix[nk * 128 + r] = ix;
-                    if (++nk == k) find_worst();
-                } else if (before(s, ix, wsc, wix)) {
-                    lsc[wpos * 128 + r] = s; lix[wpos * 128 + r] = ix;
-                    find_worst();
+        // Candidates (scores at or above the threshold) wait in this row's buffer in shared memory
+        // ([slot][row]: a warp's lanes hit consecutive words) and are inserted together, the lanes
+        // of the warp in step, once per tile after the accumulator is released, or earlier when a
+        // buffer might overflow.
+        float* cbs = s_cand;
+        int* cbi = reinterpret_cast<int*>(s_cand + kCandSlots * 128);
+        int ncb = 0;
+        auto flush = [&]() {
+            for (int c = 0; __any_sync(0xffffffffu, c < ncb); ++c) {
+                if (c < ncb) {
+                    const float v = cbs[c * 128 + r];
+                    const int iv = cbi[c * 128 + r];
+                    if (before(v, iv, wsc, wix)) insert(v, iv);
                 }
             }
-            nc = 0;
-            tau = nk == k ? wsc : -INFINITY;
+            ncb = 0;
+            __syncwarp();
         };
         auto scan16 = [&](const uint32_t (&va)[16], const float* nrm, int key0) {
-            float s[16];
+            float sv[16];
             bool any = false;
 #pragma unroll
             for (int e = 0; e < 16; e += 4) {
                 const float4 n4 = *reinterpret_cast<const float4*>(nrm + e);
-                s[e] = __uint_as_float(va[e]) * n4.x;
-                s[e + 1] = __uint_as_float(va[e + 1]) * n4.y;
-                s[e + 2] = __uint_as_float(va[e + 2]) * n4.z;
-                s[e + 3] = __uint_as_float(va[e + 3]) * n4.w;
-                any |= (s[e] >= tau) | (s[e + 1] >= tau) | (s[e + 2] >= tau) | (s[e + 3] >= tau);
+                sv[e] = __uint_as_float(va[e]) * n4.x;
+                sv[e + 1] = __uint_as_float(va[e + 1]) * n4.y;
+                sv[e + 2] = __uint_as_float(va[e + 2]) * n4.z;
+                sv[e + 3] = __uint_as_float(va[e + 3]) * n4.w;
+                any |= (sv[e] >= wsc) | (sv[e + 1] >= wsc) | (sv[e + 2] >= wsc) | (sv[e + 3] >= wsc);
             }
             if (any) {
-                // at most 16 appends: the list is merged once fewer than 16 slots are left
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
-                    if (s[e] >= tau) {
-                        lsc[(k + nc) * 128 + r] = s[e];
-                        lix[(k + nc) * 128 + r] = key0 + e;
-                        ++nc;
+                    if (sv[e] >= wsc) {
+                        cbs[ncb * 128 + r] = sv[e];
+                        cbi[ncb * 128 + r] = key0 + e;
+                        ++ncb;
                     }
-                if (nc > kCand - 16) merge();
             }
+            // room for the next 16 scores
+            if (__any_sync(0xffffffffu, ncb > kCandSlots - 16)) flush();
+            // the TMEM loads and waits that follow are warp-collective: reconverge first
+            __syncwarp();
         };
         for (int i = 0; i < nt; ++i) {
             const int ab = i & 1, st = i % kRaw;
@@ -453,15 +474,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_topk_tc(TopkParams p) {
                 mbar_arrive(&bars[bAccEmpty + ab]);
                 mbar_arrive(&bars[bRawEmpty + st]);
             }
+            if (__any_sync(0xffffffffu, ncb > 0)) flush();
         }
-        if (nc > 0) merge();
         if (qvalid && !*s_abort) {
             const float qi = p.qinv[q];
-            for (int e = 0; e < k; ++e) {
-                const size_t o = ((size_t)q * p.nsplit + split) * k + e;
-                p.part_score[o] = e < nk ? lsc[e * 128 + r] * qi : -INFINITY;
-                p.part_idx[o] = e < nk ? lix[e * 128 + r] : INT_MAX;
-            }
+#pragma unroll
+            for (int e = 0; e < KM; ++e)
+                if (e < k) {
+                    const size_t o = ((size_t)q * p.nsplit + split) * k + e;
+                    const bool got = bix[e] != INT_MAX;
+                    p.part_score[o] = got ? bsc[e] * qi : -INFINITY;
+                    p.part_idx[o] = got ? bix[e] : INT_MAX;
+                }
         }
     }
     __syncthreads();
@@ -499,16 +523,22 @@ __global__ void __launch_bounds__(256) k_topk_merge(TopkParams p) {
     }
 }
 
-template <int B, int GD, int GM>
-cudaError_t launch_scan(const TopkParams& p, cudaStream_t st) {
+template <int B, int GD, int GM, int KM>
+cudaError_t launch_scan_k(const TopkParams& p, cudaStream_t st) {
     using Lay = TopkLayout<B, GD, GM>;
     static_assert(Lay::smem <= 232448, "top-k shared memory map too large");
-    auto kern = k_topk_tc<B, GD, GM>;
+    auto kern = k_topk_tc<B, GD, GM, KM>;
     static TqLaunchCache cache;
     cudaError_t e = tq_kernel_setup(kern, kThreads, Lay::smem, cache, nullptr, nullptr);
     if (e != cudaSuccess) return e;
     kern<<<(unsigned)((int64_t)p.n_qt * p.nsplit), kThreads, Lay::smem, st>>>(p);
     return cudaGetLastError();
+}
+
+// the row's k best live in registers: 16 slots for k <= 16, 32 otherwise
+template <int B, int GD, int GM>
+cudaError_t launch_scan(const TopkParams& p, cudaStream_t st) {
+    return p.k <= 16 ? launch_scan_k<B, GD, GM, 16>(p, st) : launch_scan_k<B, GD, GM, 32>(p, st);
 }
 
 }  // namespace
