@@ -507,6 +507,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_q8_split(AttnParams
     __shared__ uint64_t bars[kAttnWarps][NS];
     __shared__ uint4 s_q[4][2][8];   // per head: hi / lo bytes of the int16 query, per 16-coordinate column
     __shared__ float s_qs[4];        // scale * fixed-point step
+    __shared__ __align__(16) float s_qf[4][128];   // the query heads in fp32 (tail logits)
 
     const int G = p.g, d = p.d;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -545,6 +546,7 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_q8_split(AttnParams
             hi[k] = (qi + 128) >> 8;
             lo[k] = qi - 256 * hi[k];
         }
+        *reinterpret_cast<float4*>(&s_qf[w][4 * lane]) = make_float4(v[0], v[1], v[2], v[3]);
         reinterpret_cast<uint32_t*>(&s_q[w][0][lane >> 2])[lane & 3] = q8_pack4(hi[0], hi[1], hi[2], hi[3]);
         reinterpret_cast<uint32_t*>(&s_q[w][1][lane >> 2])[lane & 3] = q8_pack4(lo[0], lo[1], lo[2], lo[3]);
         if (lane == 0) s_qs[w] = p.scale * step;
@@ -569,26 +571,21 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_q8_split(AttnParams
     };
     for (int k = 0; k < NS; ++k) issue(k);
 
-    // the first range of each stream writes the exact logits of its tail (read by the merge)
-    if (split == 0) {
-        for (int tt = w; tt < p.n_tail; tt += kAttnWarps) {
-            const uint16_t* kp = p.tail_k + ((size_t)stream * p.n_tail + tt) * d;
-            float kv[4];
+    // the exact logits of the stream's bf16 tail (read by the merge), one token per warp of the
+    // stream's ranges, against the queries in shared memory
+    for (int tt = split * kAttnWarps + w; tt < p.n_tail; tt += p.nsplit * kAttnWarps) {
+        const uint16_t* kp = p.tail_k + ((size_t)stream * p.n_tail + tt) * d;
+        float kv[4];
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int j = 4 * lane + k;
-                kv[k] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
-            }
-            for (int h = 0; h < G; ++h) {
-                float a = 0.f;
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int j = 4 * lane + k;
-                    if (j < d) a = fmaf(kv[k], tq_load_elem(p.q, p.q_dtype, (stream * G + h) * d + j), a);
-                }
-                a = tq_warp_sum(a);
-                if (lane == 0) p.tail_logit[(stream * G + h) * p.n_tail + tt] = p.scale * a;
-            }
+        for (int k = 0; k < 4; ++k) {
+            const int j = 4 * lane + k;   // d is a multiple of 8: lanes past d hold no coordinates
+            kv[k] = j < d ? __uint_as_float((uint32_t)kp[j] << 16) : 0.f;
+        }
+        for (int h = 0; h < G; ++h) {
+            const float4 qv = *reinterpret_cast<const float4*>(&s_qf[h][4 * lane]);
+            float a = fmaf(kv[0], qv.x, fmaf(kv[1], qv.y, fmaf(kv[2], qv.z, kv[3] * qv.w)));
+            a = tq_warp_sum(a);
+            if (lane == 0) p.tail_logit[(stream * G + h) * p.n_tail + tt] = p.scale * a;
         }
     }
 
@@ -784,10 +781,24 @@ cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
         }
         if (e != cudaSuccess) return e;
     }
-    // a plain launch: as a programmatic dependent of the split the merge measured 17 us slower
-    // per call at 8 x 32768 tokens
+    // a plain launch: as a programmatic dependent of the split the merge measured no faster
     k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
+}
+
+// Split CTAs of the 8-bit-key attention that fit one SM: two while the value table and the
+// rings take at most half of the 227 KB (values of up to 3 bits), else one (4-bit values: a
+// 32 KB table); the key ranges are sized so that the grid is one such wave.
+int tq_attention_q8_ctas_per_sm(int bv) {
+    constexpr size_t kStaticBound = 8192;   // the kernel's static shared arrays, rounded up
+    size_t smem = 0;
+    switch (bv) {
+        case 1: smem = q8_attn_smem<1>(); break;
+        case 2: smem = q8_attn_smem<2>(); break;
+        case 3: smem = q8_attn_smem<3>(); break;
+        default: smem = q8_attn_smem<4>(); break;
+    }
+    return smem + kStaticBound <= 232448 / 2 ? 2 : 1;
 }
 
 cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st) {

@@ -164,10 +164,11 @@ AttnWs attn_ws(const TqDims& tk, int64_t n_streams, int64_t n_tok, int g, int n_
 
 // attention over 8-bit keys: the tail logits, split partials (no query fragments)
 struct AttnQ8Ws { int nsplit, bps; size_t tl, part, ml, total; };
-AttnQ8Ws attn_q8_ws(int64_t n_streams, int64_t n_tok, int g, int n_tail) {
+AttnQ8Ws attn_q8_ws(int64_t n_streams, int64_t n_tok, int g, int n_tail, int vbits) {
     AttnQ8Ws w;
     const int64_t nb = (n_tok + 31) / 32;
-    int64_t bps = (nb * n_streams + 2 * tq_device_sms() - 1) / (2 * tq_device_sms());
+    const int64_t ctas = (int64_t)tq_attention_q8_ctas_per_sm(vbits) * tq_device_sms();   // one wave
+    int64_t bps = (nb * n_streams + ctas - 1) / ctas;
     bps = std::max<int64_t>(8, bps);
     bps = std::max<int64_t>(1, std::min<int64_t>(bps, nb));
     w.bps = (int)bps;
@@ -522,7 +523,7 @@ size_t tq_attention_q8_workspace_bytes(const tq_codec* vcodec, int64_t n_seq, in
                                        int n_tail) {
     if (check_codec(vcodec, true) != TQ_OK || vcodec->qjl || vcodec->d > 128) return 0;
     if (n_seq < 0 || n_kv < 1 || n_tok < 0 || n_tail < 0 || g < 1 || g > 4) return 0;
-    return attn_q8_ws(n_seq * n_kv, n_tok, g, n_tail).total;
+    return attn_q8_ws(n_seq * n_kv, n_tok, g, n_tail, vcodec->mse_bits).total;
 }
 
 int tq_attention_q8(const tq_codec* vcodec, const void* packed_k8, const void* packed_v, int64_t n_seq, int n_kv,
@@ -548,7 +549,7 @@ int tq_attention_q8(const tq_codec* vcodec, const void* packed_k8, const void* p
     const TqDims tv = dims_of(vcodec);
     const int64_t n_streams = n_seq * n_kv;
     if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
-    const AttnQ8Ws W = attn_q8_ws(n_streams, n_tok, g, n_tail);
+    const AttnQ8Ws W = attn_q8_ws(n_streams, n_tok, g, n_tail, vcodec->mse_bits);
     if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
     if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
     uint8_t* wsb = static_cast<uint8_t*>(ws);

@@ -427,6 +427,7 @@ cudaError_t tq_launch_quantize_wide(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_quantize_ws(const QuantParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st);
 cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st);
+int tq_attention_q8_ctas_per_sm(int value_bits);
 cudaError_t tq_launch_topk(const TopkParams& p, cudaStream_t st);
 int tq_topk_nsplit(int64_t n_qt, int64_t n_tiles);   // key ranges per query tile
 cudaError_t tq_launch_q8_quantize(const Q8QuantParams& p, cudaStream_t st);
