@@ -323,6 +323,12 @@ def run_gpu(args, world, rank, local):
         also["c4_append_quantize_hadamard_rotation"] = {
             "ms": hms, "vectors_per_s": vec_per_step / (hms * 1e-3), "dense_rotation_ms": t_quant,
             "GB_per_s": quant_bytes / (hms * 1e-3) / 1e9}
+        # the same c4 logits with the MSE-only estimator (no sign-plane MMAs; same records read)
+        mms = time_calls(torch, lambda i: tq.tq_logits(codec, cache, N_SEQ, N_KV, N_TOK, q, G, None, 0, scale, out, wsl,
+                                                        stream, estimator=tq.TQ_EST_MSE), 20, 3)
+        also["c4_logits_mse_only_estimator"] = {
+            "ms": mms, "keys_per_s": keys_per_step / (mms * 1e-3), "GB_per_s": logit_bytes / (mms * 1e-3) / 1e9,
+            "frac_of_measured_hbm": logit_bytes / (mms * 1e-3) / 1e9 / peaks["hbm_gbs"], "qjl_estimator_ms": t_logit}
     line = {
         "metric": METRIC, "value": keys_per_step * world / (ms_step * 1e-3), "unit": "keys/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,

@@ -408,12 +408,14 @@ struct FlatWalk {
 };
 
 // NP = estimator code planes, GD/GM = 128-coordinate groups of code / sign planes,
-// B = stored code planes, NT = n-tiles of 4 query heads, NS = ring stages per warp.
-template <int B, int GD, int GM, int NT, int NS>
+// B = stored code planes, NT = n-tiles of 4 query heads, NS = ring stages per warp;
+// QJL = false (the MSE-only estimator, kappa = 0) runs no sign-plane MMAs.
+template <int B, int GD, int GM, int NT, int NS, bool QJL>
 __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParams p) {
     constexpr int NP = B == 3 ? 4 : B;
     constexpr int NPG = B * GD + GM;       // stored plane groups
-    constexpr int NMG = NP * GD + GM;      // MMA plane groups
+    constexpr int NMG = NP * GD + GM;      // MMA plane groups of the fragments
+    constexpr int NMG_RUN = QJL ? NMG : NP * GD;   // the groups this variant multiplies
     constexpr uint32_t BB = 512u * NPG + 128u;
     // exact int32 combination of the hi/lo columns while 128 * 8 kTqQueryMax * K < 2^31
     constexpr bool kIntComb = NP * GD <= 4 && GM <= 4;
@@ -445,7 +447,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     // the copies above read only keys; the query fragments come from the prologue
     tq_pdl_wait();
     const int64_t row = p.n_tok + p.n_tail;
-    uint32_t qf[NT][NMG][4][2];
+    uint32_t qf[NT][NMG_RUN][4][2];
     float4 sc[NT];
     float* orow[NT];
     bool hv[NT];
@@ -460,7 +462,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
 #pragma unroll
-                for (int mg = 0; mg < NMG; ++mg)
+                for (int mg = 0; mg < NMG_RUN; ++mg)
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const uint2 v = *reinterpret_cast<const uint2*>(
@@ -489,8 +491,12 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
         for (int mt = 0; mt < 2; ++mt) {
             // code planes accumulate in two chains (chunks c odd / even), the sign plane in one
             int accA[NT][4], accA2[NT][4], accS[NT][4];
+            if constexpr (!QJL) {
 #pragma unroll
-            for (int mg = 0; mg < NMG; ++mg) {
+                for (int n = 0; n < NT; ++n) accS[n][0] = accS[n][1] = accS[n][2] = accS[n][3] = 0;
+            }
+#pragma unroll
+            for (int mg = 0; mg < NMG_RUN; ++mg) {
                 uint32_t w0, w1;  // words of rows g (u = 2mt) and g + 8 (u = 2mt + 1)
                 if (mg < NP * GD && mg / GD == 3) {  // b0 ^ b1 ^ b2
                     const int gr = mg % GD;
@@ -569,13 +575,13 @@ __global__ void __launch_bounds__(kStreamWarps * 32) k_logits_stream(LogitsParam
     }
 }
 
-template <int B, int GD, int GM, int NT>
+template <int B, int GD, int GM, int NT, bool QJL>
 cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
     constexpr int NS = 4;
     constexpr int NPG = B * GD + GM;
     constexpr size_t BB = 512u * NPG + 128u;
     const size_t smem = (size_t)kStreamWarps * NS * BB;
-    auto kern = k_logits_stream<B, GD, GM, NT, NS>;
+    auto kern = k_logits_stream<B, GD, GM, NT, NS, QJL>;
     static TqLaunchCache cache;
     int sms = 0, per_sm = 0;
     cudaError_t e = tq_kernel_setup(kern, kStreamWarps * 32, smem, cache, &sms, &per_sm);
@@ -590,7 +596,10 @@ cudaError_t launch_stream(const LogitsParams& p0, cudaStream_t st) {
 
 template <int B, int GD, int GM>
 cudaError_t launch_nt(const LogitsParams& p, cudaStream_t st) {
-    return p.ntiles == 1 ? launch_stream<B, GD, GM, 1>(p, st) : launch_stream<B, GD, GM, 2>(p, st);
+    // the MSE-only estimator (kappa = 0) multiplies no sign planes
+    if (p.kappa == 0.f)
+        return p.ntiles == 1 ? launch_stream<B, GD, GM, 1, false>(p, st) : launch_stream<B, GD, GM, 2, false>(p, st);
+    return p.ntiles == 1 ? launch_stream<B, GD, GM, 1, true>(p, st) : launch_stream<B, GD, GM, 2, true>(p, st);
 }
 
 }  // namespace
