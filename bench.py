@@ -323,6 +323,21 @@ def run_gpu(args, world, rank, local):
         also["c4_append_quantize_hadamard_rotation"] = {
             "ms": hms, "vectors_per_s": vec_per_step / (hms * 1e-3), "dense_rotation_ms": t_quant,
             "GB_per_s": quant_bytes / (hms * 1e-3) / 1e9}
+        # the query prologue (query rotation, sketch and operand fragments of the 2048 heads)
+        # followed by one 32-key block per stream, with the dense rotation and with the
+        # Hadamard one, whose query rotation runs as a fast Walsh-Hadamard transform; then the
+        # whole c4 logits call under the Hadamard codec (same records)
+        pro_ms = time_graph(torch, lambda i: tq.tq_logits(codec, cache, N_SEQ, N_KV, 32, q, G, None, 0, scale, out,
+                                                           wsl), 20)
+        hpro_ms = time_graph(torch, lambda i: tq.tq_logits(hcodec, cache, N_SEQ, N_KV, 32, q, G, None, 0, scale, out,
+                                                            wsl), 20)
+        hlog_ms = time_calls(torch, lambda i: tq.tq_logits(hcodec, cache, N_SEQ, N_KV, N_TOK, q, G, None, 0, scale,
+                                                            out, wsl, stream), 20, 3)
+        also["c4_query_prologue_plus_one_block"] = {"dense_rotation_ms": pro_ms, "walsh_hadamard_ms": hpro_ms,
+                                                    "q_heads": N_SEQ * N_KV * G, "keys_per_stream": 32,
+                                                    "timing": "CUDA graph of 20 calls, inputs in L2"}
+        also["c4_logits_hadamard_rotation"] = {"ms": hlog_ms, "keys_per_s": keys_per_step / (hlog_ms * 1e-3),
+                                               "dense_rotation_ms": t_logit}
         # the same c4 logits with the MSE-only estimator (no sign-plane MMAs; same records read)
         mms = time_calls(torch, lambda i: tq.tq_logits(codec, cache, N_SEQ, N_KV, N_TOK, q, G, None, 0, scale, out, wsl,
                                                         stream, estimator=tq.TQ_EST_MSE), 20, 3)

@@ -40,14 +40,18 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
 // Prologue. Grid (ceil(heads / HPC), 1 + ceil(n_tail / 16)), 512 threads; each CTA owns HPC
 // (4, 8 or 16) consecutive query heads (rows s*g + h of q), chosen so that about one CTA per
 // SM covers all heads: the kernel is latency-bound and every CTA pays one matrix load.
-//   y = 0: 1. q' = Pi q and q'' = S q as one [HPC x d] x [d x (D + Mp)] product against
-//             (Pi^T | S^T), whose rows arrive by bulk copies of 32 KB: all four chunks at once
-//             for D + Mp <= 256 (each used as it lands), else 16-row chunks in two stages. Thread (row slice, head quad,
-//             column quad) keeps 4 heads x 4 columns (x 2 for wide codecs); the row slices are
-//             added in shared memory.
+//   y = 0: 1. q' = Pi q and q'' = S q.
+//             D = Mp = 128: both products from one A operand (the 16 query rows, fp16 hi/lo) on
+//             mma.sync against the prepared swizzled images of 256 Pi and sigma_S S, which arrive
+//             by two bulk copies; for a Sylvester-ordered Hadamard Pi, q' is a fast Walsh-Hadamard
+//             transform in registers instead. Row maxima meet in shared memory by atomics.
+//             Wider codecs: one [HPC x d] x [d x (D + Mp)] FFMA product against (Pi^T | S^T),
+//             whose rows arrive by bulk copies of 32 KB in two stages; thread (row slice, head
+//             quad, column quad) keeps 4 heads x 8 columns; row slices add up in shared memory.
 //          2. per-head max -> fixed-point steps dA (codes, all planes) and dS (signs).
-//          3. one thread per fragment word: it rounds its four coordinates, packs their hi and
-//             lo bytes into two words and stores them; warp sums give the per-head constants.
+//          3. one warp per (head, plane group), one fragment word pair per lane: it rounds its
+//             four coordinates, packs their hi and lo bytes and stores them; warp sums give
+//             the per-head constants.
 //   y > 0: exact logits of 16 tail tokens for the CTA's heads, one warp per token.
 constexpr int kTailTok = 16;   // tail tokens per tail CTA (one per warp)
 // matrix rows per bulk-copied chunk (32 KB) and stages: 256-wide codecs hold all four chunks
@@ -104,12 +108,11 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         return;
     }
 
+    // MMA path (D + Mp = 256): qo [16][256] (q' then q''), A hi/lo, the four B images.
     // FFMA path (wide codecs): qT [256][HPC] query transposed, then qo [HPC][W].
-    // MMA path (D + Mp = 256): qo [16][256], then the operand tiles.
     float* qT = sm;
     float* qo = NR == 1 ? sm : qT + 256 * HPC;   // q' (0..D-1) then q'' (D..W-1)
-    __shared__ float s_inv[2][HPC], s_step[2][HPC];
-    __shared__ int s_sum[2][HPC];
+    __shared__ uint32_t s_max[2][HPC];   // max |q'|, max |q''| per head (fp32 bits)
     __shared__ uint64_t s_bar[4];   // matrix chunk stages (two bulk copies each)
     const int nmg = T.nmg;
     if (tid == 0) {
@@ -124,17 +127,28 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         uint4* fz = reinterpret_cast<uint4*>(p.qfrag + (size_t)st0 * frag_words);
         for (int e = tid; e < (st1 - st0) * frag_words / 4; e += blockDim.x) fz[e] = make_uint4(0, 0, 0, 0);
     }
-    if (tid < 2 * HPC) s_sum[tid / HPC][tid % HPC] = 0;
+    if (tid < 2 * HPC) s_max[tid / HPC][tid % HPC] = 0u;
     if constexpr (NR == 1) {
-        // 1. product on the fp16 tensor cores (mma.sync m16n8k16, hi/lo split passes):
-        //    q' = Pi q (A = queries, 16 rows, B = 256 Pi), then q'' = M q' = S q (B = 256 M,
-        //    M = S Pi^T). Warp w owns output columns 8w .. 8w + 7 of both products.
+        // 1. q' = Pi q and q'' = S q on the fp16 tensor cores (mma.sync m16n8k16, operands split
+        //    into fp16 hi + lo, three passes), both from the same A = the 16 query rows; warp w
+        //    owns output columns 8w .. 8w + 7 of each product. B = the prepared images of 256 Pi
+        //    and sigma_S S (128-byte swizzled, row = output coordinate), one bulk copy each.
+        //    A Sylvester-ordered Hadamard Pi = H diag(s) / sqrt(d) skips its images: each warp
+        //    applies it to its own head as a fast Walsh-Hadamard transform in registers.
         uint8_t* at = reinterpret_cast<uint8_t*>(sm + 16 * 256);   // A hi, A lo [16][256 B]
-        uint8_t* bt = at + 2 * 16 * 256;                            // Pi hi, Pi lo, M hi, M lo [128][256 B]
-        __shared__ float s_qsc[16];
+        uint8_t* bt = at + 2 * 16 * 256;                            // Pi hi, Pi lo, S hi, S lo
+        __shared__ float s_qa[16];
         const uint32_t sat = tq_smem_addr(at), sbt = tq_smem_addr(bt);
-        // every global load of this phase is issued before any is used: the query row of
-        // this warp's head, then the 16 B-tile chunks of this thread
+        const uint32_t flags = __ldg(p.hdr);
+        const bool wht = (flags & (TQ_PREP_PM1 | TQ_PREP_WHT)) == (TQ_PREP_PM1 | TQ_PREP_WHT);
+        const float inv_ss = 1.f / __ldg(reinterpret_cast<const float*>(p.hdr) + 3);   // a power of two
+        if (tid == 0) {
+            if (wht) tq_mbar_arrive(&s_bar[0]);
+            else tq_bulk_load(bt, p.pimg, 2 * (uint32_t)kTqImageBytes, &s_bar[0]);
+            tq_bulk_load(bt + 2 * kTqImageBytes, p.pimg + 2 * kTqImageBytes, 2 * (uint32_t)kTqImageBytes,
+                         &s_bar[0]);
+        }
+        // the query row of this warp's head: lane l holds coordinates 4l .. 4l + 3
         float xq[4];
         {
             const int h = wid;   // 16 warps, 16 rows
@@ -145,84 +159,146 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                 xq[k] = ok && j < d ? tq_load_elem(p.q, p.q_dtype, (int64_t)(h_base + h) * d + j) : 0.f;
             }
         }
-        {   // B tiles, swizzled rows
-            const uint16_t* srcs[4] = {p.pih, p.pil, p.mh, p.ml};
-            uint4 v[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int e = tid + kPrologueThreads * k;
-                const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
-                v[k] = __ldg(reinterpret_cast<const uint4*>(srcs[m] + row * 128 + ch * 8));
-            }
-#pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                const int e = tid + kPrologueThreads * k;
-                const int m = e >> 11, row = (e >> 4) & 127, ch = e & 15;
-                *reinterpret_cast<uint4*>(bt + m * 32768 + tq_swz256(row, ch)) = v[k];
-            }
-        }
-        // A rows: warp w = head w; lane l holds coordinates 4l .. 4l + 3, scaled per row by a power
-        // of two (max in [2^14, 2^15)) and split into binary16 hi + lo
-        auto put_row = [&](int row, const float (&x)[4], float scale_of_max) {
-            float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+        // A row: scaled by a power of two (max in [2^14, 2^15)) and split into binary16 hi + lo;
+        // a_lo: some lo part is nonzero (a bf16 or fp16 query is exact in the hi part)
+        bool a_lo = false;
+        {
+            float mx = fmaxf(fmaxf(fabsf(xq[0]), fabsf(xq[1])), fmaxf(fabsf(xq[2]), fabsf(xq[3])));
             mx = tq_warp_max(mx);
             int ex = 0;
             if (mx > 0.f && isfinite(mx)) ex = min(max(14 - (((__float_as_int(mx) >> 23) & 0xff) - 127), -126), 126);
             const float sc = __int_as_float((127 + ex) << 23);
-            const __half2 h0 = __floats2half2_rn(x[0] * sc, x[1] * sc), h1 = __floats2half2_rn(x[2] * sc, x[3] * sc);
+            const __half2 h0 = __floats2half2_rn(xq[0] * sc, xq[1] * sc), h1 = __floats2half2_rn(xq[2] * sc, xq[3] * sc);
             const float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
-            const __half2 l0 = __floats2half2_rn(x[0] * sc - f0.x, x[1] * sc - f0.y);
-            const __half2 l1 = __floats2half2_rn(x[2] * sc - f1.x, x[3] * sc - f1.y);
-            const uint32_t off = tq_swz256(row, lane >> 1) + (lane & 1) * 8;
+            const __half2 l0 = __floats2half2_rn(xq[0] * sc - f0.x, xq[1] * sc - f0.y);
+            const __half2 l1 = __floats2half2_rn(xq[2] * sc - f1.x, xq[3] * sc - f1.y);
+            const uint32_t off = tq_swz256(wid, lane >> 1) + (lane & 1) * 8;
             *reinterpret_cast<uint2*>(at + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&h0),
                                                             *reinterpret_cast<const uint32_t*>(&h1));
             *reinterpret_cast<uint2*>(at + 4096 + off) = make_uint2(*reinterpret_cast<const uint32_t*>(&l0),
                                                                    *reinterpret_cast<const uint32_t*>(&l1));
-            if (lane == 0) s_qsc[row] = scale_of_max / sc;
-        };
-        put_row(wid, xq, 1.f / 256.f);
-        __syncthreads();
-        // one 16 x 8 output tile per warp over K = 128: A hi/lo x B hi/lo (three passes)
-        const int mi = lane >> 3, r8 = lane & 7;
-        const int a_row = (mi & 1) * 8 + r8, a_chk = mi >> 1;
-        const int b_row = 8 * wid + r8, b_chk = mi & 1;
-        const int g = lane >> 2, t = lane & 3;
-        auto tile = [&](int bm, float (&acc)[4]) {   // bm: 0 = Pi, 2 = M
-            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            if (lane == 0) s_qa[wid] = 1.f / sc;
+            a_lo = (*reinterpret_cast<const uint32_t*>(&l0) | *reinterpret_cast<const uint32_t*>(&l1)) & 0x7fff7fffu;
+        }
+        if (wht) {
+            // q' = H (s * q) / sqrt(d), s_j = sign(Pi[0][j]) (row 0 of H is all ones), read from row
+            // 0 of the Pi hi image. Butterflies of span 1 and 2 in registers, spans 4 .. d/2 between
+            // lanes l and l ^ (span / 4); only spans below d run, so the zero coordinates from d on
+            // never mix with the first d.
+            const uint2 r0 = __ldg(reinterpret_cast<const uint2*>(p.pimg + tq_sw128_offset(0, 4 * lane)));
+            const uint32_t sg[4] = {r0.x, r0.x >> 16, r0.y, r0.y >> 16};
+            float v[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) v[k] = (sg[k] & 0x8000u) ? -xq[k] : xq[k];
+            if (d > 1) {
+                const float a0 = v[0], a2 = v[2];
+                v[0] = a0 + v[1]; v[1] = a0 - v[1];
+                v[2] = a2 + v[3]; v[3] = a2 - v[3];
+            }
+            if (d > 2) {
+                const float a0 = v[0], a1 = v[1];
+                v[0] = a0 + v[2]; v[2] = a0 - v[2];
+                v[1] = a1 + v[3]; v[3] = a1 - v[3];
+            }
+#pragma unroll
+            for (int sh = 0; sh < 5; ++sh) {
+                if ((4 << sh) >= d) break;
+                const bool hi = (lane >> sh) & 1;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float o = __shfl_xor_sync(0xffffffffu, v[k], 1 << sh);
+                    v[k] = hi ? o - v[k] : v[k] + o;
+                }
+            }
+            const float inv = fabsf(__ldg(p.piT));   // |Pi[0][0]| = 1/sqrt(d) as stored
+            float mx = 0.f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                v[k] *= inv;
+                qo[wid * 256 + 4 * lane + k] = v[k];
+                mx = fmaxf(mx, fabsf(v[k]));
+            }
+            mx = tq_warp_max(mx);
+            if (lane == 0 && wid < HPC) s_max[0][wid] = __float_as_uint(mx);
+        }
+        a_lo = __syncthreads_or(a_lo);   // A rows, s_qa (and the barrier's initialisation, before anyone waits)
+        const bool landed = __syncthreads_and(tq_mbar_wait(&s_bar[0], 0u, kWaitLimit));
+        if (!landed) {
+            // the images did not land in time: record it, give the copies a bounded time to
+            // finish before the shared memory is released, and leave the fragments unwritten
+            if (tid == 0) {
+                tq_raise(p.status, TQ_FLAG_TIMEOUT);
+                tq_mbar_wait(&s_bar[0], 0u, kWaitLimit);
+            }
+            return;
+        }
+        // one 16 x 8 output tile of each product per warp over K = 128: A hi/lo x B hi/lo
+        // (hi.hi, hi.lo and, when some A lo part is nonzero, lo.hi, in separate accumulators)
+        {
+            const int mi = lane >> 3, r8 = lane & 7;
+            const int a_row = (mi & 1) * 8 + r8, a_chk = mi >> 1;
+            const int b_row = 8 * wid + r8, b_chk = mi & 1;
+            const int g = lane >> 2, t = lane & 3;
+            // 16-byte chunk c (0..15) of row r of a 128-byte swizzled image: K-block c / 8
+            auto bsw = [](int r, int c) { return (uint32_t)((c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4)); };
+            float ap[3][4], as[3][4];
+#pragma unroll
+            for (int x = 0; x < 3; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) ap[x][y] = as[x][y] = 0.f;
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc) {
-                uint32_t ah[4], al[4], bh[2], bl[2];
+                uint32_t ah[4], al[4] = {0u, 0u, 0u, 0u}, bh[2], bl[2];
                 tq_ldsm_x4(sat + tq_swz256(a_row, 2 * kc + a_chk), ah[0], ah[1], ah[2], ah[3]);
-                tq_ldsm_x4(sat + 4096 + tq_swz256(a_row, 2 * kc + a_chk), al[0], al[1], al[2], al[3]);
-                tq_ldsm_x2(sbt + bm * 32768 + tq_swz256(b_row, 2 * kc + b_chk), bh[0], bh[1]);
-                tq_ldsm_x2(sbt + (bm + 1) * 32768 + tq_swz256(b_row, 2 * kc + b_chk), bl[0], bl[1]);
-                tq_hmma(acc, ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
-                tq_hmma(acc, ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
-                tq_hmma(acc, al[0], al[1], al[2], al[3], bh[0], bh[1]);
+                if (a_lo) tq_ldsm_x4(sat + 4096 + tq_swz256(a_row, 2 * kc + a_chk), al[0], al[1], al[2], al[3]);
+                const uint32_t bo = bsw(b_row, 2 * kc + b_chk);
+                if (!wht) {
+                    tq_ldsm_x2(sbt + bo, bh[0], bh[1]);
+                    tq_ldsm_x2(sbt + (uint32_t)kTqImageBytes + bo, bl[0], bl[1]);
+                    tq_hmma(ap[0], ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                    tq_hmma(ap[1], ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                    if (a_lo) tq_hmma(ap[2], al[0], al[1], al[2], al[3], bh[0], bh[1]);
+                }
+                tq_ldsm_x2(sbt + 2 * (uint32_t)kTqImageBytes + bo, bh[0], bh[1]);
+                tq_ldsm_x2(sbt + 3 * (uint32_t)kTqImageBytes + bo, bl[0], bl[1]);
+                tq_hmma(as[0], ah[0], ah[1], ah[2], ah[3], bh[0], bh[1]);
+                tq_hmma(as[1], ah[0], ah[1], ah[2], ah[3], bl[0], bl[1]);
+                if (a_lo) tq_hmma(as[2], al[0], al[1], al[2], al[3], bh[0], bh[1]);
             }
-        };
-        float acc[4];
-        tile(0, acc);   // q' columns 8w + 2t, +1 of rows g, g + 8
-        qo[g * 256 + 8 * wid + 2 * t] = acc[0] * s_qsc[g];
-        qo[g * 256 + 8 * wid + 2 * t + 1] = acc[1] * s_qsc[g];
-        qo[(g + 8) * 256 + 8 * wid + 2 * t] = acc[2] * s_qsc[g + 8];
-        qo[(g + 8) * 256 + 8 * wid + 2 * t + 1] = acc[3] * s_qsc[g + 8];
-        __syncthreads();
-        {
-            const int h = wid;
-            float x[4];
+            // accumulator r: row g (r < 2) or g + 8, column 8w + 2t + (r & 1)
+            const float fa[2] = {s_qa[g] * (1.f / 256.f), s_qa[g + 8] * (1.f / 256.f)};
+            const float fs[2] = {s_qa[g] * inv_ss, s_qa[g + 8] * inv_ss};
+            float mp[2] = {0.f, 0.f}, ms[2] = {0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 4; ++k) x[k] = qo[h * 256 + 4 * lane + k];
-            __syncwarp();
-            put_row(h, x, 1.f / 256.f);   // A <- q'
+            for (int r = 0; r < 4; ++r) {
+                const int row = g + 8 * (r >> 1), col = 8 * wid + 2 * t + (r & 1);
+                const float vs = ((as[0][r] + as[1][r]) + as[2][r]) * fs[r >> 1];
+                qo[row * 256 + 128 + col] = vs;
+                ms[r >> 1] = fmaxf(ms[r >> 1], fabsf(vs));
+                if (!wht) {
+                    const float vp = ((ap[0][r] + ap[1][r]) + ap[2][r]) * fa[r >> 1];
+                    qo[row * 256 + col] = vp;
+                    mp[r >> 1] = fmaxf(mp[r >> 1], fabsf(vp));
+                }
+            }
+            // row maxima: the four lanes of a row group, then one shared atomic per row
+#pragma unroll
+            for (int o = 1; o < 4; o <<= 1)
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    mp[x] = fmaxf(mp[x], __shfl_xor_sync(0xffffffffu, mp[x], o));
+                    ms[x] = fmaxf(ms[x], __shfl_xor_sync(0xffffffffu, ms[x], o));
+                }
+            if (t == 0) {
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    if (g + 8 * x >= HPC) continue;
+                    if (!wht) atomicMax(&s_max[0][g + 8 * x], __float_as_uint(mp[x]));
+                    atomicMax(&s_max[1][g + 8 * x], __float_as_uint(ms[x]));
+                }
+            }
         }
-        __syncthreads();
-        tile(2, acc);   // q'' = M q'
-        qo[g * 256 + 128 + 8 * wid + 2 * t] = acc[0] * s_qsc[g];
-        qo[g * 256 + 128 + 8 * wid + 2 * t + 1] = acc[1] * s_qsc[g];
-        qo[(g + 8) * 256 + 128 + 8 * wid + 2 * t] = acc[2] * s_qsc[g + 8];
-        qo[(g + 8) * 256 + 128 + 8 * wid + 2 * t + 1] = acc[3] * s_qsc[g + 8];
-        __syncthreads();
+        __syncthreads();   // qo, s_max
     } else {
     for (int e = tid; e < 256 * HPC; e += blockDim.x) {
         const int j = e / HPC, h = e % HPC;
@@ -318,42 +394,50 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                     for (int y = 0; y < 4; ++y) atomicAdd(qo + (4 * hq + x) * W + 256 * r + 4 * cq + y, acc[r][x][y]);
         __syncthreads();
     }
+        // 2. per-head maxima (one head per warp)
+        if (wid < H) {
+            const int h = wid;
+            float ma = 0.f, ms = 0.f;
+            for (int i = lane; i < D; i += 32) ma = fmaxf(ma, fabsf(qo[h * W + i]));
+            for (int k = lane; k < Mp; k += 32) ms = fmaxf(ms, fabsf(qo[h * W + D + k]));
+            ma = tq_warp_max(ma);
+            ms = tq_warp_max(ms);
+            if (lane == 0) {
+                s_max[0][h] = __float_as_uint(ma);
+                s_max[1][h] = __float_as_uint(ms);
+            }
+        }
+        __syncthreads();
     }
-    // 2. fixed-point steps (one head per warp)
-    float amax = 0.f;
-    for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
+    // 2. fixed-point steps dA (code planes: max |q'| times the largest plane factor) and dS
+    //    (signs), 3. fragment words and 4. per-head scales: one warp per head (HPC <= 16 warps).
+    //    Lane -> chunk c, slot t, register hh of every plane group mg; byte bb of the word is
+    //    coordinate 128 gr + 32 t + 2c + hh + 8 bb, in column 2 (head % 4) (hi) or
+    //    2 (head % 4) + 1 (lo) of n-tile head / 4.
     if (wid < H) {
         const int h = wid;
-        float ma = 0.f, ms = 0.f;
-        for (int i = lane; i < D; i += 32) ma = fmaxf(ma, fabsf(qo[h * W + i]));
-        for (int k = lane; k < Mp; k += 32) ms = fmaxf(ms, fabsf(qo[h * W + D + k]));
-        ma = tq_warp_max(ma) * amax;
-        ms = tq_warp_max(ms);
-        if (lane == 0) {
-            s_step[0][h] = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
-            s_step[1][h] = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
-            s_inv[0][h] = 1.f / s_step[0][h];
-            s_inv[1][h] = 1.f / s_step[1][h];
-        }
-    }
-    __syncthreads();
-    // 3. fragment words. Item e -> head h, plane group mg, chunk c, slot t, register hh; byte bb
-    //    of the word is coordinate 128 gr + 32 t + 2c + hh + 8 bb, in column 2 (head % 4) (hi)
-    //    or 2 (head % 4) + 1 (lo) of n-tile head / 4. A warp's 32 items share h and mg.
-    const int per_head = 32 * nmg;
-    for (int e = tid; e < HPC * per_head; e += blockDim.x) {
-        const int h = e / per_head, w = e - h * per_head;
-        const int mg = w >> 5, c = (w >> 3) & 3, t = (w >> 1) & 3, hh = w & 1;
-        const bool is_code = mg < np * T.GD;
-        int sum = 0;
-        if (h < H) {
-            const int gr = is_code ? mg % T.GD : mg - np * T.GD;
-            const float coef = is_code ? 2.f * p.cb.plane_coef[mg / T.GD] : 1.f;
-            const float inv = coef * s_inv[is_code ? 0 : 1][h];
+        float amax = 0.f;
+        for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
+        const float ma = __uint_as_float(s_max[0][h]) * amax, ms = __uint_as_float(s_max[1][h]);
+        const float dA = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
+        const float dS = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
+        const float invA = 1.f / dA, invS = 1.f / dS;
+        const int gh = h_base + h, stream = gh / G, head = gh - stream * G;
+        const int GDv = NR == 1 ? 1 : T.GD;
+        const int c = lane >> 3, t = (lane >> 1) & 3, hh = lane & 1;
+        // bit s = 2c + hh of the key bytes meets this register: factor 2^(3 - s mod 4)
+        const int f = 8 >> ((2 * c + hh) & 3);
+        uint32_t* dst = p.qfrag + ((size_t)stream * p.ntiles + (head >> 2)) * nmg * 256 + c * 64 + 16 * (head & 3) +
+                        2 * t + hh;
+        int sumA = 0, sumS = 0;
+#pragma unroll 2
+        for (int mg = 0; mg < nmg; ++mg) {
+            const bool is_code = mg < np * GDv;
+            const int gr = is_code ? mg % GDv : mg - np * GDv;
+            const float inv = is_code ? 2.f * p.cb.plane_coef[mg / GDv] * invA : invS;
             const float* src = qo + h * W + (is_code ? 0 : D) + 128 * gr + 32 * t + 2 * c + hh;
             uint32_t whi = 0, wlo = 0;
-            // bit s = 2c + hh of the key bytes meets this register: factor 2^(3 - s mod 4)
-            const int f = 8 >> ((2 * c + hh) & 3);
+            int sum = 0;
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
                 const int v = __float2int_rn(src[8 * bb] * inv);
@@ -362,27 +446,24 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                 whi |= (uint32_t)(hi & 0xff) << (8 * bb);
                 wlo |= (uint32_t)(lo & 0xff) << (8 * bb);
             }
-            const int gh = h_base + h, stream = gh / G, head = gh - stream * G;
-            const size_t wi = ((size_t)stream * p.ntiles + (head >> 2)) * nmg * 256 + mg * 256 + c * 64 +
-                              16 * (head & 3) + 2 * t + hh;
-            p.qfrag[wi] = whi;
-            p.qfrag[wi + 8] = wlo;   // lane + 4 (column lo) -> word + 8
+            if (is_code) sumA += sum;
+            else sumS += sum;
+            dst[mg * 256] = whi;
+            dst[mg * 256 + 8] = wlo;   // lane + 4 (column lo) -> word + 8
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (lane == 0 && h < H) atomicAdd(&s_sum[is_code ? 0 : 1][h], sum);
-    }
-    __syncthreads();
-    // per-head scales, folding the 128 of the u8 bit bytes and the QJL factor kappa:
-    //   l = |x| (dA/128 accA - KA + gamma (kappa 2 dS/128 accS - kappa KS))
-    if (tid < H) {
-        const int gh = h_base + tid, stream = gh / G, head = gh % G;
-        const float dA = s_step[0][tid], dS = s_step[1][tid];
-        // the attention scale is folded in as well
-        const float sa = p.scale;
-        reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
-            make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)s_sum[0][tid], sa * p.kappa * 2.f * dS / 128.f,
-                        sa * p.kappa * dS * (float)s_sum[1][tid]);
+        for (int o = 16; o > 0; o >>= 1) {
+            sumA += __shfl_xor_sync(0xffffffffu, sumA, o);
+            sumS += __shfl_xor_sync(0xffffffffu, sumS, o);
+        }
+        // scales, folding the 128 of the u8 bit bytes, the QJL factor kappa and the attention
+        // scale: l = |x| (dA/128 accA - KA + gamma (kappa 2 dS/128 accS - kappa KS))
+        if (lane == 0) {
+            const float sa = p.scale;
+            reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
+                make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)sumA, sa * p.kappa * 2.f * dS / 128.f,
+                            sa * p.kappa * dS * (float)sumS);
+        }
     }
 }
 

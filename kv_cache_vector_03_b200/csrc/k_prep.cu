@@ -70,10 +70,48 @@ __global__ void k_check_pm1(PrepParams p) {
     if (!__syncthreads_and(ok) && threadIdx.x == 0) atomicAnd(&p.hdr[0], 0u);
 }
 
+// Header: whether Pi is a Sylvester-ordered randomized Hadamard rotation H diag(s) / sqrt(d)
+// with one stored magnitude: d is a power of two, every |Pi[i][j]| equals |Pi[0][0]| bit for
+// bit, and every sign is (-1)^popcount(i & j) times the sign of row 0 (H[0][j] = 1).
+__global__ void k_check_wht(PrepParams p) {
+    bool ok = (p.d & (p.d - 1)) == 0;
+    const float mag = fabsf(p.pi[0]);
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; ok && e < (int64_t)p.d * p.d;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int i = (int)(e / p.d), j = (int)(e % p.d);
+        const bool neg = p.pi[e] < 0.f, neg0 = p.pi[j] < 0.f;
+        ok = fabsf(p.pi[e]) == mag && neg == (neg0 != ((__popc((unsigned)(i & j)) & 1) != 0));
+    }
+    if (!__syncthreads_and(ok) && threadIdx.x == 0) atomicAnd(&p.hdr[0], ~TQ_PREP_WHT);
+}
+
+// Header word 2: max |S| (fp32 bits; non-negative floats order as their bit patterns).
+__global__ void k_smax(PrepParams p) {
+    float mx = 0.f;
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < (int64_t)p.m * p.d;
+         e += (int64_t)gridDim.x * blockDim.x)
+        mx = fmaxf(mx, fabsf(p.s[e]));
+    mx = tq_warp_max(mx);
+    if ((threadIdx.x & 31) == 0) atomicMax(&p.hdr[2], __float_as_uint(mx));
+}
+
+// sigma_S = 2^(7 - floor(log2 max |S|)), so that sigma_S S stays below 256 (the range of the
+// fp16 hi/lo split the Pi images use as 256 Pi)
+__device__ float s_image_scale(uint32_t max_bits) {
+    const float mx = __uint_as_float(max_bits);
+    if (!(mx > 0.f) || !isfinite(mx)) return 1.f;
+    const int ex = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+    return __int_as_float((127 + min(max(7 - ex, -126), 127)) << 23);
+}
+
 __global__ void k_prepare_images(PrepParams p) {
     const bool pm1 = (p.hdr[0] & TQ_PREP_PM1) != 0;
     const float up = pm1 ? sqrtf((float)p.d) : 1.f;
-    if (blockIdx.x == 0 && threadIdx.x == 0) reinterpret_cast<float*>(p.hdr)[1] = pm1 ? up : 1.f;
+    const float ss = s_image_scale(p.hdr[2]);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        reinterpret_cast<float*>(p.hdr)[1] = pm1 ? up : 1.f;
+        reinterpret_cast<float*>(p.hdr)[3] = ss;
+    }
     for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < 128 * 128; e += gridDim.x * blockDim.x) {
         const int i = e >> 7, j = e & 127;
         const uint32_t off = tq_sw128_offset(i, j);
@@ -89,6 +127,13 @@ __global__ void k_prepare_images(PrepParams p) {
         *reinterpret_cast<__nv_bfloat16*>(p.img + 2 * kTqImageBytes + off) = b3;
         *reinterpret_cast<uint16_t*>(p.img + 3 * kTqImageBytes + off) = p.mh[e];
         *reinterpret_cast<uint16_t*>(p.img + 4 * kTqImageBytes + off) = p.ml[e];
+        // query prologue: 256 Pi (row i = output coordinate) and sigma_S S (row = sketch row)
+        uint8_t* pro = p.img + kTqProImage * kTqImageBytes;
+        *reinterpret_cast<uint16_t*>(pro + 0 * kTqImageBytes + off) = p.pih[e];
+        *reinterpret_cast<uint16_t*>(pro + 1 * kTqImageBytes + off) = p.pil[e];
+        const double sv = (i < p.m && j < p.d) ? (double)ss * (double)p.s[(int64_t)i * p.d + j] : 0.0;
+        split_half(sv, reinterpret_cast<uint16_t*>(pro + 2 * kTqImageBytes + off),
+                   reinterpret_cast<uint16_t*>(pro + 3 * kTqImageBytes + off));
     }
 }
 
@@ -115,9 +160,15 @@ cudaError_t tq_launch_prepare(const PrepParams& p, cudaStream_t st) {
     k_prepare_split<<<296, 256, 0, st>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (p.img) {
-        // flag word: TQ_PREP_PM1 set (bytes 0x01) until an entry disproves it
-        if ((e = cudaMemsetAsync(p.hdr, 1, 4, st)) != cudaSuccess) return e;
+        // flag word: TQ_PREP_PM1 | TQ_PREP_WHT (low byte 0x03) until an entry disproves them;
+        // max |S| from zero
+        if ((e = cudaMemsetAsync(p.hdr, 0, 16, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(p.hdr, TQ_PREP_PM1 | TQ_PREP_WHT, 1, st)) != cudaSuccess) return e;
+        k_smax<<<64, 256, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
         k_check_pm1<<<64, 256, 0, st>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        k_check_wht<<<64, 256, 0, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         k_prepare_images<<<64, 256, 0, st>>>(p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -365,10 +365,8 @@ int tq_logits_run(const tq_codec* c, const void* packed, int64_t n_seq, int n_kv
     p.out = out;
     p.piT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.piT);
     p.sT = reinterpret_cast<const float*>(static_cast<uint8_t*>(c->prep) + L.sT);
-    p.pih = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pih);
-    p.pil = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.pil);
-    p.mh = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.mh);
-    p.ml = reinterpret_cast<const uint16_t*>(static_cast<uint8_t*>(c->prep) + L.ml);
+    p.pimg = L.wimg > L.img ? static_cast<uint8_t*>(c->prep) + L.img + kTqProImage * kTqImageBytes : nullptr;
+    p.hdr = reinterpret_cast<const uint32_t*>(static_cast<uint8_t*>(c->prep) + L.hdr);
     p.qfrag = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(ws) + W.qfrag);
     p.qscale = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.qscale);
     p.n_seq = n_seq; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
@@ -479,10 +477,8 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
     lp.out = reinterpret_cast<float*>(wsb + W.tl);
     lp.piT = reinterpret_cast<const float*>(kprep + L.piT);
     lp.sT = reinterpret_cast<const float*>(kprep + L.sT);
-    lp.pih = reinterpret_cast<const uint16_t*>(kprep + L.pih);
-    lp.pil = reinterpret_cast<const uint16_t*>(kprep + L.pil);
-    lp.mh = reinterpret_cast<const uint16_t*>(kprep + L.mh);
-    lp.ml = reinterpret_cast<const uint16_t*>(kprep + L.ml);
+    lp.pimg = L.wimg > L.img ? kprep + L.img + kTqProImage * kTqImageBytes : nullptr;
+    lp.hdr = reinterpret_cast<const uint32_t*>(kprep + L.hdr);
     lp.qfrag = reinterpret_cast<uint32_t*>(wsb + W.lg.qfrag);
     lp.qscale = reinterpret_cast<float*>(wsb + W.lg.qscale);
     lp.status = static_cast<uint32_t*>(ws);

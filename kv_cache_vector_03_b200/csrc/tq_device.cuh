@@ -196,6 +196,10 @@ TQ_DEVICE void tq_mbar_init(uint64_t* bar, uint32_t count) {
 TQ_DEVICE void tq_fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
 TQ_DEVICE void tq_fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 
+TQ_DEVICE void tq_mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(tq_smem_addr(bar)) : "memory");
+}
+
 TQ_DEVICE void tq_bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(tq_smem_addr(bar)), "r"(bytes)
                  : "memory");
@@ -307,7 +311,8 @@ struct LogitsParams {
     float* out;
     const float* piT;
     const float* sT;
-    const uint16_t *pih, *pil, *mh, *ml;   // fp16 hi/lo of 256 Pi and 256 M (row = output)
+    const uint8_t* pimg;   // prologue images (256 Pi hi, lo, sigma_S S hi, lo), D = Mp = 128 only
+    const uint32_t* hdr;   // prep header (rotation flags, sigma_S), with pimg
     uint32_t* qfrag;       // [stream][ntile][nmg][4][32][2]
     float* qscale;         // [stream][ntile*4][4]: dA/128, KA, 2dS/128, KS
     uint32_t* status;

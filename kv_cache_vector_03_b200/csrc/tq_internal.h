@@ -63,10 +63,14 @@ static inline TqDims tq_dims(int d, int m, int B, int qjl) {
 
 // Prepared (derived) operands, laid out in the caller's prep buffer:
 //   header (256 B: word 0 = TQ_PREP_PM1 when every entry of the d x d Pi is +-1/sqrt(d), a
-//   scaled Hadamard rotation; float word 1 = the factor by which the Pi_1 image exceeds Pi)
+//   scaled Hadamard rotation, plus TQ_PREP_WHT when moreover d is a power of two and
+//   Pi = H diag(s) / sqrt(d) with H the Sylvester Hadamard matrix, H[i][j] = (-1)^popcount(i & j);
+//   float word 1 = the factor by which the Pi_1 image exceeds Pi; word 2 = max |S| (fp32 bits);
+//   float word 3 = sigma_S, the power of two that puts max |S| sigma_S in [128, 256))
 //   | PiT fp32 [D][D] | ST fp32 [D][Mp] | MT fp32 [D][Mp]
 //   | Pi_hi, Pi_lo fp16 [D][D] | M_hi, M_lo fp16 [Mp][D]     (tensor-core quantize)
-//   | images (keys with D = Mp = 128 only): Pi_1, Pi_2, Pi_3 bf16, M_hi, M_lo fp16
+//   | images (keys with D = Mp = 128 only): Pi_1, Pi_2, Pi_3 bf16, M_hi, M_lo fp16 (quantize),
+//     then 256 Pi hi, lo and sigma_S S hi, lo fp16 (query prologue)
 //   | wide images (keys with D = Mp = 256 only): 256 Pi then 256 M, each as 8 chunks of
 //     32 KB, chunk 4 nh + kb = rows 128 nh .. +127, columns 64 kb .. +63: fp16 hi (16 KB)
 //     then lo (16 KB), each [128 rows][128 B] with the same 128-byte swizzle
@@ -81,7 +85,10 @@ static inline TqDims tq_dims(int d, int m, int B, int qjl) {
 // (row mod 8) (the 128-byte swizzle). Pi = Pi_1 + Pi_2 + Pi_3 exactly (bf16 pieces of the
 // fp32 matrix: 8 + 8 + 8 significant bits); M_hi, M_lo as above.
 #define TQ_PREP_PM1 1u
+#define TQ_PREP_WHT 2u
 constexpr size_t kTqImageBytes = 128 * 128 * 2;
+constexpr int kTqNumImages = 9;     // Pi_1..3, M_hi, M_lo, then Pi_hi, Pi_lo, S_hi, S_lo
+constexpr int kTqProImage = 5;      // first image of the query prologue
 constexpr size_t kTqWideChunk = 32768;
 struct TqPrepLayout {
     size_t hdr, piT, sT, mT, pih, pil, mh, ml, img, wimg, total;
@@ -98,7 +105,7 @@ static inline TqPrepLayout tq_prep_layout(const TqDims& t) {
     L.pil = off; off += (size_t)t.D * t.D * 2;
     L.mh = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
     L.ml = off; off += t.qjl ? (size_t)t.Mp * t.D * 2 : 0;
-    L.img = off; off += (t.qjl && t.D == 128 && t.Mp == 128) ? 5 * kTqImageBytes : 0;
+    L.img = off; off += (t.qjl && t.D == 128 && t.Mp == 128) ? kTqNumImages * kTqImageBytes : 0;
     L.wimg = off; off += (t.qjl && t.D == 256 && t.Mp == 256) ? 16 * kTqWideChunk : 0;
     L.total = off;
     return L;

@@ -491,6 +491,48 @@ def test_hadamard_rotation_path():
         check_attention(got[h * g:(h + 1) * g], want, L, lg[h * g:(h + 1) * g], n_tok, V, vnorm)
 
 
+@pytest.mark.parametrize("d,kind", [(128, "sylvester"), (64, "sylvester"), (128, "xor_rows"),
+                                    (128, "permuted_rows"), (128, "haar")])
+def test_rotation_flags_and_wht_logits(d, kind):
+    """The prepared header marks Pi = H D / sqrt(d) with H in Sylvester order (the logits
+    prologue then rotates the query by a fast Walsh-Hadamard transform and reads no Pi tile):
+    also with rows permuted by i -> i ^ c (H's rows multiply as their indices XOR, so that is
+    H D' / sqrt(d) again), not with a generic row permutation (+-1 flag alone) nor for a Haar
+    rotation (neither). Logits against the oracle on the same codes in every case."""
+    m_ = 128
+    if kind == "haar":
+        pik = ti.haar_rotation(d, 61)
+    else:
+        pik = ti.hadamard_rotation(d, 61)
+        if kind == "xor_rows":
+            pik = pik[np.arange(d) ^ 37]
+        elif kind == "permuted_rows":
+            pik = pik[np.random.default_rng(62).permutation(d)]
+    want_flags = {"sylvester": 3, "xor_rows": 3, "permuted_rows": 1, "haar": 0}[kind]
+    sk = ti.gaussian_sketch(m_, d, 63)
+    n_kv, n_tok, n_tail, g, B = 2, 333, 3, 4, 2
+    kc = make_codec(d, m_, B, True, pik, sk)
+    flags = int(kc.prep[:4].cpu().numpy().view(np.uint32)[0])
+    assert flags == want_flags, (kind, flags)
+    keys = np.stack([ti.key_stream(4, 1, h, n_tok + n_tail, d) for h in range(n_kv)])
+    pk, st = gpu_quantize(kc, to_dev_bf16(np.ascontiguousarray(keys[:, :n_tok]).reshape(-1, d)), n_kv, n_tok)
+    assert st == tq().TQ_OK
+    kidx, ksb, knh, kgh = unpack(kc, pk, n_kv, n_tok)
+    c_k, _ = _cb(d, B)
+    kf = ti.bf16_to_f64(keys)
+    qb = ti.decode_queries(14, 1, n_kv * g, d)
+    scale = 1.0 / math.sqrt(d)
+    tk = to_dev_bf16(np.ascontiguousarray(keys[:, n_tok:]))
+    lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
+    q = ti.bf16_to_f64(qb)[0]
+    for h in range(n_kv):
+        qh = q[h * g:(h + 1) * g]
+        lo = oracle.logits(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, qh, qjl=True, scale=scale)
+        _check_logits(lg[h * g:(h + 1) * g, :n_tok], lo, qh, np.linalg.norm(kf[h, :n_tok], axis=1), scale)
+        tail = oracle.exact_dot(kf[h, n_tok:], qh, scale)
+        _check_logits(lg[h * g:(h + 1) * g, n_tok:], tail, qh, np.linalg.norm(kf[h, n_tok:], axis=1), scale)
+
+
 def _unpack_q8(packed_dev, d, n_streams, n_tok):
     """Decode the 8-bit key blocks as the header describes them: codes [column][token][16 B],
     then binary16 scales [chunk][token]."""
