@@ -11,8 +11,10 @@
 // mbarrier), computes the 32 x 4 logits on the int8 tensor cores (bit planes, as tq_logits),
 // keeps a running maximum and sum per head (online softmax), turns exp(l - m) |v| into fp16
 // hi + lo MMA columns and accumulates the values, decoded through per-lane half2 tables, on the
-// fp16 tensor cores (as tq_pv). Kernel 3 (merge): one CTA per query head combines the ranges
-// (log-sum-exp), rotates the value sum by Pi^T once and adds the exact tail.
+// fp16 tensor cores (as tq_pv). Kernel 3 (merge): a cluster of four CTAs per query head combines
+// the ranges (log-sum-exp), rotates the value sum by Pi^T once and adds the exact tail.
+#include <cooperative_groups.h>
+
 #include <algorithm>
 #include <cfloat>
 
@@ -326,39 +328,44 @@ __global__ void __launch_bounds__(kAttnWarps * 32, 2) k_attn_split(AttnParams p)
     }
 }
 
-// One CTA per query head: the ranges and the exact tail under one maximum M,
+// One cluster of four CTAs per query head: the ranges and the exact tail under one maximum M,
 //   out = (Pi^T sum_s e^{m_s - M} part_s + sum_t e^{l_t - M} v_t) / (sum_s e^{m_s - M} l_s + sum_t e^{l_t - M}).
-// Every global load is issued in one round: thread (group, coordinate quad) folds every 8th
-// range (rotated-domain partial quads) and every 8th tail token (exact logit, 8-byte load of
-// 4 bf16 coordinates; a warp reads one 256-byte row) under its own running maximum, into a
-// rotated-domain and an original-domain sum; the groups then meet in shared memory.
+// CTA r of the cluster owns rotated and output coordinates 32 r .. 32 r + 31. Thread (group,
+// quad) folds every 32nd range (its quad of the rotated-domain partial) and every 32nd tail
+// token (exact logit, 8-byte load of 4 bf16 value coordinates) under its own running maximum,
+// every load issued before any is used. All four CTAs read every range maximum and tail
+// logit in the same order, so M and the denominator come out identical in each. The quarters
+// of the rotated-domain sum meet through distributed shared memory, and CTA r rotates its 32
+// output coordinates with its 32 rows of Pi^T (loaded at the start).
 constexpr int kMergeThreads = 256;
-constexpr int kMergeGroups = kMergeThreads / 32;   // 32 coordinate quads = 128 coordinates
+constexpr int kMergeCtas = 4;
+constexpr int kMergeGroups = 32;   // x 8 coordinate quads = the CTA's 32 coordinates
 
-__global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
+__global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
     const int d = p.tv.d, ns = p.nsplit, nt = p.n_tail;   // D = 128
-    const int64_t hq = blockIdx.x;   // stream * g + head
+    const int r = (int)cluster.block_rank();
+    const int64_t hq = blockIdx.x / kMergeCtas;   // stream * g + head
     const int64_t stream = hq / p.g;
-    __shared__ __align__(16) float s_acc[kMergeGroups * 128], s_tac[kMergeGroups * 128];
+    __shared__ __align__(16) float s_acc[kMergeGroups * 32], s_tac[kMergeGroups * 32];
     __shared__ __align__(16) float s_o[128];
-    __shared__ float s_t[128], s_gm[kMergeGroups], s_gl[kMergeGroups];
-    const int tid = threadIdx.x, grp = tid >> 5, qd = tid & 31;
-    // the half row of Pi^T this thread rotates with (output j = tid / 2, half tid % 2), loaded
-    // first so that its latency overlaps the partials' (d <= 128: one pair per thread)
-    const int jr = tid >> 1, hr = tid & 1;
-    const bool rv = tid < 2 * d;
-    float4 wrow[16];
+    __shared__ float s_t[32], s_w[kMergeGroups], s_gm[kMergeGroups], s_gl[kMergeGroups], s_den;
+    const int tid = threadIdx.x, grp = tid >> 3, qd = tid & 7;
+    const int c0 = 32 * r + 4 * qd;   // this thread's coordinate quad
+    // rotation: output jr = 32 r + tid / 8, sixteen coordinates 16 er .. of its row of Pi^T
+    const int jr = 32 * r + (tid >> 3), er = tid & 7;
+    float4 wrow[4];
     {
-        const float4* rowp = reinterpret_cast<const float4*>(p.piT_v + (size_t)(rv ? jr : 0) * 128 + hr * 64);
+        const float4* rowp = reinterpret_cast<const float4*>(p.piT_v + (size_t)jr * 128 + er * 16);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) wrow[k] = __ldg(rowp + k);
+        for (int k = 0; k < 4; ++k) wrow[k] = __ldg(rowp + k);
     }
     const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
-    const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * 128) + qd;
+    const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * 128 + c0);
     float m = -INFINITY, l = 0.f;
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = make_float4(0.f, 0.f, 0.f, 0.f);
-    // batches whose loads are all issued before any is used; one rescale per batch
-    constexpr int RB = 8, TB = 16;
+    constexpr int RB = 4, TB = 4;
     for (int s0 = grp; s0 < ns; s0 += RB * kMergeGroups) {
         float2 v[RB];
         float4 x[RB];
@@ -386,8 +393,8 @@ __global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
         }
     }
     const float* tl = p.tail_logit + (size_t)hq * nt;
-    const uint2* tv = reinterpret_cast<const uint2*>(p.tail_v + (size_t)stream * nt * d) + qd;
-    const bool qv = qd < d / 4;
+    const uint2* tv = reinterpret_cast<const uint2*>(p.tail_v + (size_t)stream * nt * d) + c0 / 4;
+    const bool qv = c0 / 4 < d / 4;
     for (int t0 = grp; t0 < nt; t0 += TB * kMergeGroups) {
         float lt[TB];
         uint2 vv[TB];
@@ -415,38 +422,50 @@ __global__ void __launch_bounds__(kMergeThreads) k_attn_merge(AttnParams p) {
         }
         m = mn;
     }
-    reinterpret_cast<float4*>(s_acc)[grp * 32 + qd] = a;
-    reinterpret_cast<float4*>(s_tac)[grp * 32 + qd] = b;
+    reinterpret_cast<float4*>(s_acc)[grp * 8 + qd] = a;
+    reinterpret_cast<float4*>(s_tac)[grp * 8 + qd] = b;
     if (qd == 0) { s_gm[grp] = m; s_gl[grp] = l; }
     __syncthreads();
-    float M = -INFINITY;
+    if (tid < 32) {   // group weights under the common maximum, and the denominator
+        const float gm = s_gm[tid];
+        float M = gm;
 #pragma unroll
-    for (int q = 0; q < kMergeGroups; ++q) M = fmaxf(M, s_gm[q]);
-    float den = 0.f;
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = gm > -INFINITY ? __expf(gm - M) : 0.f;
+        float den = w * s_gl[tid];
 #pragma unroll
-    for (int q = 0; q < kMergeGroups; ++q) den += s_gm[q] > -INFINITY ? __expf(s_gm[q] - M) * s_gl[q] : 0.f;
-    {
-        const int i = tid & 127;
-        const float* accp = tid < 128 ? s_acc : s_tac;
-        float v = 0.f;
-#pragma unroll
-        for (int q = 0; q < kMergeGroups; ++q)
-            if (s_gm[q] > -INFINITY) v = fmaf(__expf(s_gm[q] - M), accp[q * 128 + i], v);
-        (tid < 128 ? s_o : s_t)[i] = v;
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        s_w[tid] = w;
+        if (tid == 0) s_den = den;
     }
     __syncthreads();
-    const float inv = 1.f / den;
-    // out[j] = (<row j of Pi^T, o> + t_j) / den; the two halves meet by a shuffle of
-    // neighbouring lanes (all 256 threads take part)
+    if (tid < 64) {   // this CTA's quarter of o (threads 0-31) and of the tail sum (32-63)
+        const int i = tid & 31;
+        const float* accp = tid < 32 ? s_acc : s_tac;
+        float v = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < kMergeGroups; ++q) v = fmaf(s_w[q], accp[q * 32 + i], v);
+        if (tid < 32) s_o[32 * r + i] = v;
+        else s_t[i] = v;
+    }
+    cluster.sync();   // every quarter of o is written
+    if (tid < 128 && (tid >> 5) != r) {
+        const float* peer = cluster.map_shared_rank(s_o, (int)(tid >> 5));
+        s_o[tid] = peer[tid];
+    }
+    cluster.sync();   // o is complete here, and no CTA leaves while a peer still reads it
+    // out[j] = (<row j of Pi^T, o> + t_j) / den; the eight parts of a row meet by shuffles
     float acc = 0.f;
-    const float4* op = reinterpret_cast<const float4*>(s_o + hr * 64);
+    const float4* op = reinterpret_cast<const float4*>(s_o + er * 16);
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
+    for (int k = 0; k < 4; ++k) {
         const float4 w = wrow[k], o = op[k];
         acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    if (rv && hr == 0) p.out[(size_t)hq * d + jr] = (acc + s_t[jr]) * inv;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (er == 0 && jr < d) p.out[(size_t)hq * d + jr] = (acc + s_t[jr - 32 * r]) / s_den;
 }
 
 template <int BK, int BV>
@@ -782,7 +801,7 @@ cudaError_t tq_launch_attention(const AttnParams& p, cudaStream_t st) {
         if (e != cudaSuccess) return e;
     }
     // a plain launch: as a programmatic dependent of the split the merge measured no faster
-    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    k_attn_merge<<<(unsigned)(p.n_streams * p.g * kMergeCtas), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
 
@@ -817,6 +836,6 @@ cudaError_t tq_launch_attention_q8(const AttnParams& p, cudaStream_t st) {
         e = cudaGetLastError();
     }
     if (e != cudaSuccess) return e;
-    k_attn_merge<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    k_attn_merge<<<(unsigned)(p.n_streams * p.g * kMergeCtas), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }

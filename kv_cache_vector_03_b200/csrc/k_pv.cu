@@ -14,8 +14,10 @@
 // table that maps a 2B-bit field (two tokens' codes of one coordinate) to a half2 of
 // centroids, and multiplied on the tensor cores. The 8 warps meet at the CTA's maximum;
 // partial sums, maxima and denominators go to the workspace.
-// Kernel 2 (merge): one CTA per query head combines the partials (log-sum-exp rescale) and
-// rotates by Pi^T.
+// Kernel 2 (merge): a cluster of four CTAs per query head (one CTA for D = 256) combines the
+// partials (log-sum-exp rescale) and rotates by Pi^T.
+#include <cooperative_groups.h>
+
 #include "tq_device.cuh"
 
 namespace {
@@ -286,14 +288,117 @@ __global__ void __launch_bounds__(kPvWarps * 32, KT == 8 ? 2 : 1) k_pv_split(PvP
     }
 }
 
-// One CTA per query head: o = sum_s e^{m_s - M} part_s / sum_s e^{m_s - M} l_s, then Pi^T o.
-// Every global load of the partials is issued in one round: thread (group, coordinate quad)
-// reads the maxima, sums and partial quads of every ngrp-th range and folds them under its
-// own running maximum; the groups then meet in shared memory under the common one.
 constexpr int kMergeThreads = 256;
 
-template <int D>   // 128 or 256
-__global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
+// D = 128: one cluster of four CTAs per query head,
+//   out = Pi^T sum_s e^{m_s - M} part_s / sum_s e^{m_s - M} l_s.
+// CTA r owns rotated and output coordinates 32 r .. 32 r + 31. Thread (group, quad) folds
+// every 32nd range (its quad of the partial) under its own running maximum, every load issued
+// before any is used; all four CTAs read every range maximum in the same order, so M and the
+// denominator come out identical in each. The quarters of o meet through distributed shared
+// memory and CTA r rotates its 32 outputs with its 32 rows of Pi^T (loaded at the start).
+constexpr int kMergeCtas = 4;
+constexpr int kMergeGroups = 32;   // x 8 coordinate quads = the CTA's 32 coordinates
+
+__global__ void __cluster_dims__(kMergeCtas, 1, 1) __launch_bounds__(kMergeThreads) k_pv_merge4(PvParams p) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int d = p.t.d, ns = p.nsplit;
+    const int r = (int)cluster.block_rank();
+    const int64_t hq = blockIdx.x / kMergeCtas;   // stream * g + head
+    __shared__ __align__(16) float s_acc[kMergeGroups * 32];
+    __shared__ __align__(16) float s_o[128];
+    __shared__ float s_w[kMergeGroups], s_gm[kMergeGroups], s_gl[kMergeGroups], s_den;
+    const int tid = threadIdx.x, grp = tid >> 3, qd = tid & 7;
+    const int c0 = 32 * r + 4 * qd;
+    const int jr = 32 * r + (tid >> 3), er = tid & 7;
+    float4 wrow[4];
+    {
+        const float4* rowp = reinterpret_cast<const float4*>(p.piT + (size_t)jr * 128 + er * 16);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) wrow[k] = __ldg(rowp + k);
+    }
+    const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
+    const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * 128 + c0);
+    float m = -INFINITY, l = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    constexpr int RB = 8;
+    for (int s0 = grp; s0 < ns; s0 += RB * kMergeGroups) {
+        float2 v[RB];
+        float4 x[RB];
+#pragma unroll
+        for (int u = 0; u < RB; ++u) {
+            const int s = s0 + u * kMergeGroups;
+            v[u] = s < ns ? ml[s] : make_float2(-INFINITY, 0.f);
+            x[u] = s < ns ? src[(size_t)s * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float mn = m;
+#pragma unroll
+        for (int u = 0; u < RB; ++u) mn = v[u].y > 0.f ? fmaxf(mn, v[u].x) : mn;
+        if (mn > -INFINITY) {   // a range with weight (every range wrote its partial)
+            const float so = __expf(m - mn);
+            a.x *= so; a.y *= so; a.z *= so; a.w *= so;
+            l *= so;
+#pragma unroll
+            for (int u = 0; u < RB; ++u) {
+                const float sn = v[u].y > 0.f ? __expf(v[u].x - mn) : 0.f;
+                a.x = fmaf(sn, x[u].x, a.x); a.y = fmaf(sn, x[u].y, a.y);
+                a.z = fmaf(sn, x[u].z, a.z); a.w = fmaf(sn, x[u].w, a.w);
+                l = fmaf(sn, v[u].y, l);
+            }
+            m = mn;
+        }
+    }
+    reinterpret_cast<float4*>(s_acc)[grp * 8 + qd] = a;
+    if (qd == 0) { s_gm[grp] = m; s_gl[grp] = l; }
+    __syncthreads();
+    if (tid < 32) {   // group weights under the common maximum, and the denominator
+        const float gm = s_gm[tid];
+        float M = gm;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = gm > -INFINITY ? __expf(gm - M) : 0.f;
+        float den = w * s_gl[tid];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+        s_w[tid] = w;
+        if (tid == 0) s_den = den;
+    }
+    __syncthreads();
+    if (tid < 32) {   // this CTA's quarter of o
+        float v = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < kMergeGroups; ++q) v = fmaf(s_w[q], s_acc[q * 32 + tid], v);
+        s_o[32 * r + tid] = v;
+    }
+    cluster.sync();   // every quarter of o is written
+    if (tid < 128 && (tid >> 5) != r) {
+        const float* peer = cluster.map_shared_rank(s_o, (int)(tid >> 5));
+        s_o[tid] = peer[tid];
+    }
+    cluster.sync();   // o is complete here, and no CTA leaves while a peer still reads it
+    // out[j] = <row j of Pi^T, o> / den (its columns i >= d are zero); the eight parts of a row
+    // meet by shuffles
+    float acc = 0.f;
+    const float4* op = reinterpret_cast<const float4*>(s_o + er * 16);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float4 w = wrow[k], o = op[k];
+        acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+    if (er == 0 && jr < d) p.out[(size_t)hq * d + jr] = acc / s_den;
+}
+
+// D = 256: one CTA per query head: o = sum_s e^{m_s - M} part_s / sum_s e^{m_s - M} l_s,
+// then Pi^T o. Every global load of the partials is issued in one round: thread (group,
+// coordinate quad) reads the maxima, sums and partial quads of every ngrp-th range and folds
+// them under its own running maximum; the groups then meet in shared memory under the common
+// one.
+__global__ void __launch_bounds__(kMergeThreads) k_pv_merge256(PvParams p) {
+    constexpr int D = 256;
     const int d = p.t.d, ns = p.nsplit;
     const int64_t hq = blockIdx.x;   // stream * g + head
     __shared__ __align__(16) float s_acc[kMergeThreads * 4];   // [group][D]
@@ -302,16 +407,6 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
     const int tid = threadIdx.x;
     constexpr int nq = D / 4, ngrp = kMergeThreads / nq;
     const int grp = tid / nq, qd = tid % nq;
-    // D = 128: the half row of Pi^T this thread rotates with (output tid / 2, half tid % 2) is
-    // loaded first so that its latency overlaps the partials'
-    const int jr = tid >> 1, hr = tid & 1;
-    const bool rv = tid < 2 * d;
-    float4 wrow[D == 128 ? 16 : 1];
-    if constexpr (D == 128) {
-        const float4* rowp = reinterpret_cast<const float4*>(p.piT + (size_t)(rv ? jr : 0) * 128 + hr * 64);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) wrow[k] = __ldg(rowp + k);
-    }
     const float2* ml = reinterpret_cast<const float2*>(p.part_ml) + (size_t)hq * ns;
     const float4* src = reinterpret_cast<const float4*>(p.part + (size_t)hq * ns * D) + qd;
     float m = -INFINITY, l = 0.f;
@@ -359,21 +454,9 @@ __global__ void __launch_bounds__(kMergeThreads) k_pv_merge(PvParams p) {
     }
     __syncthreads();
     const float inv = 1.f / den;
-    // out[j] = sum_i Pi[i][j] o_i = <row j of Pi^T, o> (its columns i >= d are zero): pair
-    // (j, half), the halves joined by a shuffle of neighbouring lanes
-    if constexpr (D == 128) {
-        float acc = 0.f;
-        const float4* op = reinterpret_cast<const float4*>(s_o + hr * 64);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float4 w = wrow[k], o = op[k];
-            acc = fmaf(w.x, o.x, fmaf(w.y, o.y, fmaf(w.z, o.z, fmaf(w.w, o.w, acc))));
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        if (rv && hr == 0) p.out[(size_t)hq * d + jr] = acc * inv;
-        return;
-    }
-    // D = 256: 16-byte loads of the row; the block-uniform trip count keeps warps whole
+    // out[j] = sum_i Pi[i][j] o_i = <row j of Pi^T, o> (its columns i >= d are zero): pairs
+    // (j, half) with 16-byte loads of the row, the halves joined by a shuffle of neighbouring
+    // lanes; the block-uniform trip count keeps warps whole
     const int hl = D / 2;
     for (int e0 = 0; e0 < 2 * d; e0 += kMergeThreads) {
         const int e = e0 + tid, j = e >> 1, hf = e & 1;
@@ -424,7 +507,7 @@ cudaError_t tq_launch_pv(const PvParams& p, cudaStream_t st) {
     else if (p.t.D == 256) e = nt == 1 ? launch_b<16, 1>(p, st) : launch_b<16, 2>(p, st);
     else return cudaErrorInvalidValue;
     if (e != cudaSuccess) return e;
-    if (p.t.D == 128) k_pv_merge<128><<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
-    else k_pv_merge<256><<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
+    if (p.t.D == 128) k_pv_merge4<<<(unsigned)(p.n_streams * p.g * kMergeCtas), kMergeThreads, 0, st>>>(p);
+    else k_pv_merge256<<<(unsigned)(p.n_streams * p.g), kMergeThreads, 0, st>>>(p);
     return cudaGetLastError();
 }
