@@ -307,6 +307,28 @@ def test_pv_d200_values(B, g):
         _check_pv(got[h * g:(h + 1) * g], want, Ph.astype(np.float64), nhat[h])
 
 
+def test_pv_p_rows_unaligned():
+    """P whose rows do not start on a 16-byte boundary (a view one float into its buffer):
+    the API takes any 4-byte aligned P; parity against the oracle as for aligned rows."""
+    torch = torch_cuda()
+    d, B, g, n_tok, n_kv = 128, 3, 4, 2048, 2
+    pi = ti.C3.pi()
+    bits = np.concatenate([ti.value_stream(h, n_tok) for h in range(n_kv)])
+    codec = make_codec(d, 0, B, False, pi, None)
+    packed, _ = gpu_quantize(codec, to_dev_bf16(bits), n_kv, n_tok)
+    P = ti.logits_p(n_kv * g, n_tok)
+    buf = torch.empty(P.size + 1, dtype=torch.float32, device="cuda")
+    p_off = buf[1:].view(1, n_kv * g, n_tok)
+    p_off.copy_(torch.from_numpy(P.astype(np.float32)).view(1, n_kv * g, n_tok))
+    got = _pv_gpu(codec, packed, 1, n_kv, n_tok, p_off, g)[0]
+    idx, nhat = unpack(codec, packed, n_kv, n_tok)
+    c, _ = _cb(d, B)
+    for h in range(n_kv):
+        Ph = P[h * g:(h + 1) * g]
+        want = oracle.pv(idx[h], nhat[h], pi, c, Ph)
+        _check_pv(got[h * g:(h + 1) * g], want, Ph.astype(np.float64), nhat[h])
+
+
 def test_pv_one_hot_and_uniform():
     d, B, n_tok = 128, 3, 300
     pi = ti.C3.pi()
