@@ -513,14 +513,16 @@ def test_hadamard_rotation_path():
         check_attention(got[h * g:(h + 1) * g], want, L, lg[h * g:(h + 1) * g], n_tok, V, vnorm)
 
 
-@pytest.mark.parametrize("d,kind", [(128, "sylvester"), (64, "sylvester"), (128, "xor_rows"),
-                                    (128, "permuted_rows"), (128, "haar")])
-def test_rotation_flags_and_wht_logits(d, kind):
+@pytest.mark.parametrize("d,kind,qf32", [(128, "sylvester", False), (64, "sylvester", False), (128, "xor_rows", False),
+                                         (128, "permuted_rows", False), (128, "haar", False), (128, "sylvester", True),
+                                         (128, "haar", True)])
+def test_rotation_flags_and_wht_logits(d, kind, qf32):
     """The prepared header marks Pi = H D / sqrt(d) with H in Sylvester order (the logits
     prologue then rotates the query by a fast Walsh-Hadamard transform and reads no Pi tile):
     also with rows permuted by i -> i ^ c (H's rows multiply as their indices XOR, so that is
     H D' / sqrt(d) again), not with a generic row permutation (+-1 flag alone) nor for a Haar
-    rotation (neither). Logits against the oracle on the same codes in every case."""
+    rotation (neither). Logits against the oracle on the same codes in every case, for bf16
+    queries and for fp32 queries (whose rows carry a nonzero fp16 lo part: the third pass)."""
     m_ = 128
     if kind == "haar":
         pik = ti.haar_rotation(d, 61)
@@ -542,11 +544,16 @@ def test_rotation_flags_and_wht_logits(d, kind):
     kidx, ksb, knh, kgh = unpack(kc, pk, n_kv, n_tok)
     c_k, _ = _cb(d, B)
     kf = ti.bf16_to_f64(keys)
-    qb = ti.decode_queries(14, 1, n_kv * g, d)
     scale = 1.0 / math.sqrt(d)
     tk = to_dev_bf16(np.ascontiguousarray(keys[:, n_tok:]))
-    lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
-    q = ti.bf16_to_f64(qb)[0]
+    if qf32:
+        qf = np.random.default_rng(64).standard_normal((1, n_kv * g, d)).astype(np.float32)
+        lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_f32(qf), g, tk, n_tail, scale)[0]
+        q = qf.astype(np.float64)[0]
+    else:
+        qb = ti.decode_queries(14, 1, n_kv * g, d)
+        lg = _logits_gpu(kc, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, tk, n_tail, scale)[0]
+        q = ti.bf16_to_f64(qb)[0]
     for h in range(n_kv):
         qh = q[h * g:(h + 1) * g]
         lo = oracle.logits(kidx[h], ksb[h], knh[h], kgh[h], pik, sk, c_k, qh, qjl=True, scale=scale)
