@@ -719,6 +719,7 @@ cudaError_t launch_prologue(const LogitsParams& p, int64_t n_heads, cudaStream_t
 cudaError_t tq_launch_logits_prologue(const LogitsParams& p, cudaStream_t st) {
     const int64_t n_heads = p.n_seq * p.n_kv * p.g;
     const bool wide = p.t.D + p.t.Mp > 256;
+    if (!wide && (p.pimg == nullptr || p.hdr == nullptr)) return cudaErrorInvalidValue;   // 256-wide: images needed
     switch (prologue_hpc(n_heads)) {
         case 4: return wide ? launch_prologue<2, 4>(p, n_heads, st) : launch_prologue<1, 4>(p, n_heads, st);
         case 8: return wide ? launch_prologue<2, 8>(p, n_heads, st) : launch_prologue<1, 8>(p, n_heads, st);
