@@ -54,10 +54,9 @@ __device__ __forceinline__ size_t qf_index(int64_t stream, int ntile, int ntiles
 //             the per-head constants.
 //   y > 0: exact logits of 16 tail tokens for the CTA's heads, one warp per token.
 constexpr int kTailTok = 16;   // tail tokens per tail CTA (one per warp)
-// matrix rows per bulk-copied chunk (32 KB) and stages: 256-wide codecs hold all four chunks
-// at once (issued together, consumed as they land), wider ones cycle two stages
-__host__ __device__ constexpr int prologue_rows(int W) { return W <= 256 ? 32 : 16; }
-__host__ __device__ constexpr int prologue_stages(int W) { return W <= 256 ? 4 : 2; }
+// FFMA path (D + Mp > 256): matrix rows per bulk-copied chunk (16 rows of W fp32, at most
+// 32 KB) and the two stages they cycle through
+constexpr int kProRows = 16, kProStages = 2;
 
 template <int NR, int HPC>   // NR: 256-column groups of (Pi^T | S^T); HPC: heads per CTA
 __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsParams p) {
@@ -312,7 +311,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
     //    4cq + 256r). A chunk holds [R][D] rows of Pi^T, then [R][Mp] rows of S^T.
     {
         constexpr int NHQ = HPC / 4, KS = kPrologueThreads / (64 * NHQ);
-        const int R = prologue_rows(W), NST = prologue_stages(W), nchunk = (d + R - 1) / R;
+        const int R = kProRows, NST = kProStages, nchunk = (d + R - 1) / R;
         float* stg = qo + HPC * W;
         auto load_chunk = [&](int c) {   // one thread
             const int j0 = c * R, rows = min(R, d - j0);
@@ -691,13 +690,13 @@ static int prologue_hpc(int64_t n_heads) {
     return n_heads <= sms * 4 ? 4 : n_heads <= sms * 8 ? 8 : 16;
 }
 
-// MMA path (D + Mp = 256): qo [16][256] fp32 + A hi/lo [16][256 B] + four [128][256 B] B tiles
+// MMA path (D + Mp = 256): qo [16][256] fp32 + A hi/lo [16][256 B] + the four 32 KB B images
 constexpr size_t kPrologueSmemMma = (size_t)16 * 256 * 4 + 2 * 16 * 256 + 4 * 128 * 256;
 
 size_t tq_logits_prologue_smem(const TqDims& t, int hpc) {
     const int W = t.D + t.Mp;
     if (W <= 256) return kPrologueSmemMma;
-    return ((size_t)256 * hpc + (size_t)hpc * W + (size_t)prologue_stages(W) * prologue_rows(W) * W) * 4;
+    return ((size_t)256 * hpc + (size_t)hpc * W + (size_t)kProStages * kProRows * W) * 4;
 }
 
 // largest prologue shared memory over the supported codecs and head counts
