@@ -204,13 +204,16 @@ def test_logits_gqa_ragged_with_tail(B, g):
             _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1), scale)
 
 
-@pytest.mark.parametrize("n_seq,n_kv,g,n_tail", [(40, 4, 4, 20), (25, 8, 8, 33)])
-def test_logits_many_heads(n_seq, n_kv, g, n_tail):
+@pytest.mark.parametrize("n_seq,n_kv,g,n_tail,rot", [(40, 4, 4, 20, "haar"), (25, 8, 8, 33, "haar"),
+                                                     (37, 5, 4, 0, "hadamard"), (61, 5, 4, 3, "hadamard")])
+def test_logits_many_heads(n_seq, n_kv, g, n_tail, rot):
     """640 / 1600 query heads: the prologue takes 8 / 16 heads per CTA; tails of 20 / 33 tokens
-    span two / three tail CTAs."""
+    span two / three tail CTAs. 740 / 1220 heads with a Sylvester-ordered Hadamard rotation (the
+    query transform by butterflies): 8 / 16 heads per CTA, the last CTA holding 4."""
     d = m = 128
     B = 2
-    pi, s = ti.haar_rotation(d, 93), ti.gaussian_sketch(m, d, 94)
+    pi = ti.haar_rotation(d, 93) if rot == "haar" else ti.hadamard_rotation(d, 93)
+    s = ti.gaussian_sketch(m, d, 94)
     n_tok = 70
     keys = np.stack([np.stack([ti.key_stream(4, sq, h, n_tok + n_tail) for h in range(n_kv)]) for sq in range(n_seq)])
     comp = np.ascontiguousarray(keys[:, :, :n_tok])
@@ -224,14 +227,16 @@ def test_logits_many_heads(n_seq, n_kv, g, n_tail):
     c, t = _cb(d, B)
     q = ti.bf16_to_f64(qb)
     kf = ti.bf16_to_f64(keys)
-    for sq in range(0, n_seq, 7):
+    for sq in sorted(set(range(0, n_seq, 7)) | {n_seq - 1}):   # the last sequence ends in the last CTA
         for h in range(n_kv):
             st = sq * n_kv + h
             qh = q[sq, h * g:(h + 1) * g]
             want = oracle.logits(idx[st], sbit[st], nhat[st], ghat[st], pi, s, c, qh, qjl=True, scale=scale)
             _check_logits(got[sq, h * g:(h + 1) * g, :n_tok], want, qh, np.linalg.norm(kf[sq, h, :n_tok], axis=1), scale)
-            wt = oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)
-            _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1), scale)
+            if n_tail:
+                wt = oracle.exact_dot(kf[sq, h, n_tok:], qh, scale)
+                _check_logits(got[sq, h * g:(h + 1) * g, n_tok:], wt, qh, np.linalg.norm(kf[sq, h, n_tok:], axis=1),
+                              scale)
 
 
 def test_logits_d200_codec():
