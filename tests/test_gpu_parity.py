@@ -275,7 +275,8 @@ def _check_pv(got, want, P, nhat):
     return err.max()
 
 
-@pytest.mark.parametrize("B,g,n_tok", [(3, 4, 5000), (4, 4, 4097), (2, 1, 100), (4, 8, 777), (1, 2, 64)])
+@pytest.mark.parametrize("B,g,n_tok", [(3, 4, 5000), (4, 4, 4097), (2, 1, 100), (4, 8, 777), (1, 2, 64),
+                                       (3, 4, 1), (2, 4, 31)])
 def test_pv(B, g, n_tok):
     d = 128
     pi = ti.C3.pi()
