@@ -568,6 +568,36 @@ def test_rotation_flags_and_wht_logits(d, kind, qf32):
         _check_logits(lg[h * g:(h + 1) * g, n_tok:], tail, qh, np.linalg.norm(kf[h, n_tok:], axis=1), scale)
 
 
+def test_wht_prologue_matches_dense_product():
+    """The Walsh-Hadamard query transform against the dense mma.sync product on the same
+    rotation: a Hadamard Pi with one entry's magnitude moved by one fp32 ulp keeps the +-1 flag
+    but not the Sylvester one, so its logits take the dense path; both codecs score the same
+    packed keys (quantized under the exact Hadamard Pi) with the same queries."""
+    d = m_ = 128
+    pik = ti.hadamard_rotation(d, 71).astype(np.float32)
+    pid = pik.copy()
+    pid[5, 7] = np.nextafter(pid[5, 7], np.float32(2.0) * pid[5, 7])
+    sk = ti.gaussian_sketch(m_, d, 72)
+    kh, kd = make_codec(d, m_, 2, True, pik, sk), make_codec(d, m_, 2, True, pid, sk)
+    assert int(kh.prep[:4].cpu().numpy().view(np.uint32)[0]) == 3
+    assert int(kd.prep[:4].cpu().numpy().view(np.uint32)[0]) == 1
+    n_kv, n_tok, g = 4, 500, 4
+    keys = np.stack([ti.key_stream(4, 2, h, n_tok) for h in range(n_kv)])
+    pk, st = gpu_quantize(kh, to_dev_bf16(np.ascontiguousarray(keys).reshape(-1, d)), n_kv, n_tok)
+    assert st == tq().TQ_OK
+    qb = ti.decode_queries(15, 1, n_kv * g)
+    scale = 1.0 / math.sqrt(d)
+    lw = _logits_gpu(kh, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, None, 0, scale)[0]
+    ld = _logits_gpu(kd, pk, 1, n_kv, n_tok, to_dev_bf16(qb), g, None, 0, scale)[0]
+    q = ti.bf16_to_f64(qb)[0]
+    kn = np.linalg.norm(ti.bf16_to_f64(keys), axis=2)
+    for h in range(n_kv):
+        qh = q[h * g:(h + 1) * g]
+        err = np.abs(lw[h * g:(h + 1) * g] - ld[h * g:(h + 1) * g]) / (
+            scale * np.linalg.norm(qh, axis=1)[:, None] * kn[h][None, :])
+        assert err.max() <= 5e-4, err.max()
+
+
 def _unpack_q8(packed_dev, d, n_streams, n_tok):
     """Decode the 8-bit key blocks as the header describes them: codes [column][token][16 B],
     then binary16 scales [chunk][token]."""
