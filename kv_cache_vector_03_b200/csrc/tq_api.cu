@@ -426,7 +426,8 @@ int tq_pv(const tq_codec* c, const void* packed_v, int64_t n_seq, int n_kv, int6
     p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + W.ml);
     p.n_streams = n_streams; p.n_tok = n_tok; p.nb = (n_tok + 31) / 32;
     p.g = g; p.nsplit = W.nsplit; p.blocks_per_split = W.bps;
-    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    // grid sizes: the split CTAs, and the merge's four CTAs per query head
+    if (n_streams * W.nsplit > 0x7fffffffLL || n_streams * g * 4 > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
     p.t = t;
     if ((st = codebook_consts(c, &p.cb)) != TQ_OK) return st;
     return cuda_status(tq_launch_pv(p, static_cast<cudaStream_t>(stream)));
@@ -463,7 +464,8 @@ int tq_attention(const tq_codec* kcodec, const tq_codec* vcodec, const void* pac
     if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
     const AttnWs W = attn_ws(tk, n_streams, n_tok, g, n_tail);
     if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
-    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    // grid sizes: the split CTAs, and the merge's four CTAs per query head
+    if (n_streams * W.nsplit > 0x7fffffffLL || n_streams * g * 4 > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     const uint8_t* kprep = static_cast<const uint8_t*>(kcodec->prep);
     const TqPrepLayout L = tq_prep_layout(tk);
@@ -547,7 +549,8 @@ int tq_attention_q8(const tq_codec* vcodec, const void* packed_k8, const void* p
     if (n_streams * g > 0x7fffffffLL || n_streams * ((n_tok + 31) / 32) > (1LL << 40)) return TQ_ERR_UNSUPPORTED;
     const AttnQ8Ws W = attn_q8_ws(n_streams, n_tok, g, n_tail, vcodec->mse_bits);
     if (ws_bytes < W.total) return TQ_ERR_WORKSPACE;
-    if (n_streams * W.nsplit > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
+    // grid sizes: the split CTAs, and the merge's four CTAs per query head
+    if (n_streams * W.nsplit > 0x7fffffffLL || n_streams * g * 4 > 0x7fffffffLL) return TQ_ERR_UNSUPPORTED;
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     AttnParams p;
     std::memset(&p, 0, sizeof(p));
