@@ -289,10 +289,12 @@ def run_gpu(args, world, rank, local):
     # kernels launched per step: quantize 1, logits 2 (prologue + stream)
     launches_per_step = 3
     dominant = "tq_logits" if t_logit >= t_quant else "tq_quantize"
+    read_gbs = read_stream_gbs(torch)
     logits_roof = {"kernel": "tq_logits (prologue + int8-MMA stream)", "bound": "hbm", "achieved": round(logit_gbs, 1),
                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(logit_gbs / peaks["hbm_gbs"], 4),
                    "traffic": ncu_traffic("tq_logits"), "peak_kind": peak_kind,
-                   "algorithmic_bytes_per_launch": logit_bytes}
+                   "algorithmic_bytes_per_launch": logit_bytes,
+                   "read_stream_gbs": round(read_gbs, 1), "frac_of_read_stream": round(logit_gbs / read_gbs, 4)}
     # quantize: the roofline time is the larger of its algorithmic bytes at the HBM peak and its
     # algorithmic flops (two d x d contractions per vector, one pass each) at the dense bf16
     # peak; the kernel runs the contractions as split passes for fp32-equivalent precision
@@ -395,6 +397,25 @@ def ncu_traffic(kernel):
         if sha is None or _src_sha(name) != sha:
             return None
     return byts
+
+
+def read_stream_gbs(torch):
+    """A read-only streaming reference measured in this run: torch's sum over a 2 GiB fp32
+    buffer (device time per pass with CUDA events, best of 5), for context beside the
+    measured copy peak."""
+    x = torch.ones(1 << 29, dtype=torch.float32, device="cuda")
+    x.sum()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        x.sum()
+        b.record()
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b))
+    del x
+    return (1 << 31) / (best * 1e-3) / 1e9
 
 
 def time_calls(torch, fn, n_iter, n_warm=3):
