@@ -231,6 +231,60 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             }
             return;
         }
+        // 16-byte chunk c (0..15) of row r of a 128-byte swizzled image: K-block c / 8
+        auto bsw = [](int r, int c) { return (uint32_t)((c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4)); };
+        if constexpr (HPC <= 8) {
+            // up to 8 heads: the products transposed, one 16-output x 8-head tile per warp (warp
+            // w: product w / 8, outputs 16 (w mod 8) ..), so no MMA rows are spent on absent
+            // heads: A = the image rows (fp16 hi / lo), B = the query rows; hi.hi, lo.hi and,
+            // when a query row has a nonzero lo part, hi.lo, in separate accumulators
+            const int pw = wid >> 3, o0 = 16 * (wid & 7);
+            const int mi = lane >> 3, r8 = lane & 7;
+            const int a_row = o0 + (mi & 1) * 8 + r8, a_chk = mi >> 1;
+            const int b_row = r8, b_chk = mi & 1;
+            const int g = lane >> 2, t = lane & 3;
+            const uint32_t img = sbt + (uint32_t)(2 * pw) * (uint32_t)kTqImageBytes;
+            float acc[3][4];
+#pragma unroll
+            for (int x = 0; x < 3; ++x) acc[x][0] = acc[x][1] = acc[x][2] = acc[x][3] = 0.f;
+            if (!(wht && pw == 0)) {
+#pragma unroll
+                for (int kc = 0; kc < 8; ++kc) {
+                    uint32_t ih[4], il[4], qh[2], ql[2] = {0u, 0u};
+                    const uint32_t ao = bsw(a_row, 2 * kc + a_chk);
+                    tq_ldsm_x4(img + ao, ih[0], ih[1], ih[2], ih[3]);
+                    tq_ldsm_x4(img + (uint32_t)kTqImageBytes + ao, il[0], il[1], il[2], il[3]);
+                    tq_ldsm_x2(sat + tq_swz256(b_row, 2 * kc + b_chk), qh[0], qh[1]);
+                    if (a_lo) tq_ldsm_x2(sat + 4096 + tq_swz256(b_row, 2 * kc + b_chk), ql[0], ql[1]);
+                    tq_hmma(acc[0], ih[0], ih[1], ih[2], ih[3], qh[0], qh[1]);
+                    tq_hmma(acc[1], il[0], il[1], il[2], il[3], qh[0], qh[1]);
+                    if (a_lo) tq_hmma(acc[2], ih[0], ih[1], ih[2], ih[3], ql[0], ql[1]);
+                }
+                // accumulator r: output o0 + g (r < 2) or o0 + g + 8, head 2t + (r & 1)
+                const float f0 = pw == 0 ? 1.f / 256.f : inv_ss;
+                const float fe = s_qa[2 * t] * f0, fo = s_qa[2 * t + 1] * f0;
+                float* qe = qo + (2 * t) * 256 + 128 * pw + o0 + g;
+                const float v0 = ((acc[0][0] + acc[1][0]) + acc[2][0]) * fe;
+                const float v1 = ((acc[0][1] + acc[1][1]) + acc[2][1]) * fo;
+                const float v2 = ((acc[0][2] + acc[1][2]) + acc[2][2]) * fe;
+                const float v3 = ((acc[0][3] + acc[1][3]) + acc[2][3]) * fo;
+                qe[0] = v0;
+                qe[256] = v1;
+                qe[8] = v2;
+                qe[256 + 8] = v3;
+                // head maxima: the eight lanes of a head pair, then one shared atomic per head
+                float me = fmaxf(fabsf(v0), fabsf(v2)), mo = fmaxf(fabsf(v1), fabsf(v3));
+#pragma unroll
+                for (int sft = 4; sft < 32; sft <<= 1) {
+                    me = fmaxf(me, __shfl_xor_sync(0xffffffffu, me, sft));
+                    mo = fmaxf(mo, __shfl_xor_sync(0xffffffffu, mo, sft));
+                }
+                if (g == 0) {
+                    if (2 * t < HPC) atomicMax(&s_max[pw][2 * t], __float_as_uint(me));
+                    if (2 * t + 1 < HPC) atomicMax(&s_max[pw][2 * t + 1], __float_as_uint(mo));
+                }
+            }
+        } else {
         // one 16 x 8 output tile of each product per warp over K = 128: A hi/lo x B hi/lo
         // (hi.hi, hi.lo and, when some A lo part is nonzero, lo.hi, in separate accumulators)
         {
@@ -238,8 +292,6 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             const int a_row = (mi & 1) * 8 + r8, a_chk = mi >> 1;
             const int b_row = 8 * wid + r8, b_chk = mi & 1;
             const int g = lane >> 2, t = lane & 3;
-            // 16-byte chunk c (0..15) of row r of a 128-byte swizzled image: K-block c / 8
-            auto bsw = [](int r, int c) { return (uint32_t)((c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4)); };
             float ap[3][4], as[3][4];
 #pragma unroll
             for (int x = 0; x < 3; ++x)
@@ -296,6 +348,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                     atomicMax(&s_max[1][g + 8 * x], __float_as_uint(ms[x]));
                 }
             }
+        }
         }
         __syncthreads();   // qo, s_max
     } else {
@@ -409,19 +462,29 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
         __syncthreads();
     }
     // 2. fixed-point steps dA (code planes: max |q'| times the largest plane factor) and dS
-    //    (signs), 3. fragment words and 4. per-head scales: one warp per head (HPC <= 16 warps).
-    //    Lane -> chunk c, slot t, register hh of every plane group mg; byte bb of the word is
-    //    coordinate 128 gr + 32 t + 2c + hh + 8 bb, in column 2 (head % 4) (hi) or
-    //    2 (head % 4) + 1 (lo) of n-tile head / 4.
-    if (wid < H) {
-        const int h = wid;
+    //    (signs), 3. fragment words and 4. per-head scales: kNW = 16 / HPC warps per head, warp
+    //    sub of a head taking plane groups sub, sub + kNW, ... Lane -> chunk c, slot t, register
+    //    hh of a plane group mg; byte bb of the word is coordinate 128 gr + 32 t + 2c + hh + 8 bb,
+    //    in column 2 (head % 4) (hi) or 2 (head % 4) + 1 (lo) of n-tile head / 4.
+    constexpr int kNW = kPrologueThreads / 32 / HPC;
+    __shared__ int s_sum[2][HPC];
+    if constexpr (kNW > 1) {
+        if (tid < 2 * HPC) s_sum[tid / HPC][tid % HPC] = 0;
+        __syncthreads();
+    }
+    const int h = wid / kNW, sub = wid % kNW;
+    float dA = 1.f, dS = 1.f;
+    int stream = 0, head = 0;
+    if (h < H) {
         float amax = 0.f;
         for (int pl = 0; pl < np; ++pl) amax = fmaxf(amax, fabsf(2.f * p.cb.plane_coef[pl]));
         const float ma = __uint_as_float(s_max[0][h]) * amax, ms = __uint_as_float(s_max[1][h]);
-        const float dA = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
-        const float dS = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
+        dA = ma > 0.f ? ma / (float)kTqQueryMax : 1.f;
+        dS = ms > 0.f ? ms / (float)kTqQueryMax : 1.f;
         const float invA = 1.f / dA, invS = 1.f / dS;
-        const int gh = h_base + h, stream = gh / G, head = gh - stream * G;
+        const int gh = h_base + h;
+        stream = gh / G;
+        head = gh - stream * G;
         const int GDv = NR == 1 ? 1 : T.GD;
         const int c = lane >> 3, t = (lane >> 1) & 3, hh = lane & 1;
         // bit s = 2c + hh of the key bytes meets this register: factor 2^(3 - s mod 4)
@@ -430,7 +493,7 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
                         2 * t + hh;
         int sumA = 0, sumS = 0;
 #pragma unroll 2
-        for (int mg = 0; mg < nmg; ++mg) {
+        for (int mg = sub; mg < nmg; mg += kNW) {
             const bool is_code = mg < np * GDv;
             const int gr = is_code ? mg % GDv : mg - np * GDv;
             const float inv = is_code ? 2.f * p.cb.plane_coef[mg / GDv] * invA : invS;
@@ -455,14 +518,24 @@ __global__ void __launch_bounds__(kPrologueThreads) k_logits_prologue(LogitsPara
             sumA += __shfl_xor_sync(0xffffffffu, sumA, o);
             sumS += __shfl_xor_sync(0xffffffffu, sumS, o);
         }
-        // scales, folding the 128 of the u8 bit bytes, the QJL factor kappa and the attention
-        // scale: l = |x| (dA/128 accA - KA + gamma (kappa 2 dS/128 accS - kappa KS))
-        if (lane == 0) {
-            const float sa = p.scale;
-            reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
-                make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)sumA, sa * p.kappa * 2.f * dS / 128.f,
-                            sa * p.kappa * dS * (float)sumS);
+        if constexpr (kNW > 1) {
+            if (lane == 0) {
+                atomicAdd(&s_sum[0][h], sumA);
+                atomicAdd(&s_sum[1][h], sumS);
+            }
+        } else if (lane == 0) {
+            s_sum[0][h] = sumA;
+            s_sum[1][h] = sumS;
         }
+    }
+    if constexpr (kNW > 1) __syncthreads();   // every warp of a head has added its sums
+    // scales, folding the 128 of the u8 bit bytes, the QJL factor kappa and the attention
+    // scale: l = |x| (dA/128 accA - KA + gamma (kappa 2 dS/128 accS - kappa KS))
+    if (h < H && sub == 0 && lane == 0) {
+        const float sa = p.scale;
+        reinterpret_cast<float4*>(p.qscale)[(size_t)stream * p.ntiles * 4 + head] =
+            make_float4(sa * dA / 128.f, sa * 0.5f * dA * (float)s_sum[0][h], sa * p.kappa * 2.f * dS / 128.f,
+                        sa * p.kappa * dS * (float)s_sum[1][h]);
     }
 }
 
