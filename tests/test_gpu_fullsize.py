@@ -187,6 +187,10 @@ def test_c5_vector_search(b):
     all_scores = oracle.logits(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, qsamp, qjl=True)
     xn = np.linalg.norm(x.astype(np.float64), axis=1)
     swaps = check_topk(gidx[samp], gsc[samp], all_scores, qsamp, xn, k)
+    # the MSE-only ranking on the same records (no sign K-blocks) against the oracle's first term
+    midx, msc = _topk_gpu(codec, packed, n_db, to_dev_f32(qs), n_q, k, estimator=tq().TQ_EST_MSE)
+    mse_scores = oracle.logits(idx[0], sbit[0], nhat[0], ghat[0], pi, s, c, qsamp, qjl=False)
+    check_topk(midx[samp], msc[samp], mse_scores, qsamp, xn, k)
     # codes of a sample of database vectors
     vs = np.sort(RNG.choice(n_db, 2000, replace=False))
     ref = oracle.quantize(x[vs].astype(np.float64), pi, s, c, t, B, qjl=True)
