@@ -337,7 +337,7 @@ def run_gpu(args, world, rank, local):
                                                             out, wsl, stream), 20, 3)
         also["c4_query_prologue_plus_one_block"] = {"dense_rotation_ms": pro_ms, "walsh_hadamard_ms": hpro_ms,
                                                     "q_heads": N_SEQ * N_KV * G, "keys_per_stream": 32,
-                                                    "timing": "CUDA graph of 20 calls, inputs in L2"}
+                                                    "timing": "CUDA graph of 20 calls, median of 7 runs of 20 replays, inputs in L2"}
         also["c4_logits_hadamard_rotation"] = {"ms": hlog_ms, "keys_per_s": keys_per_step / (hlog_ms * 1e-3),
                                                "dense_rotation_ms": t_logit}
         # the same c4 logits with the MSE-only estimator (no sign-plane MMAs; same records read)
@@ -432,9 +432,10 @@ def time_calls(torch, fn, n_iter, n_warm=3):
     return a.elapsed_time(b) / n_iter
 
 
-def time_graph(torch, fn, n_calls, n_replays=20):
-    """Mean device time per call of fn(0) .. fn(n_calls - 1) captured once in a CUDA graph and
-    replayed n_replays times (host launch overhead amortised, as in a captured decode loop)."""
+def time_graph(torch, fn, n_calls, n_replays=20, n_runs=7):
+    """Device time per call of fn(0) .. fn(n_calls - 1) captured once in a CUDA graph: the
+    median over n_runs runs of n_replays back-to-back replays each (host launch overhead
+    amortised, as in a captured decode loop)."""
     for i in range(n_calls):   # first calls (one-time launch setup) outside the capture
         fn(i)
     torch.cuda.synchronize()
@@ -444,14 +445,17 @@ def time_graph(torch, fn, n_calls, n_replays=20):
             fn(i)
     graph.replay()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(n_replays):
-        graph.replay()
-    b.record()
-    torch.cuda.synchronize()
+    runs = []
+    for _ in range(n_runs):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(n_replays):
+            graph.replay()
+        b.record()
+        torch.cuda.synchronize()
+        runs.append(a.elapsed_time(b) / (n_replays * n_calls))
     del graph
-    return a.elapsed_time(b) / (n_replays * n_calls)
+    return float(np.median(runs))
 
 
 def extra_workloads(torch, tq, ti, gen, peaks):
@@ -483,7 +487,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         out[f"c2_llama8b_decode_logits_b{b}"] = {
             "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA-graph replays of 12 calls"}
+            "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA graph of 12 calls, median of 7 runs of 20 replays"}
         # the same decode step fused: logits -> online softmax -> P.V over packed keys and values
         # (value cache at b bits, MSE only), the 128 recent keys and values in bf16
         vcodec = tq.Codec(d, 0, b, False, torch.from_numpy(ti.C3.pi().astype(np.float32)), None)
@@ -503,7 +507,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         out[f"c2_llama8b_decode_attention_k{b}v{b}"] = {
             "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA-graph replays of 12 calls"}
+            "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA graph of 12 calls, median of 7 runs of 20 replays"}
         # sparse values: blocks whose weights are all below 1e-4 of the running maximum skip
         # their values (the bytes still stream: the value block shares the key block's stage)
         ms = time_graph(torch, lambda i: tq.tq_attention(codec, vcodec, packs[i % copies], vpacks[i % copies], 1, n_kv,
@@ -512,7 +516,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         out[f"c2_llama8b_decode_attention_k{b}v{b}_sparse_v1e-4"] = {
             "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "timing": "CUDA-graph replays of 12 calls"}
+            "timing": "CUDA graph of 12 calls, median of 7 runs of 20 replays"}
         del keys, packs, vals, vpacks
     # the key side of the asymmetric configuration at c2: 8-bit keys (q8_0-style), same queries and tail
     keys = make_keys_device(torch, gen, n_kv, n_all, n_kv)
@@ -531,7 +535,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
     out["c2_llama8b_decode_logits_q8_keys"] = {
         "ms": ms, "keys_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
         "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA-graph replays of 12 calls"}
+        "l2": f"{copies} rotating copies of the packed cache", "timing": "CUDA graph of 12 calls, median of 7 runs of 20 replays"}
     # the asymmetric decode step fused: 8-bit keys, 4-bit TurboQuant values, 128 bf16 tail tokens
     vcodec = tq.Codec(d, 0, 4, False, torch.from_numpy(ti.C3.pi().astype(np.float32)), None)
     vals = torch.randn((n_kv, n_all, d), generator=gen, device="cuda").to(torch.bfloat16)
@@ -549,7 +553,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
     out["c2_llama8b_decode_attention_q8_keys_v4"] = {
         "ms": ms, "tokens_per_s": n_kv * n_all / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
         "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-        "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA-graph replays of 12 calls"}
+        "l2": f"{copies} rotating copies of the packed keys and values", "timing": "CUDA graph of 12 calls, median of 7 runs of 20 replays"}
     del keys, q8s, vals, vpacks
     # c3: values at 128K, 8 kv-heads x 131072 tokens, 32 q-heads, P ~ N(0, 4)
     n_kv, n_tok, g = 8, 131072, 4
@@ -570,7 +574,7 @@ def extra_workloads(torch, tq, ti, gen, peaks):
         out[f"c3_values_128k_pv_{B}bit"] = {
             "ms": ms, "tokens_per_s": n_kv * n_tok / (ms * 1e-3), "GB_per_s": byts / (ms * 1e-3) / 1e9,
             "frac_of_measured_hbm": byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-            "l2": f"{copies} rotating copies of the packed values, 2 of P", "timing": "CUDA-graph replays of 4 calls"}
+            "l2": f"{copies} rotating copies of the packed values, 2 of P", "timing": "CUDA graph of 4 calls, median of 7 runs of 20 replays"}
         del packs
     del vals, P
     # c5: vector search, 1M x d=200 database (anisotropic, unit rows), 10,000 queries, top-10
